@@ -1,0 +1,193 @@
+/*
+ * svdq.h -- C ABI of the SVDQuant W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (SVDQuant; SOTA-314 practice page "Do this", NOTE-257 note page
+ * "Contribution" and "Key results") computes
+ *
+ *     Y = Q(X diag(lam)^-1) Q(R) + (X diag(lam)^-1 L1) L2 + b
+ *
+ * where lam are per-input-channel smoothing factors, W_hat = diag(lam) W,
+ * L1 = U Sigma[:, :r] and L2 = V^T[:r, :] are the top-r SVD factors of W_hat
+ * (r = 32 at 4 bits), and R = W_hat - L1 L2 is the residual, quantized to NVFP4
+ * (E2M1 values, groups of 16 along K, E4M3 scales, power-of-two FP32 tensor
+ * scale) or INT4 (groups of 64, BF16 scales).
+ *
+ * Conventions shared by every entry point:
+ *   - No exception or abort crosses this ABI; each call returns an svdq_status.
+ *   - Matrices are row-major, BF16 values are passed as their uint16_t bit
+ *     patterns, and "device" pointers are CUDA global-memory addresses of the
+ *     current process on the layer's device.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Forward calls are stream-ordered and asynchronous: they enqueue kernels
+ *     and return; they never synchronise (except with SVDQ_FWD_CHECK) and never
+ *     allocate memory.  The caller owns X, Y and the workspace.
+ *   - A layer owns its device buffers; svdq_destroy frees them.  A layer may be
+ *     used by several streams only if their forward calls do not overlap in time
+ *     on the device through a shared workspace.
+ *   - Shape rules: K % 64 == 0, N % 16 == 0, M >= 1 (any M: tails are handled).
+ *     Other shapes return SVDQ_EUNSUPPORTED.
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_EINVAL = 1,          /* null pointer, bad enum, inconsistent sizes          */
+  SVDQ_EUNSUPPORTED = 2,    /* shape or option this build does not implement       */
+  SVDQ_ENOMEM = 3,          /* host or device allocation failed (prepare only)     */
+  SVDQ_ECUDA = 4,           /* a CUDA runtime/driver call failed                   */
+  SVDQ_ENOCONVERGE = 5,     /* the truncated SVD did not converge                  */
+  SVDQ_ETIMEOUT = 6,        /* a bounded device wait expired (read with CHECK)     */
+  SVDQ_ESTATE = 7           /* the layer has no device copy (prepared host-only)   */
+} svdq_status;
+
+typedef enum {
+  SVDQ_NVFP4 = 0,           /* W4A4, E2M1 g16, E4M3 scales, FP32 tensor scales     */
+  SVDQ_INT4 = 1,            /* W4A4, symmetric INT4 g64, BF16 scales               */
+  SVDQ_W4A16_INT4 = 2       /* weight-only INT4 g64 (adaptive-norm linears)        */
+} svdq_format;
+
+/* Offline configuration.  rank: 32 (or 0 = no low-rank branch); alpha:
+ * smoothing migration strength (0.5).  flags: reserved, pass 0. */
+typedef struct {
+  int format;
+  int rank;
+  float alpha;
+  unsigned flags;
+} svdq_config;
+
+typedef struct svdq_layer svdq_layer;   /* opaque */
+
+/* Read-only description of a prepared layer. */
+typedef struct {
+  int K, N, rank, format;
+  int device;               /* CUDA ordinal, or -1 for a host-only layer           */
+  int g_x_exp, g_w_exp;     /* NVFP4 tensor scales g = 2^exp (0 for INT4)          */
+  int svd_iterations;       /* subspace iterations the SVD took                    */
+  double svd_tail_energy;   /* ||W_hat||_F^2 - sum_{i<r} sigma_i^2                 */
+} svdq_layer_info;
+
+/* Forward flags. */
+#define SVDQ_FWD_GELU      0x1u  /* tanh-GELU on the output (fc1 -> fc2 chains)      */
+#define SVDQ_FWD_UNFUSED   0x2u  /* measurement variant: separate down-projection,
+                                    quantize, bare GEMM and up-projection launches   */
+#define SVDQ_FWD_NO_BRANCH 0x4u  /* measurement variant: bare W4A4 GEMM + bias,
+                                    low-rank branch skipped (output is NOT the layer) */
+#define SVDQ_FWD_CHECK     0x8u  /* synchronise the stream and report a device
+                                    timeout as SVDQ_ETIMEOUT                          */
+
+/* Tensors that svdq_export copies to the host (logical, unswizzled layouts). */
+typedef enum {
+  SVDQ_T_LAMBDA = 0,        /* float [K]       smoothing factors lam                */
+  SVDQ_T_INV_LAMBDA = 1,    /* float [K]       fp32(1 / lam)                        */
+  SVDQ_T_L1 = 2,            /* double [K][r]   U Sigma[:, :r] of W_hat              */
+  SVDQ_T_L2 = 3,            /* double [r][N]   V^T[:r, :]                           */
+  SVDQ_T_L1D = 4,           /* uint16 [K][r]   bf16(diag(1/lam) L1)  (BF16 bits)    */
+  SVDQ_T_L2B = 5,           /* uint16 [r][N]   bf16(L2)                             */
+  SVDQ_T_RESIDUAL = 6,      /* float [K][N]    R = fp32(W_hat - diag(lam) L1d L2b)  */
+  SVDQ_T_SIGMA = 7,         /* double [r]      leading singular values of W_hat     */
+  SVDQ_T_W_CODES = 8,       /* uint8 [N][K/2]  residual codes, K-major, even k low  */
+  SVDQ_T_W_SCALES = 9,      /* NVFP4: uint8 [N][K/16] E4M3; INT4: uint16 [N][K/64] BF16 */
+  SVDQ_T_BIAS = 10,         /* float [N]                                            */
+  SVDQ_T_COUNT = 11
+} svdq_tensor;
+
+/* ------------------------------------------------------------------ offline */
+
+/* svdq_prepare -- smoothing, truncated SVD and residual quantization
+ * (SOTA-314 "Do this": smooth, "compute the SVD of the smoothed weight, keep
+ * the top r singular directions in 16 bits, and quantize only the residual").
+ *
+ *   cfg        format, rank (0 or 32), alpha (> 0 and < 1; 0.5 recommended).
+ *   K, N       input and output features.
+ *   W_bf16     host, [K][N] row-major BF16 weight (Y = X W + b); read only.
+ *   bias_bf16  host, [N] BF16, or NULL for no bias.
+ *   calib_bf16 host, [M_calib][K] BF16 calibration activations (smoothing
+ *              maxima and the activation tensor scale); required for the W4A4
+ *              formats, ignored (may be NULL) for SVDQ_W4A16_INT4.
+ *   device     CUDA ordinal that receives the prepared buffers, or -1 to keep
+ *              the layer on the host (export only; forwards return SVDQ_ESTATE).
+ *   out        receives the new layer; owned by the caller, free with svdq_destroy.
+ *
+ * Runs on the host (multi-threaded), then copies the prepared buffers to
+ * `device` with blocking copies.  Errors: SVDQ_EINVAL, SVDQ_EUNSUPPORTED,
+ * SVDQ_ENOMEM, SVDQ_ECUDA, SVDQ_ENOCONVERGE (the SVD's energy check failed).
+ * On error *out is set to NULL and nothing leaks. */
+svdq_status svdq_prepare(const svdq_config* cfg, int K, int N,
+                         const uint16_t* W_bf16, const uint16_t* bias_bf16,
+                         const uint16_t* calib_bf16, int M_calib,
+                         int device, svdq_layer** out);
+
+void svdq_destroy(svdq_layer* layer);
+
+svdq_status svdq_get_info(const svdq_layer* layer, svdq_layer_info* info);
+
+/* Bytes of tensor `id` (0 if the layer's format has no such tensor). */
+size_t svdq_tensor_bytes(const svdq_layer* layer, int id);
+
+/* Copy tensor `id` into host memory `dst` of `bytes` (must equal
+ * svdq_tensor_bytes).  Host-side; no GPU work. */
+svdq_status svdq_export(const svdq_layer* layer, int id, void* dst, size_t bytes);
+
+const char* svdq_status_string(svdq_status s);
+
+/* ------------------------------------------------------------------ forward */
+
+/* Workspace bytes a forward over M tokens needs (activation codes, scales in the
+ * tensor-core layout and the BF16 down projection X L1d).  0 on bad input. */
+size_t svdq_workspace_bytes(const svdq_layer* layer, int M);
+
+/* svdq_linear_forward -- the inference path.
+ *   X          device, [M][K] BF16 row-major, 16-byte aligned.
+ *   Y          device, [M][N] BF16 row-major, 16-byte aligned; fully overwritten.
+ *   workspace  device, >= svdq_workspace_bytes(layer, M), 256-byte aligned.
+ *   flags      SVDQ_FWD_* bits.
+ * W4A4 formats enqueue two kernels: the fused down-projection + quantize pass
+ * over X ("Down Projection with Quantize, because they read the same input")
+ * and the block-scaled tensor-core GEMM whose epilogue adds the up-projection
+ * and the bias ("Up Projection with the 4-bit compute, because they write the
+ * same output"; SOTA-314 "Do this").  W4A16 enqueues one weight-only kernel. */
+svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, void* Y,
+                                void* workspace, size_t workspace_bytes,
+                                void* stream, unsigned flags);
+
+/* The first kernel alone (NVFP4/INT4): writes the activation codes
+ * (device [M][K/2], even k in the low nibble), the activation scales in the
+ * tensor-core layout (device, svdq_act_scale_bytes(layer, M) bytes) and, when
+ * the layer has a branch, XL = bf16(X L1d) (device [M][rank] BF16).
+ * xl may be NULL for rank 0.  `mode` 0 = fused, 1 = quantize only,
+ * 2 = down projection only. */
+svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int M,
+                              void* codes, void* scales, void* xl,
+                              void* stream, int mode);
+
+/* The second kernel alone: Y from the first kernel's outputs.  flags:
+ * SVDQ_FWD_GELU, SVDQ_FWD_NO_BRANCH, SVDQ_FWD_CHECK. */
+svdq_status svdq_gemm(const svdq_layer* layer, const void* codes, const void* scales,
+                      const void* xl, int M, void* Y, void* stream, unsigned flags);
+
+/* Bytes of the activation scales for M tokens in the tensor-core layout. */
+size_t svdq_act_scale_bytes(const svdq_layer* layer, int M);
+
+/* Host-side: convert a host copy of activation scales in the tensor-core layout
+ * (svdq_act_scale_bytes bytes) into the logical layout: NVFP4 uint8 [M][K/16],
+ * INT4 uint16 [M][K/64]. */
+svdq_status svdq_act_scales_to_logical(const svdq_layer* layer, const void* device_layout,
+                                       int M, void* logical);
+
+/* Synchronise `stream` and report (and clear) the layer's device error word:
+ * SVDQ_ETIMEOUT if a bounded device wait expired since the last check. */
+svdq_status svdq_check(const svdq_layer* layer, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H */

@@ -1,0 +1,207 @@
+"""SVDQuant W4A4 linear layer for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/svdq.h`` (``libsvdq.so``,
+built in-tree by ``w4a4_diffusion_transformer_b200.build``).  The binding only
+marshals arguments: every step of the layer runs in the library (host C++ for
+the offline preparation, CUDA kernels for the forward).  There is no fallback:
+if the library is missing, importing ``lib`` raises.
+
+Device memory and streams come from the caller (for example PyTorch tensors:
+anything with ``data_ptr()``, or raw integer addresses).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvdq.so")
+
+# status codes (svdq_status)
+OK, EINVAL, EUNSUPPORTED, ENOMEM, ECUDA, ENOCONVERGE, ETIMEOUT, ESTATE = range(8)
+# formats (svdq_format)
+NVFP4, INT4, W4A16_INT4 = 0, 1, 2
+FORMATS = {"nvfp4": NVFP4, "int4": INT4, "w4a16": W4A16_INT4}
+# forward flags
+FWD_GELU, FWD_UNFUSED, FWD_NO_BRANCH, FWD_CHECK = 0x1, 0x2, 0x4, 0x8
+# exportable tensors (svdq_tensor)
+TENSORS = {
+    "lambda": (0, np.float32), "inv_lambda": (1, np.float32), "L1": (2, np.float64), "L2": (3, np.float64),
+    "L1d": (4, np.uint16), "L2b": (5, np.uint16), "R": (6, np.float32), "sigma": (7, np.float64),
+    "w_codes": (8, np.uint8), "w_scales": (9, None), "bias": (10, np.float32),
+}
+
+EXPORTED = [
+    "svdq_prepare", "svdq_destroy", "svdq_get_info", "svdq_tensor_bytes", "svdq_export",
+    "svdq_status_string", "svdq_workspace_bytes", "svdq_linear_forward", "svdq_quantize_act",
+    "svdq_gemm", "svdq_act_scale_bytes", "svdq_act_scales_to_logical", "svdq_check",
+]
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("format", ctypes.c_int), ("rank", ctypes.c_int), ("alpha", ctypes.c_float),
+                ("flags", ctypes.c_uint)]
+
+
+class LayerInfo(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int), ("N", ctypes.c_int), ("rank", ctypes.c_int), ("format", ctypes.c_int),
+                ("device", ctypes.c_int), ("g_x_exp", ctypes.c_int), ("g_w_exp", ctypes.c_int),
+                ("svd_iterations", ctypes.c_int), ("svd_tail_energy", ctypes.c_double)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libsvdq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m w4a4_diffusion_transformer_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, SZ, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint
+    sig = {
+        "svdq_prepare": (I, [ctypes.POINTER(Config), I, I, P, P, P, I, I, ctypes.POINTER(P)]),
+        "svdq_destroy": (None, [P]),
+        "svdq_get_info": (I, [P, ctypes.POINTER(LayerInfo)]),
+        "svdq_tensor_bytes": (SZ, [P, I]),
+        "svdq_export": (I, [P, I, P, SZ]),
+        "svdq_status_string": (ctypes.c_char_p, [I]),
+        "svdq_workspace_bytes": (SZ, [P, I]),
+        "svdq_linear_forward": (I, [P, P, I, P, P, SZ, P, U]),
+        "svdq_quantize_act": (I, [P, P, I, P, P, P, P, I]),
+        "svdq_gemm": (I, [P, P, P, P, I, P, P, U]),
+        "svdq_act_scale_bytes": (SZ, [P, I]),
+        "svdq_act_scales_to_logical": (I, [P, P, I, P]),
+        "svdq_check": (I, [P, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def status_string(s: int) -> str:
+    return load().svdq_status_string(int(s)).decode()
+
+
+def _ptr(x) -> Optional[int]:
+    """Device/host address of a tensor-like object (data_ptr()), an int, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return int(x.data_ptr())
+    if isinstance(x, np.ndarray):
+        return int(x.ctypes.data)
+    raise TypeError(f"cannot take the address of {type(x)}")
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return int(getattr(s, "cuda_stream"))
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise SvdqError(status, what)
+
+
+class Layer:
+    """A prepared SVDQuant layer (owns its device buffers)."""
+
+    def __init__(self, handle: int):
+        self._h = ctypes.c_void_p(handle)
+
+    @classmethod
+    def prepare(cls, W_bits: np.ndarray, bias_bits: Optional[np.ndarray], calib_bits: Optional[np.ndarray],
+                fmt: str = "nvfp4", rank: int = 32, alpha: float = 0.5, device: int = 0) -> "Layer":
+        """W_bits: uint16 [K][N] BF16 bit patterns (Y = X W + b); bias_bits: uint16 [N] or None;
+        calib_bits: uint16 [M_calib][K] or None (W4A16)."""
+        L = load()
+        W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+        K, N = W.shape
+        b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        c = None if calib_bits is None else np.ascontiguousarray(calib_bits, dtype=np.uint16)
+        cfg = Config(FORMATS[fmt], rank, alpha, 0)
+        out = ctypes.c_void_p()
+        st = L.svdq_prepare(ctypes.byref(cfg), K, N, _ptr(W), _ptr(b), _ptr(c),
+                            0 if c is None else c.shape[0], device, ctypes.byref(out))
+        _check(st, "svdq_prepare")
+        return cls(out.value)
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            load().svdq_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def info(self) -> dict:
+        i = LayerInfo()
+        _check(load().svdq_get_info(self._h, ctypes.byref(i)), "svdq_get_info")
+        return {f: getattr(i, f) for f, _ in LayerInfo._fields_}
+
+    def export(self, name: str) -> np.ndarray:
+        tid, dt = TENSORS[name]
+        info = self.info
+        K, N, r = info["K"], info["N"], info["rank"]
+        if dt is None:
+            dt = np.uint8 if info["format"] == NVFP4 else np.uint16
+        nbytes = load().svdq_tensor_bytes(self._h, tid)
+        buf = np.empty(nbytes // np.dtype(dt).itemsize, dtype=dt)
+        _check(load().svdq_export(self._h, tid, _ptr(buf), nbytes), f"svdq_export({name})")
+        shapes = {"lambda": (K,), "inv_lambda": (K,), "L1": (K, r), "L2": (r, N), "L1d": (K, r),
+                  "L2b": (r, N), "R": (K, N), "sigma": (r,), "w_codes": (N, K // 2), "bias": (N,),
+                  "w_scales": (N, -1)}
+        return buf.reshape(shapes[name])
+
+    def workspace_bytes(self, M: int) -> int:
+        return int(load().svdq_workspace_bytes(self._h, M))
+
+    def act_scale_bytes(self, M: int) -> int:
+        return int(load().svdq_act_scale_bytes(self._h, M))
+
+    def forward(self, X, M: int, Y, workspace, workspace_bytes: int, stream=None, flags: int = 0):
+        _check(load().svdq_linear_forward(self._h, _ptr(X), M, _ptr(Y), _ptr(workspace), workspace_bytes,
+                                          _stream(stream), flags), "svdq_linear_forward")
+
+    def quantize_act(self, X, M: int, codes, scales, xl, stream=None, mode: int = 0):
+        _check(load().svdq_quantize_act(self._h, _ptr(X), M, _ptr(codes), _ptr(scales), _ptr(xl),
+                                        _stream(stream), mode), "svdq_quantize_act")
+
+    def gemm(self, codes, scales, xl, M: int, Y, stream=None, flags: int = 0):
+        _check(load().svdq_gemm(self._h, _ptr(codes), _ptr(scales), _ptr(xl), M, _ptr(Y), _stream(stream),
+                                flags), "svdq_gemm")
+
+    def act_scales_to_logical(self, device_layout: np.ndarray, M: int) -> np.ndarray:
+        info = self.info
+        out = np.empty((M, info["K"] // 16), dtype=np.uint8)
+        src = np.ascontiguousarray(device_layout, dtype=np.uint8)
+        _check(load().svdq_act_scales_to_logical(self._h, _ptr(src), M, _ptr(out)), "svdq_act_scales_to_logical")
+        return out
+
+    def check(self, stream=None):
+        _check(load().svdq_check(self._h, _stream(stream)), "svdq_check")

@@ -1,0 +1,470 @@
+// C ABI of the SVDQuant W4A4 library: layer lifetime, device upload, tensor
+// maps, workspace layout and the forward launches (see include/svdq.h).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "kernels.h"
+#include "svdq_internal.h"
+
+using namespace svdq;
+
+struct svdq_layer {
+  HostPrep host;
+  int device = -1;
+  int num_sms = 0;
+  unsigned long long budget_ns = 2000000000ull;
+  // device buffers (owned)
+  float* d_inv_lam = nullptr;
+  __nv_bfloat16* d_l1t = nullptr;    // [32][K]   L1d^T
+  __nv_bfloat16* d_l2s = nullptr;    // [N][32]   (L2b / alpha)^T
+  __nv_bfloat16* d_l2t = nullptr;    // [N][32]   L2b^T (unfused up projection)
+  uint8_t* d_wq = nullptr;           // [N][K/2]
+  uint8_t* d_ws = nullptr;           // weight scales, tensor-core layout
+  float* d_bias = nullptr;           // [N]
+  int* d_err = nullptr;
+  CUtensorMap tm_wq, tm_l2s, tm_l1t;
+};
+
+namespace {
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D row-major tensor [rows][cols] of `elem` bytes, box [box_rows][box_cols].
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, uint64_t cols, uint64_t rows,
+              uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * (uint64_t)elem};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ helpers
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool w4a4(const svdq_layer* L) { return L->host.format == SVDQ_NVFP4 || L->host.format == SVDQ_INT4; }
+
+size_t act_scale_bytes(const HostPrep& h, int M) {
+  if (h.format != SVDQ_NVFP4) return 0;
+  return (size_t)((M + 127) / 128) * (size_t)(h.K / 64) * 512;
+}
+
+struct WsLayout {
+  size_t codes = 0, scales = 0, xl = 0, total = 0;
+};
+
+WsLayout ws_layout(const HostPrep& h, int M) {
+  WsLayout w;
+  w.codes = 0;
+  w.scales = align_up((size_t)M * (size_t)(h.K / 2), 256);
+  w.xl = w.scales + align_up(act_scale_bytes(h, M), 256);
+  w.total = w.xl + align_up((size_t)M * 32 * 2, 256);
+  return w;
+}
+
+template <class T>
+cudaError_t upload(T** dst, const void* src, size_t bytes) {
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(dst), std::max<size_t>(bytes, 16));
+  if (e != cudaSuccess) return e;
+  if (bytes) e = cudaMemcpy(*dst, src, bytes, cudaMemcpyHostToDevice);
+  return e;
+}
+
+void free_device(svdq_layer* L) {
+  if (L->device < 0) return;
+  DeviceGuard g(L->device);
+  cudaFree(L->d_inv_lam);
+  cudaFree(L->d_l1t);
+  cudaFree(L->d_l2s);
+  cudaFree(L->d_l2t);
+  cudaFree(L->d_wq);
+  cudaFree(L->d_ws);
+  cudaFree(L->d_bias);
+  cudaFree(L->d_err);
+  L->d_inv_lam = nullptr;
+}
+
+svdq_status upload_layer(svdq_layer* L, int device) {
+  DeviceGuard g(device);
+  if (!g.ok) return SVDQ_ECUDA;
+  const HostPrep& h = L->host;
+  const int K = h.K, N = h.N, r = h.rank;
+  L->device = device;
+  if (cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return SVDQ_ECUDA;
+  if (const char* b = std::getenv("SVDQ_WAIT_BUDGET_MS")) {
+    const double ms = std::atof(b);
+    if (ms > 0) L->budget_ns = (unsigned long long)(ms * 1e6);
+  }
+  cudaError_t e = cudaSuccess;
+  auto chk = [&](cudaError_t x) {
+    if (x != cudaSuccess && e == cudaSuccess) e = x;
+  };
+  chk(cudaMalloc(reinterpret_cast<void**>(&L->d_err), sizeof(int)));
+  if (e == cudaSuccess) chk(cudaMemset(L->d_err, 0, sizeof(int)));
+  chk(upload(&L->d_bias, h.bias.data(), sizeof(float) * N));
+  if (h.format == SVDQ_NVFP4) {
+    chk(upload(&L->d_inv_lam, h.inv_lam.data(), sizeof(float) * K));
+    chk(upload(&L->d_wq, h.w_codes.data(), h.w_codes.size()));
+    // weight scales in the tensor-core layout, rows padded to a multiple of 256
+    const int npad = (N + 255) / 256 * 256;
+    std::vector<uint8_t> ws((size_t)(npad / 128) * (K / 64) * 512, 0);
+    for (int n = 0; n < N; ++n)
+      for (int gi = 0; gi < K / 16; ++gi) ws[sf_offset(n, gi, K)] = h.w_scales_e4m3[(size_t)n * (K / 16) + gi];
+    chk(upload(&L->d_ws, ws.data(), ws.size()));
+    // low-rank branch: L1d^T for the first kernel, (L2b / alpha)^T and L2b^T for the second
+    std::vector<uint16_t> l1t((size_t)32 * K, 0), l2s((size_t)N * 32, 0), l2t((size_t)N * 32, 0);
+    const double inv_alpha = std::ldexp(1.0, -(h.g_x_exp + h.g_w_exp));
+    for (int i = 0; i < r; ++i) {
+      for (int k = 0; k < K; ++k) l1t[(size_t)i * K + k] = h.L1d[(size_t)k * r + i];
+      for (int n = 0; n < N; ++n) {
+        const uint16_t b = h.L2b[(size_t)i * N + n];
+        l2t[(size_t)n * 32 + i] = b;
+        l2s[(size_t)n * 32 + i] = bf16_from_double((double)bf16_to_float(b) * inv_alpha);
+      }
+    }
+    chk(upload(&L->d_l1t, l1t.data(), l1t.size() * 2));
+    chk(upload(&L->d_l2s, l2s.data(), l2s.size() * 2));
+    chk(upload(&L->d_l2t, l2t.data(), l2t.size() * 2));
+    if (e != cudaSuccess) return SVDQ_ECUDA;
+    bool ok = make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 256,
+                       CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&L->tm_l2s, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
+                       CU_TENSOR_MAP_SWIZZLE_64B) &&
+              make_map(&L->tm_l1t, L->d_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, 32, 64, 32,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return SVDQ_ECUDA;
+  }
+  return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+}
+
+svdq_status check_forward_args(const svdq_layer* L, const void* X, int M, const void* Y) {
+  if (!L || !X || !Y || M < 1) return SVDQ_EINVAL;
+  if (L->device < 0) return SVDQ_ESTATE;
+  if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(Y) & 15)) return SVDQ_EINVAL;
+  return SVDQ_OK;
+}
+
+K1Params k1_params(const svdq_layer* L, int M, void* codes, void* scales, void* xl) {
+  const HostPrep& h = L->host;
+  K1Params p;
+  p.M = M;
+  p.K = h.K;
+  p.c_x = (float)std::ldexp((double)(1.0f / 6.0f), -h.g_x_exp);
+  p.g_x = (float)std::ldexp(1.0, h.g_x_exp);
+  p.inv_lam = L->d_inv_lam;
+  p.codes = static_cast<uint8_t*>(codes);
+  p.scales = static_cast<uint8_t*>(scales);
+  p.xl = static_cast<__nv_bfloat16*>(xl);
+  p.err = L->d_err;
+  p.budget_ns = L->budget_ns;
+  return p;
+}
+
+svdq_status run_k1(const svdq_layer* L, const void* X, int M, void* codes, void* scales, void* xl,
+                   cudaStream_t stream, int mode) {
+  const HostPrep& h = L->host;
+  CUtensorMap tm_x;
+  if (!make_map(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.K, M, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ECUDA;
+  K1Params p = k1_params(L, M, codes, scales, xl);
+  return launch_k1(tm_x, L->tm_l1t, p, mode, stream) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+}
+
+svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
+                   cudaStream_t stream, bool branch, bool gelu) {
+  const HostPrep& h = L->host;
+  CUtensorMap tm_a, tm_xl;
+  if (!make_map(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ECUDA;
+  if (branch) {
+    if (!make_map(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return SVDQ_ECUDA;
+  } else {
+    tm_xl = tm_a;   // unused by the kernel
+  }
+  K2Params p;
+  p.M = M;
+  p.N = h.N;
+  p.K = h.K;
+  p.alpha = (float)std::ldexp(1.0, h.g_x_exp + h.g_w_exp);
+  p.sfa = static_cast<const uint8_t*>(scales);
+  p.sfb = L->d_ws;
+  p.bias = L->d_bias;
+  p.y = static_cast<__nv_bfloat16*>(Y);
+  p.err = L->d_err;
+  p.budget_ns = L->budget_ns;
+  p.branch = branch ? 1 : 0;
+  p.gelu = gelu ? 1 : 0;
+  return launch_k2(tm_a, L->tm_wq, tm_xl, L->tm_l2s, p, L->num_sms, stream) == cudaSuccess ? SVDQ_OK
+                                                                                          : SVDQ_ECUDA;
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+
+extern "C" {
+
+const char* svdq_status_string(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_EINVAL: return "invalid argument";
+    case SVDQ_EUNSUPPORTED: return "unsupported shape or option";
+    case SVDQ_ENOMEM: return "out of memory";
+    case SVDQ_ECUDA: return "CUDA error";
+    case SVDQ_ENOCONVERGE: return "truncated SVD did not converge";
+    case SVDQ_ETIMEOUT: return "device wait timed out";
+    case SVDQ_ESTATE: return "layer has no device copy";
+  }
+  return "unknown status";
+}
+
+svdq_status svdq_prepare(const svdq_config* cfg, int K, int N, const uint16_t* W_bf16, const uint16_t* bias_bf16,
+                         const uint16_t* calib_bf16, int M_calib, int device, svdq_layer** out) {
+  if (!out) return SVDQ_EINVAL;
+  *out = nullptr;
+  if (!cfg || !W_bf16 || K <= 0 || N <= 0) return SVDQ_EINVAL;
+  if (cfg->format < SVDQ_NVFP4 || cfg->format > SVDQ_W4A16_INT4) return SVDQ_EINVAL;
+  const bool wo = cfg->format == SVDQ_W4A16_INT4;
+  if (!wo) {
+    if (!calib_bf16 || M_calib < 1) return SVDQ_EINVAL;
+    if (!(cfg->alpha > 0.0f && cfg->alpha < 1.0f)) return SVDQ_EINVAL;
+    if (cfg->rank != 0 && cfg->rank != 32) return SVDQ_EUNSUPPORTED;
+  }
+  if (K % 64 != 0 || N % 16 != 0) return SVDQ_EUNSUPPORTED;
+  svdq_layer* L = new (std::nothrow) svdq_layer();
+  if (!L) return SVDQ_ENOMEM;
+  svdq_status st = host_prepare(*cfg, K, N, W_bf16, bias_bf16, calib_bf16, M_calib, L->host);
+  if (st == SVDQ_OK && device >= 0) {
+    st = upload_layer(L, device);
+    if (st != SVDQ_OK) free_device(L);
+  }
+  if (st != SVDQ_OK) {
+    delete L;
+    return st;
+  }
+  *out = L;
+  return SVDQ_OK;
+}
+
+void svdq_destroy(svdq_layer* L) {
+  if (!L) return;
+  free_device(L);
+  delete L;
+}
+
+svdq_status svdq_get_info(const svdq_layer* L, svdq_layer_info* info) {
+  if (!L || !info) return SVDQ_EINVAL;
+  info->K = L->host.K;
+  info->N = L->host.N;
+  info->rank = L->host.rank;
+  info->format = L->host.format;
+  info->device = L->device;
+  info->g_x_exp = L->host.g_x_exp;
+  info->g_w_exp = L->host.g_w_exp;
+  info->svd_iterations = L->host.svd_iterations;
+  info->svd_tail_energy = L->host.svd_tail_energy;
+  return SVDQ_OK;
+}
+
+size_t svdq_tensor_bytes(const svdq_layer* L, int id) {
+  if (!L) return 0;
+  const HostPrep& h = L->host;
+  switch (id) {
+    case SVDQ_T_LAMBDA:
+    case SVDQ_T_INV_LAMBDA: return h.lam.size() * 4;
+    case SVDQ_T_L1: return h.L1.size() * 8;
+    case SVDQ_T_L2: return h.L2.size() * 8;
+    case SVDQ_T_L1D: return h.L1d.size() * 2;
+    case SVDQ_T_L2B: return h.L2b.size() * 2;
+    case SVDQ_T_RESIDUAL: return h.R.size() * 4;
+    case SVDQ_T_SIGMA: return h.sigma.size() * 8;
+    case SVDQ_T_W_CODES: return h.w_codes.size();
+    case SVDQ_T_W_SCALES: return h.format == SVDQ_NVFP4 ? h.w_scales_e4m3.size() : h.w_scales_bf16.size() * 2;
+    case SVDQ_T_BIAS: return h.bias.size() * 4;
+  }
+  return 0;
+}
+
+svdq_status svdq_export(const svdq_layer* L, int id, void* dst, size_t bytes) {
+  if (!L || !dst) return SVDQ_EINVAL;
+  const size_t need = svdq_tensor_bytes(L, id);
+  if (need == 0 || bytes != need) return SVDQ_EINVAL;
+  const HostPrep& h = L->host;
+  const void* src = nullptr;
+  switch (id) {
+    case SVDQ_T_LAMBDA: src = h.lam.data(); break;
+    case SVDQ_T_INV_LAMBDA: src = h.inv_lam.data(); break;
+    case SVDQ_T_L1: src = h.L1.data(); break;
+    case SVDQ_T_L2: src = h.L2.data(); break;
+    case SVDQ_T_L1D: src = h.L1d.data(); break;
+    case SVDQ_T_L2B: src = h.L2b.data(); break;
+    case SVDQ_T_RESIDUAL: src = h.R.data(); break;
+    case SVDQ_T_SIGMA: src = h.sigma.data(); break;
+    case SVDQ_T_W_CODES: src = h.w_codes.data(); break;
+    case SVDQ_T_W_SCALES:
+      src = h.format == SVDQ_NVFP4 ? (const void*)h.w_scales_e4m3.data() : (const void*)h.w_scales_bf16.data();
+      break;
+    case SVDQ_T_BIAS: src = h.bias.data(); break;
+    default: return SVDQ_EINVAL;
+  }
+  std::memcpy(dst, src, bytes);
+  return SVDQ_OK;
+}
+
+size_t svdq_workspace_bytes(const svdq_layer* L, int M) {
+  if (!L || M < 1) return 0;
+  if (!w4a4(L)) return 0;
+  return ws_layout(L->host, M).total;
+}
+
+size_t svdq_act_scale_bytes(const svdq_layer* L, int M) {
+  if (!L || M < 1) return 0;
+  return act_scale_bytes(L->host, M);
+}
+
+svdq_status svdq_act_scales_to_logical(const svdq_layer* L, const void* device_layout, int M, void* logical) {
+  if (!L || !device_layout || !logical || M < 1) return SVDQ_EINVAL;
+  const HostPrep& h = L->host;
+  if (h.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
+  const uint8_t* src = static_cast<const uint8_t*>(device_layout);
+  uint8_t* dst = static_cast<uint8_t*>(logical);
+  const int G = h.K / 16;
+  for (int r = 0; r < M; ++r)
+    for (int gi = 0; gi < G; ++gi) dst[(size_t)r * G + gi] = src[sf_offset(r, gi, h.K)];
+  return SVDQ_OK;
+}
+
+svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int M, void* codes, void* scales, void* xl,
+                              void* stream, int mode) {
+  svdq_status st = check_forward_args(L, X, M, codes);
+  if (st != SVDQ_OK) return st;
+  if (L->host.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
+  if (mode < 0 || mode > 2) return SVDQ_EINVAL;
+  if (!scales && mode != 2) return SVDQ_EINVAL;
+  if (L->host.rank == 0 && mode == 2) return SVDQ_EINVAL;
+  if (L->host.rank == 0 && mode == 0) mode = 1;
+  if (L->host.rank > 0 && mode != 1 && !xl) return SVDQ_EINVAL;
+  DeviceGuard g(L->device);
+  if (!g.ok) return SVDQ_ECUDA;
+  return run_k1(L, X, M, codes, scales, xl, static_cast<cudaStream_t>(stream), mode);
+}
+
+svdq_status svdq_gemm(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
+                      void* stream, unsigned flags) {
+  svdq_status st = check_forward_args(L, codes, M, Y);
+  if (st != SVDQ_OK) return st;
+  if (L->host.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
+  if (!scales) return SVDQ_EINVAL;
+  const bool branch = L->host.rank > 0 && !(flags & SVDQ_FWD_NO_BRANCH);
+  if (branch && !xl) return SVDQ_EINVAL;
+  DeviceGuard g(L->device);
+  if (!g.ok) return SVDQ_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = run_k2(L, codes, scales, xl, M, Y, s, branch, (flags & SVDQ_FWD_GELU) != 0);
+  if (st == SVDQ_OK && (flags & SVDQ_FWD_CHECK)) st = svdq_check(L, stream);
+  return st;
+}
+
+svdq_status svdq_linear_forward(const svdq_layer* L, const void* X, int M, void* Y, void* workspace,
+                                size_t workspace_bytes, void* stream, unsigned flags) {
+  svdq_status st = check_forward_args(L, X, M, Y);
+  if (st != SVDQ_OK) return st;
+  if (L->host.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
+  const WsLayout w = ws_layout(L->host, M);
+  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return SVDQ_EINVAL;
+  DeviceGuard g(L->device);
+  if (!g.ok) return SVDQ_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* codes = ws + w.codes;
+  void* scales = ws + w.scales;
+  void* xl = ws + w.xl;
+  const bool gelu = (flags & SVDQ_FWD_GELU) != 0;
+  const bool has_branch = L->host.rank > 0;
+  if ((flags & SVDQ_FWD_UNFUSED) && has_branch) {
+    // measurement variant: down projection, quantize, bare GEMM, up projection
+    st = run_k1(L, X, M, codes, scales, xl, s, 2);
+    if (st == SVDQ_OK) st = run_k1(L, X, M, codes, scales, xl, s, 1);
+    if (st == SVDQ_OK) st = run_k2(L, codes, scales, xl, M, Y, s, false, false);
+    if (st == SVDQ_OK) {
+      UpParams up;
+      up.M = M;
+      up.N = L->host.N;
+      up.xl = static_cast<const __nv_bfloat16*>(xl);
+      up.l2t = L->d_l2t;
+      up.y = static_cast<__nv_bfloat16*>(Y);
+      up.gelu = gelu ? 1 : 0;
+      st = launch_upproj(up, s) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+    }
+  } else {
+    const bool branch = has_branch && !(flags & SVDQ_FWD_NO_BRANCH);
+    st = run_k1(L, X, M, codes, scales, xl, s, branch ? 0 : 1);
+    if (st == SVDQ_OK) st = run_k2(L, codes, scales, xl, M, Y, s, branch, gelu);
+  }
+  if (st == SVDQ_OK && (flags & SVDQ_FWD_CHECK)) st = svdq_check(L, stream);
+  return st;
+}
+
+svdq_status svdq_check(const svdq_layer* L, void* stream) {
+  if (!L) return SVDQ_EINVAL;
+  if (L->device < 0) return SVDQ_ESTATE;
+  DeviceGuard g(L->device);
+  if (!g.ok) return SVDQ_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int err = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SVDQ_ECUDA;
+  if (cudaMemcpy(&err, L->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ECUDA;
+  if (err != 0) {
+    cudaMemset(L->d_err, 0, sizeof(int));
+    return SVDQ_ETIMEOUT;
+  }
+  return SVDQ_OK;
+}
+
+}  // extern "C"

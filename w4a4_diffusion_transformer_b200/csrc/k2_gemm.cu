@@ -1,0 +1,305 @@
+// K2: NVFP4 block-scaled GEMM with the low-rank up projection fused into the
+// same accumulator.
+//
+// SOTA-314 practice page, "Do this": the fusion pairs "Up Projection with the
+// 4-bit compute, because they write the same output"; NOTE-257 note page, "Key
+// results": unfused, the branch costs "the extra 16-bit write in Up
+// Projection".  For a 128 x 256 output tile:
+//
+//   acc  = XL (L2b / alpha)                        (2 BF16 MMAs, K = 32)
+//   acc += sum_k (c_x s_x) (c_w s_w)               (NVFP4 MMAs, K = 64 each)
+//   Y    = bf16( [gelu]( alpha * acc + b ) )       (one BF16 store)
+//
+// where alpha = g_x g_w is a power of two, so L2b / alpha is exact in BF16 and
+// alpha * acc reproduces Q(X^)Q(R) + XL L2b.
+//
+// Structure (one CTA per SM, persistent over output tiles):
+//   warp 0     TMA producer: per stage a 128 x 256 E2M1 A tile, a 256 x 256 E2M1
+//              B tile (128-byte swizzle), and the E4M3 scale factors (bulk
+//              copies, already in the tensor-core layout); per tile one extra
+//              stage with the XL tile and the L2b^T tile (64-byte swizzle).
+//   warp 1     allocates TMEM (512 columns: accumulator 256 + per-stage scale factors) and
+//              issues tcgen05.cp (scales smem -> TMEM) and tcgen05.mma.
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator, alpha, bias, GELU, BF16.
+// Pipelines are mbarrier rings; every wait is bounded (sm100.cuh).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace svdq {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBKBytes = 128;               // 256 E2M1 values per row per stage
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kABytes = kBM * kBKBytes;      // 16 KiB
+constexpr int kBBytes = kBN * kBKBytes;      // 32 KiB
+constexpr int kSFABytes = 4 * 512;           // 4 K-blocks x 128 rows
+constexpr int kSFBBytes = 2 * 4 * 512;       // 2 row blocks x 4 K-blocks
+constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;   // 54 KiB
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr int kTmemCols = 512;
+// Scale factors in TMEM, one region per pipeline stage (so a region is only
+// rewritten after the MMAs that read it have completed): 4 columns per 128-row
+// x 64-K block, 16 for A and 32 for B per stage.
+constexpr int kSFCol0 = 256;
+constexpr int kSFStageCols = 48;
+static_assert(kSFCol0 + kStages * kSFStageCols <= kTmemCols, "TMEM budget");
+
+__device__ __forceinline__ void record_error(int* err, volatile int* abort_flag, int code) {
+  atomicCAS(err, 0, code);
+  *abort_flag = 1;
+}
+
+__device__ __forceinline__ float gelu_tanh(float y) {
+  const float k0 = 0.7978845608028654f;   // sqrt(2/pi)
+  return 0.5f * y * (1.0f + tanhf(k0 * (y + 0.044715f * y * y * y)));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+              const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2, K2Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int M = p.M, N = p.N, K = p.K;
+  const int tiles_m = (M + kBM - 1) / kBM;
+  const int tiles_n = (N + kBN - 1) / kBN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int kblocks = K >> 6;                     // 64-element K blocks
+  const int ktiles = (kblocks + 3) >> 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      dev::mbar_init(&full[s], 1);
+      dev::mbar_init(&empty[s], 1);
+    }
+    dev::mbar_init(acc_full, 1);
+    dev::mbar_init(acc_empty, 4);
+    dev::mbar_init(drain, 1);
+    *abort_flag = 0;
+    dev::fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    dev::tmem_alloc(tmem_slot, kTmemCols);
+    dev::tmem_relinquish();
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      dev::tma_prefetch_desc(&tm_a);
+      dev::tma_prefetch_desc(&tm_b);
+      if (p.branch) {
+        dev::tma_prefetch_desc(&tm_xl);
+        dev::tma_prefetch_desc(&tm_l2);
+      }
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % tiles_m) * kBM;
+        const int n0 = (tile / tiles_m) * kBN;
+        if (p.branch) {
+          const int s = it % kStages;
+          if (!dev::mbar_wait(&empty[s], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+            record_error(p.err, abort_flag, 0x201);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStageBytes;
+          dev::mbar_arrive_expect_tx(&full[s], kBM * 64 + kBN * 64);
+          dev::tma_load_2d(st, &tm_xl, &full[s], 0, m0);
+          dev::tma_load_2d(st + kABytes, &tm_l2, &full[s], 0, n0);
+          ++it;
+        }
+        for (int kt = 0; kt < ktiles; ++kt) {
+          const int s = it % kStages;
+          if (!dev::mbar_wait(&empty[s], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+            record_error(p.err, abort_flag, 0x202);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStageBytes;
+          const int nkb = min(4, kblocks - 4 * kt);
+          const uint32_t sf_bytes = (uint32_t)nkb * 512u;
+          dev::mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + 3u * sf_bytes);
+          dev::tma_load_2d(st, &tm_a, &full[s], kt * kBKBytes, m0);
+          dev::tma_load_2d(st + kABytes, &tm_b, &full[s], kt * kBKBytes, n0);
+          const size_t a_chunk = (size_t)(m0 >> 7) * (size_t)kblocks + (size_t)(4 * kt);
+          dev::bulk_load(st + kABytes + kBBytes, p.sfa + a_chunk * 512, sf_bytes, &full[s]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const size_t b_chunk = (size_t)((n0 >> 7) + h) * (size_t)kblocks + (size_t)(4 * kt);
+            dev::bulk_load(st + kABytes + kBBytes + kSFABytes + h * 2048, p.sfb + b_chunk * 512, sf_bytes,
+                           &full[s]);
+          }
+          ++it;
+        }
+      }
+      for (int j = max(0, it - kStages); j < it; ++j)
+        if (!dev::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns)) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_f4 = dev::idesc_nvfp4(kBM, kBN);
+      const uint32_t idesc_h = dev::idesc_bf16(kBM, kBN);
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
+        if (!dev::mbar_wait(acc_empty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+          record_error(p.err, abort_flag, 0x203);
+          ok = false;
+          break;
+        }
+        dev::tc_fence_after();
+        uint32_t accumulate = 0;
+        if (p.branch) {
+          const int s = it % kStages;
+          if (!dev::mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
+            record_error(p.err, abort_flag, 0x204);
+            ok = false;
+            break;
+          }
+          dev::tc_fence_after();
+          const uint32_t a0 = dev::smem_u32(smem + s * kStageBytes);
+          const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint64_t ad = dev::smem_desc(a0 + 32 * j, 16, 512, 4);
+            const uint64_t bd = dev::smem_desc(b0 + 32 * j, 16, 512, 4);
+            dev::mma_bf16(tmem, ad, bd, idesc_h, accumulate);
+            accumulate = 1;
+          }
+          dev::tc_commit(&empty[s]);
+          ++it;
+        }
+        for (int kt = 0; kt < ktiles; ++kt) {
+          const int s = it % kStages;
+          if (!dev::mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
+            record_error(p.err, abort_flag, 0x205);
+            ok = false;
+            break;
+          }
+          dev::tc_fence_after();
+          const int nkb = min(4, kblocks - 4 * kt);
+          const uint32_t a0 = dev::smem_u32(smem + s * kStageBytes);
+          const uint32_t b0 = a0 + kABytes;
+          const uint32_t sfa0 = b0 + kBBytes;
+          const uint32_t sfb0 = sfa0 + kSFABytes;
+          const uint32_t tsfa = tmem + kSFCol0 + s * kSFStageCols;
+          const uint32_t tsfb = tsfa + 16;
+          for (int j = 0; j < nkb; ++j) {
+            dev::tmem_copy_32x128b_x4(tsfa + 4 * j, dev::smem_desc(sfa0 + 512 * j, 0, 128, 0));
+            dev::tmem_copy_32x128b_x4(tsfb + 8 * j, dev::smem_desc(sfb0 + 512 * j, 0, 128, 0));
+            dev::tmem_copy_32x128b_x4(tsfb + 8 * j + 4, dev::smem_desc(sfb0 + 2048 + 512 * j, 0, 128, 0));
+          }
+          for (int j = 0; j < nkb; ++j) {
+            const uint64_t ad = dev::smem_desc(a0 + 32 * j, 16, 1024, 2);
+            const uint64_t bd = dev::smem_desc(b0 + 32 * j, 16, 1024, 2);
+            dev::mma_nvfp4(tmem, ad, bd, idesc_f4, tsfa + 4 * j, tsfb + 8 * j, accumulate);
+            accumulate = 1;
+          }
+          dev::tc_commit(&empty[s]);
+          ++it;
+        }
+        if (!ok) break;
+        dev::tc_commit(acc_full);
+      }
+      // Wait until every MMA and copy this thread issued has completed.
+      dev::tc_commit(drain);
+      dev::mbar_wait(drain, 0, abort_flag, p.budget_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                          // TMEM lane quarter of this warp
+    const int r_in_tile = q * 32 + lane;
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+      const int m0 = (tile % tiles_m) * kBM;
+      const int n0 = (tile / tiles_m) * kBN;
+      const bool got = dev::mbar_wait(acc_full, (uint32_t)tcount & 1u, abort_flag, p.budget_ns);
+      if (!__all_sync(0xffffffffu, got)) {          // warp-uniform exit (tcgen05.ld is warp-collective)
+        if (lane == 0) record_error(p.err, abort_flag, 0x206);
+        break;
+      }
+      dev::tc_fence_after();
+      const int row = m0 + r_in_tile;
+      __nv_bfloat16* yrow = p.y + (size_t)row * (size_t)N;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t r[32];
+        dev::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
+        dev::tmem_load_wait();
+        const int nb = n0 + c * 32;
+        if (row < M && nb < N) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int n = nb + v * 8;
+            if (n < N) {
+              uint32_t packed[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float y0 = p.alpha * __uint_as_float(r[v * 8 + 2 * e]) + __ldg(p.bias + n + 2 * e);
+                float y1 = p.alpha * __uint_as_float(r[v * 8 + 2 * e + 1]) + __ldg(p.bias + n + 2 * e + 1);
+                if (p.gelu) {
+                  y0 = gelu_tanh(y0);
+                  y1 = gelu_tanh(y1);
+                }
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+                packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(yrow + n) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            }
+          }
+        }
+      }
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(acc_empty);
+    }
+  }
+
+  dev::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    dev::tc_fence_after();
+    dev::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int k2_block_n() { return kBN; }
+
+cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
+                      const CUtensorMap& tm_l2, const K2Params& p, int num_sms, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(k2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  k2_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_xl, tm_l2, p);
+  return cudaGetLastError();
+}
+
+}  // namespace svdq

@@ -1,0 +1,57 @@
+// Kernel parameter blocks and launchers (internal to the library).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "svdq_internal.h"
+
+namespace svdq {
+
+struct K1Params {
+  int M, K;
+  float c_x;                    // fp32(1/6) * 2^-g_x_exp
+  float g_x;                    // 2^g_x_exp
+  const float* inv_lam;         // [K]
+  uint8_t* codes;               // [M][K/2]
+  uint8_t* scales;              // tensor-core scale layout, ceil(M/128)*128 rows
+  __nv_bfloat16* xl;            // [M][32]
+  int* err;                     // device error word
+  unsigned long long budget_ns; // bound on each wait
+};
+
+struct K2Params {
+  int M, N, K;
+  float alpha;                  // g_x * g_w (power of two)
+  const uint8_t* sfa;           // activation scales, tensor-core layout
+  const uint8_t* sfb;           // weight scales, tensor-core layout (rows padded to 256)
+  const float* bias;            // [N]
+  __nv_bfloat16* y;             // [M][N]
+  int* err;
+  unsigned long long budget_ns;
+  int branch;                   // 1: add XL (L2b / alpha) into the accumulator
+  int gelu;                     // 1: tanh-GELU epilogue
+};
+
+struct UpParams {
+  int M, N;
+  const __nv_bfloat16* xl;      // [M][32]
+  const __nv_bfloat16* l2t;     // [N][32] = L2b^T
+  __nv_bfloat16* y;             // [M][N], read and rewritten
+  int gelu;
+};
+
+// mode 0 = fused, 1 = quantize only, 2 = down projection only
+cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const K1Params& p, int mode,
+                      cudaStream_t stream);
+int k1_rows_per_cta();
+
+cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
+                      const CUtensorMap& tm_l2, const K2Params& p, int num_sms, cudaStream_t stream);
+int k2_block_n();
+
+cudaError_t launch_upproj(const UpParams& p, cudaStream_t stream);
+
+}  // namespace svdq

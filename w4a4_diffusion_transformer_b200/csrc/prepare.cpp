@@ -1,0 +1,529 @@
+// Offline preparation of an SVDQuant W4A4 layer on the host.
+//
+// SOTA-314 practice page, "Do this": smooth the activation outliers into the
+// weights, compute the SVD of the smoothed weight W_hat, keep the top r
+// singular directions in 16 bits and quantize only the residual
+// R = W_hat - L1 L2 (rank 32 at 4 bits; INT4 groups of 64 with 16-bit scales,
+// NVFP4 groups of 16 with FP8 scales).  NOTE-257 note page, "Key results":
+// L1 = U Sigma[:, :r], L2 = V^T[:r, :]; Eckart-Young makes the truncated SVD the
+// optimal rank-r reduction.
+//
+// Choices where the pages are silent (all documented for users of the ABI):
+//  * lam_k = max|Xc[:,k]|^alpha / max|W[k,:]|^(1-alpha); alpha = 0.5 is computed
+//    as fp32(sqrt(ax)) / fp32(sqrt(aw)) in float32; a zero maximum gives lam = 1.
+//  * the down factor carries 1/lam: L1d = bf16(diag(1/lam) L1), L2b = bf16(L2),
+//    and the residual subtracts that stored branch: R = fp32(W_hat - diag(lam) L1d L2b).
+//  * NVFP4 tensor scales are powers of two: g_w = 2^ceil(log2(amax|R| / 2688)),
+//    g_x = 2^ceil(log2(4 amax|fp32(Xc / lam)| / 2688)) from the calibration batch.
+//  * RTN = round to nearest, ties to even, saturating.
+//
+// The truncated SVD is a block subspace iteration in float64 (block r + 32,
+// Gaussian start, re-orthonormalised every half step) with a Rayleigh-Ritz
+// extraction; it stops when the captured energy sum_{i<r} sigma_i^2 stops
+// changing.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <memory>
+#include <new>
+#include <vector>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#include "svdq_internal.h"
+
+namespace svdq {
+
+// ------------------------------------------------------------------ formats
+
+float bf16_to_float(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+uint16_t bf16_from_double(double x) {
+  if (x == 0.0) return std::signbit(x) ? 0x8000 : 0x0000;
+  int e;
+  std::frexp(x, &e);                                   // |x| = m 2^e, m in [0.5, 1)
+  const double q = std::ldexp(1.0, std::max(e - 8, -133));
+  const double r = std::nearbyint(x / q) * q;          // ties to even
+  const float f = (float)r;                            // exact: <= 8 significant bits
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return (uint16_t)(u >> 16);
+}
+
+uint8_t e4m3_from_nonneg(float t) {
+  if (!(t > 0.0f)) return 0;
+  if (t >= 448.0f) return 0x7E;
+  int e;
+  std::frexp((double)t, &e);
+  const double q = std::ldexp(1.0, std::max(e - 4, -9));
+  double r = std::nearbyint((double)t / q) * q;
+  if (r > 448.0) r = 448.0;
+  if (r == 0.0) return 0;
+  if (r < 0.015625) return (uint8_t)(r / 0.001953125);         // subnormal, quantum 2^-9
+  int re;
+  const double m = std::frexp(r, &re);                          // r = m 2^re
+  const int ebits = (re - 1) + 7;
+  const int mbits = (int)((2.0 * m - 1.0) * 8.0);
+  return (uint8_t)(ebits * 8 + mbits);
+}
+
+float e4m3_to_float(uint8_t b) {
+  const int e = (b >> 3) & 0xF, m = b & 7;
+  const double v = e == 0 ? m * 0.001953125 : (1.0 + m / 8.0) * std::ldexp(1.0, e - 7);
+  return (float)((b & 0x80) ? -v : v);
+}
+
+uint8_t e2m1_code(float q) {
+  const float a = std::fabs(q);
+  uint8_t mag;
+  if (a <= 0.25f) mag = 0;
+  else if (a < 0.75f) mag = 1;
+  else if (a <= 1.25f) mag = 2;
+  else if (a < 1.75f) mag = 3;
+  else if (a <= 2.5f) mag = 4;
+  else if (a < 3.5f) mag = 5;
+  else if (a <= 5.0f) mag = 6;
+  else mag = 7;
+  return (uint8_t)((std::signbit(q) ? 8 : 0) | mag);
+}
+
+int pow2_ceil_exponent(double x) {
+  if (!(x > 0.0)) return 0;
+  int e;
+  const double m = std::frexp(x, &e);
+  return m == 0.5 ? e - 1 : e;
+}
+
+// ------------------------------------------------------------------ dense helpers
+
+namespace {
+
+// Deterministic standard normals: splitmix64 + Box-Muller.
+struct Rng {
+  uint64_t s;
+  explicit Rng(uint64_t seed) : s(seed) {}
+  uint64_t next() {
+    uint64_t z = (s += 0x9E3779B97F4A7C15ull);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+  }
+  double uniform() { return ((next() >> 11) + 0.5) * (1.0 / 9007199254740992.0); }
+  double normal() {
+    const double u1 = uniform(), u2 = uniform();
+    return std::sqrt(-2.0 * std::log(u1)) * std::cos(6.283185307179586 * u2);
+  }
+};
+
+// Y[K][b] = A[K][N] * Z[N][b]   (all row-major)
+void gemm_AZ(const double* A, int K, int N, const double* Z, int b, double* Y) {
+#pragma omp parallel for schedule(static)
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    const int k1 = std::min(K, k0 + 8);
+    double acc[8][128];
+    for (int i = 0; i < k1 - k0; ++i)
+      for (int j = 0; j < b; ++j) acc[i][j] = 0.0;
+    for (int n = 0; n < N; ++n) {
+      const double* z = Z + (size_t)n * b;
+      for (int i = 0; i < k1 - k0; ++i) {
+        const double a = A[(size_t)(k0 + i) * N + n];
+        double* ac = acc[i];
+        for (int j = 0; j < b; ++j) ac[j] += a * z[j];
+      }
+    }
+    for (int i = 0; i < k1 - k0; ++i)
+      std::memcpy(Y + (size_t)(k0 + i) * b, acc[i], sizeof(double) * b);
+  }
+}
+
+// Z[N][b] = A^T * Q   with A[K][N], Q[K][b]
+void gemm_AtQ(const double* A, int K, int N, const double* Q, int b, double* Z) {
+#pragma omp parallel for schedule(static)
+  for (int n0 = 0; n0 < N; n0 += 32) {
+    const int n1 = std::min(N, n0 + 32);
+    double* zb = Z + (size_t)n0 * b;
+    std::fill(zb, zb + (size_t)(n1 - n0) * b, 0.0);
+    for (int k = 0; k < K; ++k) {
+      const double* q = Q + (size_t)k * b;
+      const double* a = A + (size_t)k * N;
+      for (int n = n0; n < n1; ++n) {
+        const double av = a[n];
+        double* z = Z + (size_t)n * b;
+        for (int j = 0; j < b; ++j) z[j] += av * q[j];
+      }
+    }
+  }
+}
+
+// Orthonormalise the b columns of row-major X[rows][b] in place (modified
+// Gram-Schmidt, two passes).  A column that vanishes is replaced by a random
+// direction orthogonal to the previous ones.
+void orthonormalize(double* X, int rows, int b, Rng& rng) {
+  std::vector<double> C((size_t)rows * b);
+  for (int r = 0; r < rows; ++r)
+    for (int j = 0; j < b; ++j) C[(size_t)j * rows + r] = X[(size_t)r * b + j];
+  for (int j = 0; j < b; ++j) {
+    double* cj = C.data() + (size_t)j * rows;
+    double n0 = 0.0;
+    for (int r = 0; r < rows; ++r) n0 += cj[r] * cj[r];
+    n0 = std::sqrt(n0);
+    for (int attempt = 0; attempt < 4; ++attempt) {
+      for (int pass = 0; pass < 2; ++pass) {
+        for (int i = 0; i < j; ++i) {
+          const double* ci = C.data() + (size_t)i * rows;
+          double d = 0.0;
+          for (int r = 0; r < rows; ++r) d += ci[r] * cj[r];
+          for (int r = 0; r < rows; ++r) cj[r] -= d * ci[r];
+        }
+      }
+      double nn = 0.0;
+      for (int r = 0; r < rows; ++r) nn += cj[r] * cj[r];
+      nn = std::sqrt(nn);
+      if (nn > 1e-10 * std::max(n0, 1e-300) && nn > 1e-200) {
+        for (int r = 0; r < rows; ++r) cj[r] /= nn;
+        break;
+      }
+      for (int r = 0; r < rows; ++r) cj[r] = rng.normal();
+      n0 = 0.0;
+      for (int r = 0; r < rows; ++r) n0 += cj[r] * cj[r];
+      n0 = std::sqrt(n0);
+    }
+  }
+  for (int r = 0; r < rows; ++r)
+    for (int j = 0; j < b; ++j) X[(size_t)r * b + j] = C[(size_t)j * rows + r];
+}
+
+// Symmetric eigen-decomposition of T[b][b] (cyclic Jacobi).  On return the
+// eigenvalues are in w (descending) and the eigenvectors are the columns of E.
+void sym_eig(std::vector<double> T, int b, std::vector<double>& w, std::vector<double>& E) {
+  E.assign((size_t)b * b, 0.0);
+  for (int i = 0; i < b; ++i) E[(size_t)i * b + i] = 1.0;
+  auto at = [&](int i, int j) -> double& { return T[(size_t)i * b + j]; };
+  for (int sweep = 0; sweep < 100; ++sweep) {
+    double off = 0.0, tot = 0.0;
+    for (int i = 0; i < b; ++i)
+      for (int j = 0; j < b; ++j) {
+        tot += at(i, j) * at(i, j);
+        if (i != j) off += at(i, j) * at(i, j);
+      }
+    if (off <= 1e-30 * tot || off == 0.0) break;
+    for (int p = 0; p < b - 1; ++p)
+      for (int q = p + 1; q < b; ++q) {
+        const double apq = at(p, q);
+        if (std::fabs(apq) < 1e-300) continue;
+        const double theta = (at(q, q) - at(p, p)) / (2.0 * apq);
+        const double t = (theta >= 0 ? 1.0 : -1.0) / (std::fabs(theta) + std::sqrt(theta * theta + 1.0));
+        const double c = 1.0 / std::sqrt(t * t + 1.0), s = t * c;
+        for (int k = 0; k < b; ++k) {
+          const double akp = at(k, p), akq = at(k, q);
+          at(k, p) = c * akp - s * akq;
+          at(k, q) = s * akp + c * akq;
+        }
+        for (int k = 0; k < b; ++k) {
+          const double apk = at(p, k), aqk = at(q, k);
+          at(p, k) = c * apk - s * aqk;
+          at(q, k) = s * apk + c * aqk;
+        }
+        for (int k = 0; k < b; ++k) {
+          const double ekp = E[(size_t)k * b + p], ekq = E[(size_t)k * b + q];
+          E[(size_t)k * b + p] = c * ekp - s * ekq;
+          E[(size_t)k * b + q] = s * ekp + c * ekq;
+        }
+      }
+  }
+  std::vector<int> idx(b);
+  for (int i = 0; i < b; ++i) idx[i] = i;
+  std::sort(idx.begin(), idx.end(), [&](int x, int y) { return at(x, x) > at(y, y); });
+  w.resize(b);
+  std::vector<double> E2((size_t)b * b);
+  for (int c = 0; c < b; ++c) {
+    w[c] = at(idx[c], idx[c]);
+    for (int k = 0; k < b; ++k) E2[(size_t)k * b + c] = E[(size_t)k * b + idx[c]];
+  }
+  E.swap(E2);
+}
+
+// G[b][b] = X^T X for row-major X[rows][b]
+void gram(const double* X, int rows, int b, std::vector<double>& G) {
+  G.assign((size_t)b * b, 0.0);
+  const int nt = 1
+#ifdef _OPENMP
+      * omp_get_max_threads()
+#endif
+      ;
+  std::vector<double> part((size_t)nt * b * b, 0.0);
+#pragma omp parallel
+  {
+    int t = 0;
+#ifdef _OPENMP
+    t = omp_get_thread_num();
+#endif
+    double* g = part.data() + (size_t)t * b * b;
+#pragma omp for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+      const double* x = X + (size_t)r * b;
+      for (int i = 0; i < b; ++i) {
+        const double xi = x[i];
+        for (int j = 0; j < b; ++j) g[(size_t)i * b + j] += xi * x[j];
+      }
+    }
+  }
+  for (int t = 0; t < nt; ++t)
+    for (size_t i = 0; i < (size_t)b * b; ++i) G[i] += part[(size_t)t * b * b + i];
+}
+
+// Top-r SVD of A[K][N]: L1 = U Sigma[:, :r] ([K][r]), L2 = V^T[:r, :] ([r][N]).
+svdq_status truncated_svd(const std::vector<double>& A, int K, int N, int r,
+                          std::vector<double>& L1, std::vector<double>& L2,
+                          std::vector<double>& sigma, int& iters, double& tail) {
+  const int b = std::min(std::min(r + 32, K), N);
+  Rng rng(0x5EED5EEDull);
+  std::vector<double> Z((size_t)N * b), Zraw((size_t)N * b), Q((size_t)K * b), T, w, E;
+  for (auto& z : Z) z = rng.normal();
+  orthonormalize(Z.data(), N, b, rng);
+  double prev = -1.0, energy = 0.0;
+  bool converged = false;
+  const bool exact_block = (b == std::min(K, N));      // the block spans the whole range
+  const int max_iter = 300;
+  int it = 0;
+  for (; it < max_iter; ++it) {
+    gemm_AZ(A.data(), K, N, Z.data(), b, Q.data());     // Q <- A Z
+    orthonormalize(Q.data(), K, b, rng);
+    gemm_AtQ(A.data(), K, N, Q.data(), b, Zraw.data()); // Zraw <- A^T Q  (= B^T, B = Q^T A)
+    gram(Zraw.data(), N, b, T);                         // B B^T
+    sym_eig(T, b, w, E);
+    energy = 0.0;
+    for (int i = 0; i < r; ++i) energy += std::max(w[i], 0.0);
+    if (exact_block || (it >= 3 && std::fabs(energy - prev) <= 1e-13 * energy)) {
+      converged = true;
+      break;
+    }
+    prev = energy;
+    Z = Zraw;
+    orthonormalize(Z.data(), N, b, rng);
+  }
+  iters = std::min(it + 1, max_iter);
+  if (!converged && std::fabs(energy - prev) > 1e-8 * std::max(energy, 1e-300))
+    return SVDQ_ENOCONVERGE;
+  const std::vector<double>& Zf = Zraw;
+  // Rayleigh-Ritz: B = Q^T A = Z^T, B B^T = E diag(w) E^T.
+  // U = Q E, sigma = sqrt(w), V^T rows = E^T B / sigma = (Z E)^T / sigma.
+  sigma.assign(r, 0.0);
+  L1.assign((size_t)K * r, 0.0);
+  L2.assign((size_t)r * N, 0.0);
+  for (int i = 0; i < r; ++i) sigma[i] = std::sqrt(std::max(w[i], 0.0));
+#pragma omp parallel for schedule(static)
+  for (int k = 0; k < K; ++k)
+    for (int i = 0; i < r; ++i) {
+      double u = 0.0;
+      for (int j = 0; j < b; ++j) u += Q[(size_t)k * b + j] * E[(size_t)j * b + i];
+      L1[(size_t)k * r + i] = u * sigma[i];
+    }
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n)
+    for (int i = 0; i < r; ++i) {
+      double v = 0.0;
+      for (int j = 0; j < b; ++j) v += Zf[(size_t)n * b + j] * E[(size_t)j * b + i];
+      L2[(size_t)i * N + n] = sigma[i] > 0 ? v / sigma[i] : 0.0;
+    }
+  double total = 0.0;
+#pragma omp parallel for reduction(+ : total) schedule(static)
+  for (size_t i = 0; i < A.size(); ++i) total += A[i] * A[i];
+  double kept = 0.0;
+  for (int i = 0; i < r; ++i) kept += sigma[i] * sigma[i];
+  tail = total - kept;
+  return SVDQ_OK;
+}
+
+// NVFP4 quantization of one group of 16 float32 values (same steps as the
+// kernel): a = max|v|, t = fp32(a c), s = E4M3(t), inv = fp32(1/(s g)),
+// code = E2M1(fp32(v inv)).  `codes` receives 16 nibbles.
+uint8_t nvfp4_group(const float* v, float c, float g, uint8_t* codes) {
+  float a = 0.0f;
+  for (int i = 0; i < 16; ++i) a = std::max(a, std::fabs(v[i]));
+  volatile float t = a * c;
+  const uint8_t sb = e4m3_from_nonneg(t);
+  const float s = e4m3_to_float(sb);
+  if (s == 0.0f) {
+    for (int i = 0; i < 16; ++i) codes[i] = 0;
+    return sb;
+  }
+  volatile float sg = s * g;
+  volatile float inv = 1.0f / sg;
+  for (int i = 0; i < 16; ++i) {
+    volatile float q = v[i] * inv;
+    codes[i] = e2m1_code(q);
+  }
+  return sb;
+}
+
+// INT4 quantization of one group of 64: s = bf16(fp32(a fp32(1/7))),
+// code = clamp(rint(fp32(v fp32(1/s))), -7, 7).
+uint16_t int4_group(const float* v, int8_t* codes) {
+  float a = 0.0f;
+  for (int i = 0; i < 64; ++i) a = std::max(a, std::fabs(v[i]));
+  const float seventh = 1.0f / 7.0f;
+  volatile float t = a * seventh;
+  const uint16_t sb = bf16_from_double((double)t);
+  const float s = bf16_to_float(sb);
+  if (s == 0.0f) {
+    for (int i = 0; i < 64; ++i) codes[i] = 0;
+    return sb;
+  }
+  volatile float inv = 1.0f / s;
+  for (int i = 0; i < 64; ++i) {
+    volatile float q = v[i] * inv;
+    float rq = std::nearbyint((float)q);
+    rq = std::min(7.0f, std::max(-7.0f, rq));
+    codes[i] = (int8_t)rq;
+  }
+  return sb;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ pipeline
+
+svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W,
+                         const uint16_t* bias, const uint16_t* calib, int M_calib,
+                         HostPrep& P) {
+  try {
+    const bool w4a16 = cfg.format == SVDQ_W4A16_INT4;
+    P.K = K; P.N = N; P.format = cfg.format;
+    P.rank = w4a16 ? 0 : cfg.rank;
+    P.alpha = cfg.alpha;
+    const int r = P.rank;
+    P.bias.assign(N, 0.0f);
+    if (bias)
+      for (int n = 0; n < N; ++n) P.bias[n] = bf16_to_float(bias[n]);
+
+    // ---- smoothing factors (float32)
+    P.lam.assign(K, 1.0f);
+    P.inv_lam.assign(K, 1.0f);
+    if (!w4a16) {
+      std::vector<float> ax(K, 0.0f), aw(K, 0.0f);
+      for (int m = 0; m < M_calib; ++m)
+        for (int k = 0; k < K; ++k)
+          ax[k] = std::max(ax[k], std::fabs(bf16_to_float(calib[(size_t)m * K + k])));
+#pragma omp parallel for schedule(static)
+      for (int k = 0; k < K; ++k) {
+        float mx = 0.0f;
+        for (int n = 0; n < N; ++n) mx = std::max(mx, std::fabs(bf16_to_float(W[(size_t)k * N + n])));
+        aw[k] = mx;
+      }
+      for (int k = 0; k < K; ++k) {
+        float lam;
+        if (ax[k] == 0.0f || aw[k] == 0.0f) {
+          lam = 1.0f;
+        } else if (cfg.alpha == 0.5f) {
+          volatile float sx = std::sqrt(ax[k]);
+          volatile float sw = std::sqrt(aw[k]);
+          lam = sx / sw;
+        } else {
+          lam = (float)(std::pow((double)ax[k], (double)cfg.alpha) /
+                        std::pow((double)aw[k], 1.0 - (double)cfg.alpha));
+        }
+        P.lam[k] = lam;
+        volatile float inv = 1.0f / lam;
+        P.inv_lam[k] = inv;
+      }
+    }
+
+    // ---- W_hat = diag(lam) W (float64)
+    std::vector<double> Wh((size_t)K * N);
+#pragma omp parallel for schedule(static)
+    for (int k = 0; k < K; ++k)
+      for (int n = 0; n < N; ++n)
+        Wh[(size_t)k * N + n] = (double)P.lam[k] * (double)bf16_to_float(W[(size_t)k * N + n]);
+
+    // ---- truncated SVD, stored 16-bit branch, residual
+    P.R.assign((size_t)K * N, 0.0f);
+    if (r > 0) {
+      svdq_status st = truncated_svd(Wh, K, N, r, P.L1, P.L2, P.sigma, P.svd_iterations, P.svd_tail_energy);
+      if (st != SVDQ_OK) return st;
+      P.L1d.resize((size_t)K * r);
+      P.L2b.resize((size_t)r * N);
+      for (int k = 0; k < K; ++k)
+        for (int i = 0; i < r; ++i)
+          P.L1d[(size_t)k * r + i] = bf16_from_double((double)P.inv_lam[k] * P.L1[(size_t)k * r + i]);
+      for (size_t i = 0; i < P.L2b.size(); ++i) P.L2b[i] = bf16_from_double(P.L2[i]);
+      std::vector<double> L2v((size_t)r * N);
+      for (size_t i = 0; i < L2v.size(); ++i) L2v[i] = bf16_to_float(P.L2b[i]);
+#pragma omp parallel for schedule(static)
+      for (int k = 0; k < K; ++k) {
+        double lk[128];
+        for (int i = 0; i < r; ++i) lk[i] = (double)P.lam[k] * (double)bf16_to_float(P.L1d[(size_t)k * r + i]);
+        for (int n = 0; n < N; ++n) {
+          double br = 0.0;
+          for (int i = 0; i < r; ++i) br += lk[i] * L2v[(size_t)i * N + n];
+          P.R[(size_t)k * N + n] = (float)(Wh[(size_t)k * N + n] - br);
+        }
+      }
+    } else {
+      for (size_t i = 0; i < Wh.size(); ++i) P.R[i] = (float)Wh[i];
+      if (!w4a16) {
+        double tot = 0.0;
+        for (double v : Wh) tot += v * v;
+        P.svd_tail_energy = tot;
+      }
+    }
+
+    // ---- residual quantization, groups along K for each output column n
+    P.w_codes.assign((size_t)N * K / 2, 0);
+    if (cfg.format == SVDQ_NVFP4) {
+      float amax = 0.0f;
+      for (float v : P.R) amax = std::max(amax, std::fabs(v));
+      P.g_w_exp = pow2_ceil_exponent((double)amax / 2688.0);
+      const float g = (float)std::ldexp(1.0, P.g_w_exp);
+      const float c = (float)std::ldexp((double)(1.0f / 6.0f), -P.g_w_exp);
+      P.w_scales_e4m3.assign((size_t)N * K / 16, 0);
+#pragma omp parallel for schedule(static)
+      for (int n = 0; n < N; ++n) {
+        float col[16];
+        uint8_t codes[16];
+        for (int g16 = 0; g16 < K / 16; ++g16) {
+          for (int i = 0; i < 16; ++i) col[i] = P.R[(size_t)(g16 * 16 + i) * N + n];
+          P.w_scales_e4m3[(size_t)n * (K / 16) + g16] = nvfp4_group(col, c, g, codes);
+          for (int i = 0; i < 8; ++i)
+            P.w_codes[(size_t)n * (K / 2) + g16 * 8 + i] = (uint8_t)(codes[2 * i] | (codes[2 * i + 1] << 4));
+        }
+      }
+      // activation tensor scale from the calibration batch, 4x headroom
+      float xa = 0.0f;
+      for (int m = 0; m < M_calib; ++m)
+        for (int k = 0; k < K; ++k) {
+          volatile float v = bf16_to_float(calib[(size_t)m * K + k]) * P.inv_lam[k];
+          xa = std::max(xa, std::fabs((float)v));
+        }
+      P.g_x_exp = pow2_ceil_exponent(4.0 * (double)xa / 2688.0);
+    } else {
+      P.w_scales_bf16.assign((size_t)N * K / 64, 0);
+#pragma omp parallel for schedule(static)
+      for (int n = 0; n < N; ++n) {
+        float col[64];
+        int8_t codes[64];
+        for (int g64 = 0; g64 < K / 64; ++g64) {
+          for (int i = 0; i < 64; ++i) col[i] = P.R[(size_t)(g64 * 64 + i) * N + n];
+          P.w_scales_bf16[(size_t)n * (K / 64) + g64] = int4_group(col, codes);
+          for (int i = 0; i < 32; ++i)
+            P.w_codes[(size_t)n * (K / 2) + g64 * 32 + i] =
+                (uint8_t)((codes[2 * i] & 0xF) | ((codes[2 * i + 1] & 0xF) << 4));
+        }
+      }
+    }
+    return SVDQ_OK;
+  } catch (const std::bad_alloc&) {
+    return SVDQ_ENOMEM;
+  } catch (...) {
+    return SVDQ_EINVAL;
+  }
+}
+
+}  // namespace svdq

@@ -1,0 +1,60 @@
+// Internal declarations shared by the host preparation code and the CUDA
+// launch code of the SVDQuant W4A4 library.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "../../include/svdq.h"
+
+#ifdef __CUDACC__
+#define SVDQ_HD __host__ __device__
+#else
+#define SVDQ_HD
+#endif
+
+namespace svdq {
+
+// Host results of the offline preparation (logical layouts).
+struct HostPrep {
+  int K = 0, N = 0, rank = 0, format = 0;
+  float alpha = 0.5f;
+  std::vector<float> lam, inv_lam;          // [K]
+  std::vector<double> L1;                   // [K][r]
+  std::vector<double> L2;                   // [r][N]
+  std::vector<double> sigma;                // [r]
+  std::vector<uint16_t> L1d;                // [K][r] BF16 bits
+  std::vector<uint16_t> L2b;                // [r][N] BF16 bits
+  std::vector<float> R;                     // [K][N]
+  int g_x_exp = 0, g_w_exp = 0;
+  std::vector<uint8_t> w_codes;             // [N][K/2]
+  std::vector<uint8_t> w_scales_e4m3;       // [N][K/16]   (NVFP4)
+  std::vector<uint16_t> w_scales_bf16;      // [N][K/64]   (INT4 / W4A16)
+  std::vector<float> bias;                  // [N]
+  int svd_iterations = 0;
+  double svd_tail_energy = 0.0;
+};
+
+// Runs the offline pipeline on the host.  Returns SVDQ_OK or an error status.
+svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W,
+                         const uint16_t* bias, const uint16_t* calib, int M_calib,
+                         HostPrep& out);
+
+// Number-format helpers (host).
+float bf16_to_float(uint16_t b);
+uint16_t bf16_from_double(double x);       // single round-to-nearest-even
+uint8_t e4m3_from_nonneg(float t);         // RNE, saturating at 448
+float e4m3_to_float(uint8_t b);
+uint8_t e2m1_code(float q);                // RNE (ties to even code), sat 6, sign kept
+int pow2_ceil_exponent(double x);          // smallest e with 2^e >= x; 0 for x <= 0
+
+// Offset in bytes of scale (row r, group-of-16 g) inside the tensor-core
+// scale-factor layout of a [rows][K] operand (see svdq_act_scale_bytes).
+SVDQ_HD inline size_t sf_offset(int r, int g, int K) {
+  const size_t kb = (size_t)(g >> 2);                 // 64-element K block
+  const size_t chunk = (size_t)(r >> 7) * (size_t)(K >> 6) + kb;
+  return chunk * 512 + (size_t)(r & 31) * 16 + (size_t)((r >> 5) & 3) * 4 + (size_t)(g & 3);
+}
+
+}  // namespace svdq
