@@ -263,7 +263,12 @@ def svd_split(W_hat: np.ndarray, rank: int):
     L2 = V_{:r,:}" -- read as the top r rows of V^T; the sign of each singular
     pair is free.]  Returns (L1, L2, singular values)."""
     U, S, Vt = np.linalg.svd(np.asarray(W_hat, dtype=np.float64), full_matrices=False)
-    return U[:, :rank] * S[:rank], Vt[:rank, :], S
+    L1, L2 = U[:, :rank] * S[:rank], Vt[:rank, :]
+    if rank > len(S):
+        # a matrix of rank < r: the branch holds all of it, the extra directions are zero
+        L1 = np.pad(L1, ((0, 0), (0, rank - len(S))))
+        L2 = np.pad(L2, ((0, rank - len(S)), (0, 0)))
+    return L1, L2, S
 
 
 def prepare(W: np.ndarray, bias: Optional[np.ndarray], Xc: np.ndarray, fmt: str = "nvfp4",

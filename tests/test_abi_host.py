@@ -178,3 +178,13 @@ def test_argument_errors():
         L.forward(16, 8, 16, 256, 1 << 20)
     assert e.value.status == lib.ESTATE
     assert L.workspace_bytes(0) == 0
+
+
+def test_rank_above_matrix_rank():
+    d = syn.custom_layer(8, M=4, K=64, N=16)
+    L = _prep_host(d)
+    L1, L2 = L.export("L1"), L.export("L2")
+    assert np.all(np.isfinite(L1)) and np.all(np.isfinite(L2))
+    assert np.all(L1[:, 16:] == 0) and np.all(L2[16:] == 0)
+    lam = L.export("lambda").astype(np.float64)
+    np.testing.assert_allclose(L1 @ L2, lam[:, None] * d["W"], rtol=1e-10, atol=1e-12)

@@ -240,3 +240,13 @@ def test_w4a16_forward():
     np.testing.assert_allclose(f["Y"], X.astype(np.float64) @ p["w_deq"].T + b, rtol=1e-13)
     s = np.repeat(p["w_scales"], 64, axis=1)
     assert np.all(np.abs(W.T - p["w_deq"]) <= s / 2 * (1 + 1e-6))
+
+
+def test_svd_split_rank_above_matrix_rank_pads_zeros():
+    # r larger than min(K, N): the branch carries the whole matrix, the residual is zero
+    rng = np.random.default_rng(8)
+    W = rng.standard_normal((64, 16))
+    L1, L2, S = o.svd_split(W, 32)
+    assert L1.shape == (64, 32) and L2.shape == (32, 16)
+    assert np.all(L1[:, 16:] == 0) and np.all(L2[16:] == 0)
+    np.testing.assert_allclose(L1 @ L2, W, atol=1e-12)

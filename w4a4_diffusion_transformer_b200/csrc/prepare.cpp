@@ -284,6 +284,7 @@ svdq_status truncated_svd(const std::vector<double>& A, int K, int N, int r,
                           std::vector<double>& L1, std::vector<double>& L2,
                           std::vector<double>& sigma, int& iters, double& tail) {
   const int b = std::min(std::min(r + 32, K), N);
+  const int re = std::min(r, b);                        // directions beyond rank(A) stay zero
   Rng rng(0x5EED5EEDull);
   std::vector<double> Z((size_t)N * b), Zraw((size_t)N * b), Q((size_t)K * b), T, w, E;
   for (auto& z : Z) z = rng.normal();
@@ -300,7 +301,7 @@ svdq_status truncated_svd(const std::vector<double>& A, int K, int N, int r,
     gram(Zraw.data(), N, b, T);                         // B B^T
     sym_eig(T, b, w, E);
     energy = 0.0;
-    for (int i = 0; i < r; ++i) energy += std::max(w[i], 0.0);
+    for (int i = 0; i < re; ++i) energy += std::max(w[i], 0.0);
     if (exact_block || (it >= 3 && std::fabs(energy - prev) <= 1e-13 * energy)) {
       converged = true;
       break;
@@ -318,17 +319,17 @@ svdq_status truncated_svd(const std::vector<double>& A, int K, int N, int r,
   sigma.assign(r, 0.0);
   L1.assign((size_t)K * r, 0.0);
   L2.assign((size_t)r * N, 0.0);
-  for (int i = 0; i < r; ++i) sigma[i] = std::sqrt(std::max(w[i], 0.0));
+  for (int i = 0; i < re; ++i) sigma[i] = std::sqrt(std::max(w[i], 0.0));
 #pragma omp parallel for schedule(static)
   for (int k = 0; k < K; ++k)
-    for (int i = 0; i < r; ++i) {
+    for (int i = 0; i < re; ++i) {
       double u = 0.0;
       for (int j = 0; j < b; ++j) u += Q[(size_t)k * b + j] * E[(size_t)j * b + i];
       L1[(size_t)k * r + i] = u * sigma[i];
     }
 #pragma omp parallel for schedule(static)
   for (int n = 0; n < N; ++n)
-    for (int i = 0; i < r; ++i) {
+    for (int i = 0; i < re; ++i) {
       double v = 0.0;
       for (int j = 0; j < b; ++j) v += Zf[(size_t)n * b + j] * E[(size_t)j * b + i];
       L2[(size_t)i * N + n] = sigma[i] > 0 ? v / sigma[i] : 0.0;
