@@ -194,7 +194,11 @@ K1Params k1_params(const svdq_layer* L, int M, void* codes, void* scales, void* 
   p.M = M;
   p.K = h.K;
   p.c_x = (float)std::ldexp((double)(1.0f / 6.0f), -h.g_x_exp);
-  p.g_x = (float)std::ldexp(1.0, h.g_x_exp);
+  p.g_x_exp = h.g_x_exp;
+  for (int m = 0; m < 8; ++m) {
+    p.rcp[m] = (float)(1.0 / (1.0 + m / 8.0));
+    p.rcp[8 + m] = m ? (float)(1.0 / m) : 0.0f;
+  }
   p.inv_lam = L->d_inv_lam;
   p.codes = static_cast<uint8_t*>(codes);
   p.scales = static_cast<uint8_t*>(scales);
@@ -217,8 +221,10 @@ svdq_status run_k1(const svdq_layer* L, const void* X, int M, void* codes, void*
 svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
                    cudaStream_t stream, bool branch, bool gelu) {
   const HostPrep& h = L->host;
-  CUtensorMap tm_a, tm_xl;
+  CUtensorMap tm_a, tm_xl, tm_y;
   if (!make_map(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ECUDA;
+  if (!make_map(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ECUDA;
   if (branch) {
     if (!make_map(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
@@ -239,7 +245,7 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
   p.budget_ns = L->budget_ns;
   p.branch = branch ? 1 : 0;
   p.gelu = gelu ? 1 : 0;
-  return launch_k2(tm_a, L->tm_wq, tm_xl, L->tm_l2s, p, L->num_sms, stream) == cudaSuccess ? SVDQ_OK
+  return launch_k2(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream) == cudaSuccess ? SVDQ_OK
                                                                                           : SVDQ_ECUDA;
 }
 

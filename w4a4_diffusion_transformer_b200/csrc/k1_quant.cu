@@ -13,15 +13,22 @@
 // Layout of the work: a CTA owns 32 token rows and streams the whole K range in
 // stages of 256 columns.  One producer warp loads each stage with TMA (X tile,
 // the matching 256 x 32 slice of L1d^T and 256 floats of inv_lam) into a
-// 4-deep shared-memory ring; eight consumer warps quantize the tile (one thread
-// per half 64-column block of a row) and run the 32 x 32 x 256 down projection
-// on the tensor cores (mma.sync BF16: the projection is 32 columns wide and the
-// pass is bound by HBM, not by the tensor pipe).
+// 4-deep shared-memory ring.  Sixteen consumer warps share each stage:
+//   * quantization: warp w owns the 16-column group w of the stage and lane l
+//     owns row l, so the inv_lam reads are broadcasts and the swizzled X reads
+//     are conflict-free;
+//   * down projection on the tensor cores (mma.sync BF16; the projection is 32
+//     columns wide and the pass is bound by memory, not by the tensor pipe):
+//     warp w computes the 16x8 tile (w & 1, (w >> 1) & 3) over half of the
+//     stage's 256 columns (w >> 3); the two halves are summed at the end.
 //
 // Quantizer arithmetic per group of 16 (bit-exact with the CPU oracle): a =
 // max|v|; t = fp32(a * c_x) with c_x = fp32(1/6) 2^-gx; s = E4M3_rn_satfinite(t);
 // s == 0 -> all codes +0; inv = fp32(1 / (s * g_x)); code =
-// E2M1_rn_satfinite(fp32(v * inv)).
+// E2M1_rn_satfinite(fp32(v * inv)).  The reciprocal is exact without a
+// division: for s = (1 + m/8) 2^(e-7) (or m 2^-9 when e = 0) it equals
+// fp32(1/(1 + m/8)) 2^(7-e-gx) (or fp32(1/m) 2^(9-gx)), a power-of-two scaling
+// of one of 15 correctly rounded constants computed on the host.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -35,13 +42,13 @@ namespace {
 constexpr int kRows = 32;
 constexpr int kBK = 256;
 constexpr int kStages = 4;
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 16;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kXBytes = kRows * kBK * 2;     // 4 sub-tiles of 32 rows x 128 B
 constexpr int kLBytes = 32 * kBK * 2;        // 4 sub-tiles of 32 rows x 128 B
 constexpr int kIBytes = kBK * 4;
 constexpr int kStageBytes = kXBytes + kLBytes + kIBytes;   // 33 KiB, 1 KiB multiple
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + (2 * 4 * 32 * 4 + 16) * 4;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -127,13 +134,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // -------------------------------------------------------------- consumers
-  const int t = threadIdx.x;            // 0..255
-  const int qr = t >> 3;                // quantizer: row in the CTA tile
-  const int qkb = (t >> 1) & 3;         //            64-column block in the stage
-  const int qh = t & 1;                 //            32-column half of the block
-  const int grow = row0 + qr;           // global row (may be >= M: zero padding)
+  float* red = reinterpret_cast<float*>(smem + kStages * kStageBytes + 256);   // k-half partial sums
+  float* rcp = red + 2 * 4 * 32 * 4;                                           // reciprocal table
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) rcp[i] = p.rcp[i];     // constant indices: stays in parameter space
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  const int grow = row0 + lane;         // quantizer: this lane's row (may be >= M: zero padding)
+  const int qcol = warp * 16;           //            16-column group of the stage
   const int mt = warp & 1;              // down projection: 16-row tile
-  const int nt = warp >> 1;             //                  8-column tile of XL
+  const int nt = (warp >> 1) & 3;       //                  8-column tile of XL
+  const int kh = warp >> 3;             //                  half of the stage's k-steps
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   bool ok = true;
 
@@ -150,63 +162,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k0 = it * kBK;
     const int kvalid = min(kBK, K - k0);
 
-    if (kQuant) {
-      const int kc = qkb * 64 + qh * 32;
-      const bool active = kc < kvalid;
-      uint32_t sb2 = 0;
-      if (active) {
-        const uint8_t* xt = st + qkb * 4096;
-        const float* inv = reinterpret_cast<const float*>(st + kXBytes + kLBytes) + kc;
-        float v[32];
+    if (kQuant && qcol < kvalid) {
+      const uint8_t* xt = st + (qcol >> 6) * 4096;
+      const int c0 = (qcol & 63) >> 3;                  // first 16-byte chunk of the group in its row
+      const float4* inv4 = reinterpret_cast<const float4*>(st + kXBytes + kLBytes) + (qcol >> 2);
+      float v[16];
+      float a = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(xt + sw128(qr, qh * 4 + i));
-          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      for (int i = 0; i < 2; ++i) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(xt + sw128(lane, c0 + i));
+        const float4 ia = inv4[2 * i], ib = inv4[2 * i + 1];
+        const float iv[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float lo = __uint_as_float(w[e] << 16);
-            const float hi = __uint_as_float(w[e] & 0xFFFF0000u);
-            v[i * 8 + 2 * e] = __fmul_rn(lo, inv[i * 8 + 2 * e]);
-            v[i * 8 + 2 * e + 1] = __fmul_rn(hi, inv[i * 8 + 2 * e + 1]);
-          }
-        }
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          a0 = fmaxf(a0, fabsf(v[i]));
-          a1 = fmaxf(a1, fabsf(v[16 + i]));
-        }
-        sb2 = dev::cvt_e4m3x2(__fmul_rn(a0, p.c_x), __fmul_rn(a1, p.c_x));
-        uint32_t packed[4];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const float sv = dev::e4m3_to_f32((sb2 >> (8 * g)) & 0xFFu);
-          if (sv == 0.0f) {
-            packed[2 * g] = 0u;
-            packed[2 * g + 1] = 0u;
-          } else {
-            const float invs = __fdiv_rn(1.0f, __fmul_rn(sv, p.g_x));
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              float q[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) q[e] = __fmul_rn(v[g * 16 + h * 8 + e], invs);
-              packed[2 * g + h] = dev::cvt_e2m1x8(q);
-            }
-          }
-        }
-        if (grow < p.M) {
-          uint8_t* dst = p.codes + (size_t)grow * (size_t)(K >> 1) + ((k0 + kc) >> 1);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        for (int e = 0; e < 4; ++e) {
+          v[i * 8 + 2 * e] = __fmul_rn(__uint_as_float(w[e] << 16), iv[2 * e]);
+          v[i * 8 + 2 * e + 1] = __fmul_rn(__uint_as_float(w[e] & 0xFFFF0000u), iv[2 * e + 1]);
         }
       }
-      // The two halves of a 64-column block hold its four scale bytes.
-      const uint32_t other = __shfl_xor_sync(0xffffffffu, sb2 & 0xFFFFu, 1);
-      if (active && qh == 0) {
-        const uint32_t word = (sb2 & 0xFFFFu) | (other << 16);
-        const int g0 = (k0 + qkb * 64) >> 4;
-        *reinterpret_cast<uint32_t*>(p.scales + sf_offset(grow, g0, K)) = word;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+      const uint32_t sb = dev::cvt_e4m3x2(__fmul_rn(a, p.c_x), 0.0f) & 0xFFu;
+      uint32_t packed0 = 0u, packed1 = 0u;
+      if (sb != 0u) {
+        const uint32_t e = sb >> 3, m = sb & 7u;
+        const int p2 = (e ? 7 - (int)e : 9) - p.g_x_exp;
+        const float invs = rcp[(e ? 0 : 8) + m] * __int_as_float((p2 + 127) << 23);
+        float q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], invs);
+        packed0 = dev::cvt_e2m1x8(q);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[8 + i], invs);
+        packed1 = dev::cvt_e2m1x8(q);
       }
+      if (grow < p.M)
+        *reinterpret_cast<uint2*>(p.codes + (size_t)grow * (size_t)(K >> 1) + ((k0 + qcol) >> 1)) =
+            make_uint2(packed0, packed1);
+      p.scales[sf_offset(grow, (k0 + qcol) >> 4, K)] = (uint8_t)sb;
     }
 
     if (kDown) {
@@ -215,8 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nsteps = kvalid >> 4;
       const int arow = mt * 16 + (lane & 15);
       const int brow = nt * 8 + (lane & 7);
-#pragma unroll 4
-      for (int kk = 0; kk < nsteps; kk += 2) {
+#pragma unroll 2
+      for (int kk = kh * 8; kk < min(nsteps, kh * 8 + 8); kk += 2) {
         const int sub = kk >> 2;
         const int cpair = (kk & 3) * 2;                 // 16B chunk of this k-step pair
         uint32_t b[4];
@@ -233,16 +226,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) dev::mbar_arrive(&empty[s]);
   }
 
-  if (kDown && ok) {
-    const int r_a = row0 + mt * 16 + (lane >> 2);
-    const int col = nt * 8 + 2 * (lane & 3);
-    if (r_a < p.M) {
-      __nv_bfloat162 v = __floats2bfloat162_rn(acc[0], acc[1]);
-      *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)r_a * 32 + col) = v;
+  if (kDown) {
+    // sum the two k-halves; every consumer warp reaches this barrier (no early exit)
+    float* slot = red + ((mt * 4 + nt) * 32 + lane) * 4;
+    if (kh == 1) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) slot[i] = acc[i];
     }
-    if (r_a + 8 < p.M) {
-      __nv_bfloat162 v = __floats2bfloat162_rn(acc[2], acc[3]);
-      *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)(r_a + 8) * 32 + col) = v;
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+    if (kh == 0 && ok && !*abort_flag) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] += slot[i];
+      const int r_a = row0 + mt * 16 + (lane >> 2);
+      const int col = nt * 8 + 2 * (lane & 3);
+      if (r_a < p.M)
+        *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)r_a * 32 + col) = __floats2bfloat162_rn(acc[0], acc[1]);
+      if (r_a + 8 < p.M)
+        *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)(r_a + 8) * 32 + col) =
+            __floats2bfloat162_rn(acc[2], acc[3]);
     }
   }
 }
@@ -250,8 +251,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <bool Q, bool D>
 cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const K1Params& p, cudaStream_t stream) {
   auto kern = k1_kernel<Q, D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
   const int mpad = (p.M + 127) / 128 * 128;
   dim3 grid(mpad / kRows);
   kern<<<grid, kThreads, kSmemBytes, stream>>>(tm_x, tm_l, p);

@@ -20,7 +20,14 @@
 //              stage with the XL tile and the L2b^T tile (64-byte swizzle).
 //   warp 1     allocates TMEM (512 columns: accumulator 256 + per-stage scale factors) and
 //              issues tcgen05.cp (scales smem -> TMEM) and tcgen05.mma.
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, alpha, bias, GELU, BF16.
+//   warps 2-9  epilogue, two warps per TMEM lane quarter (32 rows), each owning
+//              128 of the 256 columns: tcgen05.ld in 32-column chunks (the next
+//              chunk's load overlaps the current chunk's math), alpha, bias
+//              (staged in shared memory while the mainloop runs), GELU, BF16,
+//              into two 64-byte-swizzled 32 x 32 buffers per warp that the
+//              warp's lane 0 stores to Y with TMA.  The accumulator is released
+//              to the MMA warp as soon as its last chunk is in registers, so the
+//              stores of tile t overlap the mainloop of tile t+1.
 // Pipelines are mbarrier rings; every wait is bounded (sm100.cuh).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -35,14 +42,17 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBKBytes = 128;               // 256 E2M1 values per row per stage
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kStages = 3;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kEpiBufBytes = 32 * 64;        // one 32 x 32 BF16 output chunk
+constexpr int kEpiWarpBytes = 2 * kEpiBufBytes + 512;   // two chunk buffers + 128 bias floats
 constexpr int kABytes = kBM * kBKBytes;      // 16 KiB
 constexpr int kBBytes = kBN * kBKBytes;      // 32 KiB
 constexpr int kSFABytes = 4 * 512;           // 4 K-blocks x 128 rows
 constexpr int kSFBBytes = 2 * 4 * 512;       // 2 row blocks x 4 K-blocks
 constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;   // 54 KiB
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiWarpBytes + 1024 + 256;
 constexpr int kTmemCols = 512;
 // Scale factors in TMEM, one region per pipeline stage (so a region is only
 // rewritten after the MMAs that read it have completed): 4 columns per 128-row
@@ -63,10 +73,12 @@ __device__ __forceinline__ float gelu_tanh(float y) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     k2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-              const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2, K2Params p) {
+              const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2,
+              const __grid_constant__ CUtensorMap tm_y, K2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* epi_buf = smem + kStages * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_buf + kEpiWarps * kEpiWarpBytes);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
@@ -89,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(&empty[s], 1);
     }
     dev::mbar_init(acc_full, 1);
-    dev::mbar_init(acc_empty, 4);
+    dev::mbar_init(acc_empty, kEpiWarps);
     dev::mbar_init(drain, 1);
     *abort_flag = 0;
     dev::fence_mbar_init();
@@ -163,9 +175,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_f4 = dev::idesc_nvfp4(kBM, kBN);
       const uint32_t idesc_h = dev::idesc_bf16(kBM, kBN);
+      // Scale factors of k-tile kt+1 are copied into TMEM (their own per-stage
+      // region) before the MMAs of k-tile kt are issued, so the copies do not
+      // sit between a k-tile's data arriving and its MMAs.
+      auto wait_full = [&](int slot, int code) -> bool {
+        if (!dev::mbar_wait(&full[slot % kStages], (uint32_t)(slot / kStages) & 1u, abort_flag, p.budget_ns)) {
+          record_error(p.err, abort_flag, code);
+          return false;
+        }
+        dev::tc_fence_after();
+        return true;
+      };
+      auto copy_scales = [&](int slot, int kt) {
+        const int s = slot % kStages;
+        const int nkb = min(4, kblocks - 4 * kt);
+        const uint32_t sfa0 = dev::smem_u32(smem + s * kStageBytes) + kABytes + kBBytes;
+        const uint32_t sfb0 = sfa0 + kSFABytes;
+        const uint32_t tsfa = tmem + kSFCol0 + s * kSFStageCols;
+        const uint32_t tsfb = tsfa + 16;
+        for (int j = 0; j < nkb; ++j) {
+          dev::tmem_copy_32x128b_x4(tsfa + 4 * j, dev::smem_desc(sfa0 + 512 * j, 0, 128, 0));
+          dev::tmem_copy_32x128b_x4(tsfb + 8 * j, dev::smem_desc(sfb0 + 512 * j, 0, 128, 0));
+          dev::tmem_copy_32x128b_x4(tsfb + 8 * j + 4, dev::smem_desc(sfb0 + 2048 + 512 * j, 0, 128, 0));
+        }
+      };
       int it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
+        const int kslot0 = it + (p.branch ? 1 : 0);
+        // the first k-tile's scales do not touch the accumulator: copy them first
+        if (!(ok = wait_full(kslot0, 0x205))) break;
+        copy_scales(kslot0, 0);
         if (!dev::mbar_wait(acc_empty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag, p.budget_ns)) {
           record_error(p.err, abort_flag, 0x203);
           ok = false;
@@ -174,13 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::tc_fence_after();
         uint32_t accumulate = 0;
         if (p.branch) {
+          if (!(ok = wait_full(it, 0x204))) break;
           const int s = it % kStages;
-          if (!dev::mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
-            record_error(p.err, abort_flag, 0x204);
-            ok = false;
-            break;
-          }
-          dev::tc_fence_after();
           const uint32_t a0 = dev::smem_u32(smem + s * kStageBytes);
           const uint32_t b0 = a0 + kABytes;
 #pragma unroll
@@ -191,28 +226,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             accumulate = 1;
           }
           dev::tc_commit(&empty[s]);
-          ++it;
         }
         for (int kt = 0; kt < ktiles; ++kt) {
-          const int s = it % kStages;
-          if (!dev::mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
-            record_error(p.err, abort_flag, 0x205);
-            ok = false;
-            break;
+          const int slot = kslot0 + kt;
+          const int s = slot % kStages;
+          if (kt + 1 < ktiles) {
+            if (!(ok = wait_full(slot + 1, 0x205))) break;
+            copy_scales(slot + 1, kt + 1);
           }
-          dev::tc_fence_after();
           const int nkb = min(4, kblocks - 4 * kt);
           const uint32_t a0 = dev::smem_u32(smem + s * kStageBytes);
           const uint32_t b0 = a0 + kABytes;
-          const uint32_t sfa0 = b0 + kBBytes;
-          const uint32_t sfb0 = sfa0 + kSFABytes;
           const uint32_t tsfa = tmem + kSFCol0 + s * kSFStageCols;
           const uint32_t tsfb = tsfa + 16;
-          for (int j = 0; j < nkb; ++j) {
-            dev::tmem_copy_32x128b_x4(tsfa + 4 * j, dev::smem_desc(sfa0 + 512 * j, 0, 128, 0));
-            dev::tmem_copy_32x128b_x4(tsfb + 8 * j, dev::smem_desc(sfb0 + 512 * j, 0, 128, 0));
-            dev::tmem_copy_32x128b_x4(tsfb + 8 * j + 4, dev::smem_desc(sfb0 + 2048 + 512 * j, 0, 128, 0));
-          }
           for (int j = 0; j < nkb; ++j) {
             const uint64_t ad = dev::smem_desc(a0 + 32 * j, 16, 1024, 2);
             const uint64_t bd = dev::smem_desc(b0 + 32 * j, 16, 1024, 2);
@@ -220,9 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             accumulate = 1;
           }
           dev::tc_commit(&empty[s]);
-          ++it;
         }
         if (!ok) break;
+        it = kslot0 + ktiles;
         dev::tc_commit(acc_full);
       }
       // Wait until every MMA and copy this thread issued has completed.
@@ -232,51 +258,78 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                          // TMEM lane quarter of this warp
-    const int r_in_tile = q * 32 + lane;
-    int tcount = 0;
+    const int half = (warp - 2) >> 2;                // which 128 of the 256 columns
+    uint8_t* wbuf = epi_buf + (warp - 2) * kEpiWarpBytes;
+    float* bias_s = reinterpret_cast<float*>(wbuf + 2 * kEpiBufBytes);
+    if (lane == 0) dev::tma_prefetch_desc(&tm_y);
+    int tcount = 0, chunk = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
       const int m0 = (tile % tiles_m) * kBM;
-      const int n0 = (tile / tiles_m) * kBN;
+      const int n0 = (tile / tiles_m) * kBN + half * 128;
+      // stage this tile's 128 bias values (the previous tile's reads are done:
+      // every lane passed the __syncwarp after its last use)
+      {
+        const int col = n0 + lane * 4;
+        float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (col < N) b4 = __ldg(reinterpret_cast<const float4*>(p.bias + col));
+        reinterpret_cast<float4*>(bias_s)[lane] = b4;
+      }
       const bool got = dev::mbar_wait(acc_full, (uint32_t)tcount & 1u, abort_flag, p.budget_ns);
       if (!__all_sync(0xffffffffu, got)) {          // warp-uniform exit (tcgen05.ld is warp-collective)
         if (lane == 0) record_error(p.err, abort_flag, 0x206);
         break;
       }
+      __syncwarp();
       dev::tc_fence_after();
-      const int row = m0 + r_in_tile;
-      __nv_bfloat16* yrow = p.y + (size_t)row * (size_t)N;
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        dev::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
-        dev::tmem_load_wait();
-        const int nb = n0 + c * 32;
-        if (row < M && nb < N) {
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 128);
+      uint32_t va[32], vb[32];
+      dev::tmem_load_32cols(taddr, va);
+      dev::tmem_load_wait(va);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int n = nb + v * 8;
-            if (n < N) {
-              uint32_t packed[4];
+      for (int c = 0; c < 4; ++c, ++chunk) {
+        uint32_t (&cur)[32] = (c & 1) ? vb : va;
+        uint32_t (&nxt)[32] = (c & 1) ? va : vb;
+        if (c + 1 < 4) dev::tmem_load_32cols(taddr + (uint32_t)((c + 1) * 32), nxt);
+        // the buffer of this chunk was last read by the store issued two chunks ago
+        if (lane == 0) dev::bulk_wait_group_read<1>();
+        __syncwarp();
+        uint8_t* buf = wbuf + (chunk & 1) * kEpiBufBytes;
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float y0 = p.alpha * __uint_as_float(r[v * 8 + 2 * e]) + __ldg(p.bias + n + 2 * e);
-                float y1 = p.alpha * __uint_as_float(r[v * 8 + 2 * e + 1]) + __ldg(p.bias + n + 2 * e + 1);
-                if (p.gelu) {
-                  y0 = gelu_tanh(y0);
-                  y1 = gelu_tanh(y1);
-                }
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
-                packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
-              }
-              *reinterpret_cast<uint4*>(yrow + n) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        for (int j = 0; j < 4; ++j) {
+          uint32_t packed[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 b2 = reinterpret_cast<const float2*>(bias_s)[c * 16 + j * 4 + e];
+            float y0 = p.alpha * __uint_as_float(cur[j * 8 + 2 * e]) + b2.x;
+            float y1 = p.alpha * __uint_as_float(cur[j * 8 + 2 * e + 1]) + b2.y;
+            if (p.gelu) {
+              y0 = gelu_tanh(y0);
+              y1 = gelu_tanh(y1);
             }
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+            packed[e] = *reinterpret_cast<const uint32_t*>(&h2);
           }
+          // 64-byte swizzle: 16-byte chunk j of row `lane` sits at j ^ ((lane >> 1) & 3)
+          *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+        dev::fence_async_shared();                    // make the writes visible to the TMA engine
+        __syncwarp();
+        if (lane == 0) {
+          dev::tma_store_2d(&tm_y, buf, n0 + c * 32, m0 + q * 32);
+          dev::bulk_commit_group();
+        }
+        if (c + 1 < 4) dev::tmem_load_wait(nxt);
+        if (c == 2) {
+          // the last chunk is in registers: hand the accumulator back to the MMA warp
+          dev::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) dev::mbar_arrive(acc_empty);
         }
       }
-      dev::tc_fence_before();
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(acc_empty);
     }
+    if (lane == 0) dev::bulk_wait_group_all();
   }
 
   dev::tc_fence_before();
@@ -293,12 +346,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 int k2_block_n() { return kBN; }
 
 cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
-                      const CUtensorMap& tm_l2, const K2Params& p, int num_sms, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(k2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
+                      const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
+                      cudaStream_t stream) {
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(k2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  k2_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_xl, tm_l2, p);
+  k2_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_xl, tm_l2, tm_y, p);
   return cudaGetLastError();
 }
 

@@ -13,7 +13,8 @@ namespace svdq {
 struct K1Params {
   int M, K;
   float c_x;                    // fp32(1/6) * 2^-g_x_exp
-  float g_x;                    // 2^g_x_exp
+  int g_x_exp;                  // activation tensor scale g_x = 2^g_x_exp
+  float rcp[16];                // fp32(1/(1 + m/8)) for m = 0..7, then fp32(1/m) (index 8 + m)
   const float* inv_lam;         // [K]
   uint8_t* codes;               // [M][K/2]
   uint8_t* scales;              // tensor-core scale layout, ceil(M/128)*128 rows
@@ -49,7 +50,8 @@ cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const K1
 int k1_rows_per_cta();
 
 cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
-                      const CUtensorMap& tm_l2, const K2Params& p, int num_sms, cudaStream_t stream);
+                      const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
+                      cudaStream_t stream);
 int k2_block_n();
 
 cudaError_t launch_upproj(const UpParams& p, cudaStream_t stream);

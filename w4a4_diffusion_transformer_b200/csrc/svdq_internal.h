@@ -6,7 +6,7 @@
 #include <cstdint>
 #include <vector>
 
-#include "../../include/svdq.h"
+#include "svdq.h"   // include/ is on the include path
 
 #ifdef __CUDACC__
 #define SVDQ_HD __host__ __device__
