@@ -85,6 +85,10 @@ struct DeviceGuard {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Box width and swizzle of the GEMM's 4-bit operand tiles (one pipeline stage of K).
+uint32_t k2_box_bytes() { return (uint32_t)k2_stage_k_bytes(); }
+CUtensorMapSwizzle k2_swizzle() { return k2_stage_k_bytes() == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B; }
+
 bool w4a4(const svdq_layer* L) { return L->host.format == SVDQ_NVFP4 || L->host.format == SVDQ_INT4; }
 
 size_t act_scale_bytes(const HostPrep& h, int M) {
@@ -170,8 +174,8 @@ svdq_status upload_layer(svdq_layer* L, int device) {
     chk(upload(&L->d_l2s, l2s.data(), l2s.size() * 2));
     chk(upload(&L->d_l2t, l2t.data(), l2t.size() * 2));
     if (e != cudaSuccess) return SVDQ_ECUDA;
-    bool ok = make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 256,
-                       CU_TENSOR_MAP_SWIZZLE_128B) &&
+    bool ok = make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, k2_box_bytes(), 256,
+                       k2_swizzle()) &&
               make_map(&L->tm_l2s, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
                        CU_TENSOR_MAP_SWIZZLE_64B) &&
               make_map(&L->tm_l1t, L->d_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, 32, 64, 32,
@@ -211,18 +215,23 @@ K1Params k1_params(const svdq_layer* L, int M, void* codes, void* scales, void* 
 svdq_status run_k1(const svdq_layer* L, const void* X, int M, void* codes, void* scales, void* xl,
                    cudaStream_t stream, int mode) {
   const HostPrep& h = L->host;
-  CUtensorMap tm_x;
+  CUtensorMap tm_x, tm_c;
   if (!make_map(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.K, M, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ECUDA;
+  // activation codes are written in 32-row x 16-byte tiles (one per quantizer warp and stage)
+  if (mode != 2 &&
+      !make_map(&tm_c, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SVDQ_ECUDA;
+  if (mode == 2) tm_c = tm_x;   // unused by the down-projection-only kernel
   K1Params p = k1_params(L, M, codes, scales, xl);
-  return launch_k1(tm_x, L->tm_l1t, p, mode, stream) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+  return launch_k1(tm_x, L->tm_l1t, tm_c, p, mode, stream) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
 
 svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
                    cudaStream_t stream, bool branch, bool gelu) {
   const HostPrep& h = L->host;
   CUtensorMap tm_a, tm_xl, tm_y;
-  if (!make_map(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, k2_box_bytes(), 128, k2_swizzle()))
     return SVDQ_ECUDA;
   if (!make_map(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ECUDA;

@@ -11,16 +11,22 @@
 //   * XL = bf16(X L1d) (rank 32; 1/lam is folded into L1d).
 //
 // Layout of the work: a CTA owns 32 token rows and streams the whole K range in
-// stages of 256 columns.  One producer warp loads each stage with TMA (X tile,
-// the matching 256 x 32 slice of L1d^T and 256 floats of inv_lam) into a
-// 4-deep shared-memory ring.  Sixteen consumer warps share each stage:
-//   * quantization: warp w owns the 16-column group w of the stage and lane l
-//     owns row l, so the inv_lam reads are broadcasts and the swizzled X reads
-//     are conflict-free;
-//   * down projection on the tensor cores (mma.sync BF16; the projection is 32
-//     columns wide and the pass is bound by memory, not by the tensor pipe):
-//     warp w computes the 16x8 tile (w & 1, (w >> 1) & 3) over half of the
-//     stage's 256 columns (w >> 3); the two halves are summed at the end.
+// stages of 256 columns.  Two producer warps load with TMA: one feeds an
+// 8-deep ring of X tiles (+ 256 floats of inv_lam) from HBM, the other a
+// 3-deep ring of the matching 256 x 32 slices of L1d^T, which every CTA reads
+// from L2.  The consumer warps are specialized and never wait for each other
+// inside the loop:
+//   * 8 quantizer warps: warp w owns columns 32w..32w+31 of the stage (two
+//     groups) and lane l owns row l, so the inv_lam reads are broadcasts and
+//     the swizzled X reads are conflict-free.  Each warp writes its 32 x 16-byte
+//     code tile to shared memory and stores it with its own TMA store; the two
+//     scale bytes of a lane are stored as one 2-byte word;
+//   * 8 down-projection warps on the tensor cores (mma.sync BF16; the
+//     projection is 32 columns wide and the pass is bound by memory, not by the
+//     tensor pipe): warp w owns k-steps 2w, 2w+1 of every stage for all 32 rows
+//     and all 32 output columns, so every operand fragment is read from shared
+//     memory once; the eight partial sums are added through shared memory at
+//     the end.
 //
 // Quantizer arithmetic per group of 16 (bit-exact with the CPU oracle): a =
 // max|v|; t = fp32(a * c_x) with c_x = fp32(1/6) 2^-gx; s = E4M3_rn_satfinite(t);
@@ -41,14 +47,21 @@ namespace {
 
 constexpr int kRows = 32;
 constexpr int kBK = 256;
-constexpr int kStages = 4;
-constexpr int kConsumerWarps = 16;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kXStages = 8;                  // X + inv_lam ring (HBM stream)
+constexpr int kLStages = 3;                  // L1d^T ring (L2-resident)
+constexpr int kQuantWarps = 8;
+constexpr int kMmaWarps = 8;
+constexpr int kConsumerWarps = kQuantWarps + kMmaWarps;
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kXBytes = kRows * kBK * 2;     // 4 sub-tiles of 32 rows x 128 B
 constexpr int kLBytes = 32 * kBK * 2;        // 4 sub-tiles of 32 rows x 128 B
 constexpr int kIBytes = kBK * 4;
-constexpr int kStageBytes = kXBytes + kLBytes + kIBytes;   // 33 KiB, 1 KiB multiple
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + (2 * 4 * 32 * 4 + 16) * 4;
+constexpr int kXStageBytes = kXBytes + kIBytes;            // 17 KiB, 1 KiB multiple
+constexpr int kCodeTile = kRows * 16;                     // one quantizer warp's codes: 32 rows x 16 B
+constexpr int kCodeBytes = kQuantWarps * 2 * kCodeTile;     // double-buffered per warp
+constexpr int kPartBytes = kMmaWarps * 32 * 32 * 4;         // down-projection partial sums
+static_assert(kPartBytes <= kLStages * kLBytes, "partial sums reuse the L1d^T ring");
+constexpr int kSmemBytes = kXStages * kXStageBytes + kLStages * kLBytes + kCodeBytes + 1024 + 256 + 16 * 4;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -72,14 +85,24 @@ __device__ __forceinline__ void record_error(int* err, volatile int* abort_flag,
   *abort_flag = 1;
 }
 
+__device__ __forceinline__ void mma_warps_sync() { dev::named_barrier(1, kMmaWarps * 32); }
+
 template <bool kQuant, bool kDown>
 __global__ void __launch_bounds__(kThreads, 1)
-    k1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l, K1Params p) {
+    k1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l,
+              const __grid_constant__ CUtensorMap tm_c, K1Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  uint8_t* lring = smem + kXStages * kXStageBytes;              // L1d^T ring (1 KiB aligned)
+  uint8_t* cbuf = lring + kLStages * kLBytes;                    // code staging tiles
+  float4* part = reinterpret_cast<float4*>(lring);               // partial sums, after the loop
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(cbuf + kCodeBytes);
+  uint64_t* xempty = xfull + kXStages;
+  uint64_t* lfull = xempty + kXStages;
+  uint64_t* lempty = lfull + kLStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(lempty + kLStages);
+  float* rcp = reinterpret_cast<float*>(cbuf + kCodeBytes + 256);   // reciprocal table
+  constexpr int kActiveWarps = (kQuant ? kQuantWarps : 0) + (kDown ? kMmaWarps : 0);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -88,168 +111,243 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = (K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      dev::mbar_init(&full[s], 1);
-      dev::mbar_init(&empty[s], kConsumerWarps);
+    // the GEMM that consumes this kernel's outputs may start its prologue now;
+    // it waits for this grid's completion before reading them
+    dev::griddep_launch_dependents();
+    for (int s = 0; s < kXStages; ++s) {
+      dev::mbar_init(&xfull[s], 1);
+      dev::mbar_init(&xempty[s], kActiveWarps);
+    }
+    for (int s = 0; s < kLStages; ++s) {
+      dev::mbar_init(&lfull[s], 1);
+      dev::mbar_init(&lempty[s], kMmaWarps);
     }
     *abort_flag = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) rcp[i] = p.rcp[i];     // constant indices: stays in parameter space
     dev::fence_mbar_init();
   }
   __syncthreads();
 
   if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ X producer
     if (lane == 0) {
       dev::tma_prefetch_desc(&tm_x);
-      if (kDown) dev::tma_prefetch_desc(&tm_l);
       int issued = 0;
       for (int it = 0; it < nk; ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (!dev::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.budget_ns)) {
+        const int s = it % kXStages;
+        if (!dev::mbar_wait(&xempty[s], ((uint32_t)(it / kXStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
           record_error(p.err, abort_flag, 0x101);
           break;
         }
-        uint8_t* st = smem + s * kStageBytes;
+        uint8_t* st = smem + s * kXStageBytes;
         const int k0 = it * kBK;
         const int kvalid = min(kBK, K - k0);
         const int nsub = kvalid >> 6;
-        uint32_t bytes = (uint32_t)nsub * 4096u;
-        if (kDown) bytes += (uint32_t)nsub * 4096u;
-        if (kQuant) bytes += (uint32_t)kvalid * 4u;
-        dev::mbar_arrive_expect_tx(&full[s], bytes);
-        for (int j = 0; j < nsub; ++j) dev::tma_load_2d(st + j * 4096, &tm_x, &full[s], k0 + 64 * j, row0);
-        if (kDown)
-          for (int j = 0; j < nsub; ++j) dev::tma_load_2d(st + kXBytes + j * 4096, &tm_l, &full[s], k0 + 64 * j, 0);
-        if (kQuant) dev::bulk_load(st + kXBytes + kLBytes, p.inv_lam + k0, (uint32_t)kvalid * 4u, &full[s]);
+        dev::mbar_arrive_expect_tx(&xfull[s], (uint32_t)nsub * 4096u + (kQuant ? (uint32_t)kvalid * 4u : 0u));
+        for (int j = 0; j < nsub; ++j) dev::tma_load_2d(st + j * 4096, &tm_x, &xfull[s], k0 + 64 * j, row0);
+        if (kQuant) dev::bulk_load(st + kXBytes, p.inv_lam + k0, (uint32_t)kvalid * 4u, &xfull[s]);
         issued = it + 1;
       }
       // Do not leave while copies into this CTA's shared memory are in flight.
-      for (int it = max(0, issued - kStages); it < issued; ++it) {
-        const int s = it % kStages;
-        if (!dev::mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) break;
+      for (int it = max(0, issued - kXStages); it < issued; ++it)
+        if (!dev::mbar_wait(&xfull[it % kXStages], (uint32_t)(it / kXStages) & 1u, abort_flag, p.budget_ns)) break;
+    }
+    return;
+  }
+  if (warp == kConsumerWarps + 1) {
+    // ------------------------------------------------------------ L1d^T producer
+    if (kDown && lane == 0) {
+      dev::tma_prefetch_desc(&tm_l);
+      int issued = 0;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % kLStages;
+        if (!dev::mbar_wait(&lempty[s], ((uint32_t)(it / kLStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+          record_error(p.err, abort_flag, 0x104);
+          break;
+        }
+        const int k0 = it * kBK;
+        const int nsub = min(kBK, K - k0) >> 6;
+        dev::mbar_arrive_expect_tx(&lfull[s], (uint32_t)nsub * 4096u);
+        for (int j = 0; j < nsub; ++j)
+          dev::tma_load_2d(lring + s * kLBytes + j * 4096, &tm_l, &lfull[s], k0 + 64 * j, 0);
+        issued = it + 1;
       }
+      for (int it = max(0, issued - kLStages); it < issued; ++it)
+        if (!dev::mbar_wait(&lfull[it % kLStages], (uint32_t)(it / kLStages) & 1u, abort_flag, p.budget_ns)) break;
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers
-  float* red = reinterpret_cast<float*>(smem + kStages * kStageBytes + 256);   // k-half partial sums
-  float* rcp = red + 2 * 4 * 32 * 4;                                           // reciprocal table
-  if (threadIdx.x == 0) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) rcp[i] = p.rcp[i];     // constant indices: stays in parameter space
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  const int grow = row0 + lane;         // quantizer: this lane's row (may be >= M: zero padding)
-  const int qcol = warp * 16;           //            16-column group of the stage
-  const int mt = warp & 1;              // down projection: 16-row tile
-  const int nt = (warp >> 1) & 3;       //                  8-column tile of XL
-  const int kh = warp >> 3;             //                  half of the stage's k-steps
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  bool ok = true;
+  const bool quant_warp = warp < kQuantWarps;
+  if ((quant_warp && !kQuant) || (!quant_warp && !kDown)) return;   // role not used by this variant
 
+  if (quant_warp) {
+    // ---------------------------------------------------------- quantizer
+    const int grow = row0 + lane;                     // this lane's row (may be >= M: zero padding)
+    const int col0 = warp * 32;                       // 2 groups of 16 columns of each stage
+    uint16_t* scale_pair = reinterpret_cast<uint16_t*>(p.scales + sf_offset(grow, 2 * warp, K));
+    uint8_t* ctile = cbuf + warp * 2 * kCodeTile;
+    if (lane == 0) dev::tma_prefetch_desc(&tm_c);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % kXStages;
+      if (!dev::mbar_wait(&xfull[s], (uint32_t)(it / kXStages) & 1u, abort_flag, p.budget_ns)) {
+        record_error(p.err, abort_flag, 0x102);
+        break;
+      }
+      const uint8_t* st = smem + s * kXStageBytes;
+      const int k0 = it * kBK;
+      const int kvalid = min(kBK, K - k0);
+      const bool active = col0 < kvalid;              // kvalid is a multiple of 64
+      uint32_t packed[4] = {0u, 0u, 0u, 0u}, sb2 = 0u;
+      if (active) {
+        const uint8_t* xt = st + (col0 >> 6) * 4096;
+        const int c0 = (col0 & 63) >> 3;               // first 16-byte chunk of the columns in a row
+        const float4* inv4 = reinterpret_cast<const float4*>(st + kXBytes) + (col0 >> 2);
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(xt + sw128(lane, c0 + i));
+          const float4 ia = inv4[2 * i], ib = inv4[2 * i + 1];
+          const float iv[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[i * 8 + 2 * e] = __fmul_rn(__uint_as_float(w[e] << 16), iv[2 * e]);
+            v[i * 8 + 2 * e + 1] = __fmul_rn(__uint_as_float(w[e] & 0xFFFF0000u), iv[2 * e + 1]);
+          }
+        }
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          a0 = fmaxf(a0, fabsf(v[i]));
+          a1 = fmaxf(a1, fabsf(v[16 + i]));
+        }
+        sb2 = dev::cvt_e4m3x2(__fmul_rn(a0, p.c_x), __fmul_rn(a1, p.c_x));
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const uint32_t sb = (sb2 >> (8 * g)) & 0xFFu;
+          if (sb != 0u) {
+            const uint32_t e = sb >> 3, m = sb & 7u;
+            const int p2 = (e ? 7 - (int)e : 9) - p.g_x_exp;
+            const float invs = rcp[(e ? 0 : 8) + m] * __int_as_float((p2 + 127) << 23);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float q[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[g * 16 + h * 8 + i], invs);
+              packed[2 * g + h] = dev::cvt_e2m1x8(q);
+            }
+          }
+        }
+      }
+      // the stage's inputs have been read
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&xempty[s]);
+      if (active) {
+        scale_pair[(size_t)(k0 >> 6) * 256] = (uint16_t)(sb2 & 0xFFFFu);   // next 64 columns: next 512-byte chunk
+        // codes: this warp's 32 x 16-byte tile, stored with TMA once the store
+        // that last read this buffer (two stages ago) is done reading
+        uint8_t* ct = ctile + (it & 1) * kCodeTile;
+        if (lane == 0) dev::bulk_wait_group_read<1>();
+        __syncwarp();
+        *reinterpret_cast<uint4*>(ct + lane * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        dev::fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          dev::tma_store_2d(&tm_c, ct, (k0 + col0) >> 1, row0);
+          dev::bulk_commit_group();
+        }
+      }
+    }
+    if (lane == 0) dev::bulk_wait_group_all();
+    return;
+  }
+
+  // ------------------------------------------------------------ down projection
+  const int mw = warp - kQuantWarps;                  // k-steps 2mw, 2mw+1 of each stage
+  float acc[2][4][4] = {};                            // 2 row tiles x 4 column tiles
+  bool ok = true;
   for (int it = 0; it < nk; ++it) {
-    const int s = it % kStages;
-    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-    const bool got = dev::mbar_wait(&full[s], ph, abort_flag, p.budget_ns);
+    const int s = it % kXStages;
+    const int ls = it % kLStages;
+    const bool got = dev::mbar_wait(&xfull[s], (uint32_t)(it / kXStages) & 1u, abort_flag, p.budget_ns) &&
+                     dev::mbar_wait(&lfull[ls], (uint32_t)(it / kLStages) & 1u, abort_flag, p.budget_ns);
     if (!__all_sync(0xffffffffu, got)) {            // warp-uniform exit (ldmatrix/mma are warp-collective)
-      if (lane == 0) record_error(p.err, abort_flag, 0x102);
+      if (lane == 0) record_error(p.err, abort_flag, 0x103);
       ok = false;
       break;
     }
-    const uint8_t* st = smem + s * kStageBytes;
-    const int k0 = it * kBK;
-    const int kvalid = min(kBK, K - k0);
-
-    if (kQuant && qcol < kvalid) {
-      const uint8_t* xt = st + (qcol >> 6) * 4096;
-      const int c0 = (qcol & 63) >> 3;                  // first 16-byte chunk of the group in its row
-      const float4* inv4 = reinterpret_cast<const float4*>(st + kXBytes + kLBytes) + (qcol >> 2);
-      float v[16];
-      float a = 0.f;
+    const int kvalid = min(kBK, K - it * kBK);
+    const uint32_t xbase = dev::smem_u32(smem + s * kXStageBytes);
+    const uint32_t lbase = dev::smem_u32(lring + ls * kLBytes);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(xt + sw128(lane, c0 + i));
-        const float4 ia = inv4[2 * i], ib = inv4[2 * i + 1];
-        const float iv[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    for (int h = 0; h < 2; ++h) {
+      const int kk = 2 * mw + h;
+      if (kk * 16 < kvalid) {
+        const int sub = kk >> 2;
+        const int c0 = (kk & 3) * 2;                  // first 16-byte chunk of the k-step
+        uint32_t b[2][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[i * 8 + 2 * e] = __fmul_rn(__uint_as_float(w[e] << 16), iv[2 * e]);
-          v[i * 8 + 2 * e + 1] = __fmul_rn(__uint_as_float(w[e] & 0xFFFF0000u), iv[2 * e + 1]);
+        for (int np = 0; np < 2; ++np) {
+          // n-tiles 2np, 2np+1: matrices (n 0-7, k lo), (n 0-7, k hi), (n 8-15, k lo), (n 8-15, k hi)
+          const int brow = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+          ldsm_x4(lbase + sub * 4096 + sw128(brow, c0 + ((lane >> 3) & 1)), b[np]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          uint32_t a[4];
+          ldsm_x4(xbase + sub * 4096 + sw128(mt * 16 + (lane & 15), c0 + (lane >> 4)), a);
+#pragma unroll
+          for (int np = 0; np < 2; ++np) {
+            mma_16816(acc[mt][2 * np], a, b[np][0], b[np][1]);
+            mma_16816(acc[mt][2 * np + 1], a, b[np][2], b[np][3]);
+          }
         }
       }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
-      const uint32_t sb = dev::cvt_e4m3x2(__fmul_rn(a, p.c_x), 0.0f) & 0xFFu;
-      uint32_t packed0 = 0u, packed1 = 0u;
-      if (sb != 0u) {
-        const uint32_t e = sb >> 3, m = sb & 7u;
-        const int p2 = (e ? 7 - (int)e : 9) - p.g_x_exp;
-        const float invs = rcp[(e ? 0 : 8) + m] * __int_as_float((p2 + 127) << 23);
-        float q[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], invs);
-        packed0 = dev::cvt_e2m1x8(q);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[8 + i], invs);
-        packed1 = dev::cvt_e2m1x8(q);
-      }
-      if (grow < p.M)
-        *reinterpret_cast<uint2*>(p.codes + (size_t)grow * (size_t)(K >> 1) + ((k0 + qcol) >> 1)) =
-            make_uint2(packed0, packed1);
-      p.scales[sf_offset(grow, (k0 + qcol) >> 4, K)] = (uint8_t)sb;
     }
-
-    if (kDown) {
-      const uint32_t xbase = dev::smem_u32(st);
-      const uint32_t lbase = dev::smem_u32(st + kXBytes);
-      const int nsteps = kvalid >> 4;
-      const int arow = mt * 16 + (lane & 15);
-      const int brow = nt * 8 + (lane & 7);
-#pragma unroll 2
-      for (int kk = kh * 8; kk < min(nsteps, kh * 8 + 8); kk += 2) {
-        const int sub = kk >> 2;
-        const int cpair = (kk & 3) * 2;                 // 16B chunk of this k-step pair
-        uint32_t b[4];
-        ldsm_x4(lbase + sub * 4096 + sw128(brow, cpair + (lane >> 3)), b);
-        uint32_t a[4];
-        ldsm_x4(xbase + sub * 4096 + sw128(arow, cpair + (lane >> 4)), a);
-        mma_16816(acc, a, b[0], b[1]);
-        ldsm_x4(xbase + sub * 4096 + sw128(arow, cpair + 2 + (lane >> 4)), a);
-        mma_16816(acc, a, b[2], b[3]);
-      }
-    }
-
     __syncwarp();
-    if (lane == 0) dev::mbar_arrive(&empty[s]);
+    if (lane == 0) {
+      dev::mbar_arrive(&xempty[s]);
+      dev::mbar_arrive(&lempty[ls]);
+    }
   }
 
-  if (kDown) {
-    // sum the two k-halves; every consumer warp reaches this barrier (no early exit)
-    float* slot = red + ((mt * 4 + nt) * 32 + lane) * 4;
-    if (kh == 1) {
+  // Sum the eight partials through shared memory, in the L1d^T ring: only the
+  // down-projection warps read it and the producer issues no copy beyond the
+  // last k-tile, which every one of them has consumed once all of them reach
+  // this barrier.  Every down-projection warp reaches both barriers.
+  mma_warps_sync();
 #pragma unroll
-      for (int i = 0; i < 4; ++i) slot[i] = acc[i];
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-    if (kh == 0 && ok && !*abort_flag) {
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] += slot[i];
-      const int r_a = row0 + mt * 16 + (lane >> 2);
-      const int col = nt * 8 + 2 * (lane & 3);
-      if (r_a < p.M)
-        *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)r_a * 32 + col) = __floats2bfloat162_rn(acc[0], acc[1]);
-      if (r_a + 8 < p.M)
-        *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)(r_a + 8) * 32 + col) =
-            __floats2bfloat162_rn(acc[2], acc[3]);
+    for (int n = 0; n < 4; ++n)
+      part[(mw * 32 + lane) * 8 + mt * 4 + n] = make_float4(acc[mt][n][0], acc[mt][n][1], acc[mt][n][2], acc[mt][n][3]);
+  mma_warps_sync();
+  if (ok && !*abort_flag) {
+    // thread t sums one fragment (4 values) over the eight partials
+    const int t = mw * 32 + lane;                      // 0..255
+    const int fm = t >> 7, fl = (t >> 2) & 31, fn = t & 3;
+    const float4* src = part + fl * 8 + fm * 4 + fn;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int g = 0; g < kMmaWarps; ++g) {
+      const float4 v = src[g * 32 * 8];
+      sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
     }
+    const int row = row0 + fm * 16 + (fl >> 2);
+    const int col = fn * 8 + 2 * (fl & 3);
+    if (row < p.M)
+      *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)row * 32 + col) = __floats2bfloat162_rn(sum.x, sum.y);
+    if (row + 8 < p.M)
+      *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)(row + 8) * 32 + col) = __floats2bfloat162_rn(sum.z, sum.w);
   }
 }
 
 template <bool Q, bool D>
-cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const K1Params& p, cudaStream_t stream) {
+cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CUtensorMap& tm_c,
+                        const K1Params& p, cudaStream_t stream) {
   auto kern = k1_kernel<Q, D>;
   static thread_local int configured_device = -1;
   int dev = 0;
@@ -261,7 +359,7 @@ cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const 
   }
   const int mpad = (p.M + 127) / 128 * 128;
   dim3 grid(mpad / kRows);
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(tm_x, tm_l, p);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(tm_x, tm_l, tm_c, p);
   return cudaGetLastError();
 }
 
@@ -269,12 +367,12 @@ cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const 
 
 int k1_rows_per_cta() { return kRows; }
 
-cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const K1Params& p, int mode,
-                      cudaStream_t stream) {
+cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CUtensorMap& tm_c,
+                      const K1Params& p, int mode, cudaStream_t stream) {
   switch (mode) {
-    case 0: return launch_k1_t<true, true>(tm_x, tm_l, p, stream);
-    case 1: return launch_k1_t<true, false>(tm_x, tm_l, p, stream);
-    case 2: return launch_k1_t<false, true>(tm_x, tm_l, p, stream);
+    case 0: return launch_k1_t<true, true>(tm_x, tm_l, tm_c, p, stream);
+    case 1: return launch_k1_t<true, false>(tm_x, tm_l, tm_c, p, stream);
+    case 2: return launch_k1_t<false, true>(tm_x, tm_l, tm_c, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -41,24 +41,55 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBN = 256;
-constexpr int kBKBytes = 128;               // 256 E2M1 values per row per stage
-constexpr int kStages = 3;
+// Stage shape: kKB 64-element K blocks per pipeline stage.  kKB = 4 gives
+// 128-byte operand rows (128-byte swizzle), kKB = 2 gives 64-byte rows
+// (64-byte swizzle) and twice as many, half-size stages in the same memory.
+#ifndef SVDQ_K2_KB
+#define SVDQ_K2_KB 4
+#endif
+#ifndef SVDQ_K2_STAGES
+#define SVDQ_K2_STAGES 3
+#endif
+#ifndef SVDQ_K2_LOOKAHEAD
+#define SVDQ_K2_LOOKAHEAD 0
+#endif
+// Scale-factor copies issued by a dedicated warp (1) or by the MMA warp (0).
+#ifndef SVDQ_K2_CP_WARP
+#define SVDQ_K2_CP_WARP 1
+#endif
+// Epilogue drains its 128 accumulator columns into registers before any math (1),
+// or loads them chunk by chunk, overlapping each load with the previous chunk's math (0).
+#ifndef SVDQ_K2_FAST_DRAIN
+#define SVDQ_K2_FAST_DRAIN 1
+#endif
+constexpr bool kCpWarp = SVDQ_K2_CP_WARP != 0;
+constexpr bool kFastDrain = SVDQ_K2_FAST_DRAIN != 0;
+constexpr int kKB = SVDQ_K2_KB;
+constexpr int kBKBytes = kKB * 32;          // E2M1 bytes per operand row per stage
+constexpr int kStages = SVDQ_K2_STAGES;
+constexpr bool kLookahead = SVDQ_K2_LOOKAHEAD != 0;
+constexpr uint32_t kSwz = kKB == 4 ? 2u : 4u;          // descriptor layout: 128B or 64B swizzle
+constexpr uint32_t kSwzAtom = 8u * kBKBytes;           // bytes between 8-row groups
+static_assert(kKB == 2 || kKB == 4, "stage shape");
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kCpWarpIdx = 2 + kEpiWarps;
+constexpr int kThreads = (2 + kEpiWarps + (kCpWarp ? 1 : 0)) * 32;
 constexpr int kEpiBufBytes = 32 * 64;        // one 32 x 32 BF16 output chunk
 constexpr int kEpiWarpBytes = 2 * kEpiBufBytes + 512;   // two chunk buffers + 128 bias floats
 constexpr int kABytes = kBM * kBKBytes;      // 16 KiB
 constexpr int kBBytes = kBN * kBKBytes;      // 32 KiB
-constexpr int kSFABytes = 4 * 512;           // 4 K-blocks x 128 rows
-constexpr int kSFBBytes = 2 * 4 * 512;       // 2 row blocks x 4 K-blocks
-constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;   // 54 KiB
+constexpr int kSFABytes = kKB * 512;         // kKB K-blocks x 128 rows
+constexpr int kSFBBytes = 2 * kKB * 512;     // 2 row blocks x kKB K-blocks
+constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+static_assert(kStageBytes % 1024 == 0, "stage alignment");
+static_assert(kABytes >= kBM * 64 && kBBytes >= kBN * 64, "the branch stage fits a pipeline stage");
 constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiWarpBytes + 1024 + 256;
 constexpr int kTmemCols = 512;
 // Scale factors in TMEM, one region per pipeline stage (so a region is only
 // rewritten after the MMAs that read it have completed): 4 columns per 128-row
 // x 64-K block, 16 for A and 32 for B per stage.
 constexpr int kSFCol0 = 256;
-constexpr int kSFStageCols = 48;
+constexpr int kSFStageCols = 12 * kKB;       // 4 columns of A + 8 of B per K block
 static_assert(kSFCol0 + kStages * kSFStageCols <= kTmemCols, "TMEM budget");
 
 __device__ __forceinline__ void record_error(int* err, volatile int* abort_flag, int code) {
@@ -83,7 +114,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_ready = drain + 1;                  // [kStages], scale factors of a stage in TMEM
+  uint64_t* cp_drain = sf_ready + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -93,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles_n = (N + kBN - 1) / kBN;
   const int num_tiles = tiles_m * tiles_n;
   const int kblocks = K >> 6;                     // 64-element K blocks
-  const int ktiles = (kblocks + 3) >> 2;
+  const int ktiles = (kblocks + kKB - 1) / kKB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -103,6 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::mbar_init(acc_full, 1);
     dev::mbar_init(acc_empty, kEpiWarps);
     dev::mbar_init(drain, 1);
+    for (int st = 0; st < kStages; ++st) dev::mbar_init(&sf_ready[st], 1);
+    dev::mbar_init(cp_drain, 1);
     *abort_flag = 0;
     dev::fence_mbar_init();
   }
@@ -127,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int it = 0;
       bool ok = true;
+      bool deps_ready = false;     // activations come from the preceding kernel (launched as a dependency)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m0 = (tile % tiles_m) * kBM;
         const int n0 = (tile / tiles_m) * kBN;
@@ -139,8 +175,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* st = smem + s * kStageBytes;
           dev::mbar_arrive_expect_tx(&full[s], kBM * 64 + kBN * 64);
-          dev::tma_load_2d(st, &tm_xl, &full[s], 0, m0);
           dev::tma_load_2d(st + kABytes, &tm_l2, &full[s], 0, n0);
+          if (!deps_ready) {
+            dev::griddep_wait();
+            deps_ready = true;
+          }
+          dev::tma_load_2d(st, &tm_xl, &full[s], 0, m0);
           ++it;
         }
         for (int kt = 0; kt < ktiles; ++kt) {
@@ -151,19 +191,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = smem + s * kStageBytes;
-          const int nkb = min(4, kblocks - 4 * kt);
+          const int nkb = min(kKB, kblocks - kKB * kt);
           const uint32_t sf_bytes = (uint32_t)nkb * 512u;
           dev::mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + 3u * sf_bytes);
-          dev::tma_load_2d(st, &tm_a, &full[s], kt * kBKBytes, m0);
+          // weights first: they do not depend on the preceding kernel
           dev::tma_load_2d(st + kABytes, &tm_b, &full[s], kt * kBKBytes, n0);
-          const size_t a_chunk = (size_t)(m0 >> 7) * (size_t)kblocks + (size_t)(4 * kt);
-          dev::bulk_load(st + kABytes + kBBytes, p.sfa + a_chunk * 512, sf_bytes, &full[s]);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const size_t b_chunk = (size_t)((n0 >> 7) + h) * (size_t)kblocks + (size_t)(4 * kt);
-            dev::bulk_load(st + kABytes + kBBytes + kSFABytes + h * 2048, p.sfb + b_chunk * 512, sf_bytes,
+            const size_t b_chunk = (size_t)((n0 >> 7) + h) * (size_t)kblocks + (size_t)(kKB * kt);
+            dev::bulk_load(st + kABytes + kBBytes + kSFABytes + h * (kKB * 512), p.sfb + b_chunk * 512, sf_bytes,
                            &full[s]);
           }
+          if (!deps_ready) {
+            dev::griddep_wait();
+            deps_ready = true;
+          }
+          dev::tma_load_2d(st, &tm_a, &full[s], kt * kBKBytes, m0);
+          const size_t a_chunk = (size_t)(m0 >> 7) * (size_t)kblocks + (size_t)(kKB * kt);
+          dev::bulk_load(st + kABytes + kBBytes, p.sfa + a_chunk * 512, sf_bytes, &full[s]);
           ++it;
         }
       }
@@ -188,24 +233,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto copy_scales = [&](int slot, int kt) {
         const int s = slot % kStages;
-        const int nkb = min(4, kblocks - 4 * kt);
+        const int nkb = min(kKB, kblocks - kKB * kt);
         const uint32_t sfa0 = dev::smem_u32(smem + s * kStageBytes) + kABytes + kBBytes;
         const uint32_t sfb0 = sfa0 + kSFABytes;
         const uint32_t tsfa = tmem + kSFCol0 + s * kSFStageCols;
-        const uint32_t tsfb = tsfa + 16;
+        const uint32_t tsfb = tsfa + 4 * kKB;
         for (int j = 0; j < nkb; ++j) {
           dev::tmem_copy_32x128b_x4(tsfa + 4 * j, dev::smem_desc(sfa0 + 512 * j, 0, 128, 0));
           dev::tmem_copy_32x128b_x4(tsfb + 8 * j, dev::smem_desc(sfb0 + 512 * j, 0, 128, 0));
-          dev::tmem_copy_32x128b_x4(tsfb + 8 * j + 4, dev::smem_desc(sfb0 + 2048 + 512 * j, 0, 128, 0));
+          dev::tmem_copy_32x128b_x4(tsfb + 8 * j + 4, dev::smem_desc(sfb0 + kKB * 512 + 512 * j, 0, 128, 0));
         }
+      };
+      uint32_t sf_phase = 0;                          // per-stage parity of sf_ready (kCpWarp)
+      auto wait_sf = [&](int slot) -> bool {
+        const int st = slot % kStages;
+        if (!dev::mbar_wait(&sf_ready[st], (sf_phase >> st) & 1u, abort_flag, p.budget_ns)) {
+          record_error(p.err, abort_flag, 0x207);
+          return false;
+        }
+        sf_phase ^= 1u << st;
+        dev::tc_fence_after();
+        return true;
       };
       int it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
         const int kslot0 = it + (p.branch ? 1 : 0);
         // the first k-tile's scales do not touch the accumulator: copy them first
-        if (!(ok = wait_full(kslot0, 0x205))) break;
-        copy_scales(kslot0, 0);
+        if (!kCpWarp) {
+          if (!(ok = wait_full(kslot0, 0x205))) break;
+          copy_scales(kslot0, 0);
+        }
         if (!dev::mbar_wait(acc_empty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag, p.budget_ns)) {
           record_error(p.err, abort_flag, 0x203);
           ok = false;
@@ -230,18 +288,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < ktiles; ++kt) {
           const int slot = kslot0 + kt;
           const int s = slot % kStages;
-          if (kt + 1 < ktiles) {
-            if (!(ok = wait_full(slot + 1, 0x205))) break;
-            copy_scales(slot + 1, kt + 1);
+          if (kCpWarp) {
+            if (!(ok = wait_full(slot, 0x205))) break;
+            if (!(ok = wait_sf(slot))) break;
+          } else if (kLookahead) {
+            if (kt + 1 < ktiles) {
+              if (!(ok = wait_full(slot + 1, 0x205))) break;
+              copy_scales(slot + 1, kt + 1);
+            }
+          } else if (kt > 0) {
+            if (!(ok = wait_full(slot, 0x205))) break;
+            copy_scales(slot, kt);
           }
-          const int nkb = min(4, kblocks - 4 * kt);
+          const int nkb = min(kKB, kblocks - kKB * kt);
           const uint32_t a0 = dev::smem_u32(smem + s * kStageBytes);
           const uint32_t b0 = a0 + kABytes;
           const uint32_t tsfa = tmem + kSFCol0 + s * kSFStageCols;
-          const uint32_t tsfb = tsfa + 16;
+          const uint32_t tsfb = tsfa + 4 * kKB;
           for (int j = 0; j < nkb; ++j) {
-            const uint64_t ad = dev::smem_desc(a0 + 32 * j, 16, 1024, 2);
-            const uint64_t bd = dev::smem_desc(b0 + 32 * j, 16, 1024, 2);
+            const uint64_t ad = dev::smem_desc(a0 + 32 * j, 16, kSwzAtom, kSwz);
+            const uint64_t bd = dev::smem_desc(b0 + 32 * j, 16, kSwzAtom, kSwz);
             dev::mma_nvfp4(tmem, ad, bd, idesc_f4, tsfa + 4 * j, tsfb + 8 * j, accumulate);
             accumulate = 1;
           }
@@ -254,6 +320,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Wait until every MMA and copy this thread issued has completed.
       dev::tc_commit(drain);
       dev::mbar_wait(drain, 0, abort_flag, p.budget_ns);
+    }
+  } else if (kCpWarp && warp == kCpWarpIdx) {
+    // ------------------------------------------------------------ scale-factor copier
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        bool ok = true;
+        if (p.branch) ++it;
+        for (int kt = 0; kt < ktiles; ++kt, ++it) {
+          const int st = it % kStages;
+          if (!dev::mbar_wait(&full[st], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
+            record_error(p.err, abort_flag, 0x208);
+            ok = false;
+            break;
+          }
+          dev::tc_fence_after();
+          const int nkb = min(kKB, kblocks - kKB * kt);
+          const uint32_t sfa0 = dev::smem_u32(smem + st * kStageBytes) + kABytes + kBBytes;
+          const uint32_t sfb0 = sfa0 + kSFABytes;
+          const uint32_t tsfa = tmem + kSFCol0 + st * kSFStageCols;
+          const uint32_t tsfb = tsfa + 4 * kKB;
+          for (int j = 0; j < nkb; ++j) {
+            dev::tmem_copy_32x128b_x4(tsfa + 4 * j, dev::smem_desc(sfa0 + 512 * j, 0, 128, 0));
+            dev::tmem_copy_32x128b_x4(tsfb + 8 * j, dev::smem_desc(sfb0 + 512 * j, 0, 128, 0));
+            dev::tmem_copy_32x128b_x4(tsfb + 8 * j + 4, dev::smem_desc(sfb0 + kKB * 512 + 512 * j, 0, 128, 0));
+          }
+          dev::tc_commit(&sf_ready[st]);
+        }
+        if (!ok) break;
+      }
+      dev::tc_commit(cp_drain);
+      dev::mbar_wait(cp_drain, 0, abort_flag, p.budget_ns);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -282,14 +380,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       dev::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 128);
-      uint32_t va[32], vb[32];
+      uint32_t va[32], vb[32], vc[32], vd[32];
       dev::tmem_load_32cols(taddr, va);
-      dev::tmem_load_wait(va);
+      if (kFastDrain) {
+        // all 128 columns into registers, then hand the accumulator back at once
+        dev::tmem_load_32cols(taddr + 32, vb);
+        dev::tmem_load_32cols(taddr + 64, vc);
+        dev::tmem_load_32cols(taddr + 96, vd);
+        dev::tmem_load_wait(va);
+        dev::tmem_load_wait(vb);
+        dev::tmem_load_wait(vc);
+        dev::tmem_load_wait(vd);
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(acc_empty);
+      } else {
+        dev::tmem_load_wait(va);
+      }
 #pragma unroll
       for (int c = 0; c < 4; ++c, ++chunk) {
-        uint32_t (&cur)[32] = (c & 1) ? vb : va;
+        uint32_t (&cur)[32] = kFastDrain ? (c == 0 ? va : c == 1 ? vb : c == 2 ? vc : vd) : ((c & 1) ? vb : va);
         uint32_t (&nxt)[32] = (c & 1) ? va : vb;
-        if (c + 1 < 4) dev::tmem_load_32cols(taddr + (uint32_t)((c + 1) * 32), nxt);
+        if (!kFastDrain && c + 1 < 4) dev::tmem_load_32cols(taddr + (uint32_t)((c + 1) * 32), nxt);
         // the buffer of this chunk was last read by the store issued two chunks ago
         if (lane == 0) dev::bulk_wait_group_read<1>();
         __syncwarp();
@@ -319,8 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           dev::tma_store_2d(&tm_y, buf, n0 + c * 32, m0 + q * 32);
           dev::bulk_commit_group();
         }
-        if (c + 1 < 4) dev::tmem_load_wait(nxt);
-        if (c == 2) {
+        if (!kFastDrain && c + 1 < 4) dev::tmem_load_wait(nxt);
+        if (!kFastDrain && c == 2) {
           // the last chunk is in registers: hand the accumulator back to the MMA warp
           dev::tc_fence_before();
           __syncwarp();
@@ -344,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 int k2_block_n() { return kBN; }
+int k2_stage_k_bytes() { return kBKBytes; }
 
 cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
                       const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
@@ -358,8 +471,20 @@ cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CU
   }
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  k2_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_xl, tm_l2, tm_y, p);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the prologue (barriers, TMEM, descriptor
+  // prefetch, weight tiles) overlaps the tail of the kernel that produces the
+  // activations; the producer waits for it before the first activation load.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k2_kernel, tm_a, tm_b, tm_xl, tm_l2, tm_y, p);
 }
 
 }  // namespace svdq

@@ -45,14 +45,15 @@ struct UpParams {
 };
 
 // mode 0 = fused, 1 = quantize only, 2 = down projection only
-cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const K1Params& p, int mode,
-                      cudaStream_t stream);
+cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CUtensorMap& tm_c,
+                      const K1Params& p, int mode, cudaStream_t stream);
 int k1_rows_per_cta();
 
 cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
                       const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
                       cudaStream_t stream);
 int k2_block_n();
+int k2_stage_k_bytes();   // E2M1 bytes per operand row per pipeline stage (128 or 64)
 
 cudaError_t launch_upproj(const UpParams& p, cudaStream_t stream);
 
