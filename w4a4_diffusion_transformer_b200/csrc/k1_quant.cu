@@ -205,24 +205,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t* xt = st + (col0 >> 6) * 4096;
         const int c0 = (col0 & 63) >> 3;               // first 16-byte chunk of the columns in a row
         const float4* inv4 = reinterpret_cast<const float4*>(st + kXBytes) + (col0 >> 2);
-        float v[32];
+        // v = fp32(x * inv_lam), two elements per packed multiply (each lane
+        // of the pair is an IEEE round-to-nearest product)
+        float2 v[16];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint4 raw = *reinterpret_cast<const uint4*>(xt + sw128(lane, c0 + i));
           const float4 ia = inv4[2 * i], ib = inv4[2 * i + 1];
-          const float iv[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
+          const float2 iv[4] = {make_float2(ia.x, ia.y), make_float2(ia.z, ia.w), make_float2(ib.x, ib.y),
+                                make_float2(ib.z, ib.w)};
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            v[i * 8 + 2 * e] = __fmul_rn(__uint_as_float(w[e] << 16), iv[2 * e]);
-            v[i * 8 + 2 * e + 1] = __fmul_rn(__uint_as_float(w[e] & 0xFFFF0000u), iv[2 * e + 1]);
-          }
+          for (int e = 0; e < 4; ++e)
+            v[i * 4 + e] = __fmul2_rn(make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)),
+                                      iv[e]);
         }
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          a0 = fmaxf(a0, fabsf(v[i]));
-          a1 = fmaxf(a1, fabsf(v[16 + i]));
+        for (int i = 0; i < 8; ++i) {
+          a0 = dev::fmax3(a0, fabsf(v[i].x), fabsf(v[i].y));
+          a1 = dev::fmax3(a1, fabsf(v[8 + i].x), fabsf(v[8 + i].y));
         }
         sb2 = dev::cvt_e4m3x2(__fmul_rn(a0, p.c_x), __fmul_rn(a1, p.c_x));
 #pragma unroll
@@ -232,12 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t e = sb >> 3, m = sb & 7u;
             const int p2 = (e ? 7 - (int)e : 9) - p.g_x_exp;
             const float invs = rcp[(e ? 0 : 8) + m] * __int_as_float((p2 + 127) << 23);
+            const float2 inv2 = make_float2(invs, invs);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              float q[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[g * 16 + h * 8 + i], invs);
-              packed[2 * g + h] = dev::cvt_e2m1x8(q);
+              const int b = g * 8 + h * 4;
+              packed[2 * g + h] = dev::cvt_e2m1x8(__fmul2_rn(v[b], inv2), __fmul2_rn(v[b + 1], inv2),
+                                                  __fmul2_rn(v[b + 2], inv2), __fmul2_rn(v[b + 3], inv2));
             }
           }
         }

@@ -272,6 +272,15 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// ------------------------------------------------------------------ arithmetic
+
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // ------------------------------------------------------------------ conversions
 
 // Two float32 -> two E4M3 (round to nearest even, saturating): `lo` in bits
@@ -294,6 +303,22 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
       : "h"(in));
   const __half lo = __ushort_as_half((unsigned short)(h2 & 0xFFFFu));
   return __half2float(lo);
+}
+
+// Eight float32 (four pairs) -> eight E2M1 codes packed in 32 bits (round to
+// nearest even, saturating at 6); element i lands in nibble i.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+  return out;
 }
 
 // Eight float32 -> eight E2M1 codes packed in 32 bits (round to nearest even,
