@@ -186,6 +186,36 @@ svdq_status svdq_act_scales_to_logical(const svdq_layer* layer, const void* devi
  * SVDQ_ETIMEOUT if a bounded device wait expired since the last check. */
 svdq_status svdq_check(const svdq_layer* layer, void* stream);
 
+/* ------------------------------------------------------- allocation-free forward */
+
+/* Size of the library's built-in device workspace (16 MiB). */
+#define SVDQ_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/* svdq_linear_forward_static -- svdq_linear_forward without a caller workspace.
+ *
+ * (No counterpart on the method's pages: this is a deployment convenience.)
+ * For callers that cannot allocate device memory when they run a layer -- code
+ * inside a framework's memory pool or arena without access to its allocator,
+ * runtimes that forbid allocation after start-up, plug-ins that only receive
+ * input and output pointers -- the workspace is a fixed array of
+ * SVDQ_STATIC_WORKSPACE_BYTES in the library's own device memory.  The CUDA
+ * driver creates it on every device that loads the library and keeps it until
+ * the process exits.  This call allocates and frees nothing.
+ *
+ *   X, M, Y, stream, flags  as for svdq_linear_forward.
+ * Returns SVDQ_EUNSUPPORTED if svdq_workspace_bytes(layer, M) exceeds
+ * SVDQ_STATIC_WORKSPACE_BYTES (for K = 3072: M above 9,349 tokens), and
+ * SVDQ_ECUDA if the workspace address cannot be obtained.
+ *
+ * The first call on a device looks up the array's device address (once, with
+ * that device made current); make that first call before any stream capture.
+ * All calls share the one array, which keeps the last call's contents (the
+ * forward needs no zeroed workspace): calls whose work overlaps on the GPU --
+ * on different streams, or on different layers at once -- race and must not be
+ * issued. */
+svdq_status svdq_linear_forward_static(const svdq_layer* layer, const void* X, int M, void* Y,
+                                       void* stream, unsigned flags);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,7 +38,9 @@ EXPORTED = [
     "svdq_prepare", "svdq_destroy", "svdq_get_info", "svdq_tensor_bytes", "svdq_export",
     "svdq_status_string", "svdq_workspace_bytes", "svdq_linear_forward", "svdq_quantize_act",
     "svdq_gemm", "svdq_act_scale_bytes", "svdq_act_scales_to_logical", "svdq_check",
+    "svdq_linear_forward_static",
 ]
+STATIC_WORKSPACE_BYTES = 16 << 20   # SVDQ_STATIC_WORKSPACE_BYTES
 
 
 class SvdqError(RuntimeError):
@@ -85,6 +87,7 @@ def load() -> ctypes.CDLL:
         "svdq_act_scale_bytes": (SZ, [P, I]),
         "svdq_act_scales_to_logical": (I, [P, P, I, P]),
         "svdq_check": (I, [P, P]),
+        "svdq_linear_forward_static": (I, [P, P, I, P, P, U]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -187,6 +190,12 @@ class Layer:
     def forward(self, X, M: int, Y, workspace, workspace_bytes: int, stream=None, flags: int = 0):
         _check(load().svdq_linear_forward(self._h, _ptr(X), M, _ptr(Y), _ptr(workspace), workspace_bytes,
                                           _stream(stream), flags), "svdq_linear_forward")
+
+    def forward_static(self, X, M: int, Y, stream=None, flags: int = 0):
+        """Forward with the library's built-in device workspace (no caller workspace,
+        no allocation); see svdq_linear_forward_static in include/svdq.h."""
+        _check(load().svdq_linear_forward_static(self._h, _ptr(X), M, _ptr(Y), _stream(stream), flags),
+               "svdq_linear_forward_static")
 
     def quantize_act(self, X, M: int, codes, scales, xl, stream=None, mode: int = 0):
         _check(load().svdq_quantize_act(self._h, _ptr(X), M, _ptr(codes), _ptr(scales), _ptr(xl),
