@@ -55,13 +55,22 @@ def measured_peaks():
 
 
 def profile_traffic():
-    """DRAM bytes per K2 launch from the committed ncu summary, if present."""
-    path = os.path.join(ROOT, "profiles", "k2_gemm_attn_out.json")
+    """DRAM bytes (read + write) per K2 launch from the committed ncu summary,
+    or None when the summary is missing or was taken on different K2 source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "k2_gemm_attn_out.md")
+    src = os.path.join(ROOT, "w4a4_diffusion_transformer_b200", "csrc", "k2_gemm.cu")
     try:
-        with open(path) as f:
-            return json.load(f).get("dram_bytes_per_launch")
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if f"k2_gemm.cu: {sha}" not in text:
+            return None
+        for line in text.splitlines():
+            if line.startswith("dram_bytes_per_launch:"):
+                return int(line.split(":")[1])
     except Exception:
         return None
+    return None
 
 
 class ClockSampler:
