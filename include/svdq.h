@@ -24,7 +24,8 @@
  *   - A layer owns its device buffers; svdq_destroy frees them.  A layer may be
  *     used by several streams only if their forward calls do not overlap in time
  *     on the device through a shared workspace.
- *   - Shape rules: K % 64 == 0, N % 16 == 0, M >= 1 (any M: tails are handled).
+ *   - Shape rules: K % 64 == 0, N % 16 == 0 (any N >= 1 for SVDQ_W4A16_INT4),
+ *     M >= 1 (any M: tails are handled).
  *     Other shapes return SVDQ_EUNSUPPORTED.
  */
 #ifndef SVDQ_H
@@ -153,7 +154,10 @@ size_t svdq_workspace_bytes(const svdq_layer* layer, int M);
  * over X ("Down Projection with Quantize, because they read the same input")
  * and the block-scaled tensor-core GEMM whose epilogue adds the up-projection
  * and the bias ("Up Projection with the 4-bit compute, because they write the
- * same output"; SOTA-314 "Do this").  W4A16 enqueues one weight-only kernel. */
+ * same output"; SOTA-314 "Do this").  SVDQ_W4A16_INT4 (the adaptive-norm
+ * linears, "stay W4A16") enqueues one weight-only GEMV kernel meant for a few
+ * rows (M <= 16), needs no workspace (pass NULL, 0) and accepts only
+ * SVDQ_FWD_CHECK among the flags. */
 svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, void* Y,
                                 void* workspace, size_t workspace_bytes,
                                 void* stream, unsigned flags);

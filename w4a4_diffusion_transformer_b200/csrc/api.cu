@@ -28,7 +28,7 @@ struct svdq_layer {
   __nv_bfloat16* d_l2s = nullptr;    // [N][32]   (L2b / alpha)^T
   __nv_bfloat16* d_l2t = nullptr;    // [N][32]   L2b^T (unfused up projection)
   uint8_t* d_wq = nullptr;           // [N][K/2]
-  uint8_t* d_ws = nullptr;           // weight scales, tensor-core layout
+  uint8_t* d_ws = nullptr;           // weight scales, tensor-core layout (NVFP4) or BF16 [N][K/64] (INT4)
   float* d_bias = nullptr;           // [N]
   int* d_err = nullptr;
   CUtensorMap tm_wq, tm_l2s, tm_l1t;
@@ -181,6 +181,10 @@ svdq_status upload_layer(svdq_layer* L, int device) {
               make_map(&L->tm_l1t, L->d_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, 32, 64, 32,
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return SVDQ_ECUDA;
+  } else if (h.format == SVDQ_W4A16_INT4) {
+    std::vector<uint8_t> packed(w4a16_packed_bytes(N, K));
+    w4a16_pack(h.w_codes.data(), h.w_scales_bf16.data(), N, K, packed.data());
+    chk(upload(&L->d_wq, packed.data(), packed.size()));
   }
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
@@ -290,7 +294,9 @@ svdq_status svdq_prepare(const svdq_config* cfg, int K, int N, const uint16_t* W
     if (!(cfg->alpha > 0.0f && cfg->alpha < 1.0f)) return SVDQ_EINVAL;
     if (cfg->rank != 0 && cfg->rank != 32) return SVDQ_EUNSUPPORTED;
   }
-  if (K % 64 != 0 || N % 16 != 0) return SVDQ_EUNSUPPORTED;
+  // W4A4 needs N % 16 for its TMA tiles; the weight-only GEMV takes any N
+  if (K % 64 != 0 || (!wo && N % 16 != 0)) return SVDQ_EUNSUPPORTED;
+  if (wo && !w4a16_supported(K)) return SVDQ_EUNSUPPORTED;
   svdq_layer* L = new (std::nothrow) svdq_layer();
   if (!L) return SVDQ_ENOMEM;
   svdq_status st = host_prepare(*cfg, K, N, W_bf16, bias_bf16, calib_bf16, M_calib, L->host);
@@ -429,6 +435,25 @@ svdq_status svdq_linear_forward(const svdq_layer* L, const void* X, int M, void*
                                 size_t workspace_bytes, void* stream, unsigned flags) {
   svdq_status st = check_forward_args(L, X, M, Y);
   if (st != SVDQ_OK) return st;
+  if (L->host.format == SVDQ_W4A16_INT4) {
+    // weight-only path: one kernel, no workspace
+    if (flags & (SVDQ_FWD_GELU | SVDQ_FWD_UNFUSED | SVDQ_FWD_NO_BRANCH)) return SVDQ_EUNSUPPORTED;
+    DeviceGuard g(L->device);
+    if (!g.ok) return SVDQ_ECUDA;
+    W4A16Params p;
+    p.M = M;
+    p.N = L->host.N;
+    p.K = L->host.K;
+    p.x = static_cast<const __nv_bfloat16*>(X);
+    p.wt = L->d_wq;
+    p.bias = L->d_bias;
+    p.y = static_cast<__nv_bfloat16*>(Y);
+    p.err = L->d_err;
+    p.budget_ns = L->budget_ns;
+    st = launch_w4a16(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+    if (st == SVDQ_OK && (flags & SVDQ_FWD_CHECK)) st = svdq_check(L, stream);
+    return st;
+  }
   if (L->host.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
   const WsLayout w = ws_layout(L->host, M);
   if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))

@@ -44,6 +44,24 @@ struct UpParams {
   int gelu;
 };
 
+struct W4A16Params {
+  int M, N, K;
+  const __nv_bfloat16* x;       // [M][K]
+  const uint8_t* wt;            // codes and scales packed by w4a16_pack
+  const float* bias;            // [N]
+  __nv_bfloat16* y;             // [M][N]
+  int* err;                     // set to 1 if a bounded wait gave up
+  unsigned long long budget_ns;
+};
+
+// Device layout of W4A16 weights: from codes [N][K/2] (two's complement
+// nibbles, even k low) and BF16 scales [N][K/64] to the tile-packed stream the
+// GEMV reads (w4a16_packed_bytes(N, K) bytes).
+size_t w4a16_packed_bytes(int N, int K);
+bool w4a16_supported(int K);   // shared-memory bound on K
+void w4a16_pack(const uint8_t* codes, const uint16_t* scales, int N, int K, uint8_t* out);
+cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t stream);
+
 // mode 0 = fused, 1 = quantize only, 2 = down projection only
 cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CUtensorMap& tm_c,
                       const K1Params& p, int mode, cudaStream_t stream);
