@@ -154,7 +154,11 @@ size_t svdq_workspace_bytes(const svdq_layer* layer, int M);
  * over X ("Down Projection with Quantize, because they read the same input")
  * and the block-scaled tensor-core GEMM whose epilogue adds the up-projection
  * and the bias ("Up Projection with the 4-bit compute, because they write the
- * same output"; SOTA-314 "Do this").  SVDQ_W4A16_INT4 (the adaptive-norm
+ * same output"; SOTA-314 "Do this").  For SVDQ_INT4 the GEMM dequantizes each
+ * group of 64 codes times its BF16 scale into FP16 on chip (exact: 3 + 8
+ * significant bits) and multiplies on the FP16 tensor cores, since the B200
+ * has no 4-bit integer MMA; a group whose smoothed activations exceed the
+ * calibration batch's largest by more than 32x is clamped.  SVDQ_W4A16_INT4 (the adaptive-norm
  * linears, "stay W4A16") enqueues one weight-only GEMV kernel meant for a few
  * rows (M <= 16), needs no workspace (pass NULL, 0) and accepts only
  * SVDQ_FWD_CHECK among the flags. */
@@ -163,8 +167,10 @@ svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, v
                                 void* stream, unsigned flags);
 
 /* The first kernel alone (NVFP4/INT4): writes the activation codes
- * (device [M][K/2], even k in the low nibble), the activation scales in the
- * tensor-core layout (device, svdq_act_scale_bytes(layer, M) bytes) and, when
+ * (device [M][K/2], even k in the low nibble; INT4 codes are 4-bit two's
+ * complement), the activation scales (device, svdq_act_scale_bytes(layer, M)
+ * bytes: NVFP4 E4M3 in the tensor-core layout, INT4 BF16 [K/64][M rounded up
+ * to 128], group-major, padding rows zero) and, when
  * the layer has a branch, XL = bf16(X L1d) (device [M][rank] BF16).
  * xl may be NULL for rank 0.  `mode` 0 = fused, 1 = quantize only,
  * 2 = down projection only. */
@@ -177,12 +183,12 @@ svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int M,
 svdq_status svdq_gemm(const svdq_layer* layer, const void* codes, const void* scales,
                       const void* xl, int M, void* Y, void* stream, unsigned flags);
 
-/* Bytes of the activation scales for M tokens in the tensor-core layout. */
+/* Bytes of the activation scales for M tokens in the layout the GEMM reads. */
 size_t svdq_act_scale_bytes(const svdq_layer* layer, int M);
 
-/* Host-side: convert a host copy of activation scales in the tensor-core layout
+/* Host-side: convert a host copy of activation scales in the GEMM's layout
  * (svdq_act_scale_bytes bytes) into the logical layout: NVFP4 uint8 [M][K/16],
- * INT4 uint16 [M][K/64]. */
+ * INT4 uint16 [M][K/64] (BF16 bits). */
 svdq_status svdq_act_scales_to_logical(const svdq_layer* layer, const void* device_layout,
                                        int M, void* logical);
 

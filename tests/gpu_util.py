@@ -33,12 +33,13 @@ def oracle_prep_from(L) -> dict:
     """The oracle's prepared layer built from the library's exported tensors."""
     info = L.info
     r = info["rank"]
-    p = {"fmt": "nvfp4", "rank": r, "K": info["K"], "N": info["N"],
+    fmt = "int4" if info["format"] == lib.INT4 else "nvfp4"
+    p = {"fmt": fmt, "rank": r, "K": info["K"], "N": info["N"],
          "lam": L.export("lambda"), "inv_lam": L.export("inv_lambda"),
          "L1d": syn.from_bf16_bits(L.export("L1d")).astype(np.float64) if r else np.zeros((info["K"], 0)),
          "L2b": syn.from_bf16_bits(L.export("L2b")).astype(np.float64) if r else np.zeros((0, info["N"])),
          "bias": L.export("bias").astype(np.float64), "g_x_exp": info["g_x_exp"]}
-    p.update(o.quantize_weights(L.export("R"), "nvfp4"))
+    p.update(o.quantize_weights(L.export("R"), fmt))
     assert p["g_w_exp"] == info["g_w_exp"]
     return p
 

@@ -206,8 +206,12 @@ class Layer:
                                 flags), "svdq_gemm")
 
     def act_scales_to_logical(self, device_layout: np.ndarray, M: int) -> np.ndarray:
+        """NVFP4: uint8 [M][K/16] E4M3 bytes; INT4: uint16 [M][K/64] BF16 bits."""
         info = self.info
-        out = np.empty((M, info["K"] // 16), dtype=np.uint8)
+        if info["format"] == INT4:
+            out = np.empty((M, info["K"] // 64), dtype=np.uint16)
+        else:
+            out = np.empty((M, info["K"] // 16), dtype=np.uint8)
         src = np.ascontiguousarray(device_layout, dtype=np.uint8)
         _check(load().svdq_act_scales_to_logical(self._h, _ptr(src), M, _ptr(out)), "svdq_act_scales_to_logical")
         return out

@@ -2,6 +2,7 @@
 // maps, workspace layout and the forward launches (see include/svdq.h).
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -28,7 +29,8 @@ struct svdq_layer {
   __nv_bfloat16* d_l2s = nullptr;    // [N][32]   (L2b / alpha)^T
   __nv_bfloat16* d_l2t = nullptr;    // [N][32]   L2b^T (unfused up projection)
   uint8_t* d_wq = nullptr;           // [N][K/2]
-  uint8_t* d_ws = nullptr;           // weight scales, tensor-core layout (NVFP4) or BF16 [N][K/64] (INT4)
+  uint8_t* d_ws = nullptr;           // weight scales: NVFP4 tensor-core layout; INT4 FP16 [K/64][npad] (times 2^-ew)
+  int i4_ex = 0, i4_ew = 0;          // INT4: power-of-two range exponents of the FP16 GEMM operands
   float* d_bias = nullptr;           // [N]
   int* d_err = nullptr;
   CUtensorMap tm_wq, tm_l2s, tm_l1t;
@@ -91,9 +93,26 @@ CUtensorMapSwizzle k2_swizzle() { return k2_stage_k_bytes() == 128 ? CU_TENSOR_M
 
 bool w4a4(const svdq_layer* L) { return L->host.format == SVDQ_NVFP4 || L->host.format == SVDQ_INT4; }
 
+int pad_rows(int M) { return (M + 127) / 128 * 128; }
+
+// FP16 bits of a value that is exact in float32, rounded to nearest even.
+uint16_t f16_from_double(double v) { return __half_as_ushort(__float2half_rn((float)v)); }
+int pad_cols_int4(int N) { return (N + 255) / 256 * 256; }
+
 size_t act_scale_bytes(const HostPrep& h, int M) {
-  if (h.format != SVDQ_NVFP4) return 0;
-  return (size_t)((M + 127) / 128) * (size_t)(h.K / 64) * 512;
+  if (h.format == SVDQ_NVFP4) return (size_t)((M + 127) / 128) * (size_t)(h.K / 64) * 512;
+  if (h.format == SVDQ_INT4) return (size_t)(h.K / 64) * (size_t)pad_rows(M) * 2;   // BF16 [K/64][mpad]
+  return 0;
+}
+
+// FP16 range exponents of the INT4 GEMM's dequantized operands: the largest
+// |c s| of the weights maps to at most 2^14 (4x below FP16's maximum), the
+// largest smoothed calibration activation to at most 2^12 (16x headroom).
+void int4_range_exponents(const HostPrep& h, int* ex, int* ew) {
+  float amax = 0.0f;
+  for (float v : h.R) amax = std::max(amax, std::fabs(v));
+  *ew = pow2_ceil_exponent((double)amax) - 14;
+  *ex = pow2_ceil_exponent((double)h.x_amax) - 12;
 }
 
 struct WsLayout {
@@ -150,18 +169,33 @@ svdq_status upload_layer(svdq_layer* L, int device) {
   chk(cudaMalloc(reinterpret_cast<void**>(&L->d_err), sizeof(int)));
   if (e == cudaSuccess) chk(cudaMemset(L->d_err, 0, sizeof(int)));
   chk(upload(&L->d_bias, h.bias.data(), sizeof(float) * N));
-  if (h.format == SVDQ_NVFP4) {
+  if (h.format == SVDQ_NVFP4 || h.format == SVDQ_INT4) {
     chk(upload(&L->d_inv_lam, h.inv_lam.data(), sizeof(float) * K));
     chk(upload(&L->d_wq, h.w_codes.data(), h.w_codes.size()));
-    // weight scales in the tensor-core layout, rows padded to a multiple of 256
-    const int npad = (N + 255) / 256 * 256;
-    std::vector<uint8_t> ws((size_t)(npad / 128) * (K / 64) * 512, 0);
-    for (int n = 0; n < N; ++n)
-      for (int gi = 0; gi < K / 16; ++gi) ws[sf_offset(n, gi, K)] = h.w_scales_e4m3[(size_t)n * (K / 16) + gi];
-    chk(upload(&L->d_ws, ws.data(), ws.size()));
+    int alpha_exp = h.g_x_exp + h.g_w_exp;
+    if (h.format == SVDQ_NVFP4) {
+      // weight scales in the tensor-core layout, rows padded to a multiple of 256
+      const int npad = (N + 255) / 256 * 256;
+      std::vector<uint8_t> ws((size_t)(npad / 128) * (K / 64) * 512, 0);
+      for (int n = 0; n < N; ++n)
+        for (int gi = 0; gi < K / 16; ++gi) ws[sf_offset(n, gi, K)] = h.w_scales_e4m3[(size_t)n * (K / 16) + gi];
+      chk(upload(&L->d_ws, ws.data(), ws.size()));
+    } else {
+      // weight scales times 2^-ew as FP16, group-major [K/64][npad] (zero padding)
+      int4_range_exponents(h, &L->i4_ex, &L->i4_ew);
+      alpha_exp = L->i4_ex + L->i4_ew;
+      const int npad = pad_cols_int4(N), G = K / 64;
+      std::vector<uint16_t> ws((size_t)G * npad, 0);
+      for (int n = 0; n < N; ++n)
+        for (int gi = 0; gi < G; ++gi) {
+          const double v = std::ldexp((double)bf16_to_float(h.w_scales_bf16[(size_t)n * G + gi]), -L->i4_ew);
+          ws[(size_t)gi * npad + n] = f16_from_double(v);
+        }
+      chk(upload(&L->d_ws, ws.data(), ws.size() * 2));
+    }
     // low-rank branch: L1d^T for the first kernel, (L2b / alpha)^T and L2b^T for the second
     std::vector<uint16_t> l1t((size_t)32 * K, 0), l2s((size_t)N * 32, 0), l2t((size_t)N * 32, 0);
-    const double inv_alpha = std::ldexp(1.0, -(h.g_x_exp + h.g_w_exp));
+    const double inv_alpha = std::ldexp(1.0, -alpha_exp);
     for (int i = 0; i < r; ++i) {
       for (int k = 0; k < K; ++k) l1t[(size_t)i * K + k] = h.L1d[(size_t)k * r + i];
       for (int n = 0; n < N; ++n) {
@@ -174,8 +208,9 @@ svdq_status upload_layer(svdq_layer* L, int device) {
     chk(upload(&L->d_l2s, l2s.data(), l2s.size() * 2));
     chk(upload(&L->d_l2t, l2t.data(), l2t.size() * 2));
     if (e != cudaSuccess) return SVDQ_ECUDA;
-    bool ok = make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, k2_box_bytes(), 256,
-                       k2_swizzle()) &&
+    const bool nv = h.format == SVDQ_NVFP4;
+    bool ok = make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, nv ? k2_box_bytes() : 32,
+                       256, nv ? k2_swizzle() : CU_TENSOR_MAP_SWIZZLE_NONE) &&
               make_map(&L->tm_l2s, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
                        CU_TENSOR_MAP_SWIZZLE_64B) &&
               make_map(&L->tm_l1t, L->d_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, 32, 64, 32,
@@ -201,6 +236,7 @@ K1Params k1_params(const svdq_layer* L, int M, void* codes, void* scales, void* 
   K1Params p;
   p.M = M;
   p.K = h.K;
+  p.mpad = pad_rows(M);
   p.c_x = (float)std::ldexp((double)(1.0f / 6.0f), -h.g_x_exp);
   p.g_x_exp = h.g_x_exp;
   for (int m = 0; m < 8; ++m) {
@@ -222,17 +258,56 @@ svdq_status run_k1(const svdq_layer* L, const void* X, int M, void* codes, void*
   CUtensorMap tm_x, tm_c;
   if (!make_map(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.K, M, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ECUDA;
-  // activation codes are written in 32-row x 16-byte tiles (one per quantizer warp and stage)
-  if (mode != 2 &&
-      !make_map(&tm_c, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+  // activation codes are written in 32-row tiles, one per quantizer warp and stage:
+  // 16 bytes wide for NVFP4 (32 columns), 32 bytes for INT4 (64 columns)
+  const bool nv = h.format == SVDQ_NVFP4;
+  if (mode != 2 && !make_map(&tm_c, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, nv ? 16 : 32, 32,
+                             CU_TENSOR_MAP_SWIZZLE_NONE))
     return SVDQ_ECUDA;
   if (mode == 2) tm_c = tm_x;   // unused by the down-projection-only kernel
   K1Params p = k1_params(L, M, codes, scales, xl);
-  return launch_k1(tm_x, L->tm_l1t, tm_c, p, mode, stream) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+  return launch_k1(tm_x, L->tm_l1t, tm_c, p, nv ? kFmtNvfp4 : kFmtInt4, mode, stream) == cudaSuccess ? SVDQ_OK
+                                                                                                    : SVDQ_ECUDA;
+}
+
+svdq_status run_k2_int4(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M,
+                        void* Y, cudaStream_t stream, bool branch, bool gelu) {
+  const HostPrep& h = L->host;
+  CUtensorMap tm_a, tm_xl, tm_y;
+  if (!make_map(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SVDQ_ECUDA;
+  if (!make_map(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return SVDQ_ECUDA;
+  if (branch) {
+    if (!make_map(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return SVDQ_ECUDA;
+  } else {
+    tm_xl = tm_a;   // unused by the kernel
+  }
+  K2Int4Params p;
+  p.M = M;
+  p.N = h.N;
+  p.K = h.K;
+  p.mpad = pad_rows(M);
+  p.npad = pad_cols_int4(h.N);
+  p.alpha = (float)std::ldexp(1.0, L->i4_ex + L->i4_ew);
+  p.xscale = (float)std::ldexp(1.0, -L->i4_ex);
+  p.sa = static_cast<const uint16_t*>(scales);
+  p.sb = reinterpret_cast<const uint16_t*>(L->d_ws);
+  p.bias = L->d_bias;
+  p.y = static_cast<__nv_bfloat16*>(Y);
+  p.err = L->d_err;
+  p.budget_ns = L->budget_ns;
+  p.branch = branch ? 1 : 0;
+  p.gelu = gelu ? 1 : 0;
+  return launch_k2_int4(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream) == cudaSuccess
+             ? SVDQ_OK
+             : SVDQ_ECUDA;
 }
 
 svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
                    cudaStream_t stream, bool branch, bool gelu) {
+  if (L->host.format == SVDQ_INT4) return run_k2_int4(L, codes, scales, xl, M, Y, stream, branch, gelu);
   const HostPrep& h = L->host;
   CUtensorMap tm_a, tm_xl, tm_y;
   if (!make_map(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, k2_box_bytes(), 128, k2_swizzle()))
@@ -391,6 +466,14 @@ size_t svdq_act_scale_bytes(const svdq_layer* L, int M) {
 svdq_status svdq_act_scales_to_logical(const svdq_layer* L, const void* device_layout, int M, void* logical) {
   if (!L || !device_layout || !logical || M < 1) return SVDQ_EINVAL;
   const HostPrep& h = L->host;
+  if (h.format == SVDQ_INT4) {
+    const uint16_t* src = static_cast<const uint16_t*>(device_layout);
+    uint16_t* dst = static_cast<uint16_t*>(logical);
+    const int G = h.K / 64, mpad = pad_rows(M);
+    for (int r = 0; r < M; ++r)
+      for (int gi = 0; gi < G; ++gi) dst[(size_t)r * G + gi] = src[(size_t)gi * mpad + r];
+    return SVDQ_OK;
+  }
   if (h.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
   const uint8_t* src = static_cast<const uint8_t*>(device_layout);
   uint8_t* dst = static_cast<uint8_t*>(logical);
@@ -404,7 +487,7 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int M, void* c
                               void* stream, int mode) {
   svdq_status st = check_forward_args(L, X, M, codes);
   if (st != SVDQ_OK) return st;
-  if (L->host.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
+  if (!w4a4(L)) return SVDQ_EUNSUPPORTED;
   if (mode < 0 || mode > 2) return SVDQ_EINVAL;
   if (!scales && mode != 2) return SVDQ_EINVAL;
   if (L->host.rank == 0 && mode == 2) return SVDQ_EINVAL;
@@ -419,7 +502,7 @@ svdq_status svdq_gemm(const svdq_layer* L, const void* codes, const void* scales
                       void* stream, unsigned flags) {
   svdq_status st = check_forward_args(L, codes, M, Y);
   if (st != SVDQ_OK) return st;
-  if (L->host.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
+  if (!w4a4(L)) return SVDQ_EUNSUPPORTED;
   if (!scales) return SVDQ_EINVAL;
   const bool branch = L->host.rank > 0 && !(flags & SVDQ_FWD_NO_BRANCH);
   if (branch && !xl) return SVDQ_EINVAL;
@@ -454,7 +537,7 @@ svdq_status svdq_linear_forward(const svdq_layer* L, const void* X, int M, void*
     if (st == SVDQ_OK && (flags & SVDQ_FWD_CHECK)) st = svdq_check(L, stream);
     return st;
   }
-  if (L->host.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
+  if (!w4a4(L)) return SVDQ_EUNSUPPORTED;
   const WsLayout w = ws_layout(L->host, M);
   if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return SVDQ_EINVAL;

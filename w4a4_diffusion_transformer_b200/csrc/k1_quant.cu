@@ -28,7 +28,12 @@
 //     memory once; the eight partial sums are added through shared memory at
 //     the end.
 //
-// Quantizer arithmetic per group of 16 (bit-exact with the CPU oracle): a =
+// The INT4 variant (groups of 64, BF16 scales, codes in [-7, 7]; SOTA-314
+// "Do this") runs 4 quantizer warps of 64 columns each and writes its scales
+// group-major, [K/64][M padded to 128] BF16, the order the INT4 GEMM stages
+// them in.
+//
+// NVFP4 quantizer arithmetic per group of 16 (bit-exact with the CPU oracle): a =
 // max|v|; t = fp32(a * c_x) with c_x = fp32(1/6) 2^-gx; s = E4M3_rn_satfinite(t);
 // s == 0 -> all codes +0; inv = fp32(1 / (s * g_x)); code =
 // E2M1_rn_satfinite(fp32(v * inv)).  The reciprocal is exact without a
@@ -49,16 +54,23 @@ constexpr int kRows = 32;
 constexpr int kBK = 256;
 constexpr int kXStages = 8;                  // X + inv_lam ring (HBM stream)
 constexpr int kLStages = 3;                  // L1d^T ring (L2-resident)
-constexpr int kQuantWarps = 8;
 constexpr int kMmaWarps = 8;
-constexpr int kConsumerWarps = kQuantWarps + kMmaWarps;
-constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kXBytes = kRows * kBK * 2;     // 4 sub-tiles of 32 rows x 128 B
 constexpr int kLBytes = 32 * kBK * 2;        // 4 sub-tiles of 32 rows x 128 B
 constexpr int kIBytes = kBK * 4;
 constexpr int kXStageBytes = kXBytes + kIBytes;            // 17 KiB, 1 KiB multiple
-constexpr int kCodeTile = kRows * 16;                     // one quantizer warp's codes: 32 rows x 16 B
-constexpr int kCodeBytes = kQuantWarps * 2 * kCodeTile;     // double-buffered per warp
+constexpr int kCodeBytes = 8 * 1024;                       // code staging tiles, double-buffered per warp
+// Quantizer warps per format: NVFP4 warps own 32 columns of a stage (two
+// groups of 16), INT4 warps own 64 columns (one group of 64).
+template <int F>
+struct K1Shape {
+  static constexpr int quant_warps = F == kFmtNvfp4 ? 8 : 4;
+  static constexpr int cols = kBK / quant_warps;                     // columns per quantizer warp
+  static constexpr int code_tile = kRows * cols / 2;                 // its codes: 32 rows x cols/2 B
+  static constexpr int consumer_warps = quant_warps + kMmaWarps;
+  static constexpr int threads = (consumer_warps + 2) * 32;
+  static_assert(quant_warps * 2 * code_tile == kCodeBytes, "code staging size");
+};
 constexpr int kPartBytes = kMmaWarps * 32 * 32 * 4;         // down-projection partial sums
 static_assert(kPartBytes <= kLStages * kLBytes, "partial sums reuse the L1d^T ring");
 constexpr int kSmemBytes = kXStages * kXStageBytes + kLStages * kLBytes + kCodeBytes + 1024 + 256 + 16 * 4;
@@ -87,8 +99,8 @@ __device__ __forceinline__ void record_error(int* err, volatile int* abort_flag,
 
 __device__ __forceinline__ void mma_warps_sync() { dev::named_barrier(1, kMmaWarps * 32); }
 
-template <bool kQuant, bool kDown>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kFmt, bool kQuant, bool kDown>
+__global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
     k1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l,
               const __grid_constant__ CUtensorMap tm_c, K1Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -102,6 +114,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* lempty = lfull + kLStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(lempty + kLStages);
   float* rcp = reinterpret_cast<float*>(cbuf + kCodeBytes + 256);   // reciprocal table
+  constexpr int kQuantWarps = K1Shape<kFmt>::quant_warps;
+  constexpr int kConsumerWarps = K1Shape<kFmt>::consumer_warps;
+  constexpr int kCodeTile = K1Shape<kFmt>::code_tile;
   constexpr int kActiveWarps = (kQuant ? kQuantWarps : 0) + (kDown ? kMmaWarps : 0);
 
   const int warp = threadIdx.x >> 5;
@@ -183,8 +198,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool quant_warp = warp < kQuantWarps;
   if ((quant_warp && !kQuant) || (!quant_warp && !kDown)) return;   // role not used by this variant
 
+  if (quant_warp && kFmt == kFmtInt4) {
+    // ---------------------------------------------------------- INT4 quantizer
+    // Warp w owns sub-tile w of each stage (columns 64w..64w+63: one group of
+    // 64) and lane l owns row l.  Per group: a = max|v|; s = bf16(fp32(a *
+    // fp32(1/7))); s == 0 -> all codes 0; inv = fp32(1/s) (correctly rounded
+    // reciprocal); code = rint_even(fp32(v * inv)).  |v * inv| <= 7 (1 + 2^-8)
+    // because s is a > 0 divided by 7 and rounded to 8 significant bits, so the
+    // clamp to [-7, 7] never changes a code.  Rounding adds 1.5 * 2^23: the
+    // sum's low mantissa bits are then the rounded integer in two's
+    // complement, so its low nibble is the 4-bit code.
+    const int grow = row0 + lane;                     // < mpad: the grid covers the padded rows
+    uint16_t* srow = reinterpret_cast<uint16_t*>(p.scales) + grow;   // scales [K/64][mpad]
+    uint8_t* ctile = cbuf + warp * 2 * kCodeTile;
+    if (lane == 0) dev::tma_prefetch_desc(&tm_c);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % kXStages;
+      if (!dev::mbar_wait(&xfull[s], (uint32_t)(it / kXStages) & 1u, abort_flag, p.budget_ns)) {
+        record_error(p.err, abort_flag, 0x102);
+        break;
+      }
+      const uint8_t* st = smem + s * kXStageBytes;
+      const int k0 = it * kBK;
+      const bool active = warp * 64 < min(kBK, K - k0);
+      uint32_t packed[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      uint32_t sbits = 0u;
+      if (active) {
+        const uint8_t* xt = st + warp * 4096;
+        const float4* inv4 = reinterpret_cast<const float4*>(st + kXBytes) + warp * 16;
+        float2 v[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(xt + sw128(lane, i));
+          const float4 ia = inv4[2 * i], ib = inv4[2 * i + 1];
+          const float2 iv[4] = {make_float2(ia.x, ia.y), make_float2(ia.z, ia.w), make_float2(ib.x, ib.y),
+                                make_float2(ib.z, ib.w)};
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            v[i * 4 + e] = __fmul2_rn(make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)),
+                                      iv[e]);
+        }
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a = dev::fmax3(a, fabsf(v[i].x), fabsf(v[i].y));
+        const __nv_bfloat16 sb = __float2bfloat16_rn(__fmul_rn(a, 1.0f / 7.0f));
+        sbits = __bfloat16_as_ushort(sb);
+        const float sc = __bfloat162float(sb);
+        if (sc != 0.f) {
+          const float inv = __frcp_rn(sc);
+          const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            // codes 8j..8j+7: even ones form byte-lanes A, odd ones B; byte i of
+            // the word holds code 8j+2i in its low nibble and 8j+2i+1 in its high
+            uint32_t t[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              // q = fp32(v * inv) must be rounded before the integer rounding:
+              // the scalar __fadd_rn is never contracted with the multiply into
+              // a fused multiply-add (a packed add can be, which rounds the
+              // exact product and moves ties such as 2.5000000326 -> 3)
+              const float2 q = __fmul2_rn(v[4 * j + e], inv2);
+              t[2 * e] = __float_as_uint(__fadd_rn(q.x, 12582912.0f));
+              t[2 * e + 1] = __float_as_uint(__fadd_rn(q.y, 12582912.0f));
+            }
+            const uint32_t A = __byte_perm(__byte_perm(t[0], t[2], 0x0040), __byte_perm(t[4], t[6], 0x0040), 0x5410);
+            const uint32_t B = __byte_perm(__byte_perm(t[1], t[3], 0x0040), __byte_perm(t[5], t[7], 0x0040), 0x5410);
+            packed[j] = (A & 0x0F0F0F0Fu) | ((B << 4) & 0xF0F0F0F0u);
+          }
+        }
+      }
+      // the stage's inputs have been read
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&xempty[s]);
+      if (active) {
+        srow[(size_t)((k0 >> 6) + warp) * (size_t)p.mpad] = (uint16_t)sbits;
+        // codes: this warp's 32 x 32-byte tile, stored with TMA once the store
+        // that last read this buffer (two stages ago) is done reading
+        uint8_t* ct = ctile + (it & 1) * kCodeTile;
+        if (lane == 0) dev::bulk_wait_group_read<1>();
+        __syncwarp();
+        *reinterpret_cast<uint4*>(ct + lane * 32) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        *reinterpret_cast<uint4*>(ct + lane * 32 + 16) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        dev::fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          dev::tma_store_2d(&tm_c, ct, (k0 + warp * 64) >> 1, row0);
+          dev::bulk_commit_group();
+        }
+      }
+    }
+    if (lane == 0) dev::bulk_wait_group_all();
+    return;
+  }
   if (quant_warp) {
-    // ---------------------------------------------------------- quantizer
+    // ---------------------------------------------------------- NVFP4 quantizer
     const int grow = row0 + lane;                     // this lane's row (may be >= M: zero padding)
     const int col0 = warp * 32;                       // 2 groups of 16 columns of each stage
     uint16_t* scale_pair = reinterpret_cast<uint16_t*>(p.scales + sf_offset(grow, 2 * warp, K));
@@ -347,10 +456,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool Q, bool D>
+template <int F, bool Q, bool D>
 cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CUtensorMap& tm_c,
                         const K1Params& p, cudaStream_t stream) {
-  auto kern = k1_kernel<Q, D>;
+  auto kern = k1_kernel<F, Q, D>;
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -361,7 +470,7 @@ cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const 
   }
   const int mpad = (p.M + 127) / 128 * 128;
   dim3 grid(mpad / kRows);
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(tm_x, tm_l, tm_c, p);
+  kern<<<grid, K1Shape<F>::threads, kSmemBytes, stream>>>(tm_x, tm_l, tm_c, p);
   return cudaGetLastError();
 }
 
@@ -370,13 +479,16 @@ cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const 
 int k1_rows_per_cta() { return kRows; }
 
 cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CUtensorMap& tm_c,
-                      const K1Params& p, int mode, cudaStream_t stream) {
-  switch (mode) {
-    case 0: return launch_k1_t<true, true>(tm_x, tm_l, tm_c, p, stream);
-    case 1: return launch_k1_t<true, false>(tm_x, tm_l, tm_c, p, stream);
-    case 2: return launch_k1_t<false, true>(tm_x, tm_l, tm_c, p, stream);
-    default: return cudaErrorInvalidValue;
+                      const K1Params& p, int fmt, int mode, cudaStream_t stream) {
+  if (mode == 2) return launch_k1_t<kFmtNvfp4, false, true>(tm_x, tm_l, tm_c, p, stream);   // no quantizer
+  if (fmt == kFmtNvfp4) {
+    if (mode == 0) return launch_k1_t<kFmtNvfp4, true, true>(tm_x, tm_l, tm_c, p, stream);
+    if (mode == 1) return launch_k1_t<kFmtNvfp4, true, false>(tm_x, tm_l, tm_c, p, stream);
+  } else if (fmt == kFmtInt4) {
+    if (mode == 0) return launch_k1_t<kFmtInt4, true, true>(tm_x, tm_l, tm_c, p, stream);
+    if (mode == 1) return launch_k1_t<kFmtInt4, true, false>(tm_x, tm_l, tm_c, p, stream);
   }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace svdq

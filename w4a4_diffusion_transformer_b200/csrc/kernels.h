@@ -10,14 +10,19 @@
 
 namespace svdq {
 
+// Activation/weight formats of the W4A4 kernels.
+constexpr int kFmtNvfp4 = 0;
+constexpr int kFmtInt4 = 1;
+
 struct K1Params {
   int M, K;
+  int mpad;                     // M rounded up to 128 (rows of the INT4 scale array)
   float c_x;                    // fp32(1/6) * 2^-g_x_exp
   int g_x_exp;                  // activation tensor scale g_x = 2^g_x_exp
   float rcp[16];                // fp32(1/(1 + m/8)) for m = 0..7, then fp32(1/m) (index 8 + m)
   const float* inv_lam;         // [K]
   uint8_t* codes;               // [M][K/2]
-  uint8_t* scales;              // tensor-core scale layout, ceil(M/128)*128 rows
+  uint8_t* scales;              // NVFP4: tensor-core scale layout, mpad rows; INT4: BF16 [K/64][mpad]
   __nv_bfloat16* xl;            // [M][32]
   int* err;                     // device error word
   unsigned long long budget_ns; // bound on each wait
@@ -28,6 +33,21 @@ struct K2Params {
   float alpha;                  // g_x * g_w (power of two)
   const uint8_t* sfa;           // activation scales, tensor-core layout
   const uint8_t* sfb;           // weight scales, tensor-core layout (rows padded to 256)
+  const float* bias;            // [N]
+  __nv_bfloat16* y;             // [M][N]
+  int* err;
+  unsigned long long budget_ns;
+  int branch;                   // 1: add XL (L2b / alpha) into the accumulator
+  int gelu;                     // 1: tanh-GELU epilogue
+};
+
+struct K2Int4Params {
+  int M, N, K;
+  int mpad, npad;               // rows of the activation / weight scale arrays (multiples of 128 / 256)
+  float alpha;                  // 2^(ex + ew): undoes the FP16 range exponents
+  float xscale;                 // 2^-ex, applied to the BF16 activation scales
+  const uint16_t* sa;           // activation scales, BF16 [K/64][mpad]
+  const uint16_t* sb;           // weight scales times 2^-ew, FP16 [K/64][npad]
   const float* bias;            // [N]
   __nv_bfloat16* y;             // [M][N]
   int* err;
@@ -62,9 +82,9 @@ bool w4a16_supported(int K);   // shared-memory bound on K
 void w4a16_pack(const uint8_t* codes, const uint16_t* scales, int N, int K, uint8_t* out);
 cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t stream);
 
-// mode 0 = fused, 1 = quantize only, 2 = down projection only
+// fmt = kFmtNvfp4 or kFmtInt4; mode 0 = fused, 1 = quantize only, 2 = down projection only
 cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CUtensorMap& tm_c,
-                      const K1Params& p, int mode, cudaStream_t stream);
+                      const K1Params& p, int fmt, int mode, cudaStream_t stream);
 int k1_rows_per_cta();
 
 cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
@@ -72,6 +92,12 @@ cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CU
                       cudaStream_t stream);
 int k2_block_n();
 int k2_stage_k_bytes();   // E2M1 bytes per operand row per pipeline stage (128 or 64)
+
+// INT4 GEMM: A = activation codes [M][K/2] (box 32 B x 128 rows), B = weight
+// codes [N][K/2] (box 32 B x 256 rows), both unswizzled.
+cudaError_t launch_k2_int4(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
+                           const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Int4Params& p, int num_sms,
+                           cudaStream_t stream);
 
 cudaError_t launch_upproj(const UpParams& p, cudaStream_t stream);
 

@@ -476,6 +476,15 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
       }
     }
 
+    // ---- largest smoothed calibration activation, amax |fp32(Xc / lam)|
+    P.x_amax = 0.0f;
+    if (!w4a16)
+      for (int m = 0; m < M_calib; ++m)
+        for (int k = 0; k < K; ++k) {
+          volatile float v = bf16_to_float(calib[(size_t)m * K + k]) * P.inv_lam[k];
+          P.x_amax = std::max(P.x_amax, std::fabs((float)v));
+        }
+
     // ---- residual quantization, groups along K for each output column n
     P.w_codes.assign((size_t)N * K / 2, 0);
     if (cfg.format == SVDQ_NVFP4) {
@@ -497,13 +506,7 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
         }
       }
       // activation tensor scale from the calibration batch, 4x headroom
-      float xa = 0.0f;
-      for (int m = 0; m < M_calib; ++m)
-        for (int k = 0; k < K; ++k) {
-          volatile float v = bf16_to_float(calib[(size_t)m * K + k]) * P.inv_lam[k];
-          xa = std::max(xa, std::fabs((float)v));
-        }
-      P.g_x_exp = pow2_ceil_exponent(4.0 * (double)xa / 2688.0);
+      P.g_x_exp = pow2_ceil_exponent(4.0 * (double)P.x_amax / 2688.0);
     } else {
       P.w_scales_bf16.assign((size_t)N * K / 64, 0);
 #pragma omp parallel for schedule(static)
