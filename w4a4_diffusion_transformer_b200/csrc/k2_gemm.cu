@@ -18,8 +18,12 @@
 //              B tile (128-byte swizzle), and the E4M3 scale factors (bulk
 //              copies, already in the tensor-core layout); per tile one extra
 //              stage with the XL tile and the L2b^T tile (64-byte swizzle).
-//   warp 1     allocates TMEM (512 columns: accumulator 256 + per-stage scale factors) and
-//              issues tcgen05.cp (scales smem -> TMEM) and tcgen05.mma.
+//   warp 1     allocates TMEM (512 columns: accumulator 256 + per-stage scale
+//              factors) and issues tcgen05.mma.
+//   warp 10    copies each stage's scale factors into TMEM (tcgen05.cp) as soon
+//              as they land: they complete their own barrier and are loaded
+//              before the operand tiles, so the copies run while the tiles are
+//              still in flight instead of between a stage's arrival and its MMAs.
 //   warps 2-9  epilogue, two warps per TMEM lane quarter (32 rows), each owning
 //              128 of the 256 columns: tcgen05.ld in 32-column chunks (the next
 //              chunk's load overlaps the current chunk's math), alpha, bias
@@ -50,30 +54,21 @@ constexpr int kBN = 256;
 #ifndef SVDQ_K2_STAGES
 #define SVDQ_K2_STAGES 3
 #endif
-#ifndef SVDQ_K2_LOOKAHEAD
-#define SVDQ_K2_LOOKAHEAD 0
-#endif
-// Scale-factor copies issued by a dedicated warp (1) or by the MMA warp (0).
-#ifndef SVDQ_K2_CP_WARP
-#define SVDQ_K2_CP_WARP 1
-#endif
 // Epilogue drains its 128 accumulator columns into registers before any math (1),
 // or loads them chunk by chunk, overlapping each load with the previous chunk's math (0).
 #ifndef SVDQ_K2_FAST_DRAIN
 #define SVDQ_K2_FAST_DRAIN 1
 #endif
-constexpr bool kCpWarp = SVDQ_K2_CP_WARP != 0;
 constexpr bool kFastDrain = SVDQ_K2_FAST_DRAIN != 0;
 constexpr int kKB = SVDQ_K2_KB;
 constexpr int kBKBytes = kKB * 32;          // E2M1 bytes per operand row per stage
 constexpr int kStages = SVDQ_K2_STAGES;
-constexpr bool kLookahead = SVDQ_K2_LOOKAHEAD != 0;
 constexpr uint32_t kSwz = kKB == 4 ? 2u : 4u;          // descriptor layout: 128B or 64B swizzle
 constexpr uint32_t kSwzAtom = 8u * kBKBytes;           // bytes between 8-row groups
 static_assert(kKB == 2 || kKB == 4, "stage shape");
 constexpr int kEpiWarps = 8;
 constexpr int kCpWarpIdx = 2 + kEpiWarps;
-constexpr int kThreads = (2 + kEpiWarps + (kCpWarp ? 1 : 0)) * 32;
+constexpr int kThreads = (3 + kEpiWarps) * 32;
 constexpr int kEpiBufBytes = 32 * 64;        // one 32 x 32 BF16 output chunk
 constexpr int kEpiWarpBytes = 2 * kEpiBufBytes + 512;   // two chunk buffers + 128 bias floats
 constexpr int kABytes = kBM * kBKBytes;      // 16 KiB
@@ -116,7 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 1;
   uint64_t* sf_ready = drain + 1;                  // [kStages], scale factors of a stage in TMEM
   uint64_t* cp_drain = sf_ready + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drain + 1);
+  uint64_t* sf_full = cp_drain + 1;                // [kStages], a stage's scale factors in shared memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -132,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       dev::mbar_init(&full[s], 1);
       dev::mbar_init(&empty[s], 1);
+      dev::mbar_init(&sf_full[s], 1);
     }
     dev::mbar_init(acc_full, 1);
     dev::mbar_init(acc_empty, kEpiWarps);
@@ -174,6 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = smem + s * kStageBytes;
+          dev::mbar_arrive(&sf_full[s]);               // a branch stage carries no scale factors
           dev::mbar_arrive_expect_tx(&full[s], kBM * 64 + kBN * 64);
           dev::tma_load_2d(st + kABytes, &tm_l2, &full[s], 0, n0);
           if (!deps_ready) {
@@ -193,36 +191,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = smem + s * kStageBytes;
           const int nkb = min(kKB, kblocks - kKB * kt);
           const uint32_t sf_bytes = (uint32_t)nkb * 512u;
-          dev::mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + 3u * sf_bytes);
+          // The scale factors complete their own barrier and are issued first:
+          // the copy warp moves them into TMEM while the operand tiles are
+          // still in flight, so those copies are off the stage's critical path.
+          dev::mbar_arrive_expect_tx(&sf_full[s], 3u * sf_bytes);
+          dev::mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
           // weights first: they do not depend on the preceding kernel
-          dev::tma_load_2d(st + kABytes, &tm_b, &full[s], kt * kBKBytes, n0);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const size_t b_chunk = (size_t)((n0 >> 7) + h) * (size_t)kblocks + (size_t)(kKB * kt);
             dev::bulk_load(st + kABytes + kBBytes + kSFABytes + h * (kKB * 512), p.sfb + b_chunk * 512, sf_bytes,
-                           &full[s]);
+                           &sf_full[s]);
           }
+          dev::tma_load_2d(st + kABytes, &tm_b, &full[s], kt * kBKBytes, n0);
           if (!deps_ready) {
             dev::griddep_wait();
             deps_ready = true;
           }
-          dev::tma_load_2d(st, &tm_a, &full[s], kt * kBKBytes, m0);
           const size_t a_chunk = (size_t)(m0 >> 7) * (size_t)kblocks + (size_t)(kKB * kt);
-          dev::bulk_load(st + kABytes + kBBytes, p.sfa + a_chunk * 512, sf_bytes, &full[s]);
+          dev::bulk_load(st + kABytes + kBBytes, p.sfa + a_chunk * 512, sf_bytes, &sf_full[s]);
+          dev::tma_load_2d(st, &tm_a, &full[s], kt * kBKBytes, m0);
           ++it;
         }
       }
       for (int j = max(0, it - kStages); j < it; ++j)
-        if (!dev::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns)) break;
+        if (!dev::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns) ||
+            !dev::mbar_wait(&sf_full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns))
+          break;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_f4 = dev::idesc_nvfp4(kBM, kBN);
       const uint32_t idesc_h = dev::idesc_bf16(kBM, kBN);
-      // Scale factors of k-tile kt+1 are copied into TMEM (their own per-stage
-      // region) before the MMAs of k-tile kt are issued, so the copies do not
-      // sit between a k-tile's data arriving and its MMAs.
       auto wait_full = [&](int slot, int code) -> bool {
         if (!dev::mbar_wait(&full[slot % kStages], (uint32_t)(slot / kStages) & 1u, abort_flag, p.budget_ns)) {
           record_error(p.err, abort_flag, code);
@@ -231,20 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::tc_fence_after();
         return true;
       };
-      auto copy_scales = [&](int slot, int kt) {
-        const int s = slot % kStages;
-        const int nkb = min(kKB, kblocks - kKB * kt);
-        const uint32_t sfa0 = dev::smem_u32(smem + s * kStageBytes) + kABytes + kBBytes;
-        const uint32_t sfb0 = sfa0 + kSFABytes;
-        const uint32_t tsfa = tmem + kSFCol0 + s * kSFStageCols;
-        const uint32_t tsfb = tsfa + 4 * kKB;
-        for (int j = 0; j < nkb; ++j) {
-          dev::tmem_copy_32x128b_x4(tsfa + 4 * j, dev::smem_desc(sfa0 + 512 * j, 0, 128, 0));
-          dev::tmem_copy_32x128b_x4(tsfb + 8 * j, dev::smem_desc(sfb0 + 512 * j, 0, 128, 0));
-          dev::tmem_copy_32x128b_x4(tsfb + 8 * j + 4, dev::smem_desc(sfb0 + kKB * 512 + 512 * j, 0, 128, 0));
-        }
-      };
-      uint32_t sf_phase = 0;                          // per-stage parity of sf_ready (kCpWarp)
+      uint32_t sf_phase = 0;                          // per-stage parity of sf_ready
       auto wait_sf = [&](int slot) -> bool {
         const int st = slot % kStages;
         if (!dev::mbar_wait(&sf_ready[st], (sf_phase >> st) & 1u, abort_flag, p.budget_ns)) {
@@ -259,11 +247,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
         const int kslot0 = it + (p.branch ? 1 : 0);
-        // the first k-tile's scales do not touch the accumulator: copy them first
-        if (!kCpWarp) {
-          if (!(ok = wait_full(kslot0, 0x205))) break;
-          copy_scales(kslot0, 0);
-        }
         if (!dev::mbar_wait(acc_empty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag, p.budget_ns)) {
           record_error(p.err, abort_flag, 0x203);
           ok = false;
@@ -288,18 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < ktiles; ++kt) {
           const int slot = kslot0 + kt;
           const int s = slot % kStages;
-          if (kCpWarp) {
-            if (!(ok = wait_full(slot, 0x205))) break;
-            if (!(ok = wait_sf(slot))) break;
-          } else if (kLookahead) {
-            if (kt + 1 < ktiles) {
-              if (!(ok = wait_full(slot + 1, 0x205))) break;
-              copy_scales(slot + 1, kt + 1);
-            }
-          } else if (kt > 0) {
-            if (!(ok = wait_full(slot, 0x205))) break;
-            copy_scales(slot, kt);
-          }
+          if (!(ok = wait_full(slot, 0x205))) break;
+          if (!(ok = wait_sf(slot))) break;
           const int nkb = min(kKB, kblocks - kKB * kt);
           const uint32_t a0 = dev::smem_u32(smem + s * kStageBytes);
           const uint32_t b0 = a0 + kABytes;
@@ -321,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tc_commit(drain);
       dev::mbar_wait(drain, 0, abort_flag, p.budget_ns);
     }
-  } else if (kCpWarp && warp == kCpWarpIdx) {
+  } else if (warp == kCpWarpIdx) {
     // ------------------------------------------------------------ scale-factor copier
     if (lane == 0) {
       int it = 0;
@@ -330,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.branch) ++it;
         for (int kt = 0; kt < ktiles; ++kt, ++it) {
           const int st = it % kStages;
-          if (!dev::mbar_wait(&full[st], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
+          if (!dev::mbar_wait(&sf_full[st], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
             record_error(p.err, abort_flag, 0x208);
             ok = false;
             break;
