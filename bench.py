@@ -6,9 +6,14 @@ up-projection + bias epilogue (K2), on the FLUX.1-shaped attention output
 projection (M = 4608 tokens, K = N = 3072, rank 32, NVFP4 g16/E4M3), inputs
 resident in HBM, L2 flushed between steps outside the timed events (a 256 MiB
 write, then a read of the same buffer so that no dirty lines of the flush are
-left for the timed kernels to write back).  The value is whole-job TFLOP/s of the layer's algorithmic work
-2MNK + 2M*32*(K+N), device-timed with CUDA events on the launch stream, max
-over ranks.
+left for the timed kernels to write back).  The value is whole-job TFLOP/s of
+the layer's algorithmic work 2MNK + 2M*32*(K+N), device-timed with one pair of
+CUDA events around each step on the launch stream (K1 and K2 back to back, as a
+caller runs them), max over ranks.  The per-kernel durations behind the
+roofline fractions are timed after the steps, each kernel alone between its own
+events.  The JSON line also carries the other rows of the hot path on their
+FLUX.1-shaped layers (INT4 QKV, the fc1 -> GELU -> fc2 pair, the W4A16
+adaptive-norm GEMV) under "other_layers".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -225,6 +230,93 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def time_events(stream, n, flush_l2, fn):
+    """Mean device time (ms) of fn() over n calls, each bracketed by CUDA events
+    on `stream` after an L2 flush."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        flush_l2(i)
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / n
+
+
+def other_layers(pkg, syn, stream, flush_l2, n, peaks):
+    """The other hot-path rows on their FLUX.1-shaped layers (not the headline):
+    the INT4 variant (fused QKV 4608x3072->9216), the MLP pair (fc1 with the GELU
+    epilogue, fc2 on fc1's output) and the W4A16 adaptive-norm GEMV (4x3072->18432)."""
+    import torch
+    out = {}
+    bf16_peak = peaks["bf16_tflops"]
+
+    def w4a4_layer(d, fmt, X, flags, key, calib=None):
+        M, K, N = X.shape[0], d["W"].shape[0], d["W"].shape[1]
+        L = pkg.Layer.prepare(syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]),
+                              syn.bf16_bits(d["Xc"] if calib is None else calib), fmt=fmt, rank=RANK,
+                              device=torch.cuda.current_device())
+        x = X if isinstance(X, torch.Tensor) else torch.from_numpy(X).to(torch.bfloat16).cuda()
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty(L.act_scale_bytes(M), dtype=torch.uint8, device="cuda")
+        xl = torch.empty((M, RANK), dtype=torch.bfloat16, device="cuda")
+
+        def layer():
+            L.quantize_act(x, M, codes, scales, xl, stream, 0)
+            L.gemm(codes, scales, xl, M, y, stream, flags)
+
+        layer()
+        L.check(stream)
+        lay = time_events(stream, n, flush_l2, layer)
+        k2 = time_events(stream, n, flush_l2, lambda: L.gemm(codes, scales, xl, M, y, stream, flags))
+        L.check(stream)
+        k2t = k2_flops(M, K, N) / (k2 * 1e-3) / 1e12
+        peak = bf16_peak * (FP4_OVER_BF16 if fmt == "nvfp4" else 1.0)
+        out[key] = {"shape": f"{M}x{K}->{N}", "format": fmt, "us_per_layer": lay * 1e3, "k2_us": k2 * 1e3,
+                    "layer_tflops": layer_flops(M, K, N) / (lay * 1e-3) / 1e12, "k2_tflops": k2t,
+                    "k2_frac": k2t / peak,
+                    "k2_peak": f"{peak:g} TFLOP/s = measured bf16 burst" +
+                               (f" x {FP4_OVER_BF16:g}" if fmt == "nvfp4" else " (FP16 tensor rate, the INT4 "
+                                                                             "GEMM's dequantized operands)")}
+        L.close()
+        return y
+
+    # INT4 variant
+    d = syn.layer("qkv_int4")
+    w4a4_layer(d, "int4", d["X"], 0, "int4_qkv")
+    # MLP pair: fc1 (GELU), then fc2 on fc1's output; fc2 calibrates on fc1's output for its calibration batch
+    d1 = syn.layer("mlp", "fc1")
+    h = w4a4_layer(d1, "nvfp4", d1["X"], pkg.FWD_GELU, "fc1_gelu")
+    L1 = pkg.Layer.prepare(syn.bf16_bits(d1["W"]), syn.bf16_bits(d1["bias"]), syn.bf16_bits(d1["Xc"]),
+                           fmt="nvfp4", rank=RANK, device=torch.cuda.current_device())
+    xc = torch.from_numpy(d1["Xc"]).to(torch.bfloat16).cuda()
+    hc = torch.empty((xc.shape[0], d1["W"].shape[1]), dtype=torch.bfloat16, device="cuda")
+    wsc = torch.empty(L1.workspace_bytes(xc.shape[0]), dtype=torch.uint8, device="cuda")
+    L1.forward(xc, xc.shape[0], hc, wsc, wsc.numel(), stream, pkg.FWD_GELU | pkg.FWD_CHECK)
+    L1.close()
+    d2 = syn.layer("mlp", "fc2")
+    d2["Xc"] = hc.float().cpu().numpy()
+    w4a4_layer(d2, "nvfp4", h, 0, "fc2")
+    # W4A16 adaptive-norm GEMV
+    da = syn.layer("block_b4", "adaln", with_run=False)
+    La = pkg.Layer.prepare(syn.bf16_bits(da["W"]), syn.bf16_bits(da["bias"]), None, fmt="w4a16", rank=0,
+                           device=torch.cuda.current_device())
+    Ma, Ka, Na = 4, da["W"].shape[0], da["W"].shape[1]
+    xa = torch.from_numpy(syn.activations(4, 4, Ma, Ka, syn.ROLE_X_RUN, outliers=False)).to(torch.bfloat16).cuda()
+    ya = torch.empty((Ma, Na), dtype=torch.bfloat16, device="cuda")
+    La.forward(xa, Ma, ya, None, 0, stream, pkg.FWD_CHECK)
+    t = time_events(stream, n, flush_l2, lambda: La.forward(xa, Ma, ya, None, 0, stream, 0))
+    La.check(stream)
+    wbytes = Na * Ka // 2 + Na * (Ka // 64) * 2 + Ma * Ka * 2 + Ma * Na * 2 + Na * 4
+    gbs = wbytes / (t * 1e-3) / 1e9
+    out["w4a16_adaln"] = {"shape": f"{Ma}x{Ka}->{Na}", "format": "w4a16 int4 g64", "us": t * 1e3,
+                          "algorithmic_bytes": wbytes, "GBs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"]}
+    La.close()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -232,13 +324,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-layers", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
 
-    import numpy as np
     import torch
 
     import synthetic as syn
@@ -273,85 +365,69 @@ def main():
         flush.fill_(i & 0xFF)                                     # evict: write > L2
         torch.sum(flush.view(torch.int64), dim=0, keepdim=True, out=flush_sink)   # clean the lines
 
-    def step_fused():
+    def step():
+        # the layer as a caller runs it: K1 then K2 back to back on one stream (K2
+        # is a programmatic dependent launch of K1: its prologue overlaps K1's tail)
         L.quantize_act(x, M, codes, scales, xl, stream, 0)
         L.gemm(codes, scales, xl, M, y, stream, 0)
 
-    def time_variant(fn, n):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        for i in range(n):
-            flush_l2(i)
-            evs[i][0].record(stream)
-            fn()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
-        return sum(a.elapsed_time(b) for a, b in evs) / n
-
     # ---- warm-up
     for _ in range(args.warmup):
-        step_fused()
+        step()
     L.forward(x, M, y, ws, wsb, stream, pkg.FWD_CHECK)
     torch.cuda.synchronize()
 
-    # ---- timed region: exactly `steps` fused steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # ---- timed region: exactly `steps` steps, one event pair around each step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
         for i in range(args.steps):
             flush_l2(i)
             ev[i][0].record(stream)
-            L.quantize_act(x, M, codes, scales, xl, stream, 0)
+            step()
             ev[i][1].record(stream)
-            L.gemm(codes, scales, xl, M, y, stream, 0)
-            ev[i][2].record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    k1_ms = [a.elapsed_time(b) for a, b, _ in ev]
-    k2_ms = [b.elapsed_time(c) for _, b, c in ev]
-    step_ms = sum(k1_ms) / args.steps + sum(k2_ms) / args.steps
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     step_ms_max = allreduce_max(step_ms, world)
-    k2_avg = sum(k2_ms) / args.steps
-    k1_avg = sum(k1_ms) / args.steps
     value = layer_flops(M, K, N) * world / (step_ms_max * 1e-3) / 1e12
+    L.check(stream)
 
-    # ---- measurement variants (outside the timed region): bare GEMM and unfused layer
+    # ---- per-kernel durations (same launches, each bracketed by its own events)
+    n_k = max(100, min(1000, args.steps))
+    k2_ms = time_events(stream, n_k, flush_l2, lambda: L.gemm(codes, scales, xl, M, y, stream, 0))
+    k1_ms = time_events(stream, n_k, flush_l2, lambda: L.quantize_act(x, M, codes, scales, xl, stream, 0))
+
+    # ---- measurement variants: bare GEMM and unfused layer
     n_var = max(50, min(500, args.steps))
 
     def bare():
         L.quantize_act(x, M, codes, scales, xl, stream, 1)
         L.gemm(codes, scales, xl, M, y, stream, pkg.FWD_NO_BRANCH)
 
-    def unfused():
-        L.forward(x, M, y, ws, wsb, stream, pkg.FWD_UNFUSED)
-
-    def bare_gemm():
-        L.gemm(codes, scales, xl, M, y, stream, pkg.FWD_NO_BRANCH)
-
-    bare_ms = time_variant(bare, n_var)
-    unfused_ms = time_variant(unfused, n_var)
+    bare_ms = time_events(stream, n_var, flush_l2, bare)
+    unfused_ms = time_events(stream, n_var, flush_l2, lambda: L.forward(x, M, y, ws, wsb, stream, pkg.FWD_UNFUSED))
     L.quantize_act(x, M, codes, scales, xl, stream, 0)
-    bare_k2_ms = time_variant(bare_gemm, n_var)
+    bare_k2_ms = time_events(stream, n_var, flush_l2, lambda: L.gemm(codes, scales, xl, M, y, stream,
+                                                                      pkg.FWD_NO_BRANCH))
     L.check(stream)
 
     # ---- end to end through the public API with host buffers
     xh = torch.from_numpy(d["X"]).to(torch.bfloat16).pin_memory()
     yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    n_e2e = max(20, min(200, args.steps))
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
-    for i in range(n_e2e):
-        flush_l2(i)
-        e2e_ev[i][0].record(stream)
+
+    def e2e():
         x.copy_(xh, non_blocking=True)
         L.forward(x, M, y, ws, wsb, stream, 0)
         yh.copy_(y, non_blocking=True)
-        e2e_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = allreduce_max(sum(a.elapsed_time(b) for a, b in e2e_ev) / n_e2e, world)
+
+    e2e_ms = allreduce_max(time_events(stream, max(20, min(200, args.steps)), flush_l2, e2e), world)
 
     peaks, peak_src = measured_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    k2_achieved = k2_flops(M, K, N) / (k2_avg * 1e-3) / 1e12
+    k2_achieved = k2_flops(M, K, N) / (k2_ms * 1e-3) / 1e12
+    k1_bytes = M * K * 2 + M * K // 2 + M * K // 16 + M * RANK * 2 + K * 4
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
@@ -359,23 +435,30 @@ def main():
         "config": {"workload": f"{WORKLOAD} {M}x{K}->{N} NVFP4 g16 E4M3 r{RANK}", "M": M, "K": K, "N": N,
                    "rank": RANK, "parallelism": "replicas" if world > 1 else "single",
                    "l2": "flushed between steps outside the timed events (256 MiB write + read)"},
-        "us_per_layer": step_ms_max * 1e3, "k1_us": k1_avg * 1e3, "k2_us": k2_avg * 1e3,
+        "us_per_layer": step_ms_max * 1e3, "k1_us": k1_ms * 1e3, "k2_us": k2_ms * 1e3,
         "pct_nvfp4_peak": {"of_measured": value / world / fp4_peak, "of_nominal": value / world /
                            NOMINAL_FP4_DENSE_TFLOPS, "measured_peak_tflops": fp4_peak,
                            "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)"},
         "bare_us": bare_ms * 1e3, "bare_k2_us": bare_k2_ms * 1e3, "unfused_us": unfused_ms * 1e3,
-        "lowrank_overhead": step_ms / bare_ms - 1.0, "lowrank_overhead_k2": k2_avg / bare_k2_ms - 1.0,
+        "lowrank_overhead": step_ms / bare_ms - 1.0, "lowrank_overhead_k2": k2_ms / bare_k2_ms - 1.0,
         "unfused_overhead": unfused_ms / step_ms - 1.0,
         "roofline": {"bound": "tensor", "kernel": "k2_gemm (NVFP4 block-scaled tcgen05 + fused up-proj)",
                      "achieved": k2_achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": k2_achieved / fp4_peak,
                      "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16:g}",
+                     "timing": "K2 alone between CUDA events on the launch stream, L2 flushed, "
+                               f"{n_k} launches after the timed steps",
                      "traffic": profile_traffic()},
+        "k1_roofline": {"bound": "hbm", "achieved": k1_bytes / (k1_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": k1_bytes / (k1_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                        "algorithmic_bytes": k1_bytes},
         "e2e": {"value": layer_flops(M, K, N) * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
                 "path": "svdq_linear_forward with pinned host X/Y, copies inside the timed events"},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
+    if rank == 0 and world == 1 and not args.no_other_layers:
+        out["other_layers"] = other_layers(pkg, syn, stream, flush_l2, max(30, min(200, args.steps)), peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(d, M, K, N)
     L.close()
