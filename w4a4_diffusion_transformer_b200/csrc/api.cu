@@ -34,6 +34,8 @@ struct svdq_layer {
   float* d_bias = nullptr;           // [N]
   int* d_err = nullptr;
   CUtensorMap tm_wq, tm_l2s, tm_l1t;
+  CUtensorMap tm_wq_pair, tm_l2s_pair;   // 128-row boxes for the CTA-pair GEMM (NVFP4)
+  int k2_kernel = 0;                     // NVFP4 GEMM: 0 = by size, 1 = single-CTA, 2 = CTA pairs
 };
 
 namespace {
@@ -209,6 +211,17 @@ svdq_status upload_layer(svdq_layer* L, int device) {
     chk(upload(&L->d_l2t, l2t.data(), l2t.size() * 2));
     if (e != cudaSuccess) return SVDQ_ECUDA;
     const bool nv = h.format == SVDQ_NVFP4;
+    if (nv) {
+      const bool ok2 = make_map(&L->tm_wq_pair, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128,
+                                (uint32_t)k2_pair_rows_b(), CU_TENSOR_MAP_SWIZZLE_128B) &&
+                       make_map(&L->tm_l2s_pair, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32,
+                                (uint32_t)k2_pair_rows_b(), CU_TENSOR_MAP_SWIZZLE_64B);
+      if (!ok2) return SVDQ_ECUDA;
+      if (const char* k = std::getenv("SVDQ_K2_KERNEL")) {
+        if (!std::strcmp(k, "single")) L->k2_kernel = 1;
+        if (!std::strcmp(k, "pair")) L->k2_kernel = 2;
+      }
+    }
     bool ok = make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, nv ? k2_box_bytes() : 32,
                        256, nv ? k2_swizzle() : CU_TENSOR_MAP_SWIZZLE_NONE) &&
               make_map(&L->tm_l2s, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
@@ -324,6 +337,7 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
   p.M = M;
   p.N = h.N;
   p.K = h.K;
+  p.mpad = pad_rows(M);
   p.alpha = (float)std::ldexp(1.0, h.g_x_exp + h.g_w_exp);
   p.sfa = static_cast<const uint8_t*>(scales);
   p.sfb = L->d_ws;
@@ -333,8 +347,12 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
   p.budget_ns = L->budget_ns;
   p.branch = branch ? 1 : 0;
   p.gelu = gelu ? 1 : 0;
-  return launch_k2(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream) == cudaSuccess ? SVDQ_OK
-                                                                                          : SVDQ_ECUDA;
+  // The CTA-pair kernel (256 x 256 tiles) is exact but measured slower than the
+  // single-CTA kernel on this part; it runs only when SVDQ_K2_KERNEL=pair.
+  const bool pair = L->k2_kernel == 2;
+  const cudaError_t e = pair ? launch_k2_pair(tm_a, L->tm_wq_pair, tm_xl, L->tm_l2s_pair, tm_y, p, L->num_sms, stream)
+                             : launch_k2(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream);
+  return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
 
 }  // namespace

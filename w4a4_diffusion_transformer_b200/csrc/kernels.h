@@ -30,6 +30,7 @@ struct K1Params {
 
 struct K2Params {
   int M, N, K;
+  int mpad;                     // rows of the activation scale layout (M rounded up to 128)
   float alpha;                  // g_x * g_w (power of two)
   const uint8_t* sfa;           // activation scales, tensor-core layout
   const uint8_t* sfb;           // weight scales, tensor-core layout (rows padded to 256)
@@ -91,6 +92,12 @@ cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CU
                       const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
                       cudaStream_t stream);
 int k2_block_n();
+// The same GEMM on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2, clusters of
+// two): tm_b and tm_l2 have 128-row boxes (each CTA holds half of B).
+cudaError_t launch_k2_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
+                           const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
+                           cudaStream_t stream);
+int k2_pair_rows_b();
 int k2_stage_k_bytes();   // E2M1 bytes per operand row per pipeline stage (128 or 64)
 
 // INT4 GEMM: A = activation codes [M][K/2] (box 32 B x 128 rows), B = weight
