@@ -259,7 +259,7 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
                               device=torch.cuda.current_device())
         x = X if isinstance(X, torch.Tensor) else torch.from_numpy(X).to(torch.bfloat16).cuda()
         y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-        codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        codes = torch.empty(L.act_code_bytes(M), dtype=torch.uint8, device="cuda")
         scales = torch.empty(L.act_scale_bytes(M), dtype=torch.uint8, device="cuda")
         xl = torch.empty((M, RANK), dtype=torch.bfloat16, device="cuda")
 
@@ -355,7 +355,7 @@ def main():
     wsb = L.workspace_bytes(M)
     ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
     # the two kernels' intermediate buffers for the split (per-kernel timed) calls
-    codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    codes = torch.empty(L.act_code_bytes(M), dtype=torch.uint8, device="cuda")
     scales = torch.empty(L.act_scale_bytes(M), dtype=torch.uint8, device="cuda")
     xl = torch.empty((M, RANK), dtype=torch.bfloat16, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")

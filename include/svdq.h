@@ -166,9 +166,11 @@ svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, v
                                 void* workspace, size_t workspace_bytes,
                                 void* stream, unsigned flags);
 
-/* The first kernel alone (NVFP4/INT4): writes the activation codes
- * (device [M][K/2], even k in the low nibble; INT4 codes are 4-bit two's
- * complement), the activation scales (device, svdq_act_scale_bytes(layer, M)
+/* The first kernel alone (NVFP4/INT4): writes the activation codes (device,
+ * svdq_act_code_bytes(layer, M) bytes, two codes per byte with the even k in
+ * the low nibble; INT4 codes are 4-bit two's complement, row-major [M][K/2];
+ * NVFP4 codes are in the GEMM's tiled layout, see svdq_act_codes_to_logical),
+ * the activation scales (device, svdq_act_scale_bytes(layer, M)
  * bytes: NVFP4 E4M3 in the tensor-core layout, INT4 BF16 [K/64][M rounded up
  * to 128], group-major, padding rows zero) and, when
  * the layer has a branch, XL = bf16(X L1d) (device [M][rank] BF16).
@@ -182,6 +184,20 @@ svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int M,
  * SVDQ_FWD_GELU, SVDQ_FWD_NO_BRANCH, SVDQ_FWD_CHECK. */
 svdq_status svdq_gemm(const svdq_layer* layer, const void* codes, const void* scales,
                       const void* xl, int M, void* Y, void* stream, unsigned flags);
+
+/* Bytes of the activation codes for M tokens in the layout the GEMM reads:
+ * INT4 M * K/2; NVFP4 ceil(M/128)*128 * ceil(K/256) * 128 (tiled). */
+size_t svdq_act_code_bytes(const svdq_layer* layer, int M);
+
+/* Host-side: convert a host copy of activation codes in the GEMM's layout
+ * (svdq_act_code_bytes bytes) into the logical row-major [M][K/2] bytes.  The
+ * NVFP4 layout stores, for each block of 128 rows and each stage of 256 codes
+ * (128 bytes of a row), one contiguous 16 KiB block in which byte j of row r
+ * sits at (r % 128) * 128 + (((j / 16) ^ (r % 8)) * 16) + j % 16: the order in
+ * which the tensor core reads a 128-byte-swizzled operand tile, so the GEMM
+ * fetches each stage with one contiguous copy. */
+svdq_status svdq_act_codes_to_logical(const svdq_layer* layer, const void* device_layout,
+                                      int M, void* logical);
 
 /* Bytes of the activation scales for M tokens in the layout the GEMM reads. */
 size_t svdq_act_scale_bytes(const svdq_layer* layer, int M);

@@ -48,12 +48,12 @@ def run_quantize(L, X: np.ndarray, mode=0):
     import torch
     M, K = X.shape
     x = torch_bf16(X)
-    codes = torch.full((M, K // 2), 0xAB, dtype=torch.uint8, device="cuda")
+    codes = torch.full((L.act_code_bytes(M),), 0xAB, dtype=torch.uint8, device="cuda")
     scales = torch.full((L.act_scale_bytes(M),), 0xCD, dtype=torch.uint8, device="cuda")
     xl = torch.full((M, 32), float("nan"), dtype=torch.bfloat16, device="cuda")
     L.quantize_act(x, M, codes, scales, xl, torch.cuda.current_stream(), mode)
     torch.cuda.synchronize()
-    return {"codes": codes.cpu().numpy(), "scales_dev": scales.cpu().numpy(),
+    return {"codes": L.act_codes_to_logical(codes.cpu().numpy(), M), "scales_dev": scales.cpu().numpy(),
             "scales": L.act_scales_to_logical(scales.cpu().numpy(), M), "xl": to_numpy_f32(xl),
             "_t": (x, codes, scales, xl)}
 

@@ -38,7 +38,7 @@ EXPORTED = [
     "svdq_prepare", "svdq_destroy", "svdq_get_info", "svdq_tensor_bytes", "svdq_export",
     "svdq_status_string", "svdq_workspace_bytes", "svdq_linear_forward", "svdq_quantize_act",
     "svdq_gemm", "svdq_act_scale_bytes", "svdq_act_scales_to_logical", "svdq_check",
-    "svdq_linear_forward_static",
+    "svdq_linear_forward_static", "svdq_act_code_bytes", "svdq_act_codes_to_logical",
 ]
 STATIC_WORKSPACE_BYTES = 16 << 20   # SVDQ_STATIC_WORKSPACE_BYTES
 
@@ -88,6 +88,8 @@ def load() -> ctypes.CDLL:
         "svdq_act_scales_to_logical": (I, [P, P, I, P]),
         "svdq_check": (I, [P, P]),
         "svdq_linear_forward_static": (I, [P, P, I, P, P, U]),
+        "svdq_act_code_bytes": (SZ, [P, I]),
+        "svdq_act_codes_to_logical": (I, [P, P, I, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -186,6 +188,16 @@ class Layer:
 
     def act_scale_bytes(self, M: int) -> int:
         return int(load().svdq_act_scale_bytes(self._h, M))
+
+    def act_code_bytes(self, M: int) -> int:
+        return int(load().svdq_act_code_bytes(self._h, M))
+
+    def act_codes_to_logical(self, device_layout: np.ndarray, M: int) -> np.ndarray:
+        """Activation codes in the GEMM's layout -> uint8 [M][K/2] (two codes per byte)."""
+        out = np.empty((M, self.info["K"] // 2), dtype=np.uint8)
+        src = np.ascontiguousarray(device_layout, dtype=np.uint8)
+        _check(load().svdq_act_codes_to_logical(self._h, _ptr(src), M, _ptr(out)), "svdq_act_codes_to_logical")
+        return out
 
     def forward(self, X, M: int, Y, workspace, workspace_bytes: int, stream=None, flags: int = 0):
         _check(load().svdq_linear_forward(self._h, _ptr(X), M, _ptr(Y), _ptr(workspace), workspace_bytes,

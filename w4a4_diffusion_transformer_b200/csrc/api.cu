@@ -33,8 +33,8 @@ struct svdq_layer {
   int i4_ex = 0, i4_ew = 0;          // INT4: power-of-two range exponents of the FP16 GEMM operands
   float* d_bias = nullptr;           // [N]
   int* d_err = nullptr;
-  CUtensorMap tm_wq, tm_l2s, tm_l1t;
-  CUtensorMap tm_wq_pair, tm_l2s_pair;   // 128-row boxes for the CTA-pair GEMM (NVFP4)
+  CUtensorMap tm_wq, tm_l2s, tm_l1t;     // tm_wq: INT4 weight codes [N][K/2]
+  CUtensorMap tm_l2s_pair;               // 128-row boxes for the CTA-pair GEMM (NVFP4)
   int k2_kernel = 0;                     // NVFP4 GEMM: 0 = by size, 1 = single-CTA, 2 = CTA pairs
 };
 
@@ -89,13 +89,18 @@ struct DeviceGuard {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Box width and swizzle of the GEMM's 4-bit operand tiles (one pipeline stage of K).
-uint32_t k2_box_bytes() { return (uint32_t)k2_stage_k_bytes(); }
-CUtensorMapSwizzle k2_swizzle() { return k2_stage_k_bytes() == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B; }
 
 bool w4a4(const svdq_layer* L) { return L->host.format == SVDQ_NVFP4 || L->host.format == SVDQ_INT4; }
 
 int pad_rows(int M) { return (M + 127) / 128 * 128; }
+int nvfp4_stages(int K) { return (K + 255) / 256; }   // K stages of 256 codes (128-byte rows)
+
+// Bytes of the activation codes for M tokens: NVFP4 tiled (act_tile_offset),
+// INT4 row-major [M][K/2].
+size_t act_code_bytes(const HostPrep& h, int M) {
+  if (h.format == SVDQ_NVFP4) return (size_t)pad_rows(M) * (size_t)nvfp4_stages(h.K) * 128u;
+  return (size_t)M * (size_t)(h.K / 2);
+}
 
 // FP16 bits of a value that is exact in float32, rounded to nearest even.
 uint16_t f16_from_double(double v) { return __half_as_ushort(__float2half_rn((float)v)); }
@@ -124,7 +129,7 @@ struct WsLayout {
 WsLayout ws_layout(const HostPrep& h, int M) {
   WsLayout w;
   w.codes = 0;
-  w.scales = align_up((size_t)M * (size_t)(h.K / 2), 256);
+  w.scales = align_up(act_code_bytes(h, M), 256);
   w.xl = w.scales + align_up(act_scale_bytes(h, M), 256);
   w.total = w.xl + align_up((size_t)M * 32 * 2, 256);
   return w;
@@ -173,7 +178,17 @@ svdq_status upload_layer(svdq_layer* L, int device) {
   chk(upload(&L->d_bias, h.bias.data(), sizeof(float) * N));
   if (h.format == SVDQ_NVFP4 || h.format == SVDQ_INT4) {
     chk(upload(&L->d_inv_lam, h.inv_lam.data(), sizeof(float) * K));
-    chk(upload(&L->d_wq, h.w_codes.data(), h.w_codes.size()));
+    if (h.format == SVDQ_NVFP4) {
+      // weight codes in the GEMM's tiled layout (wgt_tile_offset), rows padded to 256 with zeros
+      const int nst = nvfp4_stages(K);
+      std::vector<uint8_t> tiled((size_t)((N + 255) / 256) * (size_t)nst * 32768u, 0);
+      for (int n = 0; n < N; ++n)
+        for (int b = 0; b < K / 2; ++b)
+          tiled[wgt_tile_offset(n, b >> 7, (b & 127) >> 4, nst) + (b & 15)] = h.w_codes[(size_t)n * (K / 2) + b];
+      chk(upload(&L->d_wq, tiled.data(), tiled.size()));
+    } else {
+      chk(upload(&L->d_wq, h.w_codes.data(), h.w_codes.size()));
+    }
     int alpha_exp = h.g_x_exp + h.g_w_exp;
     if (h.format == SVDQ_NVFP4) {
       // weight scales in the tensor-core layout, rows padded to a multiple of 256
@@ -212,9 +227,7 @@ svdq_status upload_layer(svdq_layer* L, int device) {
     if (e != cudaSuccess) return SVDQ_ECUDA;
     const bool nv = h.format == SVDQ_NVFP4;
     if (nv) {
-      const bool ok2 = make_map(&L->tm_wq_pair, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128,
-                                (uint32_t)k2_pair_rows_b(), CU_TENSOR_MAP_SWIZZLE_128B) &&
-                       make_map(&L->tm_l2s_pair, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32,
+      const bool ok2 = make_map(&L->tm_l2s_pair, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32,
                                 (uint32_t)k2_pair_rows_b(), CU_TENSOR_MAP_SWIZZLE_64B);
       if (!ok2) return SVDQ_ECUDA;
       if (const char* k = std::getenv("SVDQ_K2_KERNEL")) {
@@ -222,8 +235,9 @@ svdq_status upload_layer(svdq_layer* L, int device) {
         if (!std::strcmp(k, "pair")) L->k2_kernel = 2;
       }
     }
-    bool ok = make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, nv ? k2_box_bytes() : 32,
-                       256, nv ? k2_swizzle() : CU_TENSOR_MAP_SWIZZLE_NONE) &&
+    // INT4 weight codes stay row-major [N][K/2] (the INT4 GEMM loads them with TMA)
+    bool ok = (nv || make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 32, 256,
+                              CU_TENSOR_MAP_SWIZZLE_NONE)) &&
               make_map(&L->tm_l2s, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
                        CU_TENSOR_MAP_SWIZZLE_64B) &&
               make_map(&L->tm_l1t, L->d_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, 32, 64, 32,
@@ -250,6 +264,7 @@ K1Params k1_params(const svdq_layer* L, int M, void* codes, void* scales, void* 
   p.M = M;
   p.K = h.K;
   p.mpad = pad_rows(M);
+  p.nst = nvfp4_stages(h.K);
   p.c_x = (float)std::ldexp((double)(1.0f / 6.0f), -h.g_x_exp);
   p.g_x_exp = h.g_x_exp;
   for (int m = 0; m < 8; ++m) {
@@ -273,11 +288,13 @@ svdq_status run_k1(const svdq_layer* L, const void* X, int M, void* codes, void*
     return SVDQ_ECUDA;
   // activation codes are written in 32-row tiles, one per quantizer warp and stage:
   // 16 bytes wide for NVFP4 (32 columns), 32 bytes for INT4 (64 columns)
+  // NVFP4 codes are written tiled from registers; INT4 codes in 32-row x 32-byte
+  // tiles by TMA (one per quantizer warp and stage)
   const bool nv = h.format == SVDQ_NVFP4;
-  if (mode != 2 && !make_map(&tm_c, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, nv ? 16 : 32, 32,
-                             CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (mode != 2 && !nv &&
+      !make_map(&tm_c, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SVDQ_ECUDA;
-  if (mode == 2) tm_c = tm_x;   // unused by the down-projection-only kernel
+  if (mode == 2 || nv) tm_c = tm_x;   // unused
   K1Params p = k1_params(L, M, codes, scales, xl);
   return launch_k1(tm_x, L->tm_l1t, tm_c, p, nv ? kFmtNvfp4 : kFmtInt4, mode, stream) == cudaSuccess ? SVDQ_OK
                                                                                                     : SVDQ_ECUDA;
@@ -322,22 +339,22 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
                    cudaStream_t stream, bool branch, bool gelu) {
   if (L->host.format == SVDQ_INT4) return run_k2_int4(L, codes, scales, xl, M, Y, stream, branch, gelu);
   const HostPrep& h = L->host;
-  CUtensorMap tm_a, tm_xl, tm_y;
-  if (!make_map(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, k2_box_bytes(), 128, k2_swizzle()))
-    return SVDQ_ECUDA;
+  CUtensorMap tm_xl, tm_y;
   if (!make_map(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ECUDA;
   if (branch) {
     if (!make_map(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
       return SVDQ_ECUDA;
   } else {
-    tm_xl = tm_a;   // unused by the kernel
+    tm_xl = tm_y;   // unused by the kernel
   }
   K2Params p;
   p.M = M;
   p.N = h.N;
   p.K = h.K;
   p.mpad = pad_rows(M);
+  p.acodes = static_cast<const uint8_t*>(codes);
+  p.wcodes = L->d_wq;
   p.alpha = (float)std::ldexp(1.0, h.g_x_exp + h.g_w_exp);
   p.sfa = static_cast<const uint8_t*>(scales);
   p.sfb = L->d_ws;
@@ -350,8 +367,8 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
   // The CTA-pair kernel (256 x 256 tiles) is exact but measured slower than the
   // single-CTA kernel on this part; it runs only when SVDQ_K2_KERNEL=pair.
   const bool pair = L->k2_kernel == 2;
-  const cudaError_t e = pair ? launch_k2_pair(tm_a, L->tm_wq_pair, tm_xl, L->tm_l2s_pair, tm_y, p, L->num_sms, stream)
-                             : launch_k2(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream);
+  const cudaError_t e = pair ? launch_k2_pair(tm_xl, L->tm_l2s_pair, tm_y, p, L->num_sms, stream)
+                             : launch_k2(tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream);
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
 
@@ -479,6 +496,29 @@ size_t svdq_workspace_bytes(const svdq_layer* L, int M) {
 size_t svdq_act_scale_bytes(const svdq_layer* L, int M) {
   if (!L || M < 1) return 0;
   return act_scale_bytes(L->host, M);
+}
+
+size_t svdq_act_code_bytes(const svdq_layer* L, int M) {
+  if (!L || M < 1 || !w4a4(L)) return 0;
+  return act_code_bytes(L->host, M);
+}
+
+svdq_status svdq_act_codes_to_logical(const svdq_layer* L, const void* device_layout, int M, void* logical) {
+  if (!L || !device_layout || !logical || M < 1) return SVDQ_EINVAL;
+  const HostPrep& h = L->host;
+  if (!w4a4(L)) return SVDQ_EUNSUPPORTED;
+  const uint8_t* src = static_cast<const uint8_t*>(device_layout);
+  uint8_t* dst = static_cast<uint8_t*>(logical);
+  const size_t row = (size_t)(h.K / 2);
+  if (h.format == SVDQ_INT4) {
+    std::memcpy(dst, src, (size_t)M * row);
+    return SVDQ_OK;
+  }
+  const int nst = nvfp4_stages(h.K);
+  for (int r = 0; r < M; ++r)
+    for (size_t b = 0; b < row; ++b)
+      dst[(size_t)r * row + b] = src[act_tile_offset(r, (int)(b >> 7), (int)((b & 127) >> 4), nst) + (b & 15)];
+  return SVDQ_OK;
 }
 
 svdq_status svdq_act_scales_to_logical(const svdq_layer* L, const void* device_layout, int M, void* logical) {

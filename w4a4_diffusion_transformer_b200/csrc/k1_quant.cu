@@ -297,8 +297,6 @@ __global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
     const int grow = row0 + lane;                     // this lane's row (may be >= M: zero padding)
     const int col0 = warp * 32;                       // 2 groups of 16 columns of each stage
     uint16_t* scale_pair = reinterpret_cast<uint16_t*>(p.scales + sf_offset(grow, 2 * warp, K));
-    uint8_t* ctile = cbuf + warp * 2 * kCodeTile;
-    if (lane == 0) dev::tma_prefetch_desc(&tm_c);
     for (int it = 0; it < nk; ++it) {
       const int s = it % kXStages;
       if (!dev::mbar_wait(&xfull[s], (uint32_t)(it / kXStages) & 1u, abort_flag, p.budget_ns)) {
@@ -358,21 +356,13 @@ __global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
       if (lane == 0) dev::mbar_arrive(&xempty[s]);
       if (active) {
         scale_pair[(size_t)(k0 >> 6) * 256] = (uint16_t)(sb2 & 0xFFFFu);   // next 64 columns: next 512-byte chunk
-        // codes: this warp's 32 x 16-byte tile, stored with TMA once the store
-        // that last read this buffer (two stages ago) is done reading
-        uint8_t* ct = ctile + (it & 1) * kCodeTile;
-        if (lane == 0) dev::bulk_wait_group_read<1>();
-        __syncwarp();
-        *reinterpret_cast<uint4*>(ct + lane * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        dev::fence_async_shared();
-        __syncwarp();
-        if (lane == 0) {
-          dev::tma_store_2d(&tm_c, ct, (k0 + col0) >> 1, row0);
-          dev::bulk_commit_group();
-        }
+        // codes: 16 bytes = chunk `warp` of this row's 128-byte stage row, in the
+        // tiled layout the GEMM loads with one bulk copy per stage (see
+        // act_tile_offset): block (row / 128, stage), swizzled by row % 8
+        *reinterpret_cast<uint4*>(p.codes + act_tile_offset(grow, it, warp, p.nst)) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
     }
-    if (lane == 0) dev::bulk_wait_group_all();
     return;
   }
 

@@ -14,10 +14,13 @@
 // alpha * acc reproduces Q(X^)Q(R) + XL L2b.
 //
 // Structure (one CTA per SM, persistent over output tiles):
-//   warp 0     TMA producer: per stage a 128 x 256 E2M1 A tile, a 256 x 256 E2M1
-//              B tile (128-byte swizzle), and the E4M3 scale factors (bulk
-//              copies, already in the tensor-core layout); per tile one extra
-//              stage with the XL tile and the L2b^T tile (64-byte swizzle).
+//   warp 0     producer: per stage a 128 x 256 E2M1 A tile and a 256 x 256 E2M1
+//              B tile, each one contiguous bulk copy (the codes are stored in
+//              blocks already in the 128-byte-swizzled order the tensor core
+//              reads: contiguous copies reach each SM faster than row-strided
+//              tensor boxes), and the E4M3 scale factors (bulk copies, already
+//              in the tensor-core layout); per tile one extra stage with the XL
+//              tile and the L2b^T tile (TMA, 64-byte swizzle).
 //   warp 1     allocates TMEM (512 columns: accumulator 256 + per-stage scale
 //              factors) and issues tcgen05.mma.
 //   warp 10    copies each stage's scale factors into TMEM (tcgen05.cp) as soon
@@ -98,8 +101,7 @@ __device__ __forceinline__ float gelu_tanh(float y) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-              const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2,
+    k2_kernel(const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2,
               const __grid_constant__ CUtensorMap tm_y, K2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -151,8 +153,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      dev::tma_prefetch_desc(&tm_a);
-      dev::tma_prefetch_desc(&tm_b);
       if (p.branch) {
         dev::tma_prefetch_desc(&tm_xl);
         dev::tma_prefetch_desc(&tm_l2);
@@ -203,14 +203,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             dev::bulk_load(st + kABytes + kBBytes + kSFABytes + h * (kKB * 512), p.sfb + b_chunk * 512, sf_bytes,
                            &sf_full[s]);
           }
-          dev::tma_load_2d(st + kABytes, &tm_b, &full[s], kt * kBKBytes, n0);
+          // operand blocks are stored tiled and pre-swizzled: one contiguous bulk copy each
+          dev::bulk_load(st + kABytes, p.wcodes + ((size_t)(n0 >> 8) * (size_t)ktiles + (size_t)kt) * kBBytes,
+                         kBBytes, &full[s]);
           if (!deps_ready) {
             dev::griddep_wait();
             deps_ready = true;
           }
           const size_t a_chunk = (size_t)(m0 >> 7) * (size_t)kblocks + (size_t)(kKB * kt);
           dev::bulk_load(st + kABytes + kBBytes, p.sfa + a_chunk * 512, sf_bytes, &sf_full[s]);
-          dev::tma_load_2d(st, &tm_a, &full[s], kt * kBKBytes, m0);
+          dev::bulk_load(st, p.acodes + ((size_t)(m0 >> 7) * (size_t)ktiles + (size_t)kt) * kABytes, kABytes,
+                         &full[s]);
           ++it;
         }
       }
@@ -429,11 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 int k2_block_n() { return kBN; }
-int k2_stage_k_bytes() { return kBKBytes; }
 
-cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
-                      const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
-                      cudaStream_t stream) {
+cudaError_t launch_k2(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
+                      const K2Params& p, int num_sms, cudaStream_t stream) {
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -457,7 +458,7 @@ cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CU
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k2_kernel, tm_a, tm_b, tm_xl, tm_l2, tm_y, p);
+  return cudaLaunchKernelEx(&cfg, k2_kernel, tm_xl, tm_l2, tm_y, p);
 }
 
 }  // namespace svdq

@@ -81,8 +81,7 @@ __device__ __forceinline__ float gelu_tanh(float y) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k2_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                   const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2,
+    k2_pair_kernel(const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2,
                    const __grid_constant__ CUtensorMap tm_y, K2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -142,8 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
-      dev::tma_prefetch_desc(&tm_a);
-      dev::tma_prefetch_desc(&tm_b);
       if (p.branch) {
         dev::tma_prefetch_desc(&tm_xl);
         dev::tma_prefetch_desc(&tm_l2);
@@ -189,14 +186,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           // scale factors on their own barrier, issued first (their TMEM copies
           // then run while the operand tiles are still in flight)
           dev::mbar_arrive_expect_tx(&sf_full[s], (sf_a ? sf_bytes : 0u) + 2u * sf_bytes);
-          dev::mbar_arrive_expect_tx(&full[s], (rows_a ? kABytes : 0) + (rows_b ? kBBytes : 0));
+          dev::mbar_arrive_expect_tx(&full[s], (sf_a ? kABytes : 0) + kBBytes);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const size_t b_chunk = (size_t)((n0 >> 7) + h) * (size_t)kblocks + (size_t)(kKB * kt);
             dev::bulk_load(st + kABytes + kBBytes + kSFABytes + h * (kKB * 512), p.sfb + b_chunk * 512, sf_bytes,
                            &sf_full[s]);
           }
-          if (rows_b) dev::tma_load_2d(st + kABytes, &tm_b, &full[s], kt * kBKBytes, my_n);
+          // this CTA's 128-row half of the 256-row weight block (tiled, pre-swizzled)
+          dev::bulk_load(st + kABytes,
+                         p.wcodes + ((size_t)(n0 >> 8) * (size_t)ktiles + (size_t)kt) * (2 * kBBytes) + rank * kBBytes,
+                         kBBytes, &full[s]);
           if (!deps_ready) {
             dev::griddep_wait();
             deps_ready = true;
@@ -205,7 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const size_t a_chunk = (size_t)(my_m >> 7) * (size_t)kblocks + (size_t)(kKB * kt);
             dev::bulk_load(st + kABytes + kBBytes, p.sfa + a_chunk * 512, sf_bytes, &sf_full[s]);
           }
-          if (rows_a) dev::tma_load_2d(st, &tm_a, &full[s], kt * kBKBytes, my_m);
+          if (sf_a)
+            dev::bulk_load(st, p.acodes + ((size_t)(my_m >> 7) * (size_t)ktiles + (size_t)kt) * kABytes, kABytes,
+                           &full[s]);
           ++it;
         }
       }
@@ -448,9 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int k2_pair_rows_b() { return kBNh; }
 
-cudaError_t launch_k2_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
-                           const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
-                           cudaStream_t stream) {
+cudaError_t launch_k2_pair(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
+                           const K2Params& p, int num_sms, cudaStream_t stream) {
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -477,7 +478,7 @@ cudaError_t launch_k2_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, con
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k2_pair_kernel, tm_a, tm_b, tm_xl, tm_l2, tm_y, p);
+  return cudaLaunchKernelEx(&cfg, k2_pair_kernel, tm_xl, tm_l2, tm_y, p);
 }
 
 }  // namespace svdq

@@ -17,11 +17,12 @@ constexpr int kFmtInt4 = 1;
 struct K1Params {
   int M, K;
   int mpad;                     // M rounded up to 128 (rows of the INT4 scale array)
+  int nst;                      // K stages of 256 codes (rows of 128 bytes) in the NVFP4 tiled code layout
   float c_x;                    // fp32(1/6) * 2^-g_x_exp
   int g_x_exp;                  // activation tensor scale g_x = 2^g_x_exp
   float rcp[16];                // fp32(1/(1 + m/8)) for m = 0..7, then fp32(1/m) (index 8 + m)
   const float* inv_lam;         // [K]
-  uint8_t* codes;               // [M][K/2]
+  uint8_t* codes;               // NVFP4: tiled layout (act_tile_offset); INT4: [M][K/2]
   uint8_t* scales;              // NVFP4: tensor-core scale layout, mpad rows; INT4: BF16 [K/64][mpad]
   __nv_bfloat16* xl;            // [M][32]
   int* err;                     // device error word
@@ -31,6 +32,8 @@ struct K1Params {
 struct K2Params {
   int M, N, K;
   int mpad;                     // rows of the activation scale layout (M rounded up to 128)
+  const uint8_t* acodes;        // activation codes, tiled layout (act_tile_offset), mpad rows
+  const uint8_t* wcodes;        // weight codes, tiled layout (wgt_tile_offset), N rounded up to 256 rows
   float alpha;                  // g_x * g_w (power of two)
   const uint8_t* sfa;           // activation scales, tensor-core layout
   const uint8_t* sfb;           // weight scales, tensor-core layout (rows padded to 256)
@@ -88,17 +91,16 @@ cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CU
                       const K1Params& p, int fmt, int mode, cudaStream_t stream);
 int k1_rows_per_cta();
 
-cudaError_t launch_k2(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
-                      const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
-                      cudaStream_t stream);
+// NVFP4 GEMM: operands from p.acodes / p.wcodes (tiled layouts); tm_xl / tm_l2
+// the branch tiles, tm_y the output.
+cudaError_t launch_k2(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
+                      const K2Params& p, int num_sms, cudaStream_t stream);
 int k2_block_n();
 // The same GEMM on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2, clusters of
-// two): tm_b and tm_l2 have 128-row boxes (each CTA holds half of B).
-cudaError_t launch_k2_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
-                           const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Params& p, int num_sms,
-                           cudaStream_t stream);
+// two): tm_l2 has 128-row boxes (each CTA holds half of B).
+cudaError_t launch_k2_pair(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
+                           const K2Params& p, int num_sms, cudaStream_t stream);
 int k2_pair_rows_b();
-int k2_stage_k_bytes();   // E2M1 bytes per operand row per pipeline stage (128 or 64)
 
 // INT4 GEMM: A = activation codes [M][K/2] (box 32 B x 128 rows), B = weight
 // codes [N][K/2] (box 32 B x 256 rows), both unswizzled.

@@ -58,4 +58,21 @@ SVDQ_HD inline size_t sf_offset(int r, int g, int K) {
   return chunk * 512 + (size_t)(r & 31) * 16 + (size_t)((r >> 5) & 3) * 4 + (size_t)(g & 3);
 }
 
+// Tiled layout of NVFP4 activation codes (the GEMM's A operand): for row
+// block b = r / 128 and K stage t (256 codes = 128 bytes of each row), a
+// contiguous 16 KiB block at (b * nst + t) * 16384 holding the block's 128 rows
+// as the tensor core reads them (128-byte swizzle): 16-byte chunk c of row
+// r % 128 at (r % 128) * 128 + ((c ^ (r % 8)) * 16).  nst = ceil(K / 256).
+SVDQ_HD inline size_t act_tile_offset(int r, int t, int c, int nst) {
+  return ((size_t)(r >> 7) * (size_t)nst + (size_t)t) * 16384u + (size_t)(r & 127) * 128u +
+         (size_t)(((c ^ (r & 7)) & 7) << 4);
+}
+
+// The same layout for the weight codes (the GEMM's B operand) in blocks of 256
+// rows: block (r / 256, t) at (b * nst + t) * 32768.
+SVDQ_HD inline size_t wgt_tile_offset(int r, int t, int c, int nst) {
+  return ((size_t)(r >> 8) * (size_t)nst + (size_t)t) * 32768u + (size_t)(r & 255) * 128u +
+         (size_t)(((c ^ (r & 7)) & 7) << 4);
+}
+
 }  // namespace svdq
