@@ -22,20 +22,23 @@
 //                   code of pair j sits at bits 4j and the second at bits 16+4j,
 //                   so (word >> 4j) & 0x000F000F is a BF16x2-ready pair;
 //   bytes 512..543  scales (row g, row g+8) for g = 0..7.
-// A tile is therefore one contiguous stream, and any range of its groups is one
-// bulk copy.
+// A tile is therefore one contiguous block of G * 544 bytes.
 //
-// Tiling.  A CTA owns one tile and all of K; its 8 warps take contiguous ranges
-// of groups (split K) and are reduced through shared memory at the end.  Each
-// warp streams its range through a private ring of shared-memory stages with
-// cp.async.bulk (one elected lane issues; an mbarrier per stage counts the
-// bytes), so up to 4 stages per warp are in flight without holding registers.
+// Work layout: one CTA per SM with sixteen warps in eight pairs; each pair
+// owns whole weight tiles (persistent over the tiles) and splits K between its
+// two warps.  A warp streams its groups through a private ring of four chunk
+// slots (four groups each) in shared memory with 16-byte cp.async copies (its
+// 32 lanes copy one group's 512 code bytes, two lanes its 32 scale bytes),
+// three chunks ahead of the one it computes, without holding registers; the
+// weights are read once.  The two partial sums of a tile meet in shared memory
+// behind a barrier of the pair alone, so no warp waits for the rest of the CTA.
 // Inside a group the k order is permuted so that the 16 codes a thread reads
 // are exactly its A-fragment elements for the group's 4 MMAs, and the
 // activation fragments (8 consecutive BF16 pairs of X, read through L1) use the
-// same permutation; a sum over k is order-free.  Each group accumulates into a
-// fresh FP32 fragment that is then scaled by the row's group scale, so the BF16
-// operands are the exact codes.
+// same permutation; a sum over k is order-free.  The four MMAs of a group
+// accumulate into independent fragments (the MMA's latency is long) that are
+// summed and scaled by the row's group scale, so the BF16 operands are the
+// exact codes.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -53,17 +56,19 @@ namespace {
 
 using namespace dev;
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
 constexpr int kRows = 16;                              // weight rows per tile (MMA M)
 constexpr int kGroupBytes = 544;                       // 512 bytes of codes + 32 of scales
-constexpr int kStageGroups = 2;
-constexpr int kStages = 4;                             // ring depth per warp
-constexpr int kStageBytes = kStageGroups * kGroupBytes;
-static_assert(kGroupBytes % 16 == 0 && kStageBytes % 16 == 0, "bulk copies move 16-byte multiples");
+constexpr int kChunk = 4;                              // groups per chunk
+constexpr int kRing = 4;                               // chunk slots per warp (kRing - 1 chunks in flight)
+constexpr int kChunkBytes = kChunk * kGroupBytes;
+constexpr int kSmemBudget = 227 * 1024;                 // dynamic shared memory per CTA
 
 // Codes pair (bits 0-3, 16-19 of y) as an exact bf16x2 of (c + 136): the
 // biased nibble (n ^ 8) = c + 8 in the mantissa of 128.0.  The bias is removed
-// once per group through the activation sums (see the kernel).
+// once per group through the activation sums (see the kernel): one multiply-add
+// per output instead of a subtraction per code pair.
 __device__ __forceinline__ uint32_t codes_pair(uint32_t y) { return (y & 0x000F000Fu) ^ 0x43084308u; }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -74,6 +79,15 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// 16-byte asynchronous copy global -> shared, cached in L2 only (the weights are read once).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ uint4 lds128(const void* p) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -92,65 +106,58 @@ __device__ __forceinline__ float2 lds64f(const void* p) {
   return v;
 }
 
-template <int MT>
-struct W4A16Smem {
-  uint8_t ring[kWarps][kStages][kStageBytes];
-  uint64_t full[kWarps][kStages];
-  float red[2][kWarps][MT][32][4];
-  int abort_flag, never;
-  float xsum[1];   // [G][8 MT]: sum of X over each group of 64 k, per activation column
-};
+constexpr int kPairs = kWarps / 2;
 
+// Shared memory: the warps' chunk rings, the second warp's partial sums per
+// pair (double-buffered by tile parity) and the per-group activation sums.
 template <int MT>
-size_t w4a16_smem_bytes(int G) {
-  return offsetof(W4A16Smem<MT>, xsum) + sizeof(float) * (size_t)G * 8 * MT;
+__host__ __device__ inline size_t smem_bytes(int G) {
+  return (size_t)kWarps * kRing * kChunkBytes +
+         sizeof(float) * ((size_t)kPairs * 2 * MT * 32 * 4 + (size_t)G * 8 * MT);
 }
 
 // MT = number of 8-row activation tiles in this pass (1: M <= 8, 2: M <= 16).
-// Persistent: CTA c takes weight tiles c, c + gridDim.x, ...; each warp's ring
-// streams its group range of one tile after the other, so the next tile's
-// weights are in flight while this one is reduced.
 template <int MT>
-__global__ void __launch_bounds__(kWarps * 32, MT == 1 ? 4 : 3) w4a16_kernel(W4A16Params p, int m0) {
+__global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m0) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  W4A16Smem<MT>& sm = *reinterpret_cast<W4A16Smem<MT>*>(smem_raw);
+  const int K = p.K, G = K >> 6;
+  uint8_t* ring = smem_raw + (size_t)(threadIdx.x >> 5) * kRing * kChunkBytes;   // this warp's chunk slots
+  float* red = reinterpret_cast<float*>(smem_raw + (size_t)kWarps * kRing * kChunkBytes);   // [kPairs][2][MT][32][4]
+  float* xsum = red + (size_t)kPairs * 2 * MT * 32 * 4;                    // [G][8 MT]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int K = p.K, G = K >> 6;
   const int ntiles = (p.N + kRows - 1) / kRows;
-  const int my_tiles = (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-  const int gb = warp * G / kWarps, ge = (warp + 1) * G / kWarps;   // this warp's groups in every tile
-  const int ng = ge - gb, st_per_tile = (ng + kStageGroups - 1) / kStageGroups;
-  const int nst = my_tiles * st_per_tile;
+  const int pair = warp >> 1, half = warp & 1;
+  const int gpair = (int)blockIdx.x * kPairs + pair, npairs = (int)gridDim.x * kPairs;
+  const int my_tiles = gpair < ntiles ? (ntiles - gpair + npairs - 1) / npairs : 0;
+  const int gb = half * G / 2, ge = (half + 1) * G / 2;             // this warp's groups in every tile
+  const int ng = ge - gb, nchunks = (ng + kChunk - 1) / kChunk;
 
-  // Producer state (lane 0): the next stage to issue as (tile of this CTA, stage in tile, ring slot).
-  int issued = 0, p_lt = 0, p_si = 0, p_slot = 0;
-  auto issue_next = [&]() {
-    const int ngr = min(kStageGroups, ng - p_si * kStageGroups);
-    const size_t tile = (size_t)blockIdx.x + (size_t)p_lt * gridDim.x;
-    const uint8_t* src = p.wt + (tile * G + gb + (size_t)p_si * kStageGroups) * kGroupBytes;
-    mbar_arrive_expect_tx(&sm.full[warp][p_slot], (uint32_t)ngr * kGroupBytes);
-    bulk_load(sm.ring[warp][p_slot], src, (uint32_t)ngr * kGroupBytes, &sm.full[warp][p_slot]);
-    ++issued;
-    if (++p_si == st_per_tile) {
-      p_si = 0;
-      ++p_lt;
+  // Chunk i of this warp's sequence = (tile i / nchunks, chunk i % nchunks): up to
+  // kChunk groups, copied into ring slot i % kRing.  One commit group per chunk
+  // index (empty past the end), so wait_group counts stay uniform.
+  const int nseq = my_tiles * nchunks;
+  auto issue_chunk = [&](int i) {
+    if (i < nseq) {
+      const int lt = i / nchunks, c = i - lt * nchunks;
+      const size_t tile = (size_t)gpair + (size_t)lt * npairs;
+      const uint8_t* src = p.wt + (tile * G + gb + (size_t)c * kChunk) * kGroupBytes;
+      uint8_t* dst = ring + (size_t)(i % kRing) * kChunkBytes;
+      const int n = min(kChunk, ng - c * kChunk);
+      for (int j = 0; j < n; ++j) {
+        cp_async16(dst + j * kGroupBytes + lane * 16, src + (size_t)j * kGroupBytes + lane * 16);
+        if (lane < 2) cp_async16(dst + j * kGroupBytes + 512 + lane * 16, src + (size_t)j * kGroupBytes + 512 + lane * 16);
+      }
     }
-    if (++p_slot == kStages) p_slot = 0;
+    cp_async_commit();
   };
+  // the first chunks in flight while the activation sums are formed
+#pragma unroll
+  for (int i = 0; i < kRing - 1; ++i) issue_chunk(i);
 
-  if (threadIdx.x == 0) {
-    sm.abort_flag = 0;
-    sm.never = 0;
-  }
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[warp][s], 1);
-    fence_mbar_init();
-    while (issued < nst && issued < kStages) issue_next();
-  }
-  // Activation sums per (group, column) while the first weights stream in.
-  for (int i = threadIdx.x; i < G * 8 * MT; i += kWarps * 32) {
+  // Activation sums per (group, column).
+  for (int i = threadIdx.x; i < G * 8 * MT; i += kThreads) {
     const int gi = i / (8 * MT), c = i % (8 * MT), m = m0 + c;
     float sum = 0.f;
     if (m < p.M) {
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(kWarps * 32, MT == 1 ? 4 : 3) w4a16_kernel(W4A
         for (int e = 0; e < 4; ++e) sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
       }
     }
-    sm.xsum[i] = sum;
+    xsum[i] = sum;
   }
   __syncthreads();
 
@@ -192,131 +199,93 @@ __global__ void __launch_bounds__(kWarps * 32, MT == 1 ? 4 : 3) w4a16_kernel(W4A
     }
   };
 
-  bool aborted = false;
-  int consumed = 0, slot = 0;
-  uint32_t phase = 0;
   for (int lt = 0; lt < my_tiles; ++lt) {
-    const int tile = (int)blockIdx.x + lt * (int)gridDim.x;
+    const int tile = gpair + lt * npairs;
     float acc[MT][4];
 #pragma unroll
     for (int t = 0; t < MT; ++t)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[t][j] = 0.f;
-
-    int gi0 = gb;
-    for (int si = 0; si < st_per_tile && !aborted; ++si, gi0 += kStageGroups) {
-      const int n_here = min(kStageGroups, ge - gi0);
-      uint32_t P[MT][8];
-      load_x(gi0, P);   // in flight during the wait
-      const bool ok = mbar_wait(&sm.full[warp][slot], phase, &sm.abort_flag, p.budget_ns);
-      if (!__all_sync(0xffffffffu, ok)) {
-        aborted = true;
-        if (lane == 0) {
-          sm.abort_flag = 1;
-          atomicExch(p.err, 1);
-        }
-        break;
-      }
-      uint4 cw[kStageGroups];
-      uint32_t sw[kStageGroups];
+    for (int c = 0; c < nchunks; ++c) {
+      const int i = lt * nchunks + c;
+      issue_chunk(i + kRing - 1);                    // keeps kRing - 1 chunks in flight
+      cp_async_wait<kRing - 1>();                    // chunk i has landed (this lane's copies)
+      __syncwarp();                                  // ... and every lane's
+      const uint8_t* slot = ring + (size_t)(i % kRing) * kChunkBytes;
+      const int n = min(kChunk, ng - c * kChunk);
 #pragma unroll
-      for (int j = 0; j < kStageGroups; ++j) {
-        if (j < n_here) {
-          cw[j] = lds128(sm.ring[warp][slot] + j * kGroupBytes + lane * 16);
-          sw[j] = lds32(sm.ring[warp][slot] + j * kGroupBytes + 512 + g * 4);
-        }
-      }
-      __syncwarp();
-      if (lane == 0 && issued < nst) {   // refill this slot
-        fence_async_shared();
-        issue_next();
-      }
-      ++consumed;
-      if (++slot == kStages) {
-        slot = 0;
-        phase ^= 1u;
-      }
+      for (int j = 0; j < kChunk; ++j) {
+        if (j < n) {
+          const int gi = gb + c * kChunk + j;
+          uint32_t P[MT][8];
+          load_x(gi, P);
+          const uint4 cw = lds128(slot + j * kGroupBytes + lane * 16);
+          const uint32_t swj = lds32(slot + j * kGroupBytes + 512 + g * 4);
+          // the four MMA steps of a group accumulate into independent fragments
+          // (the tensor-core MMA has a long latency: no chain between them)
+          float pst[4][MT][4];
 #pragma unroll
-      for (int j = 0; j < kStageGroups; ++j) {
-        if (j >= n_here) break;
-        uint32_t Pn[MT][8];
-        if (j + 1 < n_here) load_x(gi0 + j + 1, Pn);   // next group's activations
-        // start from -136 * sum(x) so the biased codes (c + 136) give sum(x c)
-        float part[MT][4];
+          for (int st = 0; st < 4; ++st)
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          const float2 xs = lds64f(&sm.xsum[(gi0 + j) * 8 * MT + 8 * t + 2 * q]);
-          part[t][0] = -136.f * xs.x;
-          part[t][1] = -136.f * xs.y;
-          part[t][2] = -136.f * xs.x;
-          part[t][3] = -136.f * xs.y;
-        }
+            for (int t = 0; t < MT; ++t)
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          // MMA step s: positions (2q, 2q+1) <- codes 4s, 4s+1 and (2q+8, 2q+9) <- 4s+2, 4s+3
-          // of this thread's 16; those are pairs 2(s&1) and 2(s&1)+1 of word s>>1.
-          const uint32_t wa = (s < 2) ? cw[j].x : cw[j].y;   // row g
-          const uint32_t wb = (s < 2) ? cw[j].z : cw[j].w;   // row g + 8
-          const int sh = 8 * (s & 1);
-          const uint32_t a[4] = {codes_pair(wa >> sh), codes_pair(wb >> sh), codes_pair(wa >> (sh + 4)),
-                                 codes_pair(wb >> (sh + 4))};
+              for (int e = 0; e < 4; ++e) pst[st][t][e] = 0.f;
 #pragma unroll
-          for (int t = 0; t < MT; ++t) mma_bf16_16816(part[t], a, P[t][2 * s], P[t][2 * s + 1]);
-        }
-        const float s0 = __uint_as_float(sw[j] << 16), s1 = __uint_as_float(sw[j] & 0xFFFF0000u);
+          for (int st = 0; st < 4; ++st) {
+            // MMA step st: positions (2q, 2q+1) <- codes 4st, 4st+1 and (2q+8, 2q+9) <- 4st+2, 4st+3
+            // of this thread's 16; those are pairs 2(st&1) and 2(st&1)+1 of word st>>1.
+            const uint32_t wa = (st < 2) ? cw.x : cw.y;   // row g
+            const uint32_t wb = (st < 2) ? cw.z : cw.w;   // row g + 8
+            const int sh = 8 * (st & 1);
+            const uint32_t a[4] = {codes_pair(wa >> sh), codes_pair(wb >> sh), codes_pair(wa >> (sh + 4)),
+                                   codes_pair(wb >> (sh + 4))};
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          acc[t][0] = fmaf(s0, part[t][0], acc[t][0]);
-          acc[t][1] = fmaf(s0, part[t][1], acc[t][1]);
-          acc[t][2] = fmaf(s1, part[t][2], acc[t][2]);
-          acc[t][3] = fmaf(s1, part[t][3], acc[t][3]);
-        }
-        if (j + 1 < n_here) {
+            for (int t = 0; t < MT; ++t) mma_bf16_16816(pst[st][t], a, P[t][2 * st], P[t][2 * st + 1]);
+          }
+          const float s0 = __uint_as_float(swj << 16), s1 = __uint_as_float(swj & 0xFFFF0000u);
 #pragma unroll
-          for (int t = 0; t < MT; ++t)
+          for (int t = 0; t < MT; ++t) {
+            // sum the steps, minus 136 * sum(x): the biased codes (c + 136) give sum(x c)
+            const float2 xs = lds64f(&xsum[gi * 8 * MT + 8 * t + 2 * q]);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) P[t][i] = Pn[t][i];
+            for (int e = 0; e < 4; ++e) {
+              const float part =
+                  ((pst[0][t][e] + pst[1][t][e]) + (pst[2][t][e] + pst[3][t][e])) - 136.f * ((e & 1) ? xs.y : xs.x);
+              acc[t][e] = fmaf((e & 2) ? s1 : s0, part, acc[t][e]);
+            }
+          }
         }
       }
+      __syncwarp();                                  // every lane is done with the slot before it is refilled
     }
-
-    // split-K reduction of this tile over the 8 warps (double-buffered by tile parity)
+    // the pair's split-K reduction (double-buffered by tile parity): the second
+    // warp hands its partials over, the first adds and stores; fragment element
+    // e is (row g + 8 (e>>1), column 2q + (e&1)) of activation tile t
+    float* r = red + ((size_t)pair * 2 + (lt & 1)) * MT * 32 * 4;
+    if (half == 1) {
 #pragma unroll
-    for (int t = 0; t < MT; ++t)
+      for (int t = 0; t < MT; ++t)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sm.red[lt & 1][warp][t][lane][j] = acc[t][j];
-    __syncthreads();
-    // warp t finishes activation tile t: fragment element j is (row g + 8 (j>>1), column 2q + (j&1))
-    if (warp < MT && !sm.abort_flag) {
-      const int t = warp;
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] += sm.red[lt & 1][w][t][lane][j];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int n = tile * kRows + g + ((j & 2) ? 8 : 0);
-        const int m = m0 + 8 * t + 2 * q + (j & 1);
-        if (n < p.N && m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v[j] + p.bias[n]);
-      }
+        for (int e = 0; e < 4; ++e) r[(t * 32 + lane) * 4 + e] = acc[t][e];
     }
-  }
-  // After an abort, let this warp's copies still in flight land before the CTA exits.
-  if (lane == 0) {
-    for (; consumed < issued; ++consumed) {
-      mbar_wait(&sm.full[warp][slot], phase, &sm.never, p.budget_ns);
-      if (++slot == kStages) {
-        slot = 0;
-        phase ^= 1u;
-      }
+    named_barrier(1 + pair, 64);
+    if (half == 0) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int n = tile * kRows + g + ((e & 2) ? 8 : 0);
+          const int m = m0 + 8 * t + 2 * q + (e & 1);
+          const float v = acc[t][e] + r[(t * 32 + lane) * 4 + e];
+          if (n < p.N && m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v + p.bias[n]);
+        }
     }
   }
 }
 
 }  // namespace
 
-bool w4a16_supported(int K) { return w4a16_smem_bytes<2>(K / 64) <= 200u * 1024u; }
+bool w4a16_supported(int K) { return smem_bytes<2>(K / 64) <= (size_t)kSmemBudget; }
 
 size_t w4a16_packed_bytes(int N, int K) {
   return (size_t)((N + kRows - 1) / kRows) * (size_t)(K / 64) * kGroupBytes;
@@ -354,12 +323,12 @@ void w4a16_pack(const uint8_t* codes, const uint16_t* scales, int N, int K, uint
 
 namespace {
 
-// Blocks per SM for this kernel at `smem` bytes, cached per device.
+// Grid size (one CTA per SM), configured once per device and shared-memory size.
 template <int MT>
 cudaError_t grid_size(size_t smem, int ntiles, int* grid) {
   struct Entry {
     size_t smem = 0;
-    int sms = 0, per_sm = 0;
+    int sms = 0;
   };
   static Entry cache[64];
   static std::mutex mu;
@@ -369,29 +338,25 @@ cudaError_t grid_size(size_t smem, int ntiles, int* grid) {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   Entry& c = cache[dev];
-  if (c.smem != smem) {
+  if (c.smem < smem) {
     if ((e = cudaFuncSetAttribute(w4a16_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
         cudaSuccess)
       return e;
     if ((e = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c.per_sm, w4a16_kernel<MT>, kWarps * 32, smem)) !=
-        cudaSuccess)
-      return e;
-    if (c.per_sm < 1) return cudaErrorInvalidConfiguration;
     c.smem = smem;
   }
-  *grid = std::min(ntiles, c.sms * c.per_sm);
+  *grid = std::min((ntiles + kPairs - 1) / kPairs, c.sms);
   return cudaSuccess;
 }
 
 template <int MT>
 cudaError_t launch_pass(const W4A16Params& p, int m0, cudaStream_t stream) {
-  const int G = p.K / 64, ntiles = (p.N + kRows - 1) / kRows;
-  const size_t smem = w4a16_smem_bytes<MT>(G);
+  const int ntiles = (p.N + kRows - 1) / kRows;
+  const size_t smem = smem_bytes<MT>(p.K / 64);
   int grid = 0;
   cudaError_t e = grid_size<MT>(smem, ntiles, &grid);
   if (e != cudaSuccess) return e;
-  w4a16_kernel<MT><<<grid, kWarps * 32, smem, stream>>>(p, m0);
+  w4a16_kernel<MT><<<grid, kThreads, smem, stream>>>(p, m0);
   return cudaGetLastError();
 }
 
