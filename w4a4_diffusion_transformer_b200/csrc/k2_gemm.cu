@@ -23,11 +23,14 @@
 //              tile and the L2b^T tile (TMA, 64-byte swizzle).
 //   warp 1     allocates TMEM (512 columns: accumulator 256 + per-stage scale
 //              factors) and issues tcgen05.mma.
-//   warp 10    copies each stage's scale factors into TMEM (tcgen05.cp) as soon
-//              as they land: they complete their own barrier and are loaded
-//              before the operand tiles, so the copies run while the tiles are
-//              still in flight instead of between a stage's arrival and its MMAs.
-//   warps 2-9  epilogue, two warps per TMEM lane quarter (32 rows), each owning
+//   warps 4-7  move each stage's scale factors into TMEM as soon as they land
+//              (they complete their own barrier and are loaded before the
+//              operand tiles): each warp reads them from shared memory and
+//              writes its TMEM lane quarter with tcgen05.st.  Issued as
+//              tcgen05.cp copies instead, they would share the tensor pipe with
+//              the MMAs, and 12 copies per stage cost about as much pipe time as
+//              two thirds of the stage's MMAs (the copy path stays selectable).
+//   warps 8-15 epilogue, two warps per TMEM lane quarter (32 rows), each owning
 //              128 of the 256 columns: tcgen05.ld in 32-column chunks (the next
 //              chunk's load overlaps the current chunk's math), alpha, bias
 //              (staged in shared memory while the mainloop runs), GELU, BF16,
@@ -54,8 +57,14 @@ constexpr int kBN = 256;
 #ifndef SVDQ_K2_KB
 #define SVDQ_K2_KB 4
 #endif
+// Epilogue output path: BF16 rows stored from registers straight to global
+// memory (1), or staged in shared memory and written by TMA stores (0).  The
+// direct path frees the staging buffers, which makes room for a fourth stage.
+#ifndef SVDQ_K2_DIRECT_STORE
+#define SVDQ_K2_DIRECT_STORE 0
+#endif
 #ifndef SVDQ_K2_STAGES
-#define SVDQ_K2_STAGES 3
+#define SVDQ_K2_STAGES (SVDQ_K2_DIRECT_STORE ? 4 : 3)
 #endif
 // Epilogue drains its 128 accumulator columns into registers before any math (1),
 // or loads them chunk by chunk, overlapping each load with the previous chunk's math (0).
@@ -69,11 +78,31 @@ constexpr int kStages = SVDQ_K2_STAGES;
 constexpr uint32_t kSwz = kKB == 4 ? 2u : 4u;          // descriptor layout: 128B or 64B swizzle
 constexpr uint32_t kSwzAtom = 8u * kBKBytes;           // bytes between 8-row groups
 static_assert(kKB == 2 || kKB == 4, "stage shape");
+// Scale factors reach TMEM either through tcgen05.cp issued by one warp (0),
+// or from registers: four warps, one per TMEM lane quarter, read them from
+// shared memory and write them with tcgen05.st (1).  A copy occupies the
+// tensor pipe that the MMAs need; the register path keeps it for the MMAs.
+#ifndef SVDQ_K2_SF_REGS
+#define SVDQ_K2_SF_REGS 1
+#endif
+constexpr bool kSfRegs = SVDQ_K2_SF_REGS != 0;
 constexpr int kEpiWarps = 8;
-constexpr int kCpWarpIdx = 2 + kEpiWarps;
-constexpr int kThreads = (3 + kEpiWarps) * 32;
+// warp roles: 0 producer, 1 MMA issuer; register path: 4-7 scale factors,
+// 8-15 epilogue (2-3 idle); copy path: 2-9 epilogue, 10 scale factors
+constexpr int kEpiWarp0 = kSfRegs ? 8 : 2;
+constexpr int kSfWarp0 = kSfRegs ? 4 : 2 + kEpiWarps;
+constexpr int kThreads = (kSfRegs ? 16 : 3 + kEpiWarps) * 32;
+// Register split of the register path (per thread, by warpgroup): producer and
+// MMA warpgroup, scale-factor warpgroup, the two epilogue warpgroups.  The sum
+// over the block equals the launch allocation of 128 per thread, which the
+// host checks before the first launch (a larger sum would make the increase
+// wait forever).
+constexpr int kRegsCtl = 56, kRegsSf = 72, kRegsEpi = 192;
+static_assert(128 * kRegsCtl + 128 * kRegsSf + 256 * kRegsEpi == 512 * 128, "register split");
 constexpr int kEpiBufBytes = 32 * 64;        // one 32 x 32 BF16 output chunk
-constexpr int kEpiWarpBytes = 2 * kEpiBufBytes + 512;   // two chunk buffers + 128 bias floats
+constexpr bool kDirectStore = SVDQ_K2_DIRECT_STORE != 0;
+// per epilogue warp: two chunk buffers (TMA store path only) + 128 bias floats
+constexpr int kEpiWarpBytes = (kDirectStore ? 0 : 2 * kEpiBufBytes) + 512;
 constexpr int kABytes = kBM * kBKBytes;      // 16 KiB
 constexpr int kBBytes = kBN * kBKBytes;      // 32 KiB
 constexpr int kSFABytes = kKB * 512;         // kKB K-blocks x 128 rows
@@ -135,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::mbar_init(acc_full, 1);
     dev::mbar_init(acc_empty, kEpiWarps);
     dev::mbar_init(drain, 1);
-    for (int st = 0; st < kStages; ++st) dev::mbar_init(&sf_ready[st], 1);
+    for (int st = 0; st < kStages; ++st) dev::mbar_init(&sf_ready[st], kSfRegs ? 4 : 1);
     dev::mbar_init(cp_drain, 1);
     *abort_flag = 0;
     dev::fence_mbar_init();
@@ -150,8 +179,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   dev::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // (register path) each role sets its warpgroup's register budget first
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    if (kSfRegs) dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
       if (p.branch) {
         dev::tma_prefetch_desc(&tm_xl);
@@ -224,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    if (kSfRegs) dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
       const uint32_t idesc_f4 = dev::idesc_nvfp4(kBM, kBN);
       const uint32_t idesc_h = dev::idesc_bf16(kBM, kBN);
@@ -297,7 +329,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tc_commit(drain);
       dev::mbar_wait(drain, 0, abort_flag, p.budget_ns);
     }
-  } else if (warp == kCpWarpIdx) {
+  } else if (kSfRegs && warp >= kSfWarp0 && warp < kSfWarp0 + 4) {
+    // ------------------------------------------------------------ scale factors, register path
+    // Warp w writes TMEM lanes 32 (w % 4) .. +31.  The layout is the one the
+    // 32x128b.warpx4 copy produces: lane 32 q + u holds, per 64-K block j, the
+    // 16-byte unit u of A's 512-byte chunk in columns 4 j .. 4 j + 3 of the A
+    // region, and unit u of B's two chunks (rows 0-127, 128-255) in columns
+    // 8 j .. 8 j + 7 of the B region.
+    dev::setmaxnreg_dec<kRegsSf>();
+    const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      if (p.branch) ++it;
+      for (int kt = 0; kt < ktiles; ++kt, ++it) {
+        const int st = it % kStages;
+        const bool got = dev::mbar_wait(&sf_full[st], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) record_error(p.err, abort_flag, 0x208);
+          ok = false;
+          break;
+        }
+        const uint8_t* sfa = smem + st * kStageBytes + kABytes + kBBytes;
+        const uint8_t* sfb = sfa + kSFABytes;
+        uint32_t ra[16], rb[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // blocks past the K tail hold stale bytes that no MMA reads
+          const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j + lane * 16);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + kKB * 512 + 512 * j + lane * 16);
+          ra[4 * j + 0] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+          rb[8 * j + 0] = b0.x; rb[8 * j + 1] = b0.y; rb[8 * j + 2] = b0.z; rb[8 * j + 3] = b0.w;
+          rb[8 * j + 4] = b1.x; rb[8 * j + 5] = b1.y; rb[8 * j + 6] = b1.z; rb[8 * j + 7] = b1.w;
+        }
+        const uint32_t tsfa = tmem + kSFCol0 + st * kSFStageCols;
+        dev::tmem_store_16cols(tsfa + lanebase, ra);
+        dev::tmem_store_32cols(tsfa + 4 * kKB + lanebase, rb);
+        dev::tmem_store_wait();
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(&sf_ready[st]);
+      }
+    }
+  } else if (!kSfRegs && warp == kSfWarp0) {
     // ------------------------------------------------------------ scale-factor copier
     if (lane == 0) {
       int it = 0;
@@ -329,13 +404,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tc_commit(cp_drain);
       dev::mbar_wait(cp_drain, 0, abort_flag, p.budget_ns);
     }
-  } else {
+  } else if (kSfRegs && warp < kSfWarp0) {
+    dev::setmaxnreg_dec<kRegsCtl>();                 // idle warps of the first warpgroup
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
+    if (kSfRegs) dev::setmaxnreg_inc<kRegsEpi>();
     const int q = warp & 3;                          // TMEM lane quarter of this warp
-    const int half = (warp - 2) >> 2;                // which 128 of the 256 columns
-    uint8_t* wbuf = epi_buf + (warp - 2) * kEpiWarpBytes;
-    float* bias_s = reinterpret_cast<float*>(wbuf + 2 * kEpiBufBytes);
-    if (lane == 0) dev::tma_prefetch_desc(&tm_y);
+    const int half = (warp - kEpiWarp0) >> 2;       // which 128 of the 256 columns
+    uint8_t* wbuf = epi_buf + (warp - kEpiWarp0) * kEpiWarpBytes;
+    float* bias_s = reinterpret_cast<float*>(wbuf + (kDirectStore ? 0 : 2 * kEpiBufBytes));
+    if (!kDirectStore && lane == 0) dev::tma_prefetch_desc(&tm_y);
     int tcount = 0, chunk = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
       const int m0 = (tile % tiles_m) * kBM;
@@ -379,9 +457,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t (&nxt)[32] = (c & 1) ? va : vb;
         if (!kFastDrain && c + 1 < 4) dev::tmem_load_32cols(taddr + (uint32_t)((c + 1) * 32), nxt);
         // the buffer of this chunk was last read by the store issued two chunks ago
-        if (lane == 0) dev::bulk_wait_group_read<1>();
-        __syncwarp();
+        if (!kDirectStore) {
+          if (lane == 0) dev::bulk_wait_group_read<1>();
+          __syncwarp();
+        }
         uint8_t* buf = wbuf + (chunk & 1) * kEpiBufBytes;
+        const int row = m0 + q * 32 + lane;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t packed[4];
@@ -397,15 +478,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
             packed[e] = *reinterpret_cast<const uint32_t*>(&h2);
           }
-          // 64-byte swizzle: 16-byte chunk j of row `lane` sits at j ^ ((lane >> 1) & 3)
-          *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          if (kDirectStore) {
+            // 8 columns per 16-byte store; N is a multiple of 16, so a store
+            // that starts inside the row ends inside it
+            const int col = n0 + c * 32 + j * 8;
+            if (row < M && col < N)
+              *reinterpret_cast<uint4*>(p.y + (size_t)row * (size_t)N + col) =
+                  make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          } else {
+            // 64-byte swizzle: 16-byte chunk j of row `lane` sits at j ^ ((lane >> 1) & 3)
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          }
         }
-        dev::fence_async_shared();                    // make the writes visible to the TMA engine
-        __syncwarp();
-        if (lane == 0) {
-          dev::tma_store_2d(&tm_y, buf, n0 + c * 32, m0 + q * 32);
-          dev::bulk_commit_group();
+        if (!kDirectStore) {
+          dev::fence_async_shared();                  // make the writes visible to the TMA engine
+          __syncwarp();
+          if (lane == 0) {
+            dev::tma_store_2d(&tm_y, buf, n0 + c * 32, m0 + q * 32);
+            dev::bulk_commit_group();
+          }
         }
         if (!kFastDrain && c + 1 < 4) dev::tmem_load_wait(nxt);
         if (!kFastDrain && c == 2) {
@@ -417,9 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
-    if (lane == 0) dev::bulk_wait_group_all();
+    if (!kDirectStore && lane == 0) dev::bulk_wait_group_all();
   }
 
+  __syncwarp();                                      // single-lane roles rejoin their warps first
   dev::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -441,6 +534,13 @@ cudaError_t launch_k2(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const 
   if (configured_device != dev) {
     cudaError_t e = cudaFuncSetAttribute(k2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
+    if (kSfRegs) {
+      // the warpgroups' register budgets add up to exactly 128 per thread
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, k2_kernel);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs != 128) return cudaErrorInvalidConfiguration;
+    }
     configured_device = dev;
   }
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
