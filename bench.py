@@ -4,16 +4,21 @@ One step = one pass of the whole hot path over one batch: the fused
 down-projection + quantize kernel (K1) and the NVFP4 GEMM with the fused
 up-projection + bias epilogue (K2), on the FLUX.1-shaped attention output
 projection (M = 4608 tokens, K = N = 3072, rank 32, NVFP4 g16/E4M3), inputs
-resident in HBM, L2 flushed between steps outside the timed events (a 256 MiB
-write, then a read of the same buffer so that no dirty lines of the flush are
-left for the timed kernels to write back).  The value is whole-job TFLOP/s of
-the layer's algorithmic work 2MNK + 2M*32*(K+N), device-timed with one pair of
-CUDA events around each step on the launch stream (K1 and K2 back to back, as a
-caller runs them), max over ranks.  The per-kernel durations behind the
-roofline fractions are timed after the steps, each kernel alone between its own
-events.  The JSON line also carries the other rows of the hot path on their
-FLUX.1-shaped layers (INT4 QKV, the fc1 -> GELU -> fc2 pair, the W4A16
-adaptive-norm GEMV) under "other_layers".
+resident in HBM.  Steps run back to back, as the layers of a transformer do,
+and cycle through six independent sets of inputs, outputs, workspaces and
+prepared weights of about 70 MB each: 420 MB, more than the 126 MB L2, so
+every step reads its data from HBM, not from a cache warmed by the step before.
+The value is whole-job TFLOP/s of the layer's algorithmic work
+2MNK + 2M*32*(K+N), device-timed with one pair of CUDA events around the timed
+steps on the launch stream (K1 and K2 back to back per step, as a caller runs
+them), max over ranks.  The per-kernel durations behind the roofline fractions
+are timed the same way after the steps, each kernel alone over the rotating
+sets.  "isolated" repeats the layer and kernel timings one launch at a time
+between its own events after an L2 flush (a 256 MiB write, then a read of the
+same buffer), which adds the launch latency of every launch.  The JSON line
+also carries the other rows of the hot path on their FLUX.1-shaped layers
+(INT4 QKV, the fc1 -> GELU -> fc2 pair, the W4A16 adaptive-norm GEMV) under
+"other_layers", timed one launch at a time after an L2 flush.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -38,6 +43,7 @@ METRIC = "fused W4A4+rank-32 linear TFLOPS, % NVFP4 peak; µs/layer vs unfused"
 WORKLOAD = "attn_out"
 RANK = 32
 NOMINAL_FP4_DENSE_TFLOPS = 9000.0
+N_SETS = 6                   # rotating input sets, 6 x ~70 MB > L2
 FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 PF / 2.25 PF)
 
 
@@ -244,6 +250,20 @@ def time_events(stream, n, flush_l2, fn):
     return sum(a.elapsed_time(b) for a, b in evs) / n
 
 
+def time_rotating(stream, n, fn):
+    """Mean device time (ms) per call of fn(i), i = 0..n-1, run back to back
+    between one pair of CUDA events on `stream`."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(n):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
 def other_layers(pkg, syn, stream, flush_l2, n, peaks):
     """The other hot-path rows on their FLUX.1-shaped layers (not the headline):
     the INT4 variant (fused QKV 4608x3072->9216), the MLP pair (fc1 with the GELU
@@ -320,7 +340,7 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -347,17 +367,33 @@ def main():
     d = syn.layer(WORKLOAD)
     shp = d["shape"]
     M, K, N = shp.M, shp.K, shp.N
-    L = pkg.Layer.prepare(syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]), syn.bf16_bits(d["Xc"]),
-                          fmt="nvfp4", rank=RANK, device=dev)
     stream = torch.cuda.current_stream()
-    x = torch.from_numpy(d["X"]).to(torch.bfloat16).cuda()
-    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    wsb = L.workspace_bytes(M)
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
-    # the two kernels' intermediate buffers for the split (per-kernel timed) calls
-    codes = torch.empty(L.act_code_bytes(M), dtype=torch.uint8, device="cuda")
-    scales = torch.empty(L.act_scale_bytes(M), dtype=torch.uint8, device="cuda")
-    xl = torch.empty((M, RANK), dtype=torch.bfloat16, device="cuda")
+
+    class Set:
+        """One independent copy of the layer's data: prepared weights, X, Y,
+        the workspace of the one-call forward and the two kernels' buffers."""
+
+        def __init__(self):
+            self.L = pkg.Layer.prepare(syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]), syn.bf16_bits(d["Xc"]),
+                                       fmt="nvfp4", rank=RANK, device=dev)
+            self.x = torch.from_numpy(d["X"]).to(torch.bfloat16).cuda()
+            self.y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            self.wsb = self.L.workspace_bytes(M)
+            self.ws = torch.empty(self.wsb, dtype=torch.uint8, device="cuda")
+            self.codes = torch.empty(self.L.act_code_bytes(M), dtype=torch.uint8, device="cuda")
+            self.scales = torch.empty(self.L.act_scale_bytes(M), dtype=torch.uint8, device="cuda")
+            self.xl = torch.empty((M, RANK), dtype=torch.bfloat16, device="cuda")
+
+        def k1(self, mode=0):
+            self.L.quantize_act(self.x, M, self.codes, self.scales, self.xl, stream, mode)
+
+        def k2(self, flags=0):
+            self.L.gemm(self.codes, self.scales, self.xl, M, self.y, stream, flags)
+
+    sets = [Set() for _ in range(N_SETS)]
+    L, x, y, ws, wsb = sets[0].L, sets[0].x, sets[0].y, sets[0].ws, sets[0].wsb
+    set_bytes = (M * K * 2 + M * N * 2 + wsb + sets[0].codes.numel() + sets[0].scales.numel() +
+                 M * RANK * 2 + N * K // 2 + N * K // 16 + (K + N) * RANK * 2 + (K + N) * 4)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     flush_sink = torch.empty(1, dtype=torch.int64, device="cuda")
 
@@ -365,52 +401,60 @@ def main():
         flush.fill_(i & 0xFF)                                     # evict: write > L2
         torch.sum(flush.view(torch.int64), dim=0, keepdim=True, out=flush_sink)   # clean the lines
 
-    def step():
+    def step(i):
         # the layer as a caller runs it: K1 then K2 back to back on one stream (K2
         # is a programmatic dependent launch of K1: its prologue overlaps K1's tail)
-        L.quantize_act(x, M, codes, scales, xl, stream, 0)
-        L.gemm(codes, scales, xl, M, y, stream, 0)
+        st = sets[i % N_SETS]
+        st.k1()
+        st.k2()
 
     # ---- warm-up
-    for _ in range(args.warmup):
-        step()
-    L.forward(x, M, y, ws, wsb, stream, pkg.FWD_CHECK)
+    for i in range(max(args.warmup, N_SETS)):
+        step(i)
+    for st in sets:
+        st.L.forward(st.x, M, st.y, st.ws, st.wsb, stream, pkg.FWD_CHECK)
     torch.cuda.synchronize()
 
-    # ---- timed region: exactly `steps` steps, one event pair around each step
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    # ---- timed region: exactly `steps` steps back to back, one event pair around them
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
-        for i in range(args.steps):
-            flush_l2(i)
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
+        step_ms = time_rotating(stream, args.steps, step)
     barrier(world)
-    step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     step_ms_max = allreduce_max(step_ms, world)
     value = layer_flops(M, K, N) * world / (step_ms_max * 1e-3) / 1e12
-    L.check(stream)
+    for st in sets:
+        st.L.check(stream)
 
-    # ---- per-kernel durations (same launches, each bracketed by its own events)
+    # ---- per-kernel durations, each kernel alone over the rotating sets
     n_k = max(100, min(1000, args.steps))
-    k2_ms = time_events(stream, n_k, flush_l2, lambda: L.gemm(codes, scales, xl, M, y, stream, 0))
-    k1_ms = time_events(stream, n_k, flush_l2, lambda: L.quantize_act(x, M, codes, scales, xl, stream, 0))
+    k2_ms = time_rotating(stream, n_k, lambda i: sets[i % N_SETS].k2())
+    k1_ms = time_rotating(stream, n_k, lambda i: sets[i % N_SETS].k1())
 
     # ---- measurement variants: bare GEMM and unfused layer
     n_var = max(50, min(500, args.steps))
 
-    def bare():
-        L.quantize_act(x, M, codes, scales, xl, stream, 1)
-        L.gemm(codes, scales, xl, M, y, stream, pkg.FWD_NO_BRANCH)
+    def bare(i):
+        sets[i % N_SETS].k1(1)
+        sets[i % N_SETS].k2(pkg.FWD_NO_BRANCH)
 
-    bare_ms = time_events(stream, n_var, flush_l2, bare)
-    unfused_ms = time_events(stream, n_var, flush_l2, lambda: L.forward(x, M, y, ws, wsb, stream, pkg.FWD_UNFUSED))
-    L.quantize_act(x, M, codes, scales, xl, stream, 0)
-    bare_k2_ms = time_events(stream, n_var, flush_l2, lambda: L.gemm(codes, scales, xl, M, y, stream,
-                                                                      pkg.FWD_NO_BRANCH))
+    def unfused(i):
+        st = sets[i % N_SETS]
+        st.L.forward(st.x, M, st.y, st.ws, st.wsb, stream, pkg.FWD_UNFUSED)
+
+    bare_ms = time_rotating(stream, n_var, bare)
+    unfused_ms = time_rotating(stream, n_var, unfused)
+    for st in sets:
+        st.k1()
+    bare_k2_ms = time_rotating(stream, n_var, lambda i: sets[i % N_SETS].k2(pkg.FWD_NO_BRANCH))
+    for st in sets:
+        st.L.check(stream)
+
+    # ---- isolated launches: one event pair per launch after an L2 flush
+    n_iso = max(50, min(300, args.steps))
+    iso_layer_ms = time_events(stream, n_iso, flush_l2, lambda: step(0))
+    iso_k2_ms = time_events(stream, n_iso, flush_l2, lambda: sets[0].k2())
+    iso_k1_ms = time_events(stream, n_iso, flush_l2, lambda: sets[0].k1())
     L.check(stream)
 
     # ---- end to end through the public API with host buffers
@@ -434,7 +478,8 @@ def main():
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
         "config": {"workload": f"{WORKLOAD} {M}x{K}->{N} NVFP4 g16 E4M3 r{RANK}", "M": M, "K": K, "N": N,
                    "rank": RANK, "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "flushed between steps outside the timed events (256 MiB write + read)"},
+                   "l2": f"inputs larger than L2: steps back to back over {N_SETS} rotating sets of inputs, "
+                         f"outputs, workspaces and prepared weights ({N_SETS} x {set_bytes / 1e6:.0f} MB)"},
         "us_per_layer": step_ms_max * 1e3, "k1_us": k1_ms * 1e3, "k2_us": k2_ms * 1e3,
         "pct_nvfp4_peak": {"of_measured": value / world / fp4_peak, "of_nominal": value / world /
                            NOMINAL_FP4_DENSE_TFLOPS, "measured_peak_tflops": fp4_peak,
@@ -445,8 +490,8 @@ def main():
         "roofline": {"bound": "tensor", "kernel": "k2_gemm (NVFP4 block-scaled tcgen05 + fused up-proj)",
                      "achieved": k2_achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": k2_achieved / fp4_peak,
                      "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16:g}",
-                     "timing": "K2 alone between CUDA events on the launch stream, L2 flushed, "
-                               f"{n_k} launches after the timed steps",
+                     "timing": f"K2 alone, {n_k} launches back to back over the {N_SETS} rotating sets "
+                               "between one pair of CUDA events on the launch stream, after the timed steps",
                      "traffic": profile_traffic()},
         "k1_roofline": {"bound": "hbm", "achieved": k1_bytes / (k1_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                         "unit": "GB/s", "frac": k1_bytes / (k1_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -454,6 +499,8 @@ def main():
         "e2e": {"value": layer_flops(M, K, N) * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
                 "path": "svdq_linear_forward with pinned host X/Y, copies inside the timed events"},
+        "isolated": {"layer_us": iso_layer_ms * 1e3, "k1_us": iso_k1_ms * 1e3, "k2_us": iso_k2_ms * 1e3,
+                     "timing": "one launch (or one K1+K2 step) between its own CUDA events after an L2 flush"},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
@@ -461,7 +508,8 @@ def main():
         out["other_layers"] = other_layers(pkg, syn, stream, flush_l2, max(30, min(200, args.steps)), peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(d, M, K, N)
-    L.close()
+    for st in sets:
+        st.L.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
