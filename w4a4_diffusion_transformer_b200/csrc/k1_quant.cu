@@ -148,6 +148,11 @@ __global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
     // ------------------------------------------------------------ X producer
     if (lane == 0) {
       dev::tma_prefetch_desc(&tm_x);
+      // This kernel is itself a programmatic dependent launch: X may be the
+      // output of the preceding kernel, and that kernel may still read the
+      // buffers this one writes.  Every write here follows an X stage, so
+      // waiting before the first X load covers both.
+      dev::griddep_wait();
       int issued = 0;
       for (int it = 0; it < nk; ++it) {
         const int s = it % kXStages;
@@ -460,8 +465,18 @@ cudaError_t launch_k1_t(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const 
   }
   const int mpad = (p.M + 127) / 128 * 128;
   dim3 grid(mpad / kRows);
-  kern<<<grid, K1Shape<F>::threads, kSmemBytes, stream>>>(tm_x, tm_l, tm_c, p);
-  return cudaGetLastError();
+  // programmatic dependent launch: the prologue overlaps the preceding kernel's tail
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(K1Shape<F>::threads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l, tm_c, p);
 }
 
 }  // namespace

@@ -142,6 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int G = K >> 6;
 
   if (threadIdx.x == 0) {
+    // the next kernel on the stream may launch now; it waits for this grid's
+    // completion before it touches anything this grid reads or writes
+    dev::griddep_launch_dependents();
     for (int s = 0; s < kPStages; ++s) {
       dev::mbar_init(&pfull[s], 1);
       dev::mbar_init(&pempty[s], kConvWarps);
