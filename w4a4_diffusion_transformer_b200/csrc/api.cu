@@ -72,6 +72,23 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// BF16 matrix [rows][cols] seen as 64-column chunks: dimensions (64 columns,
+// rows, cols / 64 chunks), so that one box of (64, box_rows, 4) brings 4
+// consecutive chunks of box_rows rows, chunk-major, each chunk a [box_rows][128 B]
+// tile in the 128-byte swizzle: the layout four 2D boxes of (64, box_rows) give,
+// in one copy instead of four.  cols % 64 == 0.
+bool make_map_kchunks(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {64, rows, cols / 64};
+  const cuuint64_t strides[2] = {cols * 2, 128};
+  const cuuint32_t box[3] = {64, box_rows, 4};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ helpers
 
 struct DeviceGuard {
@@ -240,8 +257,7 @@ svdq_status upload_layer(svdq_layer* L, int device) {
                               CU_TENSOR_MAP_SWIZZLE_NONE)) &&
               make_map(&L->tm_l2s, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
                        CU_TENSOR_MAP_SWIZZLE_64B) &&
-              make_map(&L->tm_l1t, L->d_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, 32, 64, 32,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+              make_map_kchunks(&L->tm_l1t, L->d_l1t, K, 32, 32);
     if (!ok) return SVDQ_ECUDA;
   } else if (h.format == SVDQ_W4A16_INT4) {
     std::vector<uint8_t> packed(w4a16_packed_bytes(N, K));
@@ -284,7 +300,7 @@ svdq_status run_k1(const svdq_layer* L, const void* X, int M, void* codes, void*
                    cudaStream_t stream, int mode) {
   const HostPrep& h = L->host;
   CUtensorMap tm_x, tm_c;
-  if (!make_map(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.K, M, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map_kchunks(&tm_x, X, h.K, M, 32))
     return SVDQ_ECUDA;
   // activation codes are written in 32-row tiles, one per quantizer warp and stage:
   // 16 bytes wide for NVFP4 (32 columns), 32 bytes for INT4 (64 columns)

@@ -163,9 +163,10 @@ __global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
         uint8_t* st = smem + s * kXStageBytes;
         const int k0 = it * kBK;
         const int kvalid = min(kBK, K - k0);
-        const int nsub = kvalid >> 6;
-        dev::mbar_arrive_expect_tx(&xfull[s], (uint32_t)nsub * 4096u + (kQuant ? (uint32_t)kvalid * 4u : 0u));
-        for (int j = 0; j < nsub; ++j) dev::tma_load_2d(st + j * 4096, &tm_x, &xfull[s], k0 + 64 * j, row0);
+        // one box brings the stage's four 64-column sub-tiles (past K they
+        // are zero-filled, and no consumer reads them)
+        dev::mbar_arrive_expect_tx(&xfull[s], (uint32_t)kXBytes + (kQuant ? (uint32_t)kvalid * 4u : 0u));
+        dev::tma_load_3d(st, &tm_x, &xfull[s], 0, row0, k0 >> 6);
         if (kQuant) dev::bulk_load(st + kXBytes, p.inv_lam + k0, (uint32_t)kvalid * 4u, &xfull[s]);
         issued = it + 1;
       }
@@ -187,10 +188,8 @@ __global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
           break;
         }
         const int k0 = it * kBK;
-        const int nsub = min(kBK, K - k0) >> 6;
-        dev::mbar_arrive_expect_tx(&lfull[s], (uint32_t)nsub * 4096u);
-        for (int j = 0; j < nsub; ++j)
-          dev::tma_load_2d(lring + s * kLBytes + j * 4096, &tm_l, &lfull[s], k0 + 64 * j, 0);
+        dev::mbar_arrive_expect_tx(&lfull[s], (uint32_t)kLBytes);
+        dev::tma_load_3d(lring + s * kLBytes, &tm_l, &lfull[s], 0, 0, k0 >> 6);
         issued = it + 1;
       }
       for (int it = max(0, issued - kLStages); it < issued; ++it)

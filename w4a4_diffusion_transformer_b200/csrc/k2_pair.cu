@@ -50,8 +50,16 @@ constexpr int kBKBytes = kKB * 32;           // E2M1 bytes per operand row per s
 #endif
 constexpr int kStages = SVDQ_K2P_STAGES;
 constexpr int kEpiWarps = 8;
-constexpr int kCpWarpIdx = 2 + kEpiWarps;
-constexpr int kThreads = (3 + kEpiWarps) * 32;
+// warp roles: 0 producer, 1 MMA issuer (rank 0) or forwarder (rank 1), 2-3
+// idle, 4-7 scale factors (one per TMEM lane quarter), 8-15 epilogue
+constexpr int kSfWarp0 = 4;
+constexpr int kEpiWarp0 = 8;
+constexpr int kThreads = 16 * 32;
+// register budgets per thread by warpgroup (control, scale factors, two
+// epilogue warpgroups); they add up to the launch allocation of 128, which the
+// host checks before the first launch
+constexpr int kRegsCtl = 56, kRegsSf = 72, kRegsEpi = 192;
+static_assert(128 * kRegsCtl + 128 * kRegsSf + 256 * kRegsEpi == kThreads * 128, "register split");
 constexpr int kEpiBufBytes = 32 * 64;        // one 32 x 32 BF16 output chunk
 constexpr int kEpiWarpBytes = 2 * kEpiBufBytes;
 constexpr int kABytes = kBM * kBKBytes;      // 16 KiB
@@ -90,13 +98,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + kStages;
   uint64_t* sf_full = empty + kStages;         // this CTA's scale factors landed
   uint64_t* pfull = sf_full + kStages;         // rank 0: rank 1's stage data landed
-  uint64_t* psf_full = pfull + kStages;        // rank 0: rank 1's scale factors landed
-  uint64_t* sf_ready = psf_full + kStages;     // rank 0: a stage's scale factors are in both TMEMs
-  uint64_t* acc_full = sf_ready + kStages;
+  uint64_t* sf_ready = pfull + kStages;        // this CTA's scale factors of a stage are in its TMEM
+  uint64_t* psf_ready = sf_ready + kStages;    // rank 0: rank 1's scale factors are in rank 1's TMEM
+  uint64_t* acc_full = psf_ready + kStages;
   uint64_t* acc_empty = acc_full + 1;          // rank 0: both CTAs drained the accumulator
   uint64_t* drain = acc_empty + 1;
-  uint64_t* cp_drain = drain + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -120,13 +127,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(&empty[s], 1);
       dev::mbar_init(&sf_full[s], 1);
       dev::mbar_init(&pfull[s], 1);
-      dev::mbar_init(&psf_full[s], 1);
-      dev::mbar_init(&sf_ready[s], 1);
+      dev::mbar_init(&sf_ready[s], 4);          // this CTA's scale-factor warps
+      dev::mbar_init(&psf_ready[s], 1);
     }
     dev::mbar_init(acc_full, 1);
     dev::mbar_init(acc_empty, 2 * kEpiWarps);
     dev::mbar_init(drain, 1);
-    dev::mbar_init(cp_drain, 1);
     *abort_flag = 0;
     dev::fence_mbar_init();
   }
@@ -143,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
+    dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
       if (p.branch) {
         dev::tma_prefetch_desc(&tm_xl);
@@ -221,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && !leader) {
     // ------------------------------------------------------------ rank 1: forward "stage data landed"
+    dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
       const int uses = (num_tiles > pair_id ? (num_tiles - pair_id + npairs - 1) / npairs : 0) *
                        (ktiles + (p.branch ? 1 : 0));
@@ -233,22 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::mbar_arrive_remote(dev::map_to_rank(&pfull[s], 0));
       }
     }
-  } else if (warp == kCpWarpIdx && !leader) {
-    // ------------------------------------------------------------ rank 1: forward "scale factors landed"
-    if (lane == 0) {
-      const int uses = (num_tiles > pair_id ? (num_tiles - pair_id + npairs - 1) / npairs : 0) *
-                       (ktiles + (p.branch ? 1 : 0));
-      for (int it = 0; it < uses; ++it) {
-        const int s = it % kStages;
-        if (!dev::mbar_wait(&sf_full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
-          record_error(p.err, abort_flag, 0x224);
-          break;
-        }
-        dev::mbar_arrive_remote(dev::map_to_rank(&psf_full[s], 0));
-      }
-    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ rank 0: MMA issuer
+    dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
       const uint32_t idesc_f4 = dev::idesc_nvfp4(kPM, kBN);
       const uint32_t idesc_h = dev::idesc_bf16(kPM, kBN);
@@ -292,7 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int slot = kslot0 + kt;
           const int s = slot % kStages;
           if (!(ok = wait_data(slot, 0x227))) break;
-          if (!dev::mbar_wait(&sf_ready[s], (sf_phase >> s) & 1u, abort_flag, p.budget_ns)) {
+          if (!dev::mbar_wait(&sf_ready[s], (sf_phase >> s) & 1u, abort_flag, p.budget_ns) ||
+              !dev::mbar_wait_cluster(&psf_ready[s], (sf_phase >> s) & 1u, abort_flag, p.budget_ns)) {
             record_error(p.err, abort_flag, 0x228);
             ok = false;
             break;
@@ -319,46 +315,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tc_commit_pair(drain, kLeader);
       dev::mbar_wait(drain, 0, abort_flag, p.budget_ns);
     }
-  } else if (warp == kCpWarpIdx) {
-    // ------------------------------------------------------------ rank 0: scale-factor copies (both CTAs)
+  } else if (warp >= kSfWarp0 && warp < kSfWarp0 + 4) {
+    // ------------------------------------------------------------ scale factors (both CTAs)
+    // Warp w writes its CTA's TMEM lanes 32 (w % 4) .. +31 from registers
+    // (tcgen05.st), in the layout a 32x128b.warpx4 copy produces: per 64-K
+    // block j, unit `lane` of A's 512-byte chunk (this CTA's 128 rows) in
+    // columns 4 j .. 4 j + 3 of the A region, and of B's two chunks (all 256
+    // columns of the tile) in columns 8 j .. 8 j + 7 of the B region (rank 1's
+    // readiness reaches rank 0 through a forwarder).  The tensor pipe stays
+    // with the MMAs.
+    dev::setmaxnreg_dec<kRegsSf>();
+    const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
+    int it = 0;
+    bool ok = true;
+    for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
+      if (p.branch) ++it;
+      for (int kt = 0; kt < ktiles; ++kt, ++it) {
+        const int st = it % kStages;
+        const bool got = dev::mbar_wait(&sf_full[st], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) record_error(p.err, abort_flag, 0x229);
+          ok = false;
+          break;
+        }
+        const uint8_t* sfa = smem + st * kStageBytes + kABytes + kBBytes;
+        const uint8_t* sfb = sfa + kSFABytes;
+        uint32_t ra[16], rb[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // blocks past the K tail (and the A scales of rows past the
+          // activations' padding) hold stale bytes whose results are never used
+          const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j + lane * 16);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + kKB * 512 + 512 * j + lane * 16);
+          ra[4 * j + 0] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+          rb[8 * j + 0] = b0.x; rb[8 * j + 1] = b0.y; rb[8 * j + 2] = b0.z; rb[8 * j + 3] = b0.w;
+          rb[8 * j + 4] = b1.x; rb[8 * j + 5] = b1.y; rb[8 * j + 6] = b1.z; rb[8 * j + 7] = b1.w;
+        }
+        const uint32_t tsfa = tmem + kSFCol0 + st * kSFStageCols;
+        dev::tmem_store_16cols(tsfa + lanebase, ra);
+        dev::tmem_store_32cols(tsfa + 4 * kKB + lanebase, rb);
+        dev::tmem_store_wait();
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(&sf_ready[st]);
+      }
+    }
+  } else if (warp == 2 && !leader) {
+    // ------------------------------------------------------------ rank 1: forward "scale factors in TMEM"
+    dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
+      const uint32_t psf0 = dev::map_to_rank(psf_ready, 0);
+      uint32_t sf_phase = 0;                        // per-slot parity of sf_ready (k-stages only)
       int it = 0;
-      for (int tile = pair_id; tile < num_tiles; tile += npairs) {
-        bool ok = true;
-        if (p.branch) ++it;
+      bool ok = true;
+      for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
+        if (p.branch) ++it;                         // branch stages carry no scale factors
         for (int kt = 0; kt < ktiles; ++kt, ++it) {
-          const int st = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          if (!dev::mbar_wait(&sf_full[st], ph, abort_flag, p.budget_ns) ||
-              !dev::mbar_wait_cluster(&psf_full[st], ph, abort_flag, p.budget_ns)) {
-            record_error(p.err, abort_flag, 0x229);
+          const int s = it % kStages;
+          if (!dev::mbar_wait(&sf_ready[s], (sf_phase >> s) & 1u, abort_flag, p.budget_ns)) {
+            record_error(p.err, abort_flag, 0x22b);
             ok = false;
             break;
           }
+          sf_phase ^= 1u << s;
           dev::tc_fence_after();
-          const int nkb = min(kKB, kblocks - kKB * kt);
-          const uint32_t sfa0 = dev::smem_u32(smem + st * kStageBytes) + kABytes + kBBytes;
-          const uint32_t sfb0 = sfa0 + kSFABytes;
-          const uint32_t tsfa = tmem + kSFCol0 + st * kSFStageCols;
-          const uint32_t tsfb = tsfa + 4 * kKB;
-          for (int j = 0; j < nkb; ++j) {
-            dev::tmem_copy_32x128b_x4_pair(tsfa + 4 * j, dev::smem_desc(sfa0 + 512 * j, 0, 128, 0));
-            dev::tmem_copy_32x128b_x4_pair(tsfb + 8 * j, dev::smem_desc(sfb0 + 512 * j, 0, 128, 0));
-            dev::tmem_copy_32x128b_x4_pair(tsfb + 8 * j + 4,
-                                           dev::smem_desc(sfb0 + kKB * 512 + 512 * j, 0, 128, 0));
-          }
-          dev::tc_commit_pair(&sf_ready[st], kLeader);
+          dev::mbar_arrive_remote(psf0 + 8u * (uint32_t)s);
         }
-        if (!ok) break;
       }
-      dev::tc_commit_pair(cp_drain, kLeader);
-      dev::mbar_wait(cp_drain, 0, abort_flag, p.budget_ns);
     }
-  } else if (warp >= 2 && warp < 2 + kEpiWarps) {
+  } else if (warp >= 2 && warp < kSfWarp0) {
+    dev::setmaxnreg_dec<kRegsCtl>();                 // idle warps of the first warpgroup
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    dev::setmaxnreg_inc<kRegsEpi>();
     const int q = warp & 3;                          // TMEM lane quarter of this warp
-    const int half = (warp - 2) >> 2;                // which 128 of the 256 columns
-    uint8_t* wbuf = epi_buf + (warp - 2) * kEpiWarpBytes;
+    const int half = (warp - kEpiWarp0) >> 2;        // which 128 of the 256 columns
+    uint8_t* wbuf = epi_buf + (warp - kEpiWarp0) * kEpiWarpBytes;
     const uint32_t acc_empty_leader = dev::map_to_rank(acc_empty, 0);
     if (lane == 0) dev::tma_prefetch_desc(&tm_y);
     int tcount = 0, chunk = 0;
@@ -439,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Neither CTA leaves (nor frees TMEM) while the pair's operations may still
   // read its shared memory or write its TMEM.
+  __syncwarp();                                      // single-lane roles rejoin their warps first
   dev::tc_fence_before();
   __syncthreads();
   dev::cluster_sync();
@@ -461,6 +495,11 @@ cudaError_t launch_k2_pair(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, c
   if (configured_device != dev) {
     cudaError_t e = cudaFuncSetAttribute(k2_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
+    // the warpgroups' register budgets add up to exactly 128 per thread
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, k2_pair_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != 128) return cudaErrorInvalidConfiguration;
     configured_device = dev;
   }
   const int tiles = ((p.M + kPM - 1) / kPM) * ((p.N + kBN - 1) / kBN);
