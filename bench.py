@@ -264,6 +264,31 @@ def time_rotating(stream, n, fn):
     return a.elapsed_time(b) / n
 
 
+def library_nvfp4_gemm_us(M, K, N, n, n_sets=N_SETS):
+    """Context only: cuBLASLt's bare NVFP4 GEMM (no low-rank branch, no bias) at
+    the same shape through torch._scaled_mm, back to back over rotating operand
+    sets like the timed steps; None where this PyTorch build has no FP4 path."""
+    import torch
+    try:
+        dev = "cuda"
+        rup = lambda x, m: (x + m - 1) // m * m
+        g = torch.Generator(device=dev).manual_seed(7)
+        As = [torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+              .view(torch.float4_e2m1fn_x2) for _ in range(n_sets)]
+        Bs = [torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+              .view(torch.float4_e2m1fn_x2) for _ in range(n_sets)]
+        sa = torch.ones(rup(M, 128) * rup(K // 16, 4), device=dev).to(torch.float8_e4m3fn)
+        sb = torch.ones(rup(N, 128) * rup(K // 16, 4), device=dev).to(torch.float8_e4m3fn)
+        stream = torch.cuda.current_stream()
+        f = lambda i: torch._scaled_mm(As[i % n_sets], Bs[i % n_sets].t(), scale_a=sa, scale_b=sb,
+                                       out_dtype=torch.bfloat16)
+        for i in range(2 * n_sets):
+            f(i)
+        return time_rotating(stream, n, f) * 1e3
+    except Exception:
+        return None
+
+
 def other_layers(pkg, syn, stream, flush_l2, n, peaks):
     """The other hot-path rows on their FLUX.1-shaped layers (not the headline):
     the INT4 variant (fused QKV 4608x3072->9216), the MLP pair (fc1 with the GELU
@@ -506,6 +531,11 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_other_layers:
         out["other_layers"] = other_layers(pkg, syn, stream, flush_l2, max(30, min(200, args.steps)), peaks)
+        lib_us = library_nvfp4_gemm_us(M, K, N, n_k)
+        out["library_context"] = {
+            "cublaslt_nvfp4_gemm_us": lib_us, "k2_us": k2_ms * 1e3, "bare_k2_us": bare_k2_ms * 1e3,
+            "note": "bare NVFP4 GEMM of the same shape through torch._scaled_mm (no low-rank branch, no bias), "
+                    "back to back over rotating operand sets; context, not a baseline"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(d, M, K, N)
     for st in sets:

@@ -219,3 +219,38 @@ def test_attn_out_full_size_sampled_rows():
     yref = o.forward(p, X[rows])["Y_bf16"]
     assert_close_bf16(y[rows], yref, "attn_out sampled rows")
     assert np.all(np.isfinite(y))
+
+
+# ---------------------------------------------------------------- CTA-pair GEMM (selectable kernel)
+
+def _prepare_with_kernel(d, kernel):
+    import os
+    old = os.environ.get("SVDQ_K2_KERNEL")
+    os.environ["SVDQ_K2_KERNEL"] = kernel          # read when the layer is created
+    try:
+        return prepare_gpu(d)
+    finally:
+        if old is None:
+            del os.environ["SVDQ_K2_KERNEL"]
+        else:
+            os.environ["SVDQ_K2_KERNEL"] = old
+
+
+@pytest.mark.parametrize("M,K,N,flags", [(200, 320, 272, 0), (513, 1024, 512, 0), (300, 768, 400, lib.FWD_GELU),
+                                         (130, 512, 256, lib.FWD_NO_BRANCH)])
+def test_pair_kernel_matches_oracle_and_single(M, K, N, flags):
+    # 256 x 256 tiles on CTA pairs: same arithmetic as the single-CTA kernel,
+    # so the two outputs agree bit for bit, and both meet the oracle's bar
+    d = syn.custom_layer(M + 3 * N + K, M=M, K=K, N=N)
+    Lp = _prepare_with_kernel(d, "pair")
+    Ls = _prepare_with_kernel(d, "single")
+    yp = run_forward(Lp, d["X"], flags)
+    ys = run_forward(Ls, d["X"], flags)
+    np.testing.assert_array_equal(yp.view(np.uint32), ys.view(np.uint32))
+    p = oracle_prep_from(Lp)
+    if flags & lib.FWD_NO_BRANCH:
+        xq = o.quantize_activations(d["X"], p["inv_lam"], "nvfp4", p["g_x_exp"])
+        ref = o.bf16_round(xq["deq"] @ p["w_deq"].T + p["bias"])
+    else:
+        ref = o.forward(p, d["X"], gelu=bool(flags & lib.FWD_GELU))["Y_bf16"]
+    assert_close_bf16(yp, ref, "pair forward")
