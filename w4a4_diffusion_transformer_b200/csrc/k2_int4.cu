@@ -55,10 +55,24 @@ constexpr int kBN = 256;
 constexpr int kPStages = 3;                          // staging ring (packed codes + scales)
 constexpr int kOStages = 3;                          // operand ring (FP16 tiles)
 constexpr int kEpiWarps = 4;
-constexpr int kConvWarps = 8;
-constexpr int kConvWarp0 = 2 + kEpiWarps;
+// Warp roles by warpgroup: 0 producer, 1 MMA issuer, 2-3 idle; 4-7 epilogue
+// (one per TMEM lane quarter); 8 .. 8 + kConvWarps - 1 converters.  The
+// converters are latency-bound (a load, a short dependent chain, a store per
+// group), so there are four per scheduler; the register budget is moved to the
+// epilogue with setmaxnreg.
+constexpr int kConvWarps = 16;
+constexpr int kEpiWarp0 = 4;
+constexpr int kConvWarp0 = 8;
 constexpr int kThreads = (kConvWarp0 + kConvWarps) * 32;
+constexpr int kLaunchRegs = 80;                      // per thread: 65536 / 768, rounded down to 8
+constexpr int kRegsCtl = 40, kRegsEpi = 160, kRegsConv = 64;
+static_assert(128 * kRegsCtl + 128 * kRegsEpi + kConvWarps * 32 * kRegsConv <= kThreads * kLaunchRegs,
+              "register split");
 constexpr int kConvThreads = kConvWarps * 32;
+// conversion units of a group: 16 codes (a quarter row) of A's 128 and B's 256 rows
+constexpr int kUnits = (kBM + kBN) * 4;
+constexpr int kUnitsPerThread = kUnits / kConvThreads;
+static_assert(kUnits % kConvThreads == 0 && (kBM * 4) % 32 == 0, "converter work split");
 
 // staging stage: A codes, B codes, A scales, B scales
 constexpr int kPA = 0;
@@ -175,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
       dev::tma_prefetch_desc(&tm_a);
       dev::tma_prefetch_desc(&tm_b);
@@ -226,6 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
       const uint32_t id16 = idesc_f16(kBM, kBN);
       const uint32_t idbf = dev::idesc_bf16(kBM, kBN);
@@ -283,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kConvWarp0) {
     // ------------------------------------------------------------ converters
-    const int ct = threadIdx.x - kConvWarp0 * 32;   // 0..255
+    dev::setmaxnreg_dec<kRegsConv>();
+    const int ct = threadIdx.x - kConvWarp0 * 32;   // 0 .. kConvThreads - 1
     const float xs = p.xscale;                      // 2^-ex
     int it = 0;
     bool ok = true;
@@ -299,15 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint8_t* st = pring + ps * kPStageBytes;
-        // unit u = ct + 256 i: operand row u / 4 (rows 0-127 of A, then B's 256),
-        // 16 codes (8 bytes) at quarter u % 4 of the row
-        uint2 w[6];
-        __half2 s2[6];
+        // unit u = ct + kConvThreads i: operand row u / 4 (rows 0-127 of A, then
+        // B's 256), 16 codes (8 bytes) at quarter u % 4 of the row (a warp's
+        // units are all of A or all of B)
+        uint2 w[kUnitsPerThread];
+        __half2 s2[kUnitsPerThread];
 #pragma unroll
-        for (int i = 0; i < 6; ++i) {
+        for (int i = 0; i < kUnitsPerThread; ++i) {
           const int u = ct + kConvThreads * i;
           const int row = u >> 2, q = u & 3;
-          if (i < 2) {
+          if (row < kBM) {
             w[i] = *reinterpret_cast<const uint2*>(st + kPA + row * 32 + q * 8);
             const uint16_t sb = *reinterpret_cast<const uint16_t*>(st + kPSA + row * 2);
             const float sf = fminf(__uint_as_float((uint32_t)sb << 16) * xs, 8192.0f);
@@ -324,11 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) dev::mbar_arrive(&pempty[ps]);
         uint8_t* ob = oring + os * kOStageBytes;
 #pragma unroll
-        for (int i = 0; i < 6; ++i) {
+        for (int i = 0; i < kUnitsPerThread; ++i) {
           const int u = ct + kConvThreads * i;
           const int row = u >> 2, q = u & 3;
-          const int r = i < 2 ? row : row - kBM;
-          uint8_t* base = ob + (i < 2 ? 0 : kOABytes) + r * 128;
+          const bool is_a = row < kBM;
+          const int r = is_a ? row : row - kBM;
+          uint8_t* base = ob + (is_a ? 0 : kOABytes) + r * 128;
           uint32_t v0[4], v1[4];
           dequant_word(w[i].x, s2[i], v0);
           dequant_word(w[i].y, s2[i], v1);
@@ -341,10 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) dev::mbar_arrive(&ofull[os]);
       }
     }
+  } else if (warp < kEpiWarp0) {
+    dev::setmaxnreg_dec<kRegsCtl>();                 // idle warps of the first warpgroup
   } else {
     // ------------------------------------------------------------ epilogue
+    dev::setmaxnreg_inc<kRegsEpi>();
     const int q = warp & 3;                          // TMEM lane quarter of this warp
-    uint8_t* wbuf = epi_buf + (warp - 2) * kEpiWarpBytes;
+    uint8_t* wbuf = epi_buf + (warp - kEpiWarp0) * kEpiWarpBytes;
     if (lane == 0) dev::tma_prefetch_desc(&tm_y);
     int tcount = 0, chunk = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
@@ -421,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) dev::bulk_wait_group_all();
   }
 
+  __syncwarp();                                      // single-lane roles rejoin their warps first
   dev::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -441,6 +464,11 @@ cudaError_t launch_k2_int4(const CUtensorMap& tm_a, const CUtensorMap& tm_b, con
   if (configured_device != dev) {
     cudaError_t e = cudaFuncSetAttribute(k2_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
+    // the warpgroups' register budgets fit the launch allocation
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, k2_int4_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     configured_device = dev;
   }
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
