@@ -152,25 +152,40 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
     }
     cp_async_commit();
   };
-  // the first chunks in flight while the activation sums are formed
-#pragma unroll
-  for (int i = 0; i < kRing - 1; ++i) issue_chunk(i);
-
-  // Activation sums per (group, column).
-  for (int i = threadIdx.x; i < G * 8 * MT; i += kThreads) {
-    const int gi = i / (8 * MT), c = i % (8 * MT), m = m0 + c;
+  // Activation sums per (group, column).  Each thread's first group of X is
+  // requested before the first weight chunks, so that it does not queue behind
+  // them; the sums are formed while the chunks are in flight.
+  auto group_sum = [&](const uint4 (&u)[8]) {
     float sum = 0.f;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const uint32_t w[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+    return sum;
+  };
+  auto load_group = [&](int i, uint4 (&u)[8]) {
+    const int gi = i / (8 * MT), m = m0 + i % (8 * MT);
     if (m < p.M) {
       const uint4* xs = reinterpret_cast<const uint4*>(p.x + (size_t)m * K + 64 * (size_t)gi);
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        const uint4 u = __ldg(xs + v);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      for (int v = 0; v < 8; ++v) u[v] = __ldg(xs + v);
+    } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
-      }
+      for (int v = 0; v < 8; ++v) u[v] = make_uint4(0u, 0u, 0u, 0u);
     }
-    xsum[i] = sum;
+  };
+  uint4 u0[8];
+  const bool first = (int)threadIdx.x < G * 8 * MT;
+  if (first) load_group(threadIdx.x, u0);
+#pragma unroll
+  for (int i = 0; i < kRing - 1; ++i) issue_chunk(i);
+  if (first) xsum[threadIdx.x] = group_sum(u0);
+  for (int i = threadIdx.x + kThreads; i < G * 8 * MT; i += kThreads) {
+    uint4 u[8];
+    load_group(i, u);
+    xsum[i] = group_sum(u);
   }
   __syncthreads();
 
