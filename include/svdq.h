@@ -212,6 +212,18 @@ svdq_status svdq_act_scales_to_logical(const svdq_layer* layer, const void* devi
  * SVDQ_ETIMEOUT if a bounded device wait expired since the last check. */
 svdq_status svdq_check(const svdq_layer* layer, void* stream);
 
+/* svdq_selftest_wait_timeout -- exercise the failure-detection path.
+ *
+ * Enqueues on `stream` a one-thread kernel that waits on a device barrier
+ * nothing ever arrives at, with the same bounded wait every kernel of the
+ * library uses.  After budget_us microseconds (1 .. 10,000,000) the wait gives
+ * up, records a timeout in the layer's device error word and the kernel ends:
+ * no fault, no trap, no hang, and the device stays usable.  The next
+ * svdq_check on the layer then returns SVDQ_ETIMEOUT (and clears the word).
+ * Errors: SVDQ_EINVAL (NULL layer, budget out of range), SVDQ_ESTATE (host-only
+ * layer), SVDQ_ECUDA (launch failed). */
+svdq_status svdq_selftest_wait_timeout(const svdq_layer* layer, unsigned budget_us, void* stream);
+
 /* ------------------------------------------------------- allocation-free forward */
 
 /* Size of the library's built-in device workspace (16 MiB). */

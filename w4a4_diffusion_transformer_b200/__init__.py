@@ -39,6 +39,7 @@ EXPORTED = [
     "svdq_status_string", "svdq_workspace_bytes", "svdq_linear_forward", "svdq_quantize_act",
     "svdq_gemm", "svdq_act_scale_bytes", "svdq_act_scales_to_logical", "svdq_check",
     "svdq_linear_forward_static", "svdq_act_code_bytes", "svdq_act_codes_to_logical",
+    "svdq_selftest_wait_timeout",
 ]
 STATIC_WORKSPACE_BYTES = 16 << 20   # SVDQ_STATIC_WORKSPACE_BYTES
 
@@ -90,6 +91,7 @@ def load() -> ctypes.CDLL:
         "svdq_linear_forward_static": (I, [P, P, I, P, P, U]),
         "svdq_act_code_bytes": (SZ, [P, I]),
         "svdq_act_codes_to_logical": (I, [P, P, I, P]),
+        "svdq_selftest_wait_timeout": (I, [P, U, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -230,3 +232,8 @@ class Layer:
 
     def check(self, stream=None):
         _check(load().svdq_check(self._h, _stream(stream)), "svdq_check")
+
+    def selftest_wait_timeout(self, budget_us: int, stream=None):
+        """Enqueue a kernel whose only wait never completes and gives up after
+        budget_us; the next check() raises SvdqError with SVDQ_ETIMEOUT."""
+        _check(load().svdq_selftest_wait_timeout(self._h, budget_us, _stream(stream)), "svdq_selftest_wait_timeout")

@@ -648,6 +648,17 @@ svdq_status svdq_linear_forward(const svdq_layer* L, const void* X, int M, void*
   return st;
 }
 
+svdq_status svdq_selftest_wait_timeout(const svdq_layer* L, unsigned budget_us, void* stream) {
+  if (!L || budget_us == 0 || budget_us > 10000000u) return SVDQ_EINVAL;
+  if (L->device < 0) return SVDQ_ESTATE;
+  DeviceGuard g(L->device);
+  if (!g.ok) return SVDQ_ECUDA;
+  return launch_wait_selftest(L->d_err, (unsigned long long)budget_us * 1000ull, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? SVDQ_OK
+             : SVDQ_ECUDA;
+}
+
 svdq_status svdq_check(const svdq_layer* L, void* stream) {
   if (!L) return SVDQ_EINVAL;
   if (L->device < 0) return SVDQ_ESTATE;

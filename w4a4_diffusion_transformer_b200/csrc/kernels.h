@@ -110,4 +110,8 @@ cudaError_t launch_k2_int4(const CUtensorMap& tm_a, const CUtensorMap& tm_b, con
 
 cudaError_t launch_upproj(const UpParams& p, cudaStream_t stream);
 
+// One-thread kernel whose only wait can never complete: it gives up after
+// budget_ns and sets *err (failure-detection self-test).
+cudaError_t launch_wait_selftest(int* err, unsigned long long budget_ns, cudaStream_t stream);
+
 }  // namespace svdq
