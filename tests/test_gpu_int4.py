@@ -190,3 +190,34 @@ def test_int4_qkv_full_size_sampled_rows():
     yref = o.forward(p, X[rows])["Y_bf16"]
     assert_close_bf16(y[rows], yref, "qkv int4 sampled rows")
     assert np.all(np.isfinite(y))
+
+
+# ---------------------------------------------------------------- CTA-pair INT4 GEMM (selectable kernel)
+
+def _prepare_int4_with_kernel(d, kernel):
+    import os
+    old = os.environ.get("SVDQ_K2_KERNEL")
+    os.environ["SVDQ_K2_KERNEL"] = kernel          # read when the layer is created
+    try:
+        return prepare_gpu(d, fmt="int4")
+    finally:
+        if old is None:
+            del os.environ["SVDQ_K2_KERNEL"]
+        else:
+            os.environ["SVDQ_K2_KERNEL"] = old
+
+
+@pytest.mark.parametrize("M,K,N,flags", [(200, 320, 272, 0), (100, 512, 256, 0), (300, 768, 400, lib.FWD_GELU),
+                                         (513, 1024, 512, 0)])
+def test_int4_pair_kernel_matches_oracle_and_single(M, K, N, flags):
+    # 256 x 256 tiles on CTA pairs (M = 100 and 200 leave the second CTA of the
+    # last pair tile past the activation rows): same arithmetic as the
+    # single-CTA kernel, so the outputs agree bit for bit, and both meet the bar
+    d = syn.custom_layer(M + 5 * N + K, M=M, K=K, N=N)
+    Lp = _prepare_int4_with_kernel(d, "pair")
+    Ls = _prepare_int4_with_kernel(d, "single")
+    yp = run_forward(Lp, d["X"], flags)
+    ys = run_forward(Ls, d["X"], flags)
+    np.testing.assert_array_equal(yp.view(np.uint32), ys.view(np.uint32))
+    ref = o.forward(oracle_prep_from(Lp), d["X"], gelu=bool(flags & lib.FWD_GELU))["Y_bf16"]
+    assert_close_bf16(yp, ref, "int4 pair forward")

@@ -34,7 +34,8 @@ struct svdq_layer {
   float* d_bias = nullptr;           // [N]
   int* d_err = nullptr;
   CUtensorMap tm_wq, tm_l2s, tm_l1t;     // tm_wq: INT4 weight codes [N][K/2]
-  CUtensorMap tm_l2s_pair;               // 128-row boxes for the CTA-pair GEMM (NVFP4)
+  CUtensorMap tm_l2s_pair;               // 128-row boxes for the CTA-pair GEMMs
+  CUtensorMap tm_wq_pair;                // INT4 weight codes, 128-row boxes (CTA-pair INT4 GEMM)
   int k2_kernel = 0;                     // NVFP4 GEMM: 0 = by size, 1 = single-CTA, 2 = CTA pairs
 };
 
@@ -243,9 +244,9 @@ svdq_status upload_layer(svdq_layer* L, int device) {
     chk(upload(&L->d_l2t, l2t.data(), l2t.size() * 2));
     if (e != cudaSuccess) return SVDQ_ECUDA;
     const bool nv = h.format == SVDQ_NVFP4;
-    if (nv) {
+    {
       const bool ok2 = make_map(&L->tm_l2s_pair, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32,
-                                (uint32_t)k2_pair_rows_b(), CU_TENSOR_MAP_SWIZZLE_64B);
+                                (uint32_t)(nv ? k2_pair_rows_b() : k2_int4_pair_rows_b()), CU_TENSOR_MAP_SWIZZLE_64B);
       if (!ok2) return SVDQ_ECUDA;
       if (const char* k = std::getenv("SVDQ_K2_KERNEL")) {
         if (!std::strcmp(k, "single")) L->k2_kernel = 1;
@@ -253,8 +254,10 @@ svdq_status upload_layer(svdq_layer* L, int device) {
       }
     }
     // INT4 weight codes stay row-major [N][K/2] (the INT4 GEMM loads them with TMA)
-    bool ok = (nv || make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 32, 256,
-                              CU_TENSOR_MAP_SWIZZLE_NONE)) &&
+    bool ok = (nv || (make_map(&L->tm_wq, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 32, 256,
+                               CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                      make_map(&L->tm_wq_pair, L->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 32,
+                               (uint32_t)k2_int4_pair_rows_b(), CU_TENSOR_MAP_SWIZZLE_NONE))) &&
               make_map(&L->tm_l2s, L->d_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
                        CU_TENSOR_MAP_SWIZZLE_64B) &&
               make_map_kchunks(&L->tm_l1t, L->d_l1t, K, 32, 32);
@@ -346,9 +349,10 @@ svdq_status run_k2_int4(const svdq_layer* L, const void* codes, const void* scal
   p.budget_ns = L->budget_ns;
   p.branch = branch ? 1 : 0;
   p.gelu = gelu ? 1 : 0;
-  return launch_k2_int4(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream) == cudaSuccess
-             ? SVDQ_OK
-             : SVDQ_ECUDA;
+  const cudaError_t e = L->k2_kernel == 2
+                            ? launch_k2_int4_pair(tm_a, L->tm_wq_pair, tm_xl, L->tm_l2s_pair, tm_y, p, L->num_sms, stream)
+                            : launch_k2_int4(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream);
+  return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
 
 svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,

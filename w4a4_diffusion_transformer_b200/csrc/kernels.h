@@ -107,6 +107,12 @@ int k2_pair_rows_b();
 cudaError_t launch_k2_int4(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
                            const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Int4Params& p, int num_sms,
                            cudaStream_t stream);
+// The INT4 GEMM on CTA pairs (256 x 256 tiles, clusters of two): tm_b and tm_l2
+// with boxes of k2_int4_pair_rows_b() rows.
+int k2_int4_pair_rows_b();
+cudaError_t launch_k2_int4_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
+                                const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Int4Params& p,
+                                int num_sms, cudaStream_t stream);
 
 cudaError_t launch_upproj(const UpParams& p, cudaStream_t stream);
 
