@@ -51,12 +51,6 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBN = 256;
-// Stage shape: kKB 64-element K blocks per pipeline stage.  kKB = 4 gives
-// 128-byte operand rows (128-byte swizzle), kKB = 2 gives 64-byte rows
-// (64-byte swizzle) and twice as many, half-size stages in the same memory.
-#ifndef SVDQ_K2_KB
-#define SVDQ_K2_KB 4
-#endif
 // Epilogue output path: BF16 rows stored from registers straight to global
 // memory (1), or staged in shared memory and written by TMA stores (0).  The
 // direct path frees the staging buffers, which makes room for a fourth stage.
@@ -72,12 +66,13 @@ constexpr int kBN = 256;
 #define SVDQ_K2_FAST_DRAIN 1
 #endif
 constexpr bool kFastDrain = SVDQ_K2_FAST_DRAIN != 0;
-constexpr int kKB = SVDQ_K2_KB;
+// Stage shape: 4 blocks of 64 K per pipeline stage, i.e. 128-byte operand rows
+// in the 128-byte swizzle: the tiled layout the operands are stored in.
+constexpr int kKB = 4;
 constexpr int kBKBytes = kKB * 32;          // E2M1 bytes per operand row per stage
 constexpr int kStages = SVDQ_K2_STAGES;
-constexpr uint32_t kSwz = kKB == 4 ? 2u : 4u;          // descriptor layout: 128B or 64B swizzle
+constexpr uint32_t kSwz = 2u;                          // descriptor layout: 128-byte swizzle
 constexpr uint32_t kSwzAtom = 8u * kBKBytes;           // bytes between 8-row groups
-static_assert(kKB == 2 || kKB == 4, "stage shape");
 // Scale factors reach TMEM either through tcgen05.cp issued by one warp (0),
 // or from registers: four warps, one per TMEM lane quarter, read them from
 // shared memory and write them with tcgen05.st (1).  A copy occupies the
