@@ -165,13 +165,21 @@ def barrier(world):
 
 
 def allreduce_max(x, world):
+    """Max of x over the ranks (the slowest rank's time sets the job's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(flops_per_step, world, step_ms_max):
+    """Whole-job throughput: every rank runs its own replica of the step, and
+    the job takes as long as its slowest rank."""
+    return flops_per_step * world / (step_ms_max * 1e-3) / 1e12
 
 
 def cpu_baseline(d, M, K, N, target_s=10.0):
@@ -472,7 +480,7 @@ def main():
         step_ms = time_rotating(stream, args.steps, step)
     barrier(world)
     step_ms_max = allreduce_max(step_ms, world)
-    value = layer_flops(M, K, N) * world / (step_ms_max * 1e-3) / 1e12
+    value = whole_job_tflops(layer_flops(M, K, N), world, step_ms_max)
     for st in sets:
         st.L.check(stream)
 
