@@ -27,6 +27,13 @@
  *   - Shape rules: K % 64 == 0, N % 16 == 0 (any N >= 1 for SVDQ_W4A16_INT4),
  *     M >= 1 (any M: tails are handled).
  *     Other shapes return SVDQ_EUNSUPPORTED.
+ *   - Environment, read once when a layer is placed on its device:
+ *     SVDQ_WAIT_BUDGET_MS -- wall-clock budget of every device wait (default
+ *       2000): a wait that runs out records a timeout that svdq_check (or
+ *       SVDQ_FWD_CHECK) reports as SVDQ_ETIMEOUT, and the kernel ends;
+ *     SVDQ_K2_KERNEL=pair|single -- the W4A4 GEMM on CTA pairs (256 x 256
+ *       tiles, clusters of two, tcgen05 cta_group::2) or on single CTAs
+ *       (128 x 256 tiles, the default).  Both give bit-identical results.
  */
 #ifndef SVDQ_H
 #define SVDQ_H
