@@ -11,16 +11,16 @@
 //   * XL = bf16(X L1d) (rank 32; 1/lam is folded into L1d).
 //
 // Layout of the work: a CTA owns 32 token rows and streams the whole K range in
-// stages of 256 columns.  Two producer warps load with TMA: one feeds an
-// 8-deep ring of X tiles (+ 256 floats of inv_lam) from HBM, the other a
-// 3-deep ring of the matching 256 x 32 slices of L1d^T, which every CTA reads
-// from L2.  The consumer warps are specialized and never wait for each other
-// inside the loop:
+// stages of 256 columns.  Two producer warps load with TMA (one 3D copy per
+// stage over a 64-column-chunk view): one feeds an 8-deep ring of X tiles
+// (+ 256 floats of inv_lam) from HBM, the other a 3-deep ring of the matching
+// 256 x 32 slices of L1d^T, which every CTA reads from L2.  The consumer warps
+// are specialized and never wait for each other inside the loop:
 //   * 8 quantizer warps: warp w owns columns 32w..32w+31 of the stage (two
 //     groups) and lane l owns row l, so the inv_lam reads are broadcasts and
-//     the swizzled X reads are conflict-free.  Each warp writes its 32 x 16-byte
-//     code tile to shared memory and stores it with its own TMA store; the two
-//     scale bytes of a lane are stored as one 2-byte word;
+//     the swizzled X reads are conflict-free.  Each lane stores its 16 code
+//     bytes straight from registers into the GEMM's tiled, pre-swizzled operand
+//     layout; the two scale bytes of a lane are stored as one 2-byte word;
 //   * 8 down-projection warps on the tensor cores (mma.sync BF16; the
 //     projection is 32 columns wide and the pass is bound by memory, not by the
 //     tensor pipe): warp w owns k-steps 2w, 2w+1 of every stage for all 32 rows
@@ -29,9 +29,10 @@
 //     the end.
 //
 // The INT4 variant (groups of 64, BF16 scales, codes in [-7, 7]; SOTA-314
-// "Do this") runs 4 quantizer warps of 64 columns each and writes its scales
-// group-major, [K/64][M padded to 128] BF16, the order the INT4 GEMM stages
-// them in.
+// "Do this") runs 4 quantizer warps of 64 columns each, stores each warp's
+// 32 x 32-byte code tile (row-major [M][K/2]) with its own TMA store, and writes
+// its scales group-major, [K/64][M padded to 128] BF16, the order the INT4 GEMM
+// stages them in.
 //
 // NVFP4 quantizer arithmetic per group of 16 (bit-exact with the CPU oracle): a =
 // max|v|; t = fp32(a * c_x) with c_x = fp32(1/6) 2^-gx; s = E4M3_rn_satfinite(t);

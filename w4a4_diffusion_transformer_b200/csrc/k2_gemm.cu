@@ -31,13 +31,12 @@
 //              the MMAs, and 12 copies per stage cost about as much pipe time as
 //              two thirds of the stage's MMAs (the copy path stays selectable).
 //   warps 8-15 epilogue, two warps per TMEM lane quarter (32 rows), each owning
-//              128 of the 256 columns: tcgen05.ld in 32-column chunks (the next
-//              chunk's load overlaps the current chunk's math), alpha, bias
-//              (staged in shared memory while the mainloop runs), GELU, BF16,
-//              into two 64-byte-swizzled 32 x 32 buffers per warp that the
-//              warp's lane 0 stores to Y with TMA.  The accumulator is released
-//              to the MMA warp as soon as its last chunk is in registers, so the
-//              stores of tile t overlap the mainloop of tile t+1.
+//              128 of the 256 columns: all 128 columns into registers with four
+//              tcgen05.ld, the accumulator handed back to the MMA warp at once,
+//              then alpha, bias (staged in shared memory while the mainloop
+//              runs), GELU, BF16, into two 64-byte-swizzled 32 x 32 buffers per
+//              warp that the warp's lane 0 stores to Y with TMA, so the stores
+//              of tile t overlap the mainloop of tile t+1.
 // Pipelines are mbarrier rings; every wait is bounded (sm100.cuh).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
