@@ -28,12 +28,13 @@
 //               tile the XL and L2b/alpha tiles into a branch buffer.
 //   warp 1      TMEM (two 256-column accumulators) and the MMA issuer: 2 BF16
 //               MMAs for the branch, then 4 FP16 MMAs (K = 16) per group.
-//   warps 2-5   epilogue, one per TMEM lane quarter, 32 columns at a time
+//   warps 2-3   idle (they complete the first warpgroup).
+//   warps 4-7   epilogue, one per TMEM lane quarter, 32 columns at a time
 //               (tcgen05.ld of the next chunk overlaps the current chunk's math),
 //               BF16 out through swizzled shared memory and TMA stores.  The
 //               accumulator is double-buffered, so the epilogue of tile t runs
 //               under the mainloop of tile t+1.
-//   warps 6-13  converters: staging -> FP16 operand tiles (128-byte swizzle,
+//   warps 8-23  converters: staging -> FP16 operand tiles (128-byte swizzle,
 //               K-major) in a 3-deep operand ring.
 // Within each 8-element chunk the k order in shared memory is (0,4,1,5,2,6,3,7)
 // of the packed codes -- the order in which nibble pairs come out of a 32-bit

@@ -7,7 +7,9 @@
 // every (A tile, B tile) pair's packed codes into FP16 operand tiles.  In pair
 // mode each CTA holds its own 128 rows of A and only half (128 rows) of the
 // 256-row B tile; the two SMs' tensor cores share the B halves.  A CTA then
-// converts 256 rows per group instead of 384 for the same flops.
+// converts 256 rows per group instead of 384 for the same flops.  On this part
+// it measures slower than the single-CTA kernel all the same (pair MMAs deliver
+// less per SM than single-CTA ones), so it runs only when selected.
 //
 // Layout of the work (CTA rank r of the pair):
 //   both CTAs   warp 0 producer: packed A codes of rows m0 + 128 r, packed B
