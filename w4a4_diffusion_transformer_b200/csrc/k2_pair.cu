@@ -7,24 +7,27 @@
 // output"):
 //   acc  = XL (L2b / alpha) + sum_k (c_x s_x) (c_w s_w);   Y = bf16([gelu](alpha acc + b)).
 //
-// Why pairs: each stage of the single-CTA kernel moves 52 KB per SM from L2
-// for 16.8 MFLOP, and the per-SM delivery rate (not the tensor core) sets its
-// pace.  In pair mode each CTA holds its own 128 rows of A but only half of
-// B's 256 rows; the tensor cores of the two SMs share the B halves.  A stage
-// is then 38 KB per SM for the same work, and five of them fit.
+// Why pairs: the single-CTA kernel is bound by the stream of its operand
+// stages into each SM (54 KB per 16.8 MFLOP).  In pair mode each CTA holds its
+// own 128 rows of A but only half of B's 256 rows; the tensor cores of the two
+// SMs share the B halves.  A stage is then 38 KB per SM for the same work, and
+// five of them fit.  On this part it measures slower than the single-CTA
+// kernel all the same (pair MMAs deliver less per SM than single-CTA ones), so
+// it runs only when selected.
 //
 // Layout of the work (CTA rank r = 0, 1 of the pair; tile rows m0.., cols n0..):
 //   both CTAs   warp 0: TMA producer of this CTA's stage data: A rows m0+128r,
 //               B rows n0+128r, A's scale factors (own rows) and B's (all 256
 //               rows: each CTA's tensor core needs the scales of every column);
 //               per tile a branch stage with XL rows m0+128r and L2b/alpha rows
-//               n0+128r.  warps 2-9: epilogue of this CTA's 128 accumulator
+//               n0+128r.  Warps 4-7: scale factors from shared memory into this
+//               CTA's TMEM through registers (tcgen05.st, one warp per lane
+//               quarter).  Warps 8-15: epilogue of this CTA's 128 accumulator
 //               rows (the single-CTA kernel's epilogue).
-//   rank 0      warp 1: MMA issuer (pair MMAs, M = 256); warp 10: scale-factor
-//               copies (pair copies: each CTA's shared memory into its TMEM).
-//   rank 1      warps 1 and 10 forward "stage data landed" and "scale factors
-//               landed" to rank 0's barriers (remote mbarrier arrives), since
-//               rank 0's pair operations read both CTAs' shared memory.
+//   rank 0      warp 1: MMA issuer (pair MMAs, M = 256).
+//   rank 1      warp 1 forwards "stage data landed" and warp 2 "scale factors
+//               in TMEM" to rank 0's barriers (remote mbarrier arrives), since
+//               rank 0's pair operations read both CTAs' shared memory and TMEM.
 // Rank 0's commits arrive on both CTAs' barriers (multicast commit): a stage is
 // free in both, an accumulator is full in both.  Every epilogue warp of both
 // CTAs hands the accumulator back through rank 0's barrier.  Every wait is
