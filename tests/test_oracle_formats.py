@@ -154,3 +154,23 @@ def test_pow2_exponent_ceil():
     for x in 10.0 ** np.linspace(-20, 20, 301):
         e = o.pow2_exponent_ceil(x)
         assert 2.0 ** e >= x > 2.0 ** (e - 1)
+
+
+def test_division_free_reciprocal_of_e4m3_scales():
+    # The first kernel forms inv = fp32(1 / (s * 2^gx)) without a division: for
+    # s = (1 + m/8) 2^(e-7) it takes fp32(1 / (1 + m/8)) 2^(7-e-gx), for a
+    # subnormal s = m 2^-9 it takes fp32(1/m) 2^(9-gx) -- a power-of-two
+    # scaling of one of 15 correctly rounded constants.  Equal to the IEEE
+    # quotient for every positive E4M3 value and every tensor-scale exponent
+    # the kernel accepts.
+    rcp_norm = [np.float32(1.0 / (1.0 + m / 8.0)) for m in range(8)]
+    rcp_sub = [np.float32(1.0 / m) if m else np.float32(0.0) for m in range(8)]
+    for byte in range(1, 0x7F):
+        e, m = byte >> 3, byte & 7
+        s = (1.0 + m / 8.0) * 2.0 ** (e - 7) if e else m * 2.0 ** -9
+        assert s == o.e4m3_decode(np.array([byte]))[0]
+        for gx in range(-40, 31):
+            want = np.float32(1.0) / np.float32(s * 2.0 ** gx)      # IEEE float32 division
+            got = np.float32(float(rcp_norm[m]) * 2.0 ** (7 - e - gx)) if e else \
+                np.float32(float(rcp_sub[m]) * 2.0 ** (9 - gx))
+            assert got == want, (byte, gx)
