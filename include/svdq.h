@@ -125,8 +125,11 @@ typedef enum {
  *   out        receives the new layer; owned by the caller, free with svdq_destroy.
  *
  * Runs on the host (multi-threaded), then copies the prepared buffers to
- * `device` with blocking copies.  Errors: SVDQ_EINVAL, SVDQ_EUNSUPPORTED,
- * SVDQ_ENOMEM, SVDQ_ECUDA, SVDQ_ENOCONVERGE (the SVD's energy check failed).
+ * `device` with blocking copies.  Errors: SVDQ_EINVAL, SVDQ_EUNSUPPORTED (shape
+ * rules; for SVDQ_NVFP4 also a calibration batch whose largest smoothed
+ * magnitude puts the activation tensor-scale exponent outside [-40, 30], i.e.
+ * below about 3e-10 or above about 7e11), SVDQ_ENOMEM, SVDQ_ECUDA,
+ * SVDQ_ENOCONVERGE (the SVD's energy check failed).
  * On error *out is set to NULL and nothing leaks. */
 svdq_status svdq_prepare(const svdq_config* cfg, int K, int N,
                          const uint16_t* W_bf16, const uint16_t* bias_bf16,

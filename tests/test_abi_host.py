@@ -180,6 +180,24 @@ def test_argument_errors():
     assert L.workspace_bytes(0) == 0
 
 
+def test_activation_tensor_scale_exponent_range():
+    # the first kernel's division-free reciprocal is pinned for activation
+    # tensor-scale exponents in [-40, 30]; calibration batches outside are refused
+    d = syn.custom_layer(8, M=8, K=128, N=32)
+    W = syn.bf16_bits(d["W"])
+    for scale in (2.0 ** 80, 2.0 ** -80):
+        Xc = syn.bf16_bits(syn.to_bf16(d["Xc"].astype(np.float64) * scale))
+        with pytest.raises(lib.SvdqError) as e:
+            lib.Layer.prepare(W, None, Xc, device=-1)
+        assert e.value.status == lib.EUNSUPPORTED
+        L = lib.Layer.prepare(W, None, Xc, fmt="int4", device=-1)   # INT4 has no tensor scale
+        L.close()
+    for scale in (2.0 ** 20, 2.0 ** -20):                           # inside the range
+        L = lib.Layer.prepare(W, None, syn.bf16_bits(syn.to_bf16(d["Xc"].astype(np.float64) * scale)), device=-1)
+        assert -40 <= L.info["g_x_exp"] <= 30
+        L.close()
+
+
 def test_rank_above_matrix_rank():
     d = syn.custom_layer(8, M=4, K=64, N=16)
     L = _prep_host(d)

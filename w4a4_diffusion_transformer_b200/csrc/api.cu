@@ -430,6 +430,11 @@ svdq_status svdq_prepare(const svdq_config* cfg, int K, int N, const uint16_t* W
   svdq_layer* L = new (std::nothrow) svdq_layer();
   if (!L) return SVDQ_ENOMEM;
   svdq_status st = host_prepare(*cfg, K, N, W_bf16, bias_bf16, calib_bf16, M_calib, L->host);
+  // The first kernel's division-free reciprocal of the NVFP4 scales equals the
+  // IEEE quotient for activation tensor-scale exponents in [-40, 30], i.e.
+  // calibration maxima between about 3e-10 and 7e11.
+  if (st == SVDQ_OK && L->host.format == SVDQ_NVFP4 && (L->host.g_x_exp < -40 || L->host.g_x_exp > 30))
+    st = SVDQ_EUNSUPPORTED;
   if (st == SVDQ_OK && device >= 0) {
     st = upload_layer(L, device);
     if (st != SVDQ_OK) free_device(L);
