@@ -171,7 +171,10 @@ size_t svdq_workspace_bytes(const svdq_layer* layer, int M);
  * calibration batch's largest by more than 32x is clamped.  SVDQ_W4A16_INT4 (the adaptive-norm
  * linears, "stay W4A16") enqueues one weight-only GEMV kernel meant for a few
  * rows (M <= 16), needs no workspace (pass NULL, 0) and accepts only
- * SVDQ_FWD_CHECK among the flags. */
+ * SVDQ_FWD_CHECK among the flags.  The W4A4 kernels are programmatic dependent
+ * launches: their prologues may overlap the preceding kernel on the stream,
+ * but each waits for that kernel to complete before it reads its inputs or
+ * writes anything, so stream order is kept. */
 svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, void* Y,
                                 void* workspace, size_t workspace_bytes,
                                 void* stream, unsigned flags);
