@@ -221,3 +221,49 @@ def test_int4_pair_kernel_matches_oracle_and_single(M, K, N, flags):
     np.testing.assert_array_equal(yp.view(np.uint32), ys.view(np.uint32))
     ref = o.forward(oracle_prep_from(Lp), d["X"], gelu=bool(flags & lib.FWD_GELU))["Y_bf16"]
     assert_close_bf16(yp, ref, "int4 pair forward")
+
+
+# ---------------------------------------------------------------- range of the FP16 dequantization
+
+def _int4_activation_exponent(Xc, inv_lam):
+    # the layer's FP16 range exponent of the activation operand: the largest
+    # smoothed calibration magnitude is moved to (2^7, 2^8]
+    amax = float(np.max(np.abs(o.smoothed_activations(Xc, inv_lam))))
+    return o.pow2_exponent_ceil(amax) - 8, amax
+
+
+@pytest.mark.parametrize("gain", [64.0, 128.0, 1024.0])
+def test_int4_activations_far_above_calibration(gain):
+    # Rows of the run batch scaled by a power of two (exact in BF16) far above
+    # anything in the calibration batch.  Up to about 220x the calibration
+    # maximum every group is exact and the output meets the oracle's bar; a
+    # group beyond that is clamped to the limit: the output stays finite and
+    # equals the oracle's arithmetic with those group scales clamped.
+    d = syn.custom_layer(60, M=256, K=512, N=384)
+    L = prepare_gpu(d, fmt="int4")
+    p = oracle_prep_from(L)
+    X = d["X"].copy()
+    hot = np.arange(0, 256, 17)
+    X[hot] *= np.float32(gain)
+    ex, calib_amax = _int4_activation_exponent(d["Xc"], p["inv_lam"])
+    xq = o.quantize_activations(X, p["inv_lam"], "int4")
+    limit = 8192.0 * 2.0 ** ex                          # the clamp, in scale units
+    clamped = xq["scales"] > limit
+    row_amax = float(np.max(np.abs(o.smoothed_activations(X[hot], p["inv_lam"]))))
+    y = run_forward(L, X)
+    assert np.all(np.isfinite(y))
+    if gain <= 128.0:
+        assert row_amax >= 0.25 * gain * calib_amax       # the rows really are far above calibration
+        assert not clamped.any()
+        assert_close_bf16(y, o.forward(p, X)["Y_bf16"], f"int4 x{gain:g}")
+        return
+    assert clamped.any() and row_amax > 220 * calib_amax
+    K = X.shape[1]
+    s_eff = np.minimum(xq["scales"], limit)
+    deq = (xq["codes"].reshape(X.shape[0], K // 64, 64) * s_eff[:, :, None]).reshape(X.shape)
+    model = o.forward(p, X, xq=dict(xq, deq=deq))["Y_bf16"]
+    assert_close_bf16(y, model, f"int4 x{gain:g}, clamped groups")
+    # rows without a clamped group still meet the oracle's own bar
+    ok_rows = ~clamped.any(axis=1)
+    assert ok_rows.sum() >= 200
+    assert_close_bf16(y[ok_rows], o.forward(p, X[ok_rows])["Y_bf16"], "int4 rows without clamped groups")

@@ -132,12 +132,15 @@ size_t act_scale_bytes(const HostPrep& h, int M) {
 
 // FP16 range exponents of the INT4 GEMM's dequantized operands: the largest
 // |c s| of the weights maps to at most 2^14 (4x below FP16's maximum), the
-// largest smoothed calibration activation to at most 2^12 (16x headroom).
+// largest smoothed calibration activation to at most 2^8, so that a runtime
+// group scale up to about 220x the calibration batch's largest stays below the
+// GEMM's clamp of 8192, while every group scale down to 2^-24 of that largest
+// value stays at or above 2^-17, where FP16 holds all of its 8 bits exactly.
 void int4_range_exponents(const HostPrep& h, int* ex, int* ew) {
   float amax = 0.0f;
   for (float v : h.R) amax = std::max(amax, std::fabs(v));
   *ew = pow2_ceil_exponent((double)amax) - 14;
-  *ex = pow2_ceil_exponent((double)h.x_amax) - 12;
+  *ex = pow2_ceil_exponent((double)h.x_amax) - 8;
 }
 
 struct WsLayout {
@@ -215,6 +218,10 @@ svdq_status upload_layer(svdq_layer* L, int device) {
       for (int n = 0; n < N; ++n)
         for (int gi = 0; gi < K / 16; ++gi) ws[sf_offset(n, gi, K)] = h.w_scales_e4m3[(size_t)n * (K / 16) + gi];
       chk(upload(&L->d_ws, ws.data(), ws.size()));
+      // the CTA-pair GEMM's merged copy of both
+      std::vector<uint8_t> wpair(k2_pair_weight_bytes(N, K));
+      k2_pair_pack_weights(tiled.data(), ws.data(), N, K, wpair.data());
+      chk(upload(&L->d_wpair, wpair.data(), wpair.size()));
     } else {
       // weight scales times 2^-ew as FP16, group-major [K/64][npad] (zero padding)
       int4_range_exponents(h, &L->i4_ex, &L->i4_ew);

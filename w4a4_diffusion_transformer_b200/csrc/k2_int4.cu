@@ -12,13 +12,17 @@
 //     acc = sum_g sum_{k in g} (c_x s_x 2^-ex) (c_w s_w 2^-ew)
 // with no rounding beyond FP32 accumulation.  ex and ew are power-of-two
 // exponents fixed when the layer is prepared (ew from the weights, ex from the
-// calibration batch with 16x headroom) that keep the FP16 values in range;
+// calibration batch) that keep the FP16 values in range;
 // alpha = 2^(ex + ew) is applied in the epilogue, and the branch operand is
 // L2b / alpha (exact in BF16), exactly as in the NVFP4 kernel:
 //     acc  = XL (L2b / alpha) + sum (...)          Y = bf16([gelu](alpha acc + b)).
-// A group whose scaled activation scale exceeds 8192 is clamped there (its
-// products stay finite); with the calibration headroom this needs activations
-// 32x larger than any seen at calibration.
+// Exactness holds for every scale s with 2^-17 <= s 2^-e <= 8192: at the top
+// a group whose scaled activation scale exceeds 8192 is clamped there (its
+// products stay finite, and the group contributes less than it should); ex puts
+// that limit at about 220x the largest activation of the calibration batch.  At
+// the bottom FP16 subnormals keep every BF16 scale down to 2^-17 (2^-24 of the
+// calibration maximum, 2^-30 of the largest weight residual) exactly; smaller
+// ones are rounded to multiples of 2^-24 (operand units).
 //
 // Structure (one CTA per SM, persistent over 128 x 256 output tiles, k-step =
 // one group of 64):
@@ -236,6 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           dev::bulk_load(st + kPSA, p.sa + (size_t)g * p.mpad + m0, kBM * 2, &pfull[s]);
         }
       }
+      // every exit path waits for the preceding grid, so that this grid never
+      // completes before it (the next launch on the stream waits only for this one)
+      if (!deps_ready) dev::griddep_wait();
       for (int j = max(0, it - kPStages); j < it; ++j)
         if (!dev::mbar_wait(&pfull[j % kPStages], (uint32_t)(j / kPStages) & 1u, abort_flag, p.budget_ns)) break;
       if (p.branch && tcount > 0) dev::mbar_wait(bfull, (uint32_t)(tcount - 1) & 1u, abort_flag, p.budget_ns);
