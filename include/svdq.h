@@ -167,8 +167,11 @@ size_t svdq_workspace_bytes(const svdq_layer* layer, int M);
  * same output"; SOTA-314 "Do this").  For SVDQ_INT4 the GEMM dequantizes each
  * group of 64 codes times its BF16 scale into FP16 on chip (exact: 3 + 8
  * significant bits) and multiplies on the FP16 tensor cores, since the B200
- * has no 4-bit integer MMA; a group whose smoothed activations exceed the
- * calibration batch's largest by more than 32x is clamped.  SVDQ_W4A16_INT4 (the adaptive-norm
+ * has no 4-bit integer MMA.  Exact for every group scale between 2^-24 of
+ * the calibration batch's largest smoothed activation and about 220 times it;
+ * a group whose smoothed activations exceed that upper limit is clamped to it
+ * (its contribution shrinks by the ratio), and smaller scales are rounded to
+ * FP16 subnormals (an absolute error below 2^-32 of the calibration maximum).  SVDQ_W4A16_INT4 (the adaptive-norm
  * linears, "stay W4A16") enqueues one weight-only GEMV kernel meant for a few
  * rows (M <= 16), needs no workspace (pass NULL, 0) and accepts only
  * SVDQ_FWD_CHECK among the flags.  The W4A4 kernels are programmatic dependent
@@ -254,6 +257,8 @@ svdq_status svdq_selftest_wait_timeout(const svdq_layer* layer, unsigned budget_
  * the process exits.  This call allocates and frees nothing.
  *
  *   X, M, Y, stream, flags  as for svdq_linear_forward.
+ * A SVDQ_W4A16_INT4 layer needs no workspace and runs exactly as
+ * svdq_linear_forward(layer, X, M, Y, NULL, 0, stream, flags).
  * Returns SVDQ_EUNSUPPORTED if svdq_workspace_bytes(layer, M) exceeds
  * SVDQ_STATIC_WORKSPACE_BYTES (for K = 3072: M above 9,349 tokens), and
  * SVDQ_ECUDA if the workspace address cannot be obtained.

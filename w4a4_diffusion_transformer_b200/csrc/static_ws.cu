@@ -51,8 +51,10 @@ extern "C" svdq_status svdq_linear_forward_static(const svdq_layer* layer, const
   svdq_status st = svdq_get_info(layer, &info);
   if (st != SVDQ_OK) return st;
   if (info.device < 0) return SVDQ_ESTATE;
+  // the weight-only format runs without any workspace: nothing to substitute
+  if (info.format == SVDQ_W4A16_INT4) return svdq_linear_forward(layer, X, M, Y, nullptr, 0, stream, flags);
   const size_t need = svdq_workspace_bytes(layer, M);
-  if (need == 0) return SVDQ_EUNSUPPORTED;               // format without a workspace-based forward
+  if (need == 0) return SVDQ_EUNSUPPORTED;               // no workspace-based forward for this layer
   if (need > kStaticWorkspaceBytes) return SVDQ_EUNSUPPORTED;   // M too large for the static workspace
   int prev = -1;
   if (cudaGetDevice(&prev) != cudaSuccess) return SVDQ_ECUDA;
