@@ -97,13 +97,26 @@ class ClockSampler:
         self._period = period_s
         self.error = None
 
+    def _sample(self):
+        import pynvml
+        try:
+            self.samples.append(pynvml.nvmlDeviceGetClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+            fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            mask = fn(self._h)
+            for n, bit in self._names.items():
+                if mask & bit:
+                    self.reasons.add(n)
+        except Exception as e:       # keep sampling best-effort
+            self.error = str(e)
+
     def __enter__(self):
         try:
             import pynvml
             pynvml.nvmlInit()
-            h = pynvml.nvmlDeviceGetHandleByIndex(self._idx)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
-            names = {
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self._idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._names = {
                 "hw_slowdown": getattr(pynvml, "nvmlClocksEventReasonHwSlowdown", 0x8),
                 "hw_thermal_slowdown": getattr(pynvml, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
                 "sw_thermal_slowdown": getattr(pynvml, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
@@ -113,16 +126,7 @@ class ClockSampler:
 
             def run():
                 while not self._stop.is_set():
-                    try:
-                        self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
-                        fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
-                        mask = fn(h)
-                        for n, bit in names.items():
-                            if mask & bit:
-                                self.reasons.add(n)
-                    except Exception as e:       # keep sampling best-effort
-                        self.error = str(e)
+                    self._sample()
                     time.sleep(self._period)
 
             self._thread = threading.Thread(target=run, daemon=True)
@@ -132,6 +136,10 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        # one more sample at the end of the region (a region shorter than the
+        # sampling period still gets a sample from each end)
+        if self._thread:
+            self._sample()
         self._stop.set()
         if self._thread:
             self._thread.join()
@@ -295,6 +303,107 @@ def library_nvfp4_gemm_us(M, K, N, n, n_sets=N_SETS):
         return time_rotating(stream, n, f) * 1e3
     except Exception:
         return None
+
+
+def nvfp4_peak_probe(dev, n=200):
+    """The dense NVFP4 ceiling measured on this GPU: cuBLASLt's block-scaled
+    NVFP4 GEMM at 8192^3 (torch._scaled_mm, a library probe off the hot path),
+    back to back over three operand sets (192 MB, more than L2), with the SM
+    clock sampled while it runs."""
+    M = K = N = 8192
+    with ClockSampler(dev) as clk:
+        us = library_nvfp4_gemm_us(M, K, N, n, n_sets=3)
+    if us is None:
+        return None
+    return {"tflops": 2.0 * M * N * K / (us * 1e-6) / 1e12, "us": us, "shape": "8192x8192x8192",
+            "clocks": clk.summary(),
+            "how": "cuBLASLt block-scaled NVFP4 (E2M1, E4M3 scales per 16) GEMM through torch._scaled_mm, "
+                   f"{n} launches back to back over 3 operand sets, one pair of CUDA events"}
+
+
+def block_b4(pkg, syn, stream, n, peaks, fp4_peak):
+    """The FLUX.1-dev double-stream block linears at batch 4 (M = 18432 tokens):
+    QKV, attention output, fc1 (GELU epilogue) and fc2 on fc1's output, all
+    NVFP4 r = 32, each timed as layers run (K1 + K2 back to back) and K2 alone;
+    plus the adaptive-norm W4A16 GEMV on 4 rows.  Each layer's input and output
+    exceed L2 (113 MB or more), so one set per layer reads from HBM."""
+    import torch
+    dev = torch.cuda.current_device()
+    out = {}
+    total_us = 0.0
+    total_flops = 0.0
+    h = None
+    p1_calib = None
+    for name in ("qkv", "out", "fc1", "fc2"):
+        d = syn.layer("block_b4", name)
+        if name == "fc2":
+            d["Xc"] = p1_calib
+        L = pkg.Layer.prepare(syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]), syn.bf16_bits(d["Xc"]),
+                              fmt="nvfp4", rank=RANK, device=dev)
+        K, N = d["W"].shape
+        x = h if name == "fc2" else torch.from_numpy(d.pop("X")).to(torch.bfloat16).cuda()
+        M = x.shape[0]
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        codes = torch.empty(L.act_code_bytes(M), dtype=torch.uint8, device="cuda")
+        scales = torch.empty(L.act_scale_bytes(M), dtype=torch.uint8, device="cuda")
+        xl = torch.empty((M, RANK), dtype=torch.bfloat16, device="cuda")
+        flags = pkg.FWD_GELU if name == "fc1" else 0
+
+        def k1(i):
+            L.quantize_act(x, M, codes, scales, xl, stream, 0)
+
+        def k2(i):
+            L.gemm(codes, scales, xl, M, y, stream, flags)
+
+        def layer(i):
+            k1(i)
+            k2(i)
+
+        for i in range(3):
+            layer(i)
+        L.check(stream)
+        lay = time_rotating(stream, n, layer)
+        k2_ms = time_rotating(stream, n, k2)
+        L.check(stream)
+        k2t = k2_flops(M, K, N) / (k2_ms * 1e-3) / 1e12
+        out[name] = {"shape": f"{M}x{K}->{N}", "us_per_layer": lay * 1e3, "k2_us": k2_ms * 1e3,
+                     "layer_tflops": layer_flops(M, K, N) / (lay * 1e-3) / 1e12, "k2_tflops": k2t,
+                     "k2_frac": k2t / fp4_peak}
+        total_us += lay * 1e3
+        total_flops += layer_flops(M, K, N)
+        if name == "fc1":
+            h = y
+            # fc2 calibrates on fc1's output for fc1's calibration batch (this library, offline)
+            xc = torch.from_numpy(d["Xc"]).to(torch.bfloat16).cuda()
+            hc = torch.empty((xc.shape[0], N), dtype=torch.bfloat16, device="cuda")
+            wsc = torch.empty(L.workspace_bytes(xc.shape[0]), dtype=torch.uint8, device="cuda")
+            L.forward(xc, xc.shape[0], hc, wsc, wsc.numel(), stream, pkg.FWD_GELU | pkg.FWD_CHECK)
+            p1_calib = hc.float().cpu().numpy()
+        else:
+            del y
+        L.close()
+        del x
+    # adaptive-norm modulation, W4A16 on the 4 conditioning rows
+    da = syn.layer("block_b4", "adaln", with_run=False)
+    Ka, Na = da["W"].shape
+    La = pkg.Layer.prepare(syn.bf16_bits(da["W"]), syn.bf16_bits(da["bias"]), None, fmt="w4a16", rank=0,
+                           device=dev)
+    xa = torch.from_numpy(syn.activations(4, 4, 4, Ka, syn.ROLE_X_RUN, outliers=False)).to(torch.bfloat16).cuda()
+    ya = torch.empty((4, Na), dtype=torch.bfloat16, device="cuda")
+    La.forward(xa, 4, ya, None, 0, stream, pkg.FWD_CHECK)
+    ta = time_rotating(stream, n, lambda i: La.forward(xa, 4, ya, None, 0, stream, 0))
+    La.check(stream)
+    La.close()
+    wbytes = Na * Ka // 2 + Na * (Ka // 64) * 2 + 4 * Ka * 2 + 4 * Na * 2 + Na * 4
+    out["adaln_w4a16"] = {"shape": f"4x{Ka}->{Na}", "us": ta * 1e3,
+                          "hbm_frac": wbytes / (ta * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                          "note": "the same 30 MB of weights every launch (L2-warm after the first)"}
+    total_us += ta * 1e3
+    out["stack"] = {"us": total_us, "tflops": total_flops / (total_us * 1e-6) / 1e12,
+                    "frac": total_flops / (total_us * 1e-6) / 1e12 / fp4_peak,
+                    "note": "sum of the per-layer times (QKV, out, fc1+GELU, fc2, adaLN); "
+                            "attention itself is not part of this stack"}
+    return out
 
 
 def other_layers(pkg, syn, stream, flush_l2, n, peaks):
@@ -564,11 +673,17 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_other_layers:
         out["other_layers"] = other_layers(pkg, syn, stream, flush_l2, max(30, min(200, args.steps)), peaks)
+        out["other_layers"]["block_b4"] = block_b4(pkg, syn, stream, max(20, min(100, args.steps)), peaks, fp4_peak)
         lib_us = library_nvfp4_gemm_us(M, K, N, n_k)
         out["library_context"] = {
             "cublaslt_nvfp4_gemm_us": lib_us, "k2_us": k2_ms * 1e3, "bare_k2_us": bare_k2_ms * 1e3,
             "note": "bare NVFP4 GEMM of the same shape through torch._scaled_mm (no low-rank branch, no bias), "
                     "back to back over rotating operand sets; context, not a baseline"}
+        probe = nvfp4_peak_probe(dev)
+        if probe is not None:
+            out["nvfp4_peak_measured"] = probe
+            out["pct_nvfp4_peak"]["of_cublaslt_8192"] = value / world / probe["tflops"]
+            out["roofline"]["frac_of_cublaslt_8192"] = k2_achieved / probe["tflops"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(d, M, K, N)
     for st in sets:
