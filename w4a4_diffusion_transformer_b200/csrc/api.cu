@@ -30,6 +30,7 @@ struct svdq_layer {
   __nv_bfloat16* d_l2t = nullptr;    // [N][32]   L2b^T (unfused up projection)
   uint8_t* d_wq = nullptr;           // [N][K/2]
   uint8_t* d_ws = nullptr;           // weight scales: NVFP4 tensor-core layout; INT4 FP16 [K/64][npad] (times 2^-ew)
+  uint8_t* d_wpair = nullptr;        // NVFP4: codes and scales merged for the CTA-pair GEMM
   int i4_ex = 0, i4_ew = 0;          // INT4: power-of-two range exponents of the FP16 GEMM operands
   float* d_bias = nullptr;           // [N]
   int* d_err = nullptr;
@@ -173,6 +174,7 @@ void free_device(svdq_layer* L) {
   cudaFree(L->d_l2t);
   cudaFree(L->d_wq);
   cudaFree(L->d_ws);
+  cudaFree(L->d_wpair);
   cudaFree(L->d_bias);
   cudaFree(L->d_err);
   L->d_inv_lam = nullptr;
@@ -199,10 +201,11 @@ svdq_status upload_layer(svdq_layer* L, int device) {
   chk(upload(&L->d_bias, h.bias.data(), sizeof(float) * N));
   if (h.format == SVDQ_NVFP4 || h.format == SVDQ_INT4) {
     chk(upload(&L->d_inv_lam, h.inv_lam.data(), sizeof(float) * K));
+    std::vector<uint8_t> tiled;
     if (h.format == SVDQ_NVFP4) {
       // weight codes in the GEMM's tiled layout (wgt_tile_offset), rows padded to 256 with zeros
       const int nst = nvfp4_stages(K);
-      std::vector<uint8_t> tiled((size_t)((N + 255) / 256) * (size_t)nst * 32768u, 0);
+      tiled.assign((size_t)((N + 255) / 256) * (size_t)nst * 32768u, 0);
       for (int n = 0; n < N; ++n)
         for (int b = 0; b < K / 2; ++b)
           tiled[wgt_tile_offset(n, b >> 7, (b & 127) >> 4, nst) + (b & 15)] = h.w_codes[(size_t)n * (K / 2) + b];
@@ -385,6 +388,7 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
   p.alpha = (float)std::ldexp(1.0, h.g_x_exp + h.g_w_exp);
   p.sfa = static_cast<const uint8_t*>(scales);
   p.sfb = L->d_ws;
+  p.wpair = L->d_wpair;
   p.bias = L->d_bias;
   p.y = static_cast<__nv_bfloat16*>(Y);
   p.err = L->d_err;

@@ -245,6 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++it;
         }
       }
+      // every exit path waits for the preceding grid, so that this grid never
+      // completes before it (the next launch on the stream waits only for this one)
+      if (!deps_ready) dev::griddep_wait();
       for (int j = max(0, it - kStages); j < it; ++j)
         if (!dev::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns) ||
             !dev::mbar_wait(&sf_full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns))

@@ -231,6 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (sa_rows) dev::bulk_load(st + kPSA, p.sa + (size_t)g * p.mpad + m0, kBM * 2, &pfull[s]);
         }
       }
+      // every exit path waits for the preceding grid, so that this grid never
+      // completes before it (the next launch on the stream waits only for this one)
+      if (!deps_ready) dev::griddep_wait();
       for (int j = max(0, it - kPStages); j < it; ++j)
         if (!dev::mbar_wait(&pfull[j % kPStages], (uint32_t)(j / kPStages) & 1u, abort_flag, p.budget_ns)) break;
       if (p.branch && tcount > 0) dev::mbar_wait(bfull, (uint32_t)(tcount - 1) & 1u, abort_flag, p.budget_ns);

@@ -7,31 +7,34 @@
 // output"):
 //   acc  = XL (L2b / alpha) + sum_k (c_x s_x) (c_w s_w);   Y = bf16([gelu](alpha acc + b)).
 //
-// Why pairs: the single-CTA kernel is bound by the stream of its operand
-// stages into each SM (54 KB per 16.8 MFLOP).  In pair mode each CTA holds its
-// own 128 rows of A but only half of B's 256 rows; the tensor cores of the two
-// SMs share the B halves.  A stage is then 38 KB per SM for the same work, and
-// five of them fit.  On this part it measures slower than the single-CTA
-// kernel all the same (pair MMAs deliver less per SM than single-CTA ones), so
-// it runs only when selected.
+// Why pairs: the operand stream into each SM bounds the single-CTA kernel
+// (54 KB per 128 x 256 x 256 stage).  In pair mode each CTA holds its own 128
+// rows of A and only half of B's 256 rows -- the two SMs' tensor cores share
+// the B halves -- so a stage is 38 KB per SM for the same work.
 //
-// Layout of the work (CTA rank r = 0, 1 of the pair; tile rows m0.., cols n0..):
-//   both CTAs   warp 0: TMA producer of this CTA's stage data: A rows m0+128r,
-//               B rows n0+128r, A's scale factors (own rows) and B's (all 256
-//               rows: each CTA's tensor core needs the scales of every column);
-//               per tile a branch stage with XL rows m0+128r and L2b/alpha rows
-//               n0+128r.  Warps 4-7: scale factors from shared memory into this
-//               CTA's TMEM through registers (tcgen05.st, one warp per lane
-//               quarter).  Warps 8-15: epilogue of this CTA's 128 accumulator
-//               rows (the single-CTA kernel's epilogue).
-//   rank 0      warp 1: MMA issuer (pair MMAs, M = 256).
-//   rank 1      warp 1 forwards "stage data landed" and warp 2 "scale factors
-//               in TMEM" to rank 0's barriers (remote mbarrier arrives), since
-//               rank 0's pair operations read both CTAs' shared memory and TMEM.
-// Rank 0's commits arrive on both CTAs' barriers (multicast commit): a stage is
-// free in both, an accumulator is full in both.  Every epilogue warp of both
-// CTAs hands the accumulator back through rank 0's barrier.  Every wait is
-// bounded (sm100.cuh).
+// What makes the stream fast here: a bulk copy occupies its issuing thread for
+// about a tenth of a microsecond whatever its size, so each CTA moves a stage
+// in two large copies from two producer warps: the weight half and the scale
+// factors of all 256 weight rows are stored next to each other (one 20 KB block
+// per CTA and stage, prepared once), and the activation codes (16 KB) plus
+// their scales (2 KB) come from the first kernel's output.
+//
+// Roles (CTA rank r = 0, 1 of the pair; tile rows m0.., columns n0..):
+//   both CTAs   warp 0: activation producer (A rows m0 + 128 r and their
+//               scale factors; per tile the XL rows of the branch stage).
+//               warp 2: weight producer (the B half n0 + 128 r with the scale
+//               factors of all 256 columns; per tile the L2b / alpha rows).
+//               Both complete the CTA's own `full` barrier of the stage.
+//               warps 4-7: wait for the CTA's stage, write its scale factors
+//               into the CTA's TMEM from registers (tcgen05.st, one warp per
+//               lane quarter) and arrive on the leader's `ready` barrier of the
+//               stage -- directly, across the cluster: once all eight warps of
+//               both CTAs have arrived, every operand of the stage is in place.
+//               warps 8-15: epilogue of the CTA's 128 accumulator rows.
+//   rank 0      warp 1: the MMA issuer: pair MMAs (M = 256), whose commits
+//               arrive on both CTAs' barriers (multicast): a stage is free in
+//               both, an accumulator full in both.
+// Every wait is bounded (sm100.cuh).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -51,12 +54,21 @@ constexpr int kBKBytes = kKB * 32;           // E2M1 bytes per operand row per s
 #ifndef SVDQ_K2P_STAGES
 #define SVDQ_K2P_STAGES 5
 #endif
+#ifndef SVDQ_K2P_EPI_BUFS
+#define SVDQ_K2P_EPI_BUFS 2
+#endif
+// How the MMA issuer waits on barriers that the other CTA's warps complete:
+// 1 polls with test_wait, 2 with a short try_wait hint, 0 plain try_wait.
+#ifndef SVDQ_K2P_REMOTE_WAIT
+#define SVDQ_K2P_REMOTE_WAIT 1
+#endif
+constexpr int kRemoteWait = SVDQ_K2P_REMOTE_WAIT;
 constexpr int kStages = SVDQ_K2P_STAGES;
+constexpr int kEpiBufs = SVDQ_K2P_EPI_BUFS;  // 32 x 32 output buffers per epilogue warp
 constexpr int kEpiWarps = 8;
-// warp roles: 0 producer, 1 MMA issuer (rank 0) or forwarder (rank 1), 2-3
-// idle, 4-7 scale factors (one per TMEM lane quarter), 8-15 epilogue
-constexpr int kSfWarp0 = 4;
-constexpr int kEpiWarp0 = 8;
+// warp roles: 0 activation producer, 1 MMA issuer (rank 0), 2 weight producer,
+// 3 idle, 4-7 scale factors / stage readiness, 8-15 epilogue
+constexpr int kProdA = 0, kMmaWarp = 1, kProdB = 2, kSfWarp0 = 4, kEpiWarp0 = 8;
 constexpr int kThreads = 16 * 32;
 // register budgets per thread by warpgroup (control, scale factors, two
 // epilogue warpgroups); they add up to the launch allocation of 128, which the
@@ -64,12 +76,17 @@ constexpr int kThreads = 16 * 32;
 constexpr int kRegsCtl = 56, kRegsSf = 72, kRegsEpi = 192;
 static_assert(128 * kRegsCtl + 128 * kRegsSf + 256 * kRegsEpi == kThreads * 128, "register split");
 constexpr int kEpiBufBytes = 32 * 64;        // one 32 x 32 BF16 output chunk
-constexpr int kEpiWarpBytes = 2 * kEpiBufBytes;
+constexpr int kEpiWarpBytes = kEpiBufs * kEpiBufBytes;
+// stage: [A codes 16 KB][B half codes 16 KB][B scales, 256 rows, 4 KB][A scales 2 KB]
 constexpr int kABytes = kBM * kBKBytes;      // 16 KiB
 constexpr int kBBytes = kBNh * kBKBytes;     // 16 KiB
-constexpr int kSFABytes = kKB * 512;         // kKB K-blocks x 128 rows
-constexpr int kSFBBytes = 2 * kKB * 512;     // 2 row blocks (all 256 columns) x kKB K-blocks
-constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+constexpr int kSFBBytes = 2 * kKB * 512;     // both 128-row halves x kKB K-blocks
+constexpr int kSFABytes = kKB * 512;
+constexpr int kOffB = kABytes;
+constexpr int kOffSFB = kOffB + kBBytes;
+constexpr int kOffSFA = kOffSFB + kSFBBytes;
+constexpr int kStageBytes = kOffSFA + kSFABytes;
+constexpr int kWBlockBytes = kBBytes + kSFBBytes;      // one CTA's weight block per stage (20 KB)
 static_assert(kStageBytes % 1024 == 0, "stage alignment");
 static_assert(kABytes >= kBM * 64 && kBBytes >= kBNh * 64, "the branch stage fits a pipeline stage");
 constexpr int kBarBytes = 512;
@@ -98,12 +115,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* epi_buf = smem + kStages * kStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(epi_buf + kEpiWarps * kEpiWarpBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* sf_full = empty + kStages;         // this CTA's scale factors landed
-  uint64_t* pfull = sf_full + kStages;         // rank 0: rank 1's stage data landed
-  uint64_t* sf_ready = pfull + kStages;        // this CTA's scale factors of a stage are in its TMEM
-  uint64_t* psf_ready = sf_ready + kStages;    // rank 0: rank 1's scale factors are in rank 1's TMEM
-  uint64_t* acc_full = psf_ready + kStages;
+  uint64_t* empty = full + kStages;            // this CTA's copy of "stage consumed" (multicast commit)
+  uint64_t* ready = empty + kStages;           // rank 0: the stage is in place in both CTAs
+  uint64_t* acc_full = ready + kStages;
   uint64_t* acc_empty = acc_full + 1;          // rank 0: both CTAs drained the accumulator
   uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -126,12 +140,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // completion before it touches anything this grid reads or writes
     dev::griddep_launch_dependents();
     for (int s = 0; s < kStages; ++s) {
-      dev::mbar_init(&full[s], 1);
+      dev::mbar_init(&full[s], 2);              // the two producer warps
       dev::mbar_init(&empty[s], 1);
-      dev::mbar_init(&sf_full[s], 1);
-      dev::mbar_init(&pfull[s], 1);
-      dev::mbar_init(&sf_ready[s], 4);          // this CTA's scale-factor warps
-      dev::mbar_init(&psf_ready[s], 1);
+      dev::mbar_init(&ready[s], 8);             // the scale-factor warps of both CTAs
     }
     dev::mbar_init(acc_full, 1);
     dev::mbar_init(acc_empty, 2 * kEpiWarps);
@@ -139,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     dev::fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     dev::tmem_alloc_pair(tmem_slot, kTmemCols);
     dev::tmem_relinquish_pair();
@@ -150,24 +161,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   dev::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
+  if (warp == kProdA) {
+    // ------------------------------------------------------------ activation producer (both CTAs)
     dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
-      if (p.branch) {
-        dev::tma_prefetch_desc(&tm_xl);
-        dev::tma_prefetch_desc(&tm_l2);
-      }
+      if (p.branch) dev::tma_prefetch_desc(&tm_xl);
+      // the activations come from the preceding kernel (launched as a dependency)
+      dev::griddep_wait();
       int it = 0;
       bool ok = true;
-      bool deps_ready = false;     // activations come from the preceding kernel (launched as a dependency)
       for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
-        const int m0 = (tile % tiles_m) * kPM;
-        const int n0 = (tile / tiles_m) * kBN;
-        const int my_m = m0 + kBM * (int)rank, my_n = n0 + kBNh * (int)rank;
-        const bool rows_a = my_m < M, rows_b = my_n < N;      // this CTA's rows exist (else they stay stale:
-                                                              // their results are never stored)
-        const bool sf_a = my_m < p.mpad;                      // the activation scales cover these rows
+        const int my_m = (tile % tiles_m) * kPM + kBM * (int)rank;
+        const bool rows_xl = my_m < M;                        // the branch rows exist
+        const bool rows_a = my_m < p.mpad;                    // the code and scale layouts cover these rows
+        // (rows that do not exist leave stale shared memory: their results are never stored)
         if (p.branch) {
           const int s = it % kStages;
           if (!dev::mbar_wait_cluster(&empty[s], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
@@ -176,14 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = smem + s * kStageBytes;
-          dev::mbar_arrive(&sf_full[s]);               // a branch stage carries no scale factors
-          dev::mbar_arrive_expect_tx(&full[s], (rows_a ? kBM * 64 : 0) + (rows_b ? kBNh * 64 : 0));
-          if (rows_b) dev::tma_load_2d(st + kABytes, &tm_l2, &full[s], 0, my_n);
-          if (!deps_ready) {
-            dev::griddep_wait();
-            deps_ready = true;
-          }
-          if (rows_a) dev::tma_load_2d(st, &tm_xl, &full[s], 0, my_m);
+          dev::mbar_arrive_expect_tx(&full[s], rows_xl ? kBM * 64 : 0);
+          if (rows_xl) dev::tma_load_2d(st, &tm_xl, &full[s], 0, my_m);
           ++it;
         }
         for (int kt = 0; kt < ktiles; ++kt) {
@@ -194,79 +195,82 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = smem + s * kStageBytes;
-          const int nkb = min(kKB, kblocks - kKB * kt);
-          const uint32_t sf_bytes = (uint32_t)nkb * 512u;
-          // scale factors on their own barrier, issued first (their TMEM copies
-          // then run while the operand tiles are still in flight)
-          dev::mbar_arrive_expect_tx(&sf_full[s], (sf_a ? sf_bytes : 0u) + 2u * sf_bytes);
-          dev::mbar_arrive_expect_tx(&full[s], (sf_a ? kABytes : 0) + kBBytes);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const size_t b_chunk = (size_t)((n0 >> 7) + h) * (size_t)kblocks + (size_t)(kKB * kt);
-            dev::bulk_load(st + kABytes + kBBytes + kSFABytes + h * (kKB * 512), p.sfb + b_chunk * 512, sf_bytes,
-                           &sf_full[s]);
-          }
-          // this CTA's 128-row half of the 256-row weight block (tiled, pre-swizzled)
-          dev::bulk_load(st + kABytes,
-                         p.wcodes + ((size_t)(n0 >> 8) * (size_t)ktiles + (size_t)kt) * (2 * kBBytes) + rank * kBBytes,
-                         kBBytes, &full[s]);
-          if (!deps_ready) {
-            dev::griddep_wait();
-            deps_ready = true;
-          }
-          if (sf_a) {
+          const uint32_t sf_bytes = (uint32_t)min(kKB, kblocks - kKB * kt) * 512u;
+          dev::mbar_arrive_expect_tx(&full[s], rows_a ? (uint32_t)kABytes + sf_bytes : 0u);
+          if (rows_a) {
             const size_t a_chunk = (size_t)(my_m >> 7) * (size_t)kblocks + (size_t)(kKB * kt);
-            dev::bulk_load(st + kABytes + kBBytes, p.sfa + a_chunk * 512, sf_bytes, &sf_full[s]);
-          }
-          if (sf_a)
             dev::bulk_load(st, p.acodes + ((size_t)(my_m >> 7) * (size_t)ktiles + (size_t)kt) * kABytes, kABytes,
                            &full[s]);
+            dev::bulk_load(st + kOffSFA, p.sfa + a_chunk * 512, sf_bytes, &full[s]);
+          }
           ++it;
         }
       }
       for (int j = max(0, it - kStages); j < it; ++j)
-        if (!dev::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns) ||
-            !dev::mbar_wait(&sf_full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns))
-          break;
+        if (!dev::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns)) break;
     }
-  } else if (warp == 1 && !leader) {
-    // ------------------------------------------------------------ rank 1: forward "stage data landed"
+  } else if (warp == kProdB) {
+    // ------------------------------------------------------------ weight producer (both CTAs)
     dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
-      const int uses = (num_tiles > pair_id ? (num_tiles - pair_id + npairs - 1) / npairs : 0) *
-                       (ktiles + (p.branch ? 1 : 0));
-      for (int it = 0; it < uses; ++it) {
-        const int s = it % kStages;
-        if (!dev::mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
-          record_error(p.err, abort_flag, 0x223);
-          break;
+      if (p.branch) dev::tma_prefetch_desc(&tm_l2);
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
+        const int n0 = (tile / tiles_m) * kBN;
+        const int my_n = n0 + kBNh * (int)rank;
+        if (p.branch) {
+          const int s = it % kStages;
+          if (!dev::mbar_wait_cluster(&empty[s], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+            record_error(p.err, abort_flag, 0x223);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStageBytes;
+          const bool rows_b = my_n < N;
+          dev::mbar_arrive_expect_tx(&full[s], rows_b ? kBNh * 64 : 0);
+          if (rows_b) dev::tma_load_2d(st + kOffB, &tm_l2, &full[s], 0, my_n);
+          ++it;
         }
-        dev::mbar_arrive_remote(dev::map_to_rank(&pfull[s], 0));
+        for (int kt = 0; kt < ktiles; ++kt) {
+          const int s = it % kStages;
+          if (!dev::mbar_wait_cluster(&empty[s], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+            record_error(p.err, abort_flag, 0x224);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStageBytes;
+          // this CTA's 128-row half of the 256-row weight block followed by the
+          // scale factors of all 256 rows: one contiguous 20 KB block
+          dev::mbar_arrive_expect_tx(&full[s], kWBlockBytes);
+          dev::bulk_load(st + kOffB,
+                         p.wpair + (((size_t)(n0 >> 8) * (size_t)ktiles + (size_t)kt) * 2 + rank) * kWBlockBytes,
+                         kWBlockBytes, &full[s]);
+          ++it;
+        }
       }
+      for (int j = max(0, it - kStages); j < it; ++j)
+        if (!dev::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns)) break;
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp && leader) {
     // ------------------------------------------------------------ rank 0: MMA issuer
     dev::setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
       const uint32_t idesc_f4 = dev::idesc_nvfp4(kPM, kBN);
       const uint32_t idesc_h = dev::idesc_bf16(kPM, kBN);
-      auto wait_data = [&](int slot, int code) -> bool {
-        const int s = slot % kStages;
-        const uint32_t ph = (uint32_t)(slot / kStages) & 1u;
-        if (!dev::mbar_wait(&full[s], ph, abort_flag, p.budget_ns) ||
-            !dev::mbar_wait_cluster(&pfull[s], ph, abort_flag, p.budget_ns)) {
+      auto wait_ready = [&](int slot, int code) -> bool {
+        if (!dev::mbar_wait_remote<kRemoteWait>(&ready[slot % kStages], (uint32_t)(slot / kStages) & 1u, abort_flag,
+                                                p.budget_ns)) {
           record_error(p.err, abort_flag, code);
           return false;
         }
         dev::tc_fence_after();
         return true;
       };
-      uint32_t sf_phase = 0;                          // per-stage parity of sf_ready
       int it = 0, tcount = 0;
       bool ok = true;
       for (int tile = pair_id; tile < num_tiles && ok; tile += npairs, ++tcount) {
-        const int kslot0 = it + (p.branch ? 1 : 0);
-        if (!dev::mbar_wait_cluster(acc_empty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+        if (!dev::mbar_wait_remote<kRemoteWait>(acc_empty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag, p.budget_ns)) {
           record_error(p.err, abort_flag, 0x225);
           ok = false;
           break;
@@ -274,10 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::tc_fence_after();
         uint32_t accumulate = 0;
         if (p.branch) {
-          if (!(ok = wait_data(it, 0x226))) break;
+          if (!(ok = wait_ready(it, 0x226))) break;
           const int s = it % kStages;
           const uint32_t a0 = dev::smem_u32(smem + s * kStageBytes);
-          const uint32_t b0 = a0 + kABytes;
+          const uint32_t b0 = a0 + kOffB;
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             dev::mma_f16_pair(tmem, dev::smem_desc(a0 + 32 * j, 16, 512, 4), dev::smem_desc(b0 + 32 * j, 16, 512, 4),
@@ -285,22 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             accumulate = 1;
           }
           dev::tc_commit_pair(&empty[s], kBoth);
+          ++it;
         }
-        for (int kt = 0; kt < ktiles; ++kt) {
-          const int slot = kslot0 + kt;
-          const int s = slot % kStages;
-          if (!(ok = wait_data(slot, 0x227))) break;
-          if (!dev::mbar_wait(&sf_ready[s], (sf_phase >> s) & 1u, abort_flag, p.budget_ns) ||
-              !dev::mbar_wait_cluster(&psf_ready[s], (sf_phase >> s) & 1u, abort_flag, p.budget_ns)) {
-            record_error(p.err, abort_flag, 0x228);
-            ok = false;
-            break;
-          }
-          sf_phase ^= 1u << s;
-          dev::tc_fence_after();
+        for (int kt = 0; kt < ktiles; ++kt, ++it) {
+          const int s = it % kStages;
+          if (!(ok = wait_ready(it, 0x227))) break;
           const int nkb = min(kKB, kblocks - kKB * kt);
           const uint32_t a0 = dev::smem_u32(smem + s * kStageBytes);
-          const uint32_t b0 = a0 + kABytes;
+          const uint32_t b0 = a0 + kOffB;
           const uint32_t tsfa = tmem + kSFCol0 + s * kSFStageCols;
           const uint32_t tsfb = tsfa + 4 * kKB;
           for (int j = 0; j < nkb; ++j) {
@@ -311,7 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           dev::tc_commit_pair(&empty[s], kBoth);
         }
         if (!ok) break;
-        it = kslot0 + ktiles;
         dev::tc_commit_pair(acc_full, kBoth);
       }
       // Wait until every pair operation this thread issued has completed.
@@ -319,75 +314,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_wait(drain, 0, abort_flag, p.budget_ns);
     }
   } else if (warp >= kSfWarp0 && warp < kSfWarp0 + 4) {
-    // ------------------------------------------------------------ scale factors (both CTAs)
+    // ------------------------------------------------------------ scale factors / stage readiness (both CTAs)
     // Warp w writes its CTA's TMEM lanes 32 (w % 4) .. +31 from registers
     // (tcgen05.st), in the layout a 32x128b.warpx4 copy produces: per 64-K
     // block j, unit `lane` of A's 512-byte chunk (this CTA's 128 rows) in
     // columns 4 j .. 4 j + 3 of the A region, and of B's two chunks (all 256
-    // columns of the tile) in columns 8 j .. 8 j + 7 of the B region (rank 1's
-    // readiness reaches rank 0 through a forwarder).  The tensor pipe stays
-    // with the MMAs.
+    // columns of the tile) in columns 8 j .. 8 j + 7 of the B region.  Then it
+    // tells the leader that this CTA's part of the stage is in place.
     dev::setmaxnreg_dec<kRegsSf>();
     const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t ready0 = dev::map_to_rank(ready, 0);
     int it = 0;
     bool ok = true;
     for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
-      if (p.branch) ++it;
-      for (int kt = 0; kt < ktiles; ++kt, ++it) {
+      const int nst = ktiles + (p.branch ? 1 : 0);
+      for (int u = 0; u < nst; ++u, ++it) {
         const int st = it % kStages;
-        const bool got = dev::mbar_wait(&sf_full[st], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns);
+        const bool got = dev::mbar_wait(&full[st], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns);
         if (!__all_sync(0xffffffffu, got)) {
           if (lane == 0) record_error(p.err, abort_flag, 0x229);
           ok = false;
           break;
         }
-        const uint8_t* sfa = smem + st * kStageBytes + kABytes + kBBytes;
-        const uint8_t* sfb = sfa + kSFABytes;
-        uint32_t ra[16], rb[32];
+        const bool kstage = !(p.branch && u == 0);
+        if (kstage) {
+          // K blocks past the tail hold stale bytes that no MMA reads; so do the
+          // A scales of rows past the activations' padding
+          const uint8_t* sfa = smem + st * kStageBytes + kOffSFA;
+          const uint8_t* sfb = smem + st * kStageBytes + kOffSFB;
+          uint32_t ra[16], rb[32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // blocks past the K tail (and the A scales of rows past the
-          // activations' padding) hold stale bytes whose results are never used
-          const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j + lane * 16);
-          const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
-          const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + kKB * 512 + 512 * j + lane * 16);
-          ra[4 * j + 0] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
-          rb[8 * j + 0] = b0.x; rb[8 * j + 1] = b0.y; rb[8 * j + 2] = b0.z; rb[8 * j + 3] = b0.w;
-          rb[8 * j + 4] = b1.x; rb[8 * j + 5] = b1.y; rb[8 * j + 6] = b1.z; rb[8 * j + 7] = b1.w;
+          for (int j = 0; j < 4; ++j) {
+            const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j + lane * 16);
+            const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
+            const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + kKB * 512 + 512 * j + lane * 16);
+            ra[4 * j + 0] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+            rb[8 * j + 0] = b0.x; rb[8 * j + 1] = b0.y; rb[8 * j + 2] = b0.z; rb[8 * j + 3] = b0.w;
+            rb[8 * j + 4] = b1.x; rb[8 * j + 5] = b1.y; rb[8 * j + 6] = b1.z; rb[8 * j + 7] = b1.w;
+          }
+          const uint32_t tsfa = tmem + kSFCol0 + st * kSFStageCols;
+          dev::tmem_store_16cols(tsfa + lanebase, ra);
+          dev::tmem_store_32cols(tsfa + 4 * kKB + lanebase, rb);
+          dev::tmem_store_wait();
         }
-        const uint32_t tsfa = tmem + kSFCol0 + st * kSFStageCols;
-        dev::tmem_store_16cols(tsfa + lanebase, ra);
-        dev::tmem_store_32cols(tsfa + 4 * kKB + lanebase, rb);
-        dev::tmem_store_wait();
         dev::tc_fence_before();
         __syncwarp();
-        if (lane == 0) dev::mbar_arrive(&sf_ready[st]);
+        if (lane == 0) dev::mbar_arrive_remote(ready0 + 8u * (uint32_t)st);
       }
     }
-  } else if (warp == 2 && !leader) {
-    // ------------------------------------------------------------ rank 1: forward "scale factors in TMEM"
-    dev::setmaxnreg_dec<kRegsCtl>();
-    if (lane == 0) {
-      const uint32_t psf0 = dev::map_to_rank(psf_ready, 0);
-      uint32_t sf_phase = 0;                        // per-slot parity of sf_ready (k-stages only)
-      int it = 0;
-      bool ok = true;
-      for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
-        if (p.branch) ++it;                         // branch stages carry no scale factors
-        for (int kt = 0; kt < ktiles; ++kt, ++it) {
-          const int s = it % kStages;
-          if (!dev::mbar_wait(&sf_ready[s], (sf_phase >> s) & 1u, abort_flag, p.budget_ns)) {
-            record_error(p.err, abort_flag, 0x22b);
-            ok = false;
-            break;
-          }
-          sf_phase ^= 1u << s;
-          dev::tc_fence_after();
-          dev::mbar_arrive_remote(psf0 + 8u * (uint32_t)s);
-        }
-      }
-    }
-  } else if (warp >= 2 && warp < kSfWarp0) {
+  } else if (warp < kSfWarp0) {
     dev::setmaxnreg_dec<kRegsCtl>();                 // idle warps of the first warpgroup
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
@@ -438,10 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           bias[4 * f + 2] = b4.z;
           bias[4 * f + 3] = b4.w;
         }
-        // the buffer of this chunk was last read by the store issued two chunks ago
-        if (lane == 0) dev::bulk_wait_group_read<1>();
+        // the buffer of this chunk was last read by the store issued kEpiBufs chunks ago
+        if (lane == 0) dev::bulk_wait_group_read<kEpiBufs - 1>();
         __syncwarp();
-        uint8_t* buf = wbuf + (chunk & 1) * kEpiBufBytes;
+        uint8_t* buf = wbuf + (chunk % kEpiBufs) * kEpiBufBytes;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t packed[4];
@@ -479,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   dev::tc_fence_before();
   __syncthreads();
   dev::cluster_sync();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     dev::tc_fence_after();
     dev::tmem_dealloc_pair(tmem, kTmemCols);
@@ -489,6 +464,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 int k2_pair_rows_b() { return kBNh; }
+
+size_t k2_pair_weight_bytes(int N, int K) {
+  const size_t nb = (size_t)((N + 255) / 256), ktiles = (size_t)((K / 64 + kKB - 1) / kKB);
+  return nb * ktiles * 2u * (size_t)kWBlockBytes;
+}
+
+void k2_pair_pack_weights(const uint8_t* tiled_codes, const uint8_t* sf, int N, int K, uint8_t* out) {
+  // tiled_codes: the single-CTA layout (wgt_tile_offset), 32 KB per (256-row
+  // block, stage); sf: the tensor-core scale layout, 512-byte chunks per
+  // (128-row block, 64-K block), rows padded to 256
+  const int nbl = (N + 255) / 256, kblocks = K / 64, ktiles = (kblocks + kKB - 1) / kKB;
+  for (int b = 0; b < nbl; ++b)
+    for (int t = 0; t < ktiles; ++t)
+      for (int h = 0; h < 2; ++h) {
+        uint8_t* dst = out + (((size_t)b * ktiles + t) * 2 + h) * kWBlockBytes;
+        const uint8_t* src = tiled_codes + ((size_t)b * ktiles + t) * 32768u + (size_t)h * kBBytes;
+        for (int i = 0; i < kBBytes; ++i) dst[i] = src[i];
+        for (int hh = 0; hh < 2; ++hh)
+          for (int j = 0; j < kKB; ++j) {
+            uint8_t* d = dst + kBBytes + hh * (kKB * 512) + j * 512;
+            const int kb = kKB * t + j;
+            if (kb < kblocks) {
+              const uint8_t* s = sf + ((size_t)(2 * b + hh) * kblocks + kb) * 512u;
+              for (int i = 0; i < 512; ++i) d[i] = s[i];
+            } else {
+              for (int i = 0; i < 512; ++i) d[i] = 0;
+            }
+          }
+      }
+}
 
 cudaError_t launch_k2_pair(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
                            const K2Params& p, int num_sms, cudaStream_t stream) {
@@ -517,8 +522,9 @@ cudaError_t launch_k2_pair(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, c
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  // programmatic dependent launch: the prologue overlaps the tail of the kernel
-  // that produces the activations; the producers wait for it before loading them
+  // programmatic dependent launch: the prologue and the weight stream overlap
+  // the tail of the kernel that produces the activations; the activation
+  // producer waits for it before its first load
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;

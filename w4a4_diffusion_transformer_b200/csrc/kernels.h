@@ -37,6 +37,7 @@ struct K2Params {
   float alpha;                  // g_x * g_w (power of two)
   const uint8_t* sfa;           // activation scales, tensor-core layout
   const uint8_t* sfb;           // weight scales, tensor-core layout (rows padded to 256)
+  const uint8_t* wpair;         // CTA-pair GEMM: weight codes and scales merged (k2_pair_pack_weights)
   const float* bias;            // [N]
   __nv_bfloat16* y;             // [M][N]
   int* err;
@@ -101,6 +102,13 @@ int k2_block_n();
 cudaError_t launch_k2_pair(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
                            const K2Params& p, int num_sms, cudaStream_t stream);
 int k2_pair_rows_b();
+// The pair GEMM's weight layout: per (256-row block, 256-K stage) and CTA half
+// h, the half's 16 KB of tiled codes followed by the 4 KB of scale factors of
+// all 256 rows (tensor-core layout, zero past K), so that each CTA moves its
+// weights of a stage in one contiguous copy.  Built from the single-CTA tiled
+// codes (wgt_tile_offset) and the tensor-core scale layout (rows padded to 256).
+size_t k2_pair_weight_bytes(int N, int K);
+void k2_pair_pack_weights(const uint8_t* tiled_codes, const uint8_t* sf, int N, int K, uint8_t* out);
 
 // INT4 GEMM: A = activation codes [M][K/2] (box 32 B x 128 rows), B = weight
 // codes [N][K/2] (box 32 B x 256 rows), both unswizzled.

@@ -346,9 +346,15 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
   return r;
 }
 
-// Arrive on an mbarrier of another CTA of the cluster (address from map_to_rank).
+// Arrive on an mbarrier of another CTA of the cluster (address from map_to_rank),
+// with release semantics at CTA scope (the instruction's default).  A release
+// at cluster scope waits for the CTA's outstanding memory traffic -- here the
+// bulk copies in flight -- and costs about a microsecond per arrive; the data
+// this arrive publishes (operand tiles whose copies have completed, TMEM
+// writes finished with tcgen05.wait::st or reads with tcgen05.wait::ld) is
+// complete before it.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
@@ -372,6 +378,54 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((++n & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > budget_ns) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait_cluster for barriers completed by arrivals from ANOTHER CTA of the
+// cluster (mbarrier.arrive on a shared::cluster address): a thread suspended
+// in try_wait is not woken promptly by such arrivals (about a microsecond
+// late on B200), so this polls without suspending (test_wait; mode 1) or with
+// a short suspend-time hint (try_wait; mode 2).
+template <int kMode = 1>
+__device__ __forceinline__ bool mbar_wait_remote(uint64_t* bar, uint32_t parity, const volatile int* abort_flag,
+                                                 uint64_t budget_ns) {
+  auto probe = [&]() {
+    return kMode == 1 ? mbar_test_wait_cluster(bar, parity)
+                      : kMode == 2 ? mbar_try_wait_cluster_hint(bar, parity, 20u) : mbar_try_wait_cluster(bar, parity);
+  };
+  if (probe()) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (probe()) return true;
+    if ((++n & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > budget_ns) return false;
     }
