@@ -655,9 +655,15 @@ svdq_status svdq_linear_forward(const svdq_layer* L, const void* X, int M, void*
       up.N = L->host.N;
       up.xl = static_cast<const __nv_bfloat16*>(xl);
       up.l2t = L->d_l2t;
-      up.y = static_cast<__nv_bfloat16*>(Y);
       up.gelu = gelu ? 1 : 0;
-      st = launch_upproj(up, s) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+      up.err = L->d_err;
+      up.budget_ns = L->budget_ns;
+      CUtensorMap tm_up;
+      if (!make_map(&tm_up, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L->host.N, M, 64, (uint32_t)upproj_box_rows(),
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+        st = SVDQ_ECUDA;
+      else
+        st = launch_upproj(tm_up, up, s) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
     }
   } else {
     const bool branch = has_branch && !(flags & SVDQ_FWD_NO_BRANCH);

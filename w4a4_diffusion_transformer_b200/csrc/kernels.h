@@ -65,8 +65,9 @@ struct UpParams {
   int M, N;
   const __nv_bfloat16* xl;      // [M][32]
   const __nv_bfloat16* l2t;     // [N][32] = L2b^T
-  __nv_bfloat16* y;             // [M][N], read and rewritten
   int gelu;
+  int* err;                     // device error word (a wait that ran out)
+  unsigned long long budget_ns;
 };
 
 struct W4A16Params {
@@ -122,7 +123,10 @@ cudaError_t launch_k2_int4_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b
                                 const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Int4Params& p,
                                 int num_sms, cudaStream_t stream);
 
-cudaError_t launch_upproj(const UpParams& p, cudaStream_t stream);
+// Y is read and rewritten through tm_y: a BF16 [M][N] map with boxes of 64
+// columns x upproj_box_rows() rows and the 128-byte swizzle.
+cudaError_t launch_upproj(const CUtensorMap& tm_y, const UpParams& p, cudaStream_t stream);
+int upproj_box_rows();
 
 // One-thread kernel whose only wait can never complete: it gives up after
 // budget_ns and sets *err (failure-detection self-test).
