@@ -60,8 +60,8 @@ constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRows = 16;                              // weight rows per tile (MMA M)
 constexpr int kGroupBytes = 544;                       // 512 bytes of codes + 32 of scales
-constexpr int kChunk = 4;                              // groups per chunk
-constexpr int kRing = 4;                               // chunk slots per warp (kRing - 1 chunks in flight)
+constexpr int kChunk = 6;                              // groups per chunk (one bulk copy)
+constexpr int kRing = 3;                               // chunk slots per warp (all of them in flight)
 constexpr int kChunkBytes = kChunk * kGroupBytes;
 constexpr int kSmemBudget = 227 * 1024;                 // dynamic shared memory per CTA
 
@@ -79,15 +79,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// 16-byte asynchronous copy global -> shared, cached in L2 only (the weights are read once).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 __device__ __forceinline__ uint4 lds128(const void* p) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -109,21 +100,35 @@ __device__ __forceinline__ float2 lds64f(const void* p) {
 constexpr int kPairs = kWarps / 2;
 
 // Shared memory: the warps' chunk rings, the second warp's partial sums per
-// pair (double-buffered by tile parity) and the per-group activation sums.
+// pair (double-buffered by tile parity), the per-group activation sums, one
+// mbarrier per chunk slot and, when it fits (XS), the pass's 8 MT activation
+// rows (rows padded by 16 bytes, so that the eight rows a fragment load reads
+// fall into different banks).
 template <int MT>
-__host__ __device__ inline size_t smem_bytes(int G) {
+__host__ __device__ inline size_t smem_fixed(int G) {
   return (size_t)kWarps * kRing * kChunkBytes +
-         sizeof(float) * ((size_t)kPairs * 2 * MT * 32 * 4 + (size_t)G * 8 * MT);
+         sizeof(float) * ((size_t)kPairs * 2 * MT * 32 * 4 + (size_t)G * 8 * MT) + 8u * kWarps * kRing + 8u;
+}
+__host__ __device__ inline size_t xs_stride(int G) { return (size_t)G * 128 + 16; }
+template <int MT, bool XS>
+__host__ __device__ inline size_t smem_bytes(int G) {
+  return (smem_fixed<MT>(G) + 15) / 16 * 16 + (XS ? (size_t)8 * MT * xs_stride(G) : 0);
 }
 
-// MT = number of 8-row activation tiles in this pass (1: M <= 8, 2: M <= 16).
-template <int MT>
+// MT = number of 8-row activation tiles in this pass (1: M <= 8, 2: M <= 16);
+// XS: the activation rows are staged in shared memory once per CTA (else every
+// group's fragments are read from global memory, on the critical path).
+template <int MT, bool XS>
 __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m0) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int K = p.K, G = K >> 6;
   uint8_t* ring = smem_raw + (size_t)(threadIdx.x >> 5) * kRing * kChunkBytes;   // this warp's chunk slots
   float* red = reinterpret_cast<float*>(smem_raw + (size_t)kWarps * kRing * kChunkBytes);   // [kPairs][2][MT][32][4]
   float* xsum = red + (size_t)kPairs * 2 * MT * 32 * 4;                    // [G][8 MT]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xsum + (size_t)G * 8 * MT) + (threadIdx.x >> 5) * kRing;
+  uint8_t* xs_smem = smem_raw + (smem_fixed<MT>(G) + 15) / 16 * 16;      // [8 MT][xs_stride] (XS)
+  int dummy_abort = 0;
+  const volatile int* no_abort = &dummy_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
@@ -135,22 +140,26 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
   const int ng = ge - gb, nchunks = (ng + kChunk - 1) / kChunk;
 
   // Chunk i of this warp's sequence = (tile i / nchunks, chunk i % nchunks): up to
-  // kChunk groups, copied into ring slot i % kRing.  One commit group per chunk
-  // index (empty past the end), so wait_group counts stay uniform.
+  // kChunk groups, which are contiguous in the packed layout, so lane 0 moves
+  // them with one bulk copy into ring slot i % kRing, completing that slot's
+  // mbarrier.  (Issued one by one from each of the 32 lanes, the copies made
+  // the kernel bound by instruction issue rather than by the weight stream.)
   const int nseq = my_tiles * nchunks;
+  if (lane == 0) {
+    for (int s = 0; s < kRing; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
   auto issue_chunk = [&](int i) {
-    if (i < nseq) {
+    if (i < nseq && lane == 0) {
       const int lt = i / nchunks, c = i - lt * nchunks;
       const size_t tile = (size_t)gpair + (size_t)lt * npairs;
       const uint8_t* src = p.wt + (tile * G + gb + (size_t)c * kChunk) * kGroupBytes;
-      uint8_t* dst = ring + (size_t)(i % kRing) * kChunkBytes;
-      const int n = min(kChunk, ng - c * kChunk);
-      for (int j = 0; j < n; ++j) {
-        cp_async16(dst + j * kGroupBytes + lane * 16, src + (size_t)j * kGroupBytes + lane * 16);
-        if (lane < 2) cp_async16(dst + j * kGroupBytes + 512 + lane * 16, src + (size_t)j * kGroupBytes + 512 + lane * 16);
-      }
+      const uint32_t bytes = (uint32_t)min(kChunk, ng - c * kChunk) * kGroupBytes;
+      uint64_t* bar = &bars[i % kRing];
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_load(ring + (size_t)(i % kRing) * kChunkBytes, src, bytes, bar);
     }
-    cp_async_commit();
   };
   // Activation sums per (group, column).  Each thread's first group of X is
   // requested before the first weight chunks, so that it does not queue behind
@@ -176,16 +185,63 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
       for (int v = 0; v < 8; ++v) u[v] = make_uint4(0u, 0u, 0u, 0u);
     }
   };
-  uint4 u0[8];
-  const bool first = (int)threadIdx.x < G * 8 * MT;
-  if (first) load_group(threadIdx.x, u0);
+  if (XS) {
+    // the pass's activation rows into shared memory (zeros past M), then the
+    // group sums from there.  Each thread's loads (eight at a time) go out
+    // before the weight copies, which would otherwise put them behind tens of
+    // megabytes of weights; the copies then fly while the rows are stored.
+    const int cpr = K / 8;                                          // 16-byte pieces per row
+    const int total = 8 * MT * cpr;
+    uint4 v[8];
+    auto load_batch = [&](int base) {
 #pragma unroll
-  for (int i = 0; i < kRing - 1; ++i) issue_chunk(i);
-  if (first) xsum[threadIdx.x] = group_sum(u0);
-  for (int i = threadIdx.x + kThreads; i < G * 8 * MT; i += kThreads) {
-    uint4 u[8];
-    load_group(i, u);
-    xsum[i] = group_sum(u);
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * kThreads;
+        const int r = i / cpr, c = i - r * cpr;
+        v[u] = (i < total && m0 + r < p.M) ? __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)(m0 + r) * K) + c)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    auto store_batch = [&](int base) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * kThreads;
+        const int r = i / cpr, c = i - r * cpr;
+        if (i < total) *reinterpret_cast<uint4*>(xs_smem + (size_t)r * xs_stride(G) + (size_t)c * 16) = v[u];
+      }
+    };
+    load_batch(threadIdx.x);
+    // every warp, whatever its share of X: the first chunk now, the rest of
+    // the ring once the rows are stored, so that the first chunks of all warps
+    // are not held up behind everyone's later ones
+    issue_chunk(0);
+    store_batch(threadIdx.x);
+    for (int base = threadIdx.x + 8 * kThreads; base < total; base += 8 * kThreads) {
+      load_batch(base);
+      store_batch(base);
+    }
+#pragma unroll
+    for (int i = 1; i < kRing; ++i) issue_chunk(i);
+    __syncthreads();
+    for (int i = threadIdx.x; i < G * 8 * MT; i += kThreads) {
+      const int gi = i / (8 * MT), r = i % (8 * MT);
+      uint4 u[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) u[v] = lds128(xs_smem + (size_t)r * xs_stride(G) + (size_t)gi * 128 + v * 16);
+      xsum[i] = group_sum(u);
+    }
+  } else {
+    uint4 u0[8];
+    const bool first = (int)threadIdx.x < G * 8 * MT;
+    if (first) load_group(threadIdx.x, u0);
+#pragma unroll
+    for (int i = 0; i < kRing; ++i) issue_chunk(i);
+    if (first) xsum[threadIdx.x] = group_sum(u0);
+    for (int i = threadIdx.x + kThreads; i < G * 8 * MT; i += kThreads) {
+      uint4 u[8];
+      load_group(i, u);
+      xsum[i] = group_sum(u);
+    }
   }
   __syncthreads();
 
@@ -202,7 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
   auto load_x = [&](int gi, uint32_t (&P)[MT][8]) {
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
-      if (xv[t]) {
+      if (XS) {
+        const uint8_t* xp = xs_smem + (size_t)(8 * t + g) * xs_stride(G) + (size_t)gi * 128 + q * 32;
+        const uint4 a = lds128(xp), b = lds128(xp + 16);
+        P[t][0] = a.x; P[t][1] = a.y; P[t][2] = a.z; P[t][3] = a.w;
+        P[t][4] = b.x; P[t][5] = b.y; P[t][6] = b.z; P[t][7] = b.w;
+      } else if (xv[t]) {
         const uint4* xs = reinterpret_cast<const uint4*>(xr[t] + 64 * (size_t)gi);
         const uint4 a = __ldg(xs), b = __ldg(xs + 1);
         P[t][0] = a.x; P[t][1] = a.y; P[t][2] = a.z; P[t][3] = a.w;
@@ -214,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
     }
   };
 
+  bool ok = true;
   for (int lt = 0; lt < my_tiles; ++lt) {
     const int tile = gpair + lt * npairs;
     float acc[MT][4];
@@ -223,9 +285,16 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
       for (int j = 0; j < 4; ++j) acc[t][j] = 0.f;
     for (int c = 0; c < nchunks; ++c) {
       const int i = lt * nchunks + c;
-      issue_chunk(i + kRing - 1);                    // keeps kRing - 1 chunks in flight
-      cp_async_wait<kRing - 1>();                    // chunk i has landed (this lane's copies)
-      __syncwarp();                                  // ... and every lane's
+      // chunk i has landed (bounded wait: a copy that never completes ends the
+      // kernel with the error word set instead of hanging it)
+      if (!ok || !__all_sync(0xffffffffu, mbar_wait(&bars[i % kRing], (uint32_t)(i / kRing) & 1u, no_abort,
+                                                     p.budget_ns))) {
+        // the warp stops computing but still meets its partner at the
+        // reduction barrier below, so neither warp of the pair is left waiting
+        if (ok && lane == 0) atomicExch(p.err, 1);
+        ok = false;
+        break;
+      }
       const uint8_t* slot = ring + (size_t)(i % kRing) * kChunkBytes;
       const int n = min(kChunk, ng - c * kChunk);
 #pragma unroll
@@ -236,15 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
           load_x(gi, P);
           const uint4 cw = lds128(slot + j * kGroupBytes + lane * 16);
           const uint32_t swj = lds32(slot + j * kGroupBytes + 512 + g * 4);
-          // the four MMA steps of a group accumulate into independent fragments
-          // (the tensor-core MMA has a long latency: no chain between them)
-          float pst[4][MT][4];
+          // the four MMA steps of a group accumulate into one fragment: with
+          // sixteen warps per SM the chain's latency is hidden by the other
+          // warps, and the kernel is bound by instruction issue, so fewer
+          // instructions per group is what counts
+          float pst[MT][4];
 #pragma unroll
-          for (int st = 0; st < 4; ++st)
+          for (int t = 0; t < MT; ++t)
 #pragma unroll
-            for (int t = 0; t < MT; ++t)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) pst[st][t][e] = 0.f;
+            for (int e = 0; e < 4; ++e) pst[t][e] = 0.f;
 #pragma unroll
           for (int st = 0; st < 4; ++st) {
             // MMA step st: positions (2q, 2q+1) <- codes 4st, 4st+1 and (2q+8, 2q+9) <- 4st+2, 4st+3
@@ -255,23 +324,23 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
             const uint32_t a[4] = {codes_pair(wa >> sh), codes_pair(wb >> sh), codes_pair(wa >> (sh + 4)),
                                    codes_pair(wb >> (sh + 4))};
 #pragma unroll
-            for (int t = 0; t < MT; ++t) mma_bf16_16816(pst[st][t], a, P[t][2 * st], P[t][2 * st + 1]);
+            for (int t = 0; t < MT; ++t) mma_bf16_16816(pst[t], a, P[t][2 * st], P[t][2 * st + 1]);
           }
           const float s0 = __uint_as_float(swj << 16), s1 = __uint_as_float(swj & 0xFFFF0000u);
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
-            // sum the steps, minus 136 * sum(x): the biased codes (c + 136) give sum(x c)
+            // minus 136 * sum(x): the biased codes (c + 136) give sum(x c)
             const float2 xs = lds64f(&xsum[gi * 8 * MT + 8 * t + 2 * q]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float part =
-                  ((pst[0][t][e] + pst[1][t][e]) + (pst[2][t][e] + pst[3][t][e])) - 136.f * ((e & 1) ? xs.y : xs.x);
-              acc[t][e] = fmaf((e & 2) ? s1 : s0, part, acc[t][e]);
-            }
+            for (int e = 0; e < 4; ++e)
+              acc[t][e] = fmaf((e & 2) ? s1 : s0, pst[t][e] - 136.f * ((e & 1) ? xs.y : xs.x), acc[t][e]);
           }
         }
       }
-      __syncwarp();                                  // every lane is done with the slot before it is refilled
+      // every lane is done with the slot before the copy engine refills it
+      fence_async_shared();
+      __syncwarp();
+      issue_chunk(i + kRing);
     }
     // the pair's split-K reduction (double-buffered by tile parity): the second
     // warp hands its partials over, the first adds and stores; fragment element
@@ -292,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
           const int n = tile * kRows + g + ((e & 2) ? 8 : 0);
           const int m = m0 + 8 * t + 2 * q + (e & 1);
           const float v = acc[t][e] + r[(t * 32 + lane) * 4 + e];
-          if (n < p.N && m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v + p.bias[n]);
+          if (ok && n < p.N && m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v + p.bias[n]);
         }
     }
   }
@@ -300,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(W4A16Params p, int m
 
 }  // namespace
 
-bool w4a16_supported(int K) { return smem_bytes<2>(K / 64) <= (size_t)kSmemBudget; }
+bool w4a16_supported(int K) { return smem_bytes<2, false>(K / 64) <= (size_t)kSmemBudget; }
 
 size_t w4a16_packed_bytes(int N, int K) {
   return (size_t)((N + kRows - 1) / kRows) * (size_t)(K / 64) * kGroupBytes;
@@ -339,7 +408,7 @@ void w4a16_pack(const uint8_t* codes, const uint16_t* scales, int N, int K, uint
 namespace {
 
 // Grid size (one CTA per SM), configured once per device and shared-memory size.
-template <int MT>
+template <int MT, bool XS>
 cudaError_t grid_size(size_t smem, int ntiles, int* grid) {
   struct Entry {
     size_t smem = 0;
@@ -354,7 +423,7 @@ cudaError_t grid_size(size_t smem, int ntiles, int* grid) {
   std::lock_guard<std::mutex> lock(mu);
   Entry& c = cache[dev];
   if (c.smem < smem) {
-    if ((e = cudaFuncSetAttribute(w4a16_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+    if ((e = cudaFuncSetAttribute(w4a16_kernel<MT, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
         cudaSuccess)
       return e;
     if ((e = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
@@ -364,15 +433,22 @@ cudaError_t grid_size(size_t smem, int ntiles, int* grid) {
   return cudaSuccess;
 }
 
+template <int MT, bool XS>
+cudaError_t launch_pass_t(const W4A16Params& p, int m0, cudaStream_t stream) {
+  const int ntiles = (p.N + kRows - 1) / kRows;
+  const size_t smem = smem_bytes<MT, XS>(p.K / 64);
+  int grid = 0;
+  cudaError_t e = grid_size<MT, XS>(smem, ntiles, &grid);
+  if (e != cudaSuccess) return e;
+  w4a16_kernel<MT, XS><<<grid, kThreads, smem, stream>>>(p, m0);
+  return cudaGetLastError();
+}
+
 template <int MT>
 cudaError_t launch_pass(const W4A16Params& p, int m0, cudaStream_t stream) {
-  const int ntiles = (p.N + kRows - 1) / kRows;
-  const size_t smem = smem_bytes<MT>(p.K / 64);
-  int grid = 0;
-  cudaError_t e = grid_size<MT>(smem, ntiles, &grid);
-  if (e != cudaSuccess) return e;
-  w4a16_kernel<MT><<<grid, kThreads, smem, stream>>>(p, m0);
-  return cudaGetLastError();
+  // activations staged in shared memory whenever they fit beside the rings
+  return smem_bytes<MT, true>(p.K / 64) <= (size_t)kSmemBudget ? launch_pass_t<MT, true>(p, m0, stream)
+                                                                : launch_pass_t<MT, false>(p, m0, stream);
 }
 
 }  // namespace
