@@ -12,8 +12,8 @@
 //
 // Layout of the work: a CTA owns 32 token rows and streams the whole K range in
 // stages of 256 columns.  Two producer warps load with TMA (one 3D copy per
-// stage over a 64-column-chunk view): one feeds an 8-deep ring of X tiles
-// (+ 256 floats of inv_lam) from HBM, the other a 3-deep ring of the matching
+// stage over a 64-column-chunk view): one feeds a 6-deep ring of X tiles
+// (+ 256 floats of inv_lam) from HBM, the other a 5-deep ring of the matching
 // 256 x 32 slices of L1d^T, which every CTA reads from L2.  The consumer warps
 // are specialized and never wait for each other inside the loop:
 //   * 8 quantizer warps: warp w owns columns 32w..32w+31 of the stage (two
@@ -53,8 +53,16 @@ namespace {
 
 constexpr int kRows = 32;
 constexpr int kBK = 256;
-constexpr int kXStages = 8;                  // X + inv_lam ring (HBM stream)
-constexpr int kLStages = 3;                  // L1d^T ring (L2-resident)
+// Ring depths (measured at the attention-output shape: 6 X + 5 L1d^T stages
+// 12.8 us per launch back to back, 8 + 3 stages 13.1 us).
+#ifndef SVDQ_K1_XSTAGES
+#define SVDQ_K1_XSTAGES 6
+#endif
+#ifndef SVDQ_K1_LSTAGES
+#define SVDQ_K1_LSTAGES 5
+#endif
+constexpr int kXStages = SVDQ_K1_XSTAGES;     // X + inv_lam ring (HBM stream)
+constexpr int kLStages = SVDQ_K1_LSTAGES;     // L1d^T ring (L2-resident)
 constexpr int kMmaWarps = 8;
 constexpr int kXBytes = kRows * kBK * 2;     // 4 sub-tiles of 32 rows x 128 B
 constexpr int kLBytes = 32 * kBK * 2;        // 4 sub-tiles of 32 rows x 128 B
