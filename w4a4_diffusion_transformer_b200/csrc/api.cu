@@ -28,8 +28,9 @@ struct svdq_layer {
   __nv_bfloat16* d_l1t = nullptr;    // [32][K]   L1d^T
   __nv_bfloat16* d_l2s = nullptr;    // [N][32]   (L2b / alpha)^T
   __nv_bfloat16* d_l2t = nullptr;    // [N][32]   L2b^T (unfused up projection)
-  uint8_t* d_wq = nullptr;           // [N][K/2]
-  uint8_t* d_ws = nullptr;           // weight scales: NVFP4 tensor-core layout; INT4 FP16 [K/64][npad] (times 2^-ew)
+  uint8_t* d_wq = nullptr;           // INT4: codes [N][K/2]; W4A16: the GEMV's packed weights
+  uint8_t* d_ws = nullptr;           // INT4: weight scales, FP16 [K/64][npad] (times 2^-ew)
+  uint8_t* d_wmerged = nullptr;      // NVFP4: codes and scales merged for the single-CTA GEMM
   uint8_t* d_wpair = nullptr;        // NVFP4: codes and scales merged for the CTA-pair GEMM
   int i4_ex = 0, i4_ew = 0;          // INT4: power-of-two range exponents of the FP16 GEMM operands
   float* d_bias = nullptr;           // [N]
@@ -174,6 +175,7 @@ void free_device(svdq_layer* L) {
   cudaFree(L->d_l2t);
   cudaFree(L->d_wq);
   cudaFree(L->d_ws);
+  cudaFree(L->d_wmerged);
   cudaFree(L->d_wpair);
   cudaFree(L->d_bias);
   cudaFree(L->d_err);
@@ -209,7 +211,6 @@ svdq_status upload_layer(svdq_layer* L, int device) {
       for (int n = 0; n < N; ++n)
         for (int b = 0; b < K / 2; ++b)
           tiled[wgt_tile_offset(n, b >> 7, (b & 127) >> 4, nst) + (b & 15)] = h.w_codes[(size_t)n * (K / 2) + b];
-      chk(upload(&L->d_wq, tiled.data(), tiled.size()));
     } else {
       chk(upload(&L->d_wq, h.w_codes.data(), h.w_codes.size()));
     }
@@ -220,8 +221,10 @@ svdq_status upload_layer(svdq_layer* L, int device) {
       std::vector<uint8_t> ws((size_t)(npad / 128) * (K / 64) * 512, 0);
       for (int n = 0; n < N; ++n)
         for (int gi = 0; gi < K / 16; ++gi) ws[sf_offset(n, gi, K)] = h.w_scales_e4m3[(size_t)n * (K / 16) + gi];
-      chk(upload(&L->d_ws, ws.data(), ws.size()));
-      // the CTA-pair GEMM's merged copy of both
+      // codes and scales merged, one layout per GEMM variant
+      std::vector<uint8_t> wm(k2_weight_bytes(N, K));
+      k2_pack_weights(tiled.data(), ws.data(), N, K, wm.data());
+      chk(upload(&L->d_wmerged, wm.data(), wm.size()));
       std::vector<uint8_t> wpair(k2_pair_weight_bytes(N, K));
       k2_pair_pack_weights(tiled.data(), ws.data(), N, K, wpair.data());
       chk(upload(&L->d_wpair, wpair.data(), wpair.size()));
@@ -384,10 +387,9 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
   p.K = h.K;
   p.mpad = pad_rows(M);
   p.acodes = static_cast<const uint8_t*>(codes);
-  p.wcodes = L->d_wq;
   p.alpha = (float)std::ldexp(1.0, h.g_x_exp + h.g_w_exp);
   p.sfa = static_cast<const uint8_t*>(scales);
-  p.sfb = L->d_ws;
+  p.wmerged = L->d_wmerged;
   p.wpair = L->d_wpair;
   p.bias = L->d_bias;
   p.y = static_cast<__nv_bfloat16*>(Y);

@@ -33,10 +33,9 @@ struct K2Params {
   int M, N, K;
   int mpad;                     // rows of the activation scale layout (M rounded up to 128)
   const uint8_t* acodes;        // activation codes, tiled layout (act_tile_offset), mpad rows
-  const uint8_t* wcodes;        // weight codes, tiled layout (wgt_tile_offset), N rounded up to 256 rows
   float alpha;                  // g_x * g_w (power of two)
   const uint8_t* sfa;           // activation scales, tensor-core layout
-  const uint8_t* sfb;           // weight scales, tensor-core layout (rows padded to 256)
+  const uint8_t* wmerged;       // single-CTA GEMM: weight codes and scales merged (k2_pack_weights)
   const uint8_t* wpair;         // CTA-pair GEMM: weight codes and scales merged (k2_pair_pack_weights)
   const float* bias;            // [N]
   __nv_bfloat16* y;             // [M][N]
@@ -93,11 +92,16 @@ cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CU
                       const K1Params& p, int fmt, int mode, cudaStream_t stream);
 int k1_rows_per_cta();
 
-// NVFP4 GEMM: operands from p.acodes / p.wcodes (tiled layouts); tm_xl / tm_l2
-// the branch tiles, tm_y the output.
+// NVFP4 GEMM: operands from p.acodes / p.sfa (the first kernel's layouts) and
+// p.wmerged; tm_xl / tm_l2 the branch tiles, tm_y the output.
 cudaError_t launch_k2(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
                       const K2Params& p, int num_sms, cudaStream_t stream);
 int k2_block_n();
+// The single-CTA GEMM's weight layout: per (256-row block, 256-K stage) the 32 KB
+// of tiled codes (wgt_tile_offset) followed by the 4 KB of scale factors of the
+// block's 256 rows (tensor-core layout, zero past K): one contiguous copy per stage.
+size_t k2_weight_bytes(int N, int K);
+void k2_pack_weights(const uint8_t* tiled_codes, const uint8_t* sf, int N, int K, uint8_t* out);
 // The same GEMM on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2, clusters of
 // two): tm_l2 has 128-row boxes (each CTA holds half of B).
 cudaError_t launch_k2_pair(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
