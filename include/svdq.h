@@ -63,13 +63,41 @@ typedef enum {
 } svdq_format;
 
 /* Offline configuration.  rank: 32 (or 0 = no low-rank branch); alpha:
- * smoothing migration strength (0.5).  flags: reserved, pass 0. */
+ * smoothing migration strength (0.5).  flags: SVDQ_PREP_* bits (0 = the
+ * round-to-nearest residual). */
 typedef struct {
   int format;
   int rank;
   float alpha;
   unsigned flags;
 } svdq_config;
+
+/* Preparation flags.
+ *
+ * SVDQ_PREP_GPTQ quantizes the residual with GPTQ instead of round-to-nearest
+ * (SOTA-314 practice page, "Do this": the residual is quantized with GPTQ, which
+ * improves quality in most of the paper's settings).  The pages do not restate
+ * GPTQ; this is the published algorithm (Frantar et al. 2022) in its plain
+ * column-by-column form:
+ *   H = X_hat^T X_hat over the calibration batch, X_hat = fp32(Xc / lam) (the
+ *       smoothed activations the residual multiplies); a channel with H_kk = 0
+ *       gets H_kk = 1; every H_kk then grows by 1% of the mean diagonal;
+ *   U = the upper-triangular Cholesky factor of H^-1 (H^-1 = U^T U);
+ *   the input channels k are visited in order: where k starts a group (16 for
+ *       NVFP4, 64 for INT4) that group's scale is fixed from the current
+ *       values, w_k is quantized with it exactly as round-to-nearest would,
+ *       err = (w_k - deq_k) / U_kk, and every later channel j moves by
+ *       -U_kj err.  Working values are float64; the quantizer sees their
+ *       float32 rounding.  The NVFP4 tensor scale g_w still comes from R.
+ * Only the W4A4 formats (it needs the calibration batch); the forward kernels
+ * and the layout of the prepared codes are unchanged.  Host cost: a K x K
+ * factorisation (about K^3 / 3 multiply-adds twice) and K^2 N / 2 updates.
+ *
+ * SVDQ_PREP_KEEP_GPTQ_FACTOR (with SVDQ_PREP_GPTQ) keeps U on the host for
+ * svdq_export(SVDQ_T_GPTQ_U) -- K^2 doubles, e.g. 75 MB at K = 3072; without it
+ * U is freed when svdq_prepare returns. */
+#define SVDQ_PREP_GPTQ             0x1u
+#define SVDQ_PREP_KEEP_GPTQ_FACTOR 0x2u
 
 typedef struct svdq_layer svdq_layer;   /* opaque */
 
@@ -104,7 +132,9 @@ typedef enum {
   SVDQ_T_W_CODES = 8,       /* uint8 [N][K/2]  residual codes, K-major, even k low  */
   SVDQ_T_W_SCALES = 9,      /* NVFP4: uint8 [N][K/16] E4M3; INT4: uint16 [N][K/64] BF16 */
   SVDQ_T_BIAS = 10,         /* float [N]                                            */
-  SVDQ_T_COUNT = 11
+  SVDQ_T_GPTQ_U = 11,       /* double [K][K]   GPTQ factor U (upper, H^-1 = U^T U); only
+                               with SVDQ_PREP_GPTQ | SVDQ_PREP_KEEP_GPTQ_FACTOR      */
+  SVDQ_T_COUNT = 12
 } svdq_tensor;
 
 /* ------------------------------------------------------------------ offline */
@@ -113,7 +143,9 @@ typedef enum {
  * (SOTA-314 "Do this": smooth, "compute the SVD of the smoothed weight, keep
  * the top r singular directions in 16 bits, and quantize only the residual").
  *
- *   cfg        format, rank (0 or 32), alpha (> 0 and < 1; 0.5 recommended).
+ *   cfg        format, rank (0 or 32), alpha (> 0 and < 1; 0.5 recommended),
+ *              flags (SVDQ_PREP_*; unknown bits, or SVDQ_PREP_GPTQ with
+ *              SVDQ_W4A16_INT4, or KEEP without GPTQ give SVDQ_EINVAL).
  *   K, N       input and output features.
  *   W_bf16     host, [K][N] row-major BF16 weight (Y = X W + b); read only.
  *   bias_bf16  host, [N] BF16, or NULL for no bias.
@@ -129,7 +161,8 @@ typedef enum {
  * rules; for SVDQ_NVFP4 also a calibration batch whose largest smoothed
  * magnitude puts the activation tensor-scale exponent outside [-40, 30], i.e.
  * below about 3e-10 or above about 7e11), SVDQ_ENOMEM, SVDQ_ECUDA,
- * SVDQ_ENOCONVERGE (the SVD's energy check failed).
+ * SVDQ_ENOCONVERGE (the SVD's energy check failed, or the GPTQ Hessian was
+ * not positive definite after damping -- only with non-finite calibration).
  * On error *out is set to NULL and nothing leaks. */
 svdq_status svdq_prepare(const svdq_config* cfg, int K, int N,
                          const uint16_t* W_bf16, const uint16_t* bias_bf16,

@@ -38,7 +38,12 @@ design notes of the repository):
   * the code of a group element is E2M1(fp32(v * fp32(1/(s*g)))), with v the
     float32 value fed to the quantizer;
   * INT4 is symmetric in [-7, 7], its 16-bit scale is BF16: s = bf16(fp32(a * fp32(1/7)));
-  * two codes per byte, the even k in the low nibble.
+  * two codes per byte, the even k in the low nibble;
+  * GPTQ (the pages' residual quantizer, named but not restated) is the
+    published column-by-column algorithm: H = X_hat^T X_hat of the smoothed
+    calibration batch, dead channels H_kk = 1, damping 1% of the mean
+    diagonal, U = upper Cholesky factor of H^-1, channels in natural order,
+    a group's scale fixed from the updated values when the group starts.
 """
 from __future__ import annotations
 
@@ -176,6 +181,28 @@ def pow2_exponent_ceil(x: float) -> int:
     return e - 1 if m == 0.5 else e
 
 
+def nvfp4_group_scale(a: np.ndarray, g_exp: int):
+    """Scale of NVFP4 groups with float32 maxima a: t = fp32(a * c) with
+    c = fp32(1/6) * 2^-g_exp; s = E4M3(t).  Returns s (float64 holding the E4M3
+    value) and inv = fp32(1 / fp32(s * g)), 0 where s == 0."""
+    a = np.asarray(a, dtype=F32)
+    c = F32(np.ldexp(np.float64(F32(1.0 / 6.0)), -g_exp))
+    t = (a * c).astype(F32)                                      # one float32 multiply
+    s = e4m3_round_satfinite(t.astype(np.float64))
+    sg = fp32(s * np.ldexp(1.0, g_exp))                          # exact (power-of-two scaling)
+    with np.errstate(divide="ignore"):
+        inv = (F32(1.0) / sg).astype(F32)                        # IEEE float32 division
+    return s, np.where(s == 0, F32(0.0), inv).astype(F32)
+
+
+def nvfp4_codes(v: np.ndarray, s: np.ndarray, inv: np.ndarray) -> np.ndarray:
+    """E2M1 codes of float32 values v under scales s / reciprocals inv
+    (broadcast against v): code = E2M1(fp32(v * inv)); +0 where s == 0."""
+    q = (np.asarray(v, dtype=F32) * inv).astype(F32)             # one float32 multiply
+    codes = e2m1_encode(q.astype(np.float64))
+    return np.where(s == 0, np.uint8(0), codes).astype(np.uint8)
+
+
 def nvfp4_quantize(v: np.ndarray, g_exp: int) -> Dict[str, np.ndarray]:
     """NVFP4 quantization of the rows of v (float32, [rows, K]) in groups of 16
     consecutive k, with tensor scale g = 2^g_exp.
@@ -190,20 +217,27 @@ def nvfp4_quantize(v: np.ndarray, g_exp: int) -> Dict[str, np.ndarray]:
     assert K % NVFP4_GROUP == 0
     grp = v.reshape(rows, K // NVFP4_GROUP, NVFP4_GROUP)
     a = np.max(np.abs(grp), axis=2)                              # float32, exact
-    c = F32(np.ldexp(np.float64(F32(1.0 / 6.0)), -g_exp))
-    t = (a * c).astype(F32)                                      # one float32 multiply
-    s = e4m3_round_satfinite(t.astype(np.float64))               # float64 holding an E4M3 value
-    g = np.ldexp(1.0, g_exp)
-    sg = fp32(s * g)                                             # exact (power-of-two scaling)
-    with np.errstate(divide="ignore"):
-        inv = (F32(1.0) / sg).astype(F32)                        # IEEE float32 division
-    inv = np.where(s == 0, F32(0.0), inv).astype(F32)
-    q = (grp * inv[:, :, None]).astype(F32)                      # one float32 multiply
-    codes = e2m1_encode(q.astype(np.float64))
-    codes = np.where((s == 0)[:, :, None], np.uint8(0), codes).astype(np.uint8)
-    deq = e2m1_decode(codes) * (s * g)[:, :, None]
+    s, inv = nvfp4_group_scale(a, g_exp)
+    codes = nvfp4_codes(grp, s[:, :, None], inv[:, :, None])
+    deq = e2m1_decode(codes) * (s * np.ldexp(1.0, g_exp))[:, :, None]
     return {"codes": codes.reshape(rows, K), "scale_bytes": e4m3_encode(s),
             "scales": s, "deq": deq.reshape(rows, K)}
+
+
+def int4_group_scale(a: np.ndarray):
+    """Scale of INT4 groups with float32 maxima a: s = bf16(fp32(a * fp32(1/7)));
+    returns s (float64 holding the BF16 value) and inv = fp32(1 / s), 0 where s == 0."""
+    a = np.asarray(a, dtype=F32)
+    s = bf16_round((a * F32(1.0 / 7.0)).astype(F32))
+    with np.errstate(divide="ignore"):
+        inv = (F32(1.0) / s.astype(F32)).astype(F32)
+    return s, np.where(s == 0, F32(0.0), inv).astype(F32)
+
+
+def int4_codes(v: np.ndarray, inv: np.ndarray) -> np.ndarray:
+    """code = clamp(rint_even(fp32(v * inv)), -7, 7) as int8 (0 where inv == 0)."""
+    q = (np.asarray(v, dtype=F32) * inv).astype(F32)
+    return np.clip(np.rint(q.astype(np.float64)), -INT4_QMAX, INT4_QMAX).astype(np.int8)
 
 
 def int4_quantize(v: np.ndarray) -> Dict[str, np.ndarray]:
@@ -217,13 +251,8 @@ def int4_quantize(v: np.ndarray) -> Dict[str, np.ndarray]:
     assert K % INT4_GROUP == 0
     grp = v.reshape(rows, K // INT4_GROUP, INT4_GROUP)
     a = np.max(np.abs(grp), axis=2)
-    s = bf16_round((a * F32(1.0 / 7.0)).astype(F32))
-    s32 = s.astype(F32)
-    with np.errstate(divide="ignore"):
-        inv = (F32(1.0) / s32).astype(F32)
-    inv = np.where(s == 0, F32(0.0), inv).astype(F32)
-    q = (grp * inv[:, :, None]).astype(F32)
-    codes = np.clip(np.rint(q.astype(np.float64)), -INT4_QMAX, INT4_QMAX).astype(np.int8)
+    s, inv = int4_group_scale(a)
+    codes = int4_codes(grp, inv[:, :, None])
     deq = codes.astype(np.float64) * s[:, :, None]
     return {"codes": codes.reshape(rows, K), "scales": s, "deq": deq.reshape(rows, K)}
 
@@ -272,14 +301,17 @@ def svd_split(W_hat: np.ndarray, rank: int):
 
 
 def prepare(W: np.ndarray, bias: Optional[np.ndarray], Xc: np.ndarray, fmt: str = "nvfp4",
-            rank: int = 32, alpha: float = 0.5, svd=None) -> Dict[str, np.ndarray]:
+            rank: int = 32, alpha: float = 0.5, svd=None, method: str = "rtn",
+            gptq_U: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """Offline pipeline: smooth -> SVD of W_hat -> keep the top r directions in
     16 bits -> quantize only the residual.  [P "Do this": "Compute the SVD of
     the smoothed weight W_hat, keep the top r singular directions in 16 bits,
     and quantize only the residual R = W_hat - L1 L2"; rank 32 at 4 bits.]
 
     ``svd`` may supply (L1, L2) to replace the LAPACK split (used to compare
-    against another implementation's factors on shared inputs)."""
+    against another implementation's factors on shared inputs).  ``method``
+    picks the residual quantizer: "rtn" (round to nearest) or "gptq"; ``gptq_U``
+    may supply the GPTQ factor (same purpose as ``svd``)."""
     W = np.asarray(W, dtype=np.float64)
     K, N = W.shape
     lam, inv = smoothing_factors(Xc, W, alpha)
@@ -301,7 +333,14 @@ def prepare(W: np.ndarray, bias: Optional[np.ndarray], Xc: np.ndarray, fmt: str 
            "lam": lam, "inv_lam": inv, "L1": L1, "L2": L2, "S": S,
            "L1d": L1d, "L2b": L2b, "R": R,
            "bias": np.zeros(N) if bias is None else np.asarray(bias, dtype=np.float64)}
-    out.update(quantize_weights(R, fmt))
+    if method == "rtn":
+        out.update(quantize_weights(R, fmt))
+    elif method == "gptq":
+        U = gptq_factor(gptq_hessian(Xc, inv)) if gptq_U is None else gptq_U
+        out.update(gptq_quantize(R, U, fmt))
+        out["gptq_U"] = U
+    else:
+        raise ValueError(method)
     out["g_x_exp"] = activation_tensor_exponent(Xc, inv) if fmt == "nvfp4" else 0
     return out
 
@@ -330,6 +369,91 @@ def quantize_weights(R: np.ndarray, fmt: str, g_exp: Optional[int] = None) -> Di
         q = int4_quantize(Rt)
         return {"g_w_exp": 0, "w_codes": q["codes"], "w_scales": q["scales"], "w_deq": q["deq"]}
     raise ValueError(fmt)
+
+
+# --------------------------------------------------------------------------
+# GPTQ residual quantization  [P "Do this": the residual is quantized with
+# GPTQ rather than round-to-nearest; N "Key results", the quality table rows]
+#
+# The pages name GPTQ without restating it; this is the published algorithm
+# (Frantar et al., "GPTQ: Accurate Post-Training Quantization for Generative
+# Pre-trained Transformers", 2022) in its plain column-by-column form: the
+# lazy block updates of that paper only reorder the same arithmetic.
+#   * the loss of output column n is ||X_hat (r_n - q_n)||^2 with X_hat the
+#     smoothed calibration activations, so H = X_hat^T X_hat for every n;
+#   * a channel that never fires (H_kk = 0) gets H_kk = 1, then every H_kk
+#     grows by 1% of the mean diagonal (the paper's damping);
+#   * U = upper Cholesky factor of H^-1 (H^-1 = U^T U);
+#   * input channels k are visited in order; when k starts a group, that
+#     group's scale is fixed from the current (already updated) values;
+#     w_k is quantized with it, err = (w_k - deq_k) / U_kk and every later
+#     channel j > k moves by -U_kj err.
+# Working values are float64; the quantizer sees their float32 rounding and
+# takes its decisions exactly as round-to-nearest does.
+# --------------------------------------------------------------------------
+
+GPTQ_DAMP = 0.01
+
+
+def gptq_hessian(Xc: np.ndarray, inv_lam: np.ndarray, damp: float = GPTQ_DAMP) -> np.ndarray:
+    """Damped H = X_hat^T X_hat (float64), X_hat = fp32(Xc * inv_lam)."""
+    Xh = smoothed_activations(Xc, inv_lam).astype(np.float64)
+    H = Xh.T @ Xh
+    d = np.diag(H).copy()
+    dead = np.flatnonzero(d == 0)
+    H[dead, dead] = 1.0
+    H[np.diag_indices_from(H)] += damp * float(np.mean(np.diag(H)))
+    return H
+
+
+def gptq_factor(H: np.ndarray) -> np.ndarray:
+    """Upper-triangular U with positive diagonal and U^T U = H^-1."""
+    Hinv = np.linalg.inv(np.asarray(H, dtype=np.float64))
+    Hinv = 0.5 * (Hinv + Hinv.T)
+    return np.linalg.cholesky(Hinv).T
+
+
+def gptq_quantize(R: np.ndarray, U: np.ndarray, fmt: str, g_exp: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """GPTQ quantization of the residual R [K, N] with factor U [K, K]; the
+    result has the keys of quantize_weights (codes [N, K], K-major).  For NVFP4
+    the tensor scale g_w comes from the unmodified R, as round-to-nearest's does."""
+    W = np.array(R, dtype=F32).astype(np.float64)
+    K, N = W.shape
+    U = np.asarray(U, dtype=np.float64)
+    if fmt == "nvfp4":
+        G = NVFP4_GROUP
+        e = weight_tensor_exponent(R) if g_exp is None else g_exp
+        g = np.ldexp(1.0, e)
+    elif fmt in ("int4", "w4a16"):
+        G = INT4_GROUP
+        e = 0
+    else:
+        raise ValueError(fmt)
+    codes = np.zeros((N, K), dtype=np.uint8 if fmt == "nvfp4" else np.int8)
+    scales = np.zeros((N, K // G))
+    deq = np.zeros((N, K))
+    fed = np.zeros((N, K))                  # the working value of w_k when it is quantized
+    for k in range(K):
+        if k % G == 0:
+            a = np.max(np.abs(W[k:k + G, :].astype(F32)), axis=0)
+            s, inv = nvfp4_group_scale(a, e) if fmt == "nvfp4" else int4_group_scale(a)
+            scales[:, k // G] = s
+        fed[:, k] = W[k, :]
+        v = W[k, :].astype(F32)
+        if fmt == "nvfp4":
+            c = nvfp4_codes(v, s, inv)
+            d = e2m1_decode(c) * (s * g)
+        else:
+            c = int4_codes(v, inv)
+            d = c.astype(np.float64) * s
+        codes[:, k] = c
+        deq[:, k] = d
+        err = (W[k, :] - d) / U[k, k]
+        W[k + 1:, :] -= np.outer(U[k, k + 1:], err)
+    out = {"g_w_exp": e, "w_codes": codes, "w_scales": scales, "w_deq": deq, "w_fed": fed}
+    if fmt == "nvfp4":
+        out["w_scale_bytes"] = e4m3_encode(scales)
+    return out
 
 
 def smoothed_activations(X: np.ndarray, inv_lam: np.ndarray) -> np.ndarray:

@@ -40,6 +40,7 @@ ROLE_X_RUN = 4
 ROLE_X_CALIB = 5
 ROLE_BIAS = 6
 ROLE_X_HELDOUT = 7
+ROLE_X_LATENT = 8
 
 CALIB_TOKENS = 256
 SPIKES = 32
@@ -47,6 +48,7 @@ OUTLIER_FRACTION = 0.01
 OUTLIER_GAIN = 50.0
 SPIKE_DECAY = 0.85
 BIAS_VARIANCE = 0.02
+LATENT_NOISE = 0.5
 
 
 @dataclasses.dataclass(frozen=True)
@@ -135,6 +137,21 @@ def activations(workload_id: int, layer_id: int, M: int, K: int, role: int,
     return to_bf16(x)
 
 
+def correlated_activations(workload_id: int, layer_id: int, M: int, K: int, role: int,
+                           latent_rank: int, outliers: bool = True) -> np.ndarray:
+    """X = Z A + 0.5 E: every channel mixes the same latent_rank directions
+    (Z ~ N(0,1) [M, r] drawn per batch, A ~ N(0, 1/r) [r, K] fixed per layer),
+    plus independent N(0,1) noise E; outlier channels x50; rounded to BF16.
+    Channels of a real layer's input are correlated like this, and GPTQ's
+    error feedback works through exactly that correlation."""
+    g = rng(workload_id, layer_id, role)
+    A = rng(workload_id, layer_id, ROLE_X_LATENT).standard_normal((latent_rank, K)) / np.sqrt(latent_rank)
+    x = g.standard_normal((M, latent_rank)) @ A + LATENT_NOISE * g.standard_normal((M, K))
+    if outliers:
+        x[:, outlier_channels(workload_id, layer_id, K)] *= OUTLIER_GAIN
+    return to_bf16(x)
+
+
 def weights(workload_id: int, layer_id: int, K: int, N: int, sigma0: float,
             spikes: int = SPIKES) -> np.ndarray:
     """W = N(0, 1/K) + sum_i sigma_i u_i v_i^T, rounded to BF16."""
@@ -182,12 +199,23 @@ def layer(workload: str, layer_name: Optional[str] = None, M: Optional[int] = No
 
 
 def custom_layer(seed: int, M: int, K: int, N: int, sigma0: float = 20.0,
-                 outliers: bool = True, calib_tokens: int = CALIB_TOKENS) -> dict:
-    """Same recipe at an arbitrary shape (parity sweeps over tails and sizes)."""
+                 outliers: bool = True, calib_tokens: int = CALIB_TOKENS,
+                 latent_rank: int = 0, with_heldout: bool = False) -> dict:
+    """Same recipe at an arbitrary shape (parity sweeps over tails and sizes).
+    latent_rank > 0 draws the activations from ``correlated_activations``."""
     wid, lid = 1000 + seed, 0
     shp = LayerShape(f"custom{seed}", M, K, N, sigma0, outliers=outliers)
-    return {"shape": shp,
-            "W": weights(wid, lid, K, N, sigma0, spikes=min(SPIKES, K, N)),
-            "bias": bias(wid, lid, N),
-            "Xc": activations(wid, lid, calib_tokens, K, ROLE_X_CALIB, outliers),
-            "X": activations(wid, lid, M, K, ROLE_X_RUN, outliers)}
+
+    def acts(m, role):
+        if latent_rank > 0:
+            return correlated_activations(wid, lid, m, K, role, latent_rank, outliers)
+        return activations(wid, lid, m, K, role, outliers)
+
+    out = {"shape": shp,
+           "W": weights(wid, lid, K, N, sigma0, spikes=min(SPIKES, K, N)),
+           "bias": bias(wid, lid, N),
+           "Xc": acts(calib_tokens, ROLE_X_CALIB),
+           "X": acts(M, ROLE_X_RUN)}
+    if with_heldout:
+        out["Xh"] = acts(calib_tokens, ROLE_X_HELDOUT)
+    return out

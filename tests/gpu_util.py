@@ -29,8 +29,9 @@ def prepare_gpu(d, fmt="nvfp4", rank=32):
                              fmt=fmt, rank=rank, device=0)
 
 
-def oracle_prep_from(L) -> dict:
-    """The oracle's prepared layer built from the library's exported tensors."""
+def oracle_prep_from(L, gptq_U=None) -> dict:
+    """The oracle's prepared layer built from the library's exported tensors
+    (residual quantized by GPTQ with factor ``gptq_U`` when one is given)."""
     info = L.info
     r = info["rank"]
     fmt = "int4" if info["format"] == lib.INT4 else "nvfp4"
@@ -39,7 +40,10 @@ def oracle_prep_from(L) -> dict:
          "L1d": syn.from_bf16_bits(L.export("L1d")).astype(np.float64) if r else np.zeros((info["K"], 0)),
          "L2b": syn.from_bf16_bits(L.export("L2b")).astype(np.float64) if r else np.zeros((0, info["N"])),
          "bias": L.export("bias").astype(np.float64), "g_x_exp": info["g_x_exp"]}
-    p.update(o.quantize_weights(L.export("R"), fmt))
+    if gptq_U is None:
+        p.update(o.quantize_weights(L.export("R"), fmt))
+    else:
+        p.update(o.gptq_quantize(L.export("R"), gptq_U, fmt))
     assert p["g_w_exp"] == info["g_w_exp"]
     return p
 

@@ -31,8 +31,10 @@ FWD_GELU, FWD_UNFUSED, FWD_NO_BRANCH, FWD_CHECK = 0x1, 0x2, 0x4, 0x8
 TENSORS = {
     "lambda": (0, np.float32), "inv_lambda": (1, np.float32), "L1": (2, np.float64), "L2": (3, np.float64),
     "L1d": (4, np.uint16), "L2b": (5, np.uint16), "R": (6, np.float32), "sigma": (7, np.float64),
-    "w_codes": (8, np.uint8), "w_scales": (9, None), "bias": (10, np.float32),
+    "w_codes": (8, np.uint8), "w_scales": (9, None), "bias": (10, np.float32), "gptq_U": (11, np.float64),
 }
+# preparation flags (svdq_config.flags)
+PREP_GPTQ, PREP_KEEP_GPTQ_FACTOR = 0x1, 0x2
 
 EXPORTED = [
     "svdq_prepare", "svdq_destroy", "svdq_get_info", "svdq_tensor_bytes", "svdq_export",
@@ -139,15 +141,16 @@ class Layer:
 
     @classmethod
     def prepare(cls, W_bits: np.ndarray, bias_bits: Optional[np.ndarray], calib_bits: Optional[np.ndarray],
-                fmt: str = "nvfp4", rank: int = 32, alpha: float = 0.5, device: int = 0) -> "Layer":
+                fmt: str = "nvfp4", rank: int = 32, alpha: float = 0.5, device: int = 0,
+                flags: int = 0) -> "Layer":
         """W_bits: uint16 [K][N] BF16 bit patterns (Y = X W + b); bias_bits: uint16 [N] or None;
-        calib_bits: uint16 [M_calib][K] or None (W4A16)."""
+        calib_bits: uint16 [M_calib][K] or None (W4A16); flags: PREP_* bits."""
         L = load()
         W = np.ascontiguousarray(W_bits, dtype=np.uint16)
         K, N = W.shape
         b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
         c = None if calib_bits is None else np.ascontiguousarray(calib_bits, dtype=np.uint16)
-        cfg = Config(FORMATS[fmt], rank, alpha, 0)
+        cfg = Config(FORMATS[fmt], rank, alpha, flags)
         out = ctypes.c_void_p()
         st = L.svdq_prepare(ctypes.byref(cfg), K, N, _ptr(W), _ptr(b), _ptr(c),
                             0 if c is None else c.shape[0], device, ctypes.byref(out))
@@ -182,7 +185,7 @@ class Layer:
         _check(load().svdq_export(self._h, tid, _ptr(buf), nbytes), f"svdq_export({name})")
         shapes = {"lambda": (K,), "inv_lambda": (K,), "L1": (K, r), "L2": (r, N), "L1d": (K, r),
                   "L2b": (r, N), "R": (K, N), "sigma": (r,), "w_codes": (N, K // 2), "bias": (N,),
-                  "w_scales": (N, -1)}
+                  "w_scales": (N, -1), "gptq_U": (K, K)}
         return buf.reshape(shapes[name])
 
     def workspace_bytes(self, M: int) -> int:

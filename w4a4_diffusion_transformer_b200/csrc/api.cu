@@ -139,9 +139,9 @@ size_t act_scale_bytes(const HostPrep& h, int M) {
 // GEMM's clamp of 8192, while every group scale down to 2^-24 of that largest
 // value stays at or above 2^-17, where FP16 holds all of its 8 bits exactly.
 void int4_range_exponents(const HostPrep& h, int* ex, int* ew) {
-  float amax = 0.0f;
-  for (float v : h.R) amax = std::max(amax, std::fabs(v));
-  *ew = pow2_ceil_exponent((double)amax) - 14;
+  // w_amax: the largest group maximum the quantizer saw (amax |R| for
+  // round-to-nearest; GPTQ's updated values may move it either way)
+  *ew = pow2_ceil_exponent((double)h.w_amax) - 14;
   *ex = pow2_ceil_exponent((double)h.x_amax) - 8;
 }
 
@@ -432,6 +432,9 @@ svdq_status svdq_prepare(const svdq_config* cfg, int K, int N, const uint16_t* W
   if (!cfg || !W_bf16 || K <= 0 || N <= 0) return SVDQ_EINVAL;
   if (cfg->format < SVDQ_NVFP4 || cfg->format > SVDQ_W4A16_INT4) return SVDQ_EINVAL;
   const bool wo = cfg->format == SVDQ_W4A16_INT4;
+  if (cfg->flags & ~(SVDQ_PREP_GPTQ | SVDQ_PREP_KEEP_GPTQ_FACTOR)) return SVDQ_EINVAL;
+  if ((cfg->flags & SVDQ_PREP_KEEP_GPTQ_FACTOR) && !(cfg->flags & SVDQ_PREP_GPTQ)) return SVDQ_EINVAL;
+  if (wo && (cfg->flags & SVDQ_PREP_GPTQ)) return SVDQ_EINVAL;   // GPTQ needs the calibration batch
   if (!wo) {
     if (!calib_bf16 || M_calib < 1) return SVDQ_EINVAL;
     if (!(cfg->alpha > 0.0f && cfg->alpha < 1.0f)) return SVDQ_EINVAL;
@@ -495,6 +498,7 @@ size_t svdq_tensor_bytes(const svdq_layer* L, int id) {
     case SVDQ_T_W_CODES: return h.w_codes.size();
     case SVDQ_T_W_SCALES: return h.format == SVDQ_NVFP4 ? h.w_scales_e4m3.size() : h.w_scales_bf16.size() * 2;
     case SVDQ_T_BIAS: return h.bias.size() * 4;
+    case SVDQ_T_GPTQ_U: return h.gptq_U.size() * 8;
   }
   return 0;
 }
@@ -519,6 +523,7 @@ svdq_status svdq_export(const svdq_layer* L, int id, void* dst, size_t bytes) {
       src = h.format == SVDQ_NVFP4 ? (const void*)h.w_scales_e4m3.data() : (const void*)h.w_scales_bf16.data();
       break;
     case SVDQ_T_BIAS: src = h.bias.data(); break;
+    case SVDQ_T_GPTQ_U: src = h.gptq_U.data(); break;
     default: return SVDQ_EINVAL;
   }
   std::memcpy(dst, src, bytes);

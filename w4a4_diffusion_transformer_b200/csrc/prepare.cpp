@@ -388,6 +388,206 @@ uint16_t int4_group(const float* v, int8_t* codes) {
   return sb;
 }
 
+// ------------------------------------------------------------------ GPTQ
+//
+// SOTA-314 practice page, "Do this": the residual is quantized with GPTQ rather
+// than round-to-nearest.  The published algorithm (Frantar et al. 2022) in its
+// column-by-column form; its lazy block updates only reorder the same
+// arithmetic.  The loss of output column n is ||X_hat (r_n - q_n)||^2, so one
+// Hessian H = X_hat^T X_hat serves every column.
+
+constexpr double kGptqDamp = 0.01;          // fraction of the mean diagonal added to H
+
+// Damped Hessian of the smoothed calibration activations X_hat = fp32(Xc * inv_lam).
+void gptq_hessian(const uint16_t* calib, int M, int K, const std::vector<float>& inv_lam,
+                  std::vector<double>& H) {
+  std::vector<double> xt((size_t)K * M);    // X_hat^T, [K][M]
+#pragma omp parallel for schedule(static)
+  for (int k = 0; k < K; ++k)
+    for (int m = 0; m < M; ++m) {
+      volatile float v = bf16_to_float(calib[(size_t)m * K + k]) * inv_lam[k];
+      xt[(size_t)k * M + m] = (double)(float)v;
+    }
+  H.assign((size_t)K * K, 0.0);
+  constexpr int T = 32;
+  const int nb = (K + T - 1) / T;
+  std::vector<int> ti, tj;
+  for (int i = 0; i < nb; ++i)
+    for (int j = i; j < nb; ++j) {
+      ti.push_back(i);
+      tj.push_back(j);
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int t = 0; t < (int)ti.size(); ++t) {
+    const int i0 = ti[t] * T, j0 = tj[t] * T;
+    for (int i = i0; i < std::min(K, i0 + T); ++i) {
+      const double* xi = xt.data() + (size_t)i * M;
+      for (int j = std::max(i, j0); j < std::min(K, j0 + T); ++j) {
+        const double* xj = xt.data() + (size_t)j * M;
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+        int m = 0;
+        for (; m + 4 <= M; m += 4) {
+          s0 += xi[m] * xj[m];
+          s1 += xi[m + 1] * xj[m + 1];
+          s2 += xi[m + 2] * xj[m + 2];
+          s3 += xi[m + 3] * xj[m + 3];
+        }
+        for (; m < M; ++m) s0 += xi[m] * xj[m];
+        H[(size_t)i * K + j] = H[(size_t)j * K + i] = (s0 + s1) + (s2 + s3);
+      }
+    }
+  }
+  double tr = 0.0;
+  for (int k = 0; k < K; ++k) {
+    double& d = H[(size_t)k * K + k];
+    if (d == 0.0) d = 1.0;                  // a channel the calibration never fires
+    tr += d;
+  }
+  const double add = kGptqDamp * (tr / K);
+  for (int k = 0; k < K; ++k) H[(size_t)k * K + k] += add;
+}
+
+// In place: the upper triangle of A (symmetric positive definite, [K][K]) becomes
+// the upper-triangular T with positive diagonal and A = T T^T -- Cholesky run
+// from the last column backwards.  false if a pivot is not positive.
+bool reverse_cholesky(std::vector<double>& A, int K) {
+  for (int j = K - 1; j >= 0; --j) {
+    double* rj = A.data() + (size_t)j * K;
+    double d = rj[j];
+    for (int k = j + 1; k < K; ++k) d -= rj[k] * rj[k];
+    if (!(d > 0.0) || !std::isfinite(d)) return false;
+    const double tjj = std::sqrt(d);
+    rj[j] = tjj;
+#pragma omp parallel for schedule(static) if (j >= 64)
+    for (int i = 0; i < j; ++i) {
+      double* ri = A.data() + (size_t)i * K;
+      double s = ri[j];                     // still H_ij: column j is being formed
+      for (int k = j + 1; k < K; ++k) s -= ri[k] * rj[k];
+      ri[j] = s / tjj;
+    }
+  }
+  return true;
+}
+
+// U = T^-1 for the upper-triangular T in the upper triangle of A; then
+// H^-1 = T^-T T^-1 = U^T U, so U is the upper Cholesky factor of H^-1.
+void upper_inverse(const std::vector<double>& A, int K, std::vector<double>& U) {
+  U.assign((size_t)K * K, 0.0);
+#pragma omp parallel
+  {
+    std::vector<double> u(K);
+#pragma omp for schedule(dynamic, 8)
+    for (int j = K - 1; j >= 0; --j) {
+      u[j] = 1.0 / A[(size_t)j * K + j];
+      for (int i = j - 1; i >= 0; --i) {
+        const double* ti = A.data() + (size_t)i * K;
+        double s = 0.0;
+        for (int k = i + 1; k <= j; ++k) s += ti[k] * u[k];
+        u[i] = -s / ti[i];
+      }
+      for (int i = 0; i <= j; ++i) U[(size_t)i * K + j] = u[i];
+    }
+  }
+}
+
+// Magnitude of a 3-bit E2M1 code.
+double e2m1_magnitude(uint8_t c) {
+  static const double grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  return grid[c & 7];
+}
+
+// GPTQ over the columns of the residual R [K][N] with factor U; writes codes and
+// scales into P exactly where round-to-nearest writes them.  Columns are
+// independent given U; each thread carries kNB of them through the K steps.
+void gptq_columns(const std::vector<float>& R, int K, int N, const std::vector<double>& U, bool nvfp4,
+                  HostPrep& P) {
+  constexpr int kNB = 16;
+  const int G = nvfp4 ? 16 : 64;
+  const float g = nvfp4 ? (float)std::ldexp(1.0, P.g_w_exp) : 1.0f;
+  const float cc = nvfp4 ? (float)std::ldexp((double)(1.0f / 6.0f), -P.g_w_exp) : 0.0f;
+  const double gd = (double)g;
+  float amax_all = 0.0f;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : amax_all)
+  for (int b = 0; b < (N + kNB - 1) / kNB; ++b) {
+    const int n0 = b * kNB, nc = std::min(kNB, N - n0);
+    std::vector<double> w((size_t)K * kNB, 0.0);      // working values, [K][kNB]
+    for (int k = 0; k < K; ++k)
+      for (int c = 0; c < nc; ++c) w[(size_t)k * kNB + c] = (double)R[(size_t)k * N + n0 + c];
+    float inv[kNB], sc[kNB];
+    double err[kNB];
+    for (int k = 0; k < K; ++k) {
+      if (k % G == 0) {
+        for (int c = 0; c < nc; ++c) {
+          float a = 0.0f;
+          for (int i = 0; i < G; ++i) a = std::max(a, std::fabs((float)w[(size_t)(k + i) * kNB + c]));
+          amax_all = std::max(amax_all, a);
+          const int n = n0 + c;
+          if (nvfp4) {
+            volatile float t = a * cc;
+            const uint8_t sb = e4m3_from_nonneg(t);
+            sc[c] = e4m3_to_float(sb);
+            P.w_scales_e4m3[(size_t)n * (K / 16) + k / 16] = sb;
+            if (sc[c] == 0.0f) {
+              inv[c] = 0.0f;
+            } else {
+              volatile float sg = sc[c] * g;
+              volatile float iv = 1.0f / sg;
+              inv[c] = iv;
+            }
+          } else {
+            const float seventh = 1.0f / 7.0f;
+            volatile float t = a * seventh;
+            const uint16_t sb = bf16_from_double((double)t);
+            sc[c] = bf16_to_float(sb);
+            P.w_scales_bf16[(size_t)n * (K / 64) + k / 64] = sb;
+            if (sc[c] == 0.0f) {
+              inv[c] = 0.0f;
+            } else {
+              volatile float iv = 1.0f / sc[c];
+              inv[c] = iv;
+            }
+          }
+        }
+      }
+      const double ukk = U[(size_t)k * K + k];
+      for (int c = 0; c < nc; ++c) {
+        const double wk = w[(size_t)k * kNB + c];
+        const float v = (float)wk;
+        uint8_t nib;
+        double deq;
+        if (nvfp4) {
+          if (sc[c] == 0.0f) {
+            nib = 0;
+            deq = 0.0;
+          } else {
+            volatile float q = v * inv[c];
+            nib = e2m1_code(q);
+            const double mag = e2m1_magnitude(nib) * ((double)sc[c] * gd);
+            deq = (nib & 8) ? -mag : mag;
+          }
+        } else {
+          volatile float q = v * inv[c];
+          float rq = std::nearbyint((float)q);
+          rq = std::min(7.0f, std::max(-7.0f, rq));
+          const int code = (int)rq;
+          nib = (uint8_t)(code & 0xF);
+          deq = (double)code * (double)sc[c];
+        }
+        uint8_t& byte = P.w_codes[(size_t)(n0 + c) * (K / 2) + k / 2];
+        byte = (k & 1) ? (uint8_t)((byte & 0x0F) | (nib << 4)) : (uint8_t)((byte & 0xF0) | nib);
+        err[c] = (wk - deq) / ukk;
+      }
+      const double* uk = U.data() + (size_t)k * K;
+      for (int j = k + 1; j < K; ++j) {
+        const double ukj = uk[j];
+        double* wj = w.data() + (size_t)j * kNB;
+        for (int c = 0; c < nc; ++c) wj[c] = wj[c] - ukj * err[c];
+      }
+    }
+  }
+  P.w_amax = amax_all;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ pipeline
@@ -487,9 +687,28 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
 
     // ---- residual quantization, groups along K for each output column n
     P.w_codes.assign((size_t)N * K / 2, 0);
+    float amax = 0.0f;
+    for (float v : P.R) amax = std::max(amax, std::fabs(v));
+    P.w_amax = amax;
+    if (cfg.flags & SVDQ_PREP_GPTQ) {
+      const bool nvfp4 = cfg.format == SVDQ_NVFP4;
+      if (nvfp4) {
+        P.g_w_exp = pow2_ceil_exponent((double)amax / 2688.0);
+        P.w_scales_e4m3.assign((size_t)N * K / 16, 0);
+      } else {
+        P.w_scales_bf16.assign((size_t)N * K / 64, 0);
+      }
+      std::vector<double> H, U;
+      gptq_hessian(calib, M_calib, K, P.inv_lam, H);
+      if (!reverse_cholesky(H, K)) return SVDQ_ENOCONVERGE;
+      upper_inverse(H, K, U);
+      std::vector<double>().swap(H);
+      gptq_columns(P.R, K, N, U, nvfp4, P);
+      if (nvfp4) P.g_x_exp = pow2_ceil_exponent(4.0 * (double)P.x_amax / 2688.0);
+      if (cfg.flags & SVDQ_PREP_KEEP_GPTQ_FACTOR) P.gptq_U.swap(U);
+      return SVDQ_OK;
+    }
     if (cfg.format == SVDQ_NVFP4) {
-      float amax = 0.0f;
-      for (float v : P.R) amax = std::max(amax, std::fabs(v));
       P.g_w_exp = pow2_ceil_exponent((double)amax / 2688.0);
       const float g = (float)std::ldexp(1.0, P.g_w_exp);
       const float c = (float)std::ldexp((double)(1.0f / 6.0f), -P.g_w_exp);

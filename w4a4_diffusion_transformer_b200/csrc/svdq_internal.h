@@ -29,6 +29,8 @@ struct HostPrep {
   std::vector<float> R;                     // [K][N]
   int g_x_exp = 0, g_w_exp = 0;
   float x_amax = 0.0f;                      // max |fp32(Xc / lam)| over the calibration batch
+  float w_amax = 0.0f;                      // largest group maximum the residual quantizer saw
+  std::vector<double> gptq_U;               // [K][K] GPTQ factor (kept only on request)
   std::vector<uint8_t> w_codes;             // [N][K/2]
   std::vector<uint8_t> w_scales_e4m3;       // [N][K/16]   (NVFP4)
   std::vector<uint16_t> w_scales_bf16;      // [N][K/64]   (INT4 / W4A16)
