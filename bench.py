@@ -480,6 +480,52 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
     d2 = syn.layer("mlp", "fc2")
     d2["Xc"] = hc.float().cpu().numpy()
     w4a4_layer(d2, "nvfp4", h, 0, "fc2")
+    del h
+    # the same pair through the chain: fc1's epilogue writes fc2's quantized
+    # input (codes, scales, down-projection partials), against the two layers
+    # one after the other with fc1's BF16 output through HBM
+    M1, K1, N1 = d1["X"].shape[0], d1["W"].shape[0], d1["W"].shape[1]
+    N2 = d2["W"].shape[1]
+    csets = []
+    for _ in range(2):
+        L1c = pkg.Layer.prepare(syn.bf16_bits(d1["W"]), syn.bf16_bits(d1["bias"]), syn.bf16_bits(d1["Xc"]),
+                                fmt="nvfp4", rank=RANK, device=dev)
+        L2c = pkg.Layer.prepare(syn.bf16_bits(d2["W"]), syn.bf16_bits(d2["bias"]), syn.bf16_bits(d2["Xc"]),
+                                fmt="nvfp4", rank=RANK, device=dev)
+        wsb = max(pkg.mlp_workspace_bytes(L1c, L2c, M1, pkg.FWD_GELU),
+                  pkg.mlp_workspace_bytes(L1c, L2c, M1, pkg.FWD_GELU | pkg.FWD_UNFUSED))
+        csets.append((L1c, L2c, torch.from_numpy(d1["X"]).to(torch.bfloat16).cuda(),
+                      torch.empty((M1, N2), dtype=torch.bfloat16, device="cuda"),
+                      torch.empty(wsb, dtype=torch.uint8, device="cuda"), wsb))
+
+    def chain(flags):
+        def f(i):
+            L1c, L2c, x, y, ws, wsb = csets[i % len(csets)]
+            pkg.mlp_forward(L1c, L2c, x, M1, y, ws, wsb, stream, flags)
+        return f
+
+    for fl in (pkg.FWD_GELU, pkg.FWD_GELU | pkg.FWD_UNFUSED):
+        for i in range(4):
+            chain(fl)(i)
+    for st in csets:
+        st[0].check(stream)
+        st[1].check(stream)
+    t_chain = time_rotating(stream, n, chain(pkg.FWD_GELU))
+    t_sep = time_rotating(stream, n, chain(pkg.FWD_GELU | pkg.FWD_UNFUSED))
+    for st in csets:
+        st[0].check(stream)
+        st[1].check(stream)
+    fl2 = layer_flops(M1, K1, N1) + layer_flops(M1, N1, N2)
+    out["mlp_chain"] = {"shape": f"{M1}x{K1}->{N1}->{N2}", "format": "nvfp4", "us_chain": t_chain * 1e3,
+                        "us_separate": t_sep * 1e3, "tflops_chain": fl2 / (t_chain * 1e-3) / 1e12,
+                        "tflops_separate": fl2 / (t_sep * 1e-3) / 1e12, "speedup": t_sep / t_chain,
+                        "note": "fc1 (GELU) -> fc2; chain: fc2's input quantized in fc1's epilogue "
+                                "(svdq_mlp_forward), separate: the two layers' forwards with fc1's BF16 "
+                                "output through HBM (SVDQ_FWD_UNFUSED)"}
+    for st in csets:
+        st[0].close()
+        st[1].close()
+    del csets
     # W4A16 adaptive-norm GEMV (30 MB of weights per set)
     da = syn.layer("block_b4", "adaln", with_run=False)
     Ma, Ka, Na = 4, da["W"].shape[0], da["W"].shape[1]

@@ -134,7 +134,9 @@ typedef enum {
   SVDQ_T_BIAS = 10,         /* float [N]                                            */
   SVDQ_T_GPTQ_U = 11,       /* double [K][K]   GPTQ factor U (upper, H^-1 = U^T U); only
                                with SVDQ_PREP_GPTQ | SVDQ_PREP_KEEP_GPTQ_FACTOR      */
-  SVDQ_T_COUNT = 12
+  SVDQ_T_LORA_A = 12,       /* uint16 [K][r]   LoRA down factor A as attached (BF16)  */
+  SVDQ_T_LORA_B = 13,       /* uint16 [r][N]   bf16(scale * B), the stored up factor  */
+  SVDQ_T_COUNT = 14
 } svdq_tensor;
 
 /* ------------------------------------------------------------------ offline */
@@ -182,6 +184,34 @@ svdq_status svdq_export(const svdq_layer* layer, int id, void* dst, size_t bytes
 
 const char* svdq_status_string(svdq_status s);
 
+/* svdq_set_lora -- attach a LoRA adapter (W -> W + scale A B) to the layer's
+ * 16-bit low-rank branch without re-quantizing anything.  SOTA-314 practice
+ * page, "Known implementations": the paper's engine loads off-the-shelf LoRA
+ * adapters without re-quantization.  The branch becomes
+ *     X L1d L2b + X A bf16(scale B),
+ * i.e. L1d' = [L1d | A], L2b' = [L2b ; bf16(scale B)] (rank 32 + r); smoothing,
+ * residual codes and scales are untouched.
+ *
+ *   r          adapter rank, 1..32; 0 removes the adapter (A, B ignored).
+ *   A_bf16     host, [K][r] BF16 (acts on the unsmoothed input X); copied.
+ *   B_bf16     host, [r][N] BF16; copied as bf16(scale * B), one rounding.
+ *   scale      the adapter's scaling (e.g. alpha / r); finite.
+ *
+ * Forward cost: one more pass of the first kernel's down projection over X
+ * (XL columns 32..63 = bf16(X A)), and one more pipeline stage per output tile
+ * in the NVFP4 GEMM (XL_lora times bf16(scale B) into the same accumulator);
+ * the INT4 GEMM reloads its branch buffer with the adapter's tiles within each
+ * tile, into the same accumulator as well.  With an adapter attached, XL is [M][64]
+ * BF16 (columns 32..63: X A, zero-padded past r) wherever the API exposes it,
+ * and svdq_workspace_bytes grows accordingly.  Blocking: synchronizes the
+ * device before replacing the adapter's device buffers, so no forward of this
+ * layer may be pending on another thread.  Errors: SVDQ_EINVAL (r < 0, null
+ * factors, non-finite scale), SVDQ_EUNSUPPORTED (r > 32, SVDQ_W4A16_INT4),
+ * SVDQ_ENOMEM, SVDQ_ECUDA.  The fc1 -> fc2 chain (svdq_mlp_*) does not take
+ * layers with an adapter (SVDQ_EUNSUPPORTED). */
+svdq_status svdq_set_lora(svdq_layer* layer, int r, const uint16_t* A_bf16, const uint16_t* B_bf16,
+                          float scale);
+
 /* ------------------------------------------------------------------ forward */
 
 /* Workspace bytes a forward over M tokens needs (activation codes, scales in the
@@ -222,9 +252,9 @@ svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, v
  * the activation scales (device, svdq_act_scale_bytes(layer, M)
  * bytes: NVFP4 E4M3 in the tensor-core layout, INT4 BF16 [K/64][M rounded up
  * to 128], group-major, padding rows zero) and, when
- * the layer has a branch, XL = bf16(X L1d) (device [M][rank] BF16).
- * xl may be NULL for rank 0.  `mode` 0 = fused, 1 = quantize only,
- * 2 = down projection only. */
+ * the layer has a branch, XL = bf16(X L1d) (device [M][rank] BF16; [M][64]
+ * with a LoRA adapter, see svdq_set_lora).  xl may be NULL for rank 0 without
+ * an adapter.  `mode` 0 = fused, 1 = quantize only, 2 = down projection only. */
 svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int M,
                               void* codes, void* scales, void* xl,
                               void* stream, int mode);
@@ -260,6 +290,47 @@ svdq_status svdq_act_scales_to_logical(const svdq_layer* layer, const void* devi
 /* Synchronise `stream` and report (and clear) the layer's device error word:
  * SVDQ_ETIMEOUT if a bounded device wait expired since the last check. */
 svdq_status svdq_check(const svdq_layer* layer, void* stream);
+
+/* ------------------------------------------------------------------ fc1 -> fc2 chain */
+
+/* The transformer MLP fc1 -> tanh-GELU -> fc2 with fc2's input produced
+ * already quantized by fc1's GEMM epilogue.  The pages fuse the down projection
+ * with the quantizer "because they read the same input" (SOTA-314 practice
+ * page, "Do this"; NOTE-257 note page, "Key results"); in the MLP that input
+ * is fc1's output, so fc1's epilogue rounds y = [gelu](fc1 output) to BF16
+ * -- the value fc2 would read -- and writes fc2's NVFP4 codes and scales from
+ * it with fc2's own quantizer arithmetic, bit for bit what svdq_quantize_act
+ * would write for that y, plus partial sums of fc2's down projection y L1d2
+ * over the fc1 tiles each CTA owns.  A second small kernel adds the partials
+ * of each row in a fixed order (deterministic; XL2 = bf16 of an FP32 sum whose
+ * order differs from the first kernel's, so XL2 may differ from it by a BF16
+ * rounding).  fc1's BF16 output and fc2's first kernel disappear from the path.
+ *
+ * Both layers: SVDQ_NVFP4, prepared on the same device, fc1's N equal to
+ * fc2's K (else SVDQ_EUNSUPPORTED).  fc2's calibration batch (its lam and
+ * activation tensor scale) is used as is.
+ *
+ * svdq_mlp_workspace_bytes: workspace of svdq_mlp_forward (and of
+ *   svdq_mlp_fc1) for M tokens; flags as for svdq_mlp_forward (UNFUSED needs
+ *   room for fc1's BF16 output).  0 on bad input.
+ * svdq_mlp_fc1: fc1's first kernel, fc1's GEMM in chain mode and the partial
+ *   sum.  codes2 / scales2 / xl2 (device, 16-byte aligned) receive fc2's
+ *   activation codes (svdq_act_code_bytes(fc2, M)), scales
+ *   (svdq_act_scale_bytes(fc2, M)) and XL2 ([M][32] BF16; may be NULL when fc2
+ *   has rank 0) in the layouts svdq_quantize_act(fc2, ...) writes, ready for
+ *   svdq_gemm(fc2, ...).  flags: SVDQ_FWD_GELU, SVDQ_FWD_CHECK.
+ * svdq_mlp_forward: svdq_mlp_fc1, then fc2's GEMM: Y (device, [M][fc2 N]
+ *   BF16).  flags: SVDQ_FWD_GELU (GELU after fc1; the MLP), SVDQ_FWD_CHECK, and
+ *   SVDQ_FWD_UNFUSED (measurement variant: the two layers' forwards one after
+ *   the other, fc1's BF16 output through HBM).
+ * X, workspace: as for svdq_linear_forward.  Errors as for svdq_linear_forward;
+ * a device timeout in either layer is reported with SVDQ_FWD_CHECK. */
+size_t svdq_mlp_workspace_bytes(const svdq_layer* fc1, const svdq_layer* fc2, int M, unsigned flags);
+svdq_status svdq_mlp_fc1(const svdq_layer* fc1, const svdq_layer* fc2, const void* X, int M,
+                         void* codes2, void* scales2, void* xl2,
+                         void* workspace, size_t workspace_bytes, void* stream, unsigned flags);
+svdq_status svdq_mlp_forward(const svdq_layer* fc1, const svdq_layer* fc2, const void* X, int M, void* Y,
+                             void* workspace, size_t workspace_bytes, void* stream, unsigned flags);
 
 /* svdq_selftest_wait_timeout -- exercise the failure-detection path.
  *

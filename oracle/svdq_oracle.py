@@ -39,6 +39,10 @@ design notes of the repository):
     float32 value fed to the quantizer;
   * INT4 is symmetric in [-7, 7], its 16-bit scale is BF16: s = bf16(fp32(a * fp32(1/7)));
   * two codes per byte, the even k in the low nibble;
+  * W8A8 (rank 16 at 8 bits; the pages give no 8-bit group size): INT8
+    symmetric in [-127, 127] with one group per row -- per token for the
+    activations, per output channel for the residual -- and float32 scales
+    s = fp32(a * fp32(1/127)), code = rint_even(fp32(v * fp32(1/s)));
   * GPTQ (the pages' residual quantizer, named but not restated) is the
     published column-by-column algorithm: H = X_hat^T X_hat of the smoothed
     calibration batch, dead channels H_kk = 1, damping 1% of the mean
@@ -60,6 +64,7 @@ E2M1_MAX = 6.0
 NVFP4_GROUP = 16
 INT4_GROUP = 64
 INT4_QMAX = 7
+INT8_QMAX = 127
 
 
 # --------------------------------------------------------------------------
@@ -257,6 +262,30 @@ def int4_quantize(v: np.ndarray) -> Dict[str, np.ndarray]:
     return {"codes": codes.reshape(rows, K), "scales": s, "deq": deq.reshape(rows, K)}
 
 
+def int8_row_scale(a: np.ndarray):
+    """Scale of INT8 rows with float32 maxima a: s = fp32(a * fp32(1/127));
+    returns s (float32) and inv = fp32(1 / s), 0 where s == 0."""
+    a = np.asarray(a, dtype=F32)
+    s = (a * F32(1.0 / 127.0)).astype(F32)
+    with np.errstate(divide="ignore"):
+        inv = (F32(1.0) / s).astype(F32)
+    return s, np.where(s == 0, F32(0.0), inv).astype(F32)
+
+
+def int8_quantize_rows(v: np.ndarray) -> Dict[str, np.ndarray]:
+    """Symmetric INT8 quantization of the rows of v (float32, [rows, K]), one
+    scale per row: a = max|v|; s = fp32(a * fp32(1/127)); s == 0 -> codes 0;
+    else code = clamp(rint_even(fp32(v * fp32(1/s))), -127, 127).  Returns
+    codes [rows, K] (int8), scales [rows] (float32 values, as float64) and deq."""
+    v = np.asarray(v, dtype=F32)
+    a = np.max(np.abs(v), axis=1)
+    s, inv = int8_row_scale(a)
+    q = (v * inv[:, None]).astype(F32)
+    codes = np.clip(np.rint(q.astype(np.float64)), -INT8_QMAX, INT8_QMAX).astype(np.int8)
+    s64 = s.astype(np.float64)
+    return {"codes": codes, "scales": s64, "deq": codes.astype(np.float64) * s64[:, None]}
+
+
 def int4_nibbles(codes: np.ndarray) -> np.ndarray:
     return (np.asarray(codes, dtype=np.int64) & 0xF).astype(np.uint8)
 
@@ -345,6 +374,23 @@ def prepare(W: np.ndarray, bias: Optional[np.ndarray], Xc: np.ndarray, fmt: str 
     return out
 
 
+def attach_lora(prep: Dict[str, np.ndarray], A: np.ndarray, B: np.ndarray, scale: float) -> Dict[str, np.ndarray]:
+    """A LoRA adapter W -> W + scale A B concatenated into the 16-bit branch
+    without re-quantizing anything [P "Known implementations": the paper's
+    engine loads off-the-shelf LoRA adapters without re-quantization]:
+        L1d' = [L1d | bf16(A)],  L2b' = [L2b ; bf16(fp32(scale) B)],
+    rank 32 + r; lam, the residual and its codes and scales are unchanged.  A
+    acts on the unsmoothed input, like L1d (which carries 1/lam)."""
+    A = bf16_round(np.asarray(A, dtype=np.float64))
+    Bs = bf16_round(bf16_round(np.asarray(B, dtype=np.float64)) * float(np.float32(scale)))
+    out = dict(prep)
+    out["L1d"] = np.hstack([np.asarray(prep["L1d"], dtype=np.float64).reshape(prep["K"], -1), A])
+    out["L2b"] = np.vstack([np.asarray(prep["L2b"], dtype=np.float64).reshape(-1, prep["N"]), Bs])
+    out["rank"] = out["L1d"].shape[1]
+    out["lora_r"] = A.shape[1]
+    return out
+
+
 def weight_tensor_exponent(R: np.ndarray) -> int:
     """g_w = 2^ceil(log2(amax|R| / (6 * 448)))."""
     return pow2_exponent_ceil(float(np.max(np.abs(R))) / (E2M1_MAX * E4M3_MAX))
@@ -367,6 +413,9 @@ def quantize_weights(R: np.ndarray, fmt: str, g_exp: Optional[int] = None) -> Di
                 "w_scales": q["scales"], "w_deq": q["deq"]}
     if fmt in ("int4", "w4a16"):
         q = int4_quantize(Rt)
+        return {"g_w_exp": 0, "w_codes": q["codes"], "w_scales": q["scales"], "w_deq": q["deq"]}
+    if fmt == "w8a8":
+        q = int8_quantize_rows(Rt)                    # one scale per output channel
         return {"g_w_exp": 0, "w_codes": q["codes"], "w_scales": q["scales"], "w_deq": q["deq"]}
     raise ValueError(fmt)
 
@@ -462,10 +511,12 @@ def smoothed_activations(X: np.ndarray, inv_lam: np.ndarray) -> np.ndarray:
 
 
 def quantize_activations(X: np.ndarray, inv_lam: np.ndarray, fmt: str, g_x_exp: int = 0):
-    """Q(X diag(lam)^-1), per token in groups along K."""
+    """Q(X diag(lam)^-1), per token in groups along K (W8A8: one group per token)."""
     v = smoothed_activations(X, inv_lam)
     if fmt == "nvfp4":
         return nvfp4_quantize(v, g_x_exp)
+    if fmt == "w8a8":
+        return int8_quantize_rows(v)
     return int4_quantize(v)
 
 
@@ -477,8 +528,15 @@ def down_projection(X: np.ndarray, L1d: np.ndarray) -> np.ndarray:
 
 
 def gelu_tanh(y: np.ndarray) -> np.ndarray:
-    """tanh approximation of GELU: 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3)))."""
-    return 0.5 * y * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (y + 0.044715 * y ** 3)))
+    """tanh approximation of GELU: 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715 y^3).
+
+    Evaluated as y / (1 + exp(-2u)), the same function (0.5 (1 + tanh u) is the
+    logistic function of 2u) without the cancellation of 1 + tanh(u) for u << 0,
+    which loses every digit below y = -5.6 in float64."""
+    y = np.asarray(y, dtype=np.float64)
+    u = math.sqrt(2.0 / math.pi) * (y + 0.044715 * y ** 3)
+    with np.errstate(over="ignore"):
+        return y / (1.0 + np.exp(-2.0 * u))
 
 
 def forward(prep: Dict[str, np.ndarray], X: np.ndarray, gelu: bool = False,

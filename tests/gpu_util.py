@@ -44,8 +44,16 @@ def oracle_prep_from(L, gptq_U=None) -> dict:
         p.update(o.quantize_weights(L.export("R"), fmt))
     else:
         p.update(o.gptq_quantize(L.export("R"), gptq_U, fmt))
+    if lib.load().svdq_tensor_bytes(L._h, lib.TENSORS["lora_A"][0]):
+        # an attached LoRA adapter: its stored factors (bf16(scale B) already scaled)
+        p = o.attach_lora(p, syn.from_bf16_bits(L.export("lora_A")), syn.from_bf16_bits(L.export("lora_B")), 1.0)
     assert p["g_w_exp"] == info["g_w_exp"]
     return p
+
+
+def xl_width(L) -> int:
+    """Columns of XL: 64 with a LoRA adapter attached (X A in columns 32..63), else 32."""
+    return 64 if lib.load().svdq_tensor_bytes(L._h, lib.TENSORS["lora_A"][0]) else 32
 
 
 def run_quantize(L, X: np.ndarray, mode=0):
@@ -54,7 +62,7 @@ def run_quantize(L, X: np.ndarray, mode=0):
     x = torch_bf16(X)
     codes = torch.full((L.act_code_bytes(M),), 0xAB, dtype=torch.uint8, device="cuda")
     scales = torch.full((L.act_scale_bytes(M),), 0xCD, dtype=torch.uint8, device="cuda")
-    xl = torch.full((M, 32), float("nan"), dtype=torch.bfloat16, device="cuda")
+    xl = torch.full((M, xl_width(L)), float("nan"), dtype=torch.bfloat16, device="cuda")
     L.quantize_act(x, M, codes, scales, xl, torch.cuda.current_stream(), mode)
     torch.cuda.synchronize()
     return {"codes": L.act_codes_to_logical(codes.cpu().numpy(), M), "scales_dev": scales.cpu().numpy(),

@@ -26,7 +26,7 @@ def built():
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "svdq.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(svdq_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(svdq_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported():

@@ -130,3 +130,40 @@ def test_block_b4_adaln_w4a16():
     torch.cuda.synchronize()
     ref = o.w4a16_forward(o.w4a16_prepare(d["W"], d["bias"]), X)["Y_bf16"]
     assert_close_bf16(to_numpy_f32(y), ref, "adaLN 4x3072->18432")
+
+
+def test_mlp_chain_full_size_sampled_rows():
+    """fc1 -> GELU -> fc2 through the chain at 4608 tokens: fc2's codes and
+    scales from fc1's epilogue bit-exact on sampled rows against the oracle's
+    quantizer on fc1's BF16 output (computed by a separate fc1 forward), XL2 and
+    the output within tolerance, every output element finite."""
+    import torch
+    from gpu_util import torch_bf16
+    d1 = syn.layer("mlp", "fc1")
+    M = d1["X"].shape[0]
+    L1 = prepare_gpu(d1)
+    p1 = oracle_prep_from(L1)
+    L2 = fc2_layer(d1, p1, syn.layer("mlp", "fc2"))
+    p2 = oracle_prep_from(L2)
+    x = torch_bf16(d1["X"])
+    h, _, _ = run_device(L1, x, lib.FWD_GELU)
+    stream = torch.cuda.current_stream()
+    codes = torch.empty(L2.act_code_bytes(M), dtype=torch.uint8, device="cuda")
+    scales = torch.empty(L2.act_scale_bytes(M), dtype=torch.uint8, device="cuda")
+    xl = torch.empty((M, 32), dtype=torch.bfloat16, device="cuda")
+    wsb = lib.mlp_workspace_bytes(L1, L2, M)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    lib.mlp_fc1(L1, L2, x, M, codes, scales, xl, ws, wsb, stream, lib.FWD_GELU | lib.FWD_CHECK)
+    y = torch.full((M, L2.info["N"]), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lib.mlp_forward(L1, L2, x, M, y, ws, wsb, stream, lib.FWD_GELU | lib.FWD_CHECK)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(y).all())
+    rows = sample_rows(M, 8)
+    idx = torch.from_numpy(rows).cuda()
+    hr = to_numpy_f32(h[idx])
+    ref = o.quantize_activations(hr, p2["inv_lam"], "nvfp4", p2["g_x_exp"])
+    np.testing.assert_array_equal(L2.act_scales_to_logical(scales.cpu().numpy(), M)[rows], ref["scale_bytes"])
+    np.testing.assert_array_equal(L2.act_codes_to_logical(codes.cpu().numpy(), M)[rows], o.pack_nibbles(ref["codes"]))
+    ref_xl = o.down_projection(hr, p2["L1d"])
+    np.testing.assert_allclose(to_numpy_f32(xl[idx]), ref_xl, rtol=2 ** -7, atol=1e-6 * np.max(np.abs(ref_xl)))
+    assert_close_bf16(to_numpy_f32(y[idx]), o.forward(p2, hr)["Y_bf16"], "chain fc2 output 4608x12288->3072")

@@ -161,6 +161,25 @@ def test_forward_zero_input_gives_bias():
     np.testing.assert_array_equal(y, np.broadcast_to(o.bf16_round(L.export("bias")), y.shape))
 
 
+def test_forward_zero_input_gelu_of_bias():
+    # X = 0 makes the accumulator zero, so the GELU epilogue sees y = b exactly:
+    # Y = bf16(GELU(b)) for a bias sweep over [-12, 12], within one BF16 ulp of
+    # the float64 tanh form rounded once (the GPU evaluates it in float32), or
+    # within 2^-122 (about 1.9e-37) where float32 runs out of range: for b below
+    # about -10 the denominator 1 + e^(-2u) exceeds 2^126, the fast division
+    # returns zero, and the true value is below 1.2e-37 in magnitude
+    d = syn.custom_layer(38, M=64, K=256, N=512)
+    b = syn.to_bf16(np.linspace(-12.0, 12.0, 512))
+    d = dict(d, bias=b, X=np.zeros((64, 256), dtype=np.float32))
+    L = prepare_gpu(d)
+    y = run_forward(L, d["X"], lib.FWD_GELU)
+    ref = o.bf16_round(o.gelu_tanh(b.astype(np.float64)))
+    ulp = np.ldexp(1.0, np.frexp(np.maximum(np.abs(ref), 2.0 ** -126))[1] - 8)
+    tol = np.maximum(ulp, 2.0 ** -122)
+    assert np.all(np.abs(y - ref[None, :]) <= tol[None, :])
+    assert np.mean(y == ref[None, :]) > 0.97
+
+
 def test_forward_deterministic():
     d = syn.custom_layer(36, M=384, K=512, N=512)
     L = prepare_gpu(d)

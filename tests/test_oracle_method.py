@@ -6,6 +6,7 @@ Sources: SOTA-314 practice page ("Do this"); NOTE-257 note page ("Key
 results": Propositions 4.1/4.2, Eckart-Young, Figure 5, the LoRC control;
 "Claims" C1 and C3).
 """
+import math
 from fractions import Fraction
 
 import numpy as np
@@ -193,6 +194,29 @@ def test_gelu_tanh_matches_torch():
     y = np.linspace(-8, 8, 2001)
     want = torch.nn.functional.gelu(torch.from_numpy(y), approximate="tanh").numpy()
     np.testing.assert_allclose(o.gelu_tanh(y), want, rtol=1e-14, atol=1e-15)
+
+
+def test_gelu_tanh_tail_against_300_digit_tanh_form():
+    # the tanh form 0.5 y (1 + tanh(u)) evaluated with 300 significant digits
+    # (decimal arithmetic, tanh from exp) keeps its relative accuracy where
+    # float64's 1 + tanh(u) cancels: the oracle must match it all the way down
+    # the negative tail, to 1e-12 relative (float64's exp(-2u) carries the
+    # rounding of u amplified by |2u| <= 300)
+    from decimal import Decimal, getcontext
+    getcontext().prec = 300
+    k0 = (Decimal(2) / Decimal(str(math.pi))).sqrt()
+
+    def ref(v):
+        y = Decimal(float(v))
+        u = k0 * (y + Decimal("0.044715") * y ** 3)
+        e = (2 * u).exp()
+        return float(Decimal("0.5") * y * (1 + (e - 1) / (e + 1)))
+
+    ys = np.array([-12.0, -10.0, -9.5, -8.0, -6.0, -5.0, -3.0, -1.0, -0.25, 0.0, 0.5, 2.0, 7.0])
+    got = o.gelu_tanh(ys)
+    want = np.array([ref(v) for v in ys])
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=0.0)
+    assert got[0] < 0 and abs(got[0]) > 1e-70               # about -1.6e-61: not flushed to zero
 
 
 # ---------------------------------------------------------------- theory and ablation

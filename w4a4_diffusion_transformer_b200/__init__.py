@@ -32,6 +32,7 @@ TENSORS = {
     "lambda": (0, np.float32), "inv_lambda": (1, np.float32), "L1": (2, np.float64), "L2": (3, np.float64),
     "L1d": (4, np.uint16), "L2b": (5, np.uint16), "R": (6, np.float32), "sigma": (7, np.float64),
     "w_codes": (8, np.uint8), "w_scales": (9, None), "bias": (10, np.float32), "gptq_U": (11, np.float64),
+    "lora_A": (12, np.uint16), "lora_B": (13, np.uint16),
 }
 # preparation flags (svdq_config.flags)
 PREP_GPTQ, PREP_KEEP_GPTQ_FACTOR = 0x1, 0x2
@@ -41,7 +42,8 @@ EXPORTED = [
     "svdq_status_string", "svdq_workspace_bytes", "svdq_linear_forward", "svdq_quantize_act",
     "svdq_gemm", "svdq_act_scale_bytes", "svdq_act_scales_to_logical", "svdq_check",
     "svdq_linear_forward_static", "svdq_act_code_bytes", "svdq_act_codes_to_logical",
-    "svdq_selftest_wait_timeout",
+    "svdq_selftest_wait_timeout", "svdq_mlp_workspace_bytes", "svdq_mlp_fc1", "svdq_mlp_forward",
+    "svdq_set_lora",
 ]
 STATIC_WORKSPACE_BYTES = 16 << 20   # SVDQ_STATIC_WORKSPACE_BYTES
 
@@ -94,6 +96,10 @@ def load() -> ctypes.CDLL:
         "svdq_act_code_bytes": (SZ, [P, I]),
         "svdq_act_codes_to_logical": (I, [P, P, I, P]),
         "svdq_selftest_wait_timeout": (I, [P, U, P]),
+        "svdq_mlp_workspace_bytes": (SZ, [P, P, I, U]),
+        "svdq_mlp_fc1": (I, [P, P, P, I, P, P, P, P, SZ, P, U]),
+        "svdq_mlp_forward": (I, [P, P, P, I, P, P, SZ, P, U]),
+        "svdq_set_lora": (I, [P, I, P, P, ctypes.c_float]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -185,8 +191,21 @@ class Layer:
         _check(load().svdq_export(self._h, tid, _ptr(buf), nbytes), f"svdq_export({name})")
         shapes = {"lambda": (K,), "inv_lambda": (K,), "L1": (K, r), "L2": (r, N), "L1d": (K, r),
                   "L2b": (r, N), "R": (K, N), "sigma": (r,), "w_codes": (N, K // 2), "bias": (N,),
-                  "w_scales": (N, -1), "gptq_U": (K, K)}
+                  "w_scales": (N, -1), "gptq_U": (K, K), "lora_A": (K, -1), "lora_B": (-1, N)}
         return buf.reshape(shapes[name])
+
+    def set_lora(self, A_bits: Optional[np.ndarray], B_bits: Optional[np.ndarray], scale: float = 1.0):
+        """Attach a LoRA adapter W -> W + scale A B (A_bits uint16 [K][r], B_bits
+        uint16 [r][N], BF16 patterns) to the low-rank branch; None removes it."""
+        if A_bits is None:
+            _check(load().svdq_set_lora(self._h, 0, None, None, 0.0), "svdq_set_lora")
+            return
+        A = np.ascontiguousarray(A_bits, dtype=np.uint16)
+        B = np.ascontiguousarray(B_bits, dtype=np.uint16)
+        r = A.shape[1]
+        if B.shape[0] != r:
+            raise ValueError("A is [K][r] and B is [r][N]")
+        _check(load().svdq_set_lora(self._h, r, _ptr(A), _ptr(B), float(scale)), "svdq_set_lora")
 
     def workspace_bytes(self, M: int) -> int:
         return int(load().svdq_workspace_bytes(self._h, M))
@@ -240,3 +259,24 @@ class Layer:
         """Enqueue a kernel whose only wait never completes and gives up after
         budget_us; the next check() raises SvdqError with SVDQ_ETIMEOUT."""
         _check(load().svdq_selftest_wait_timeout(self._h, budget_us, _stream(stream)), "svdq_selftest_wait_timeout")
+
+
+# ---------------------------------------------------------------- fc1 -> fc2 chain
+
+def mlp_workspace_bytes(fc1: Layer, fc2: Layer, M: int, flags: int = 0) -> int:
+    """Workspace of mlp_forward / mlp_fc1 for M tokens (svdq_mlp_workspace_bytes)."""
+    return int(load().svdq_mlp_workspace_bytes(fc1._h, fc2._h, M, flags))
+
+
+def mlp_fc1(fc1: Layer, fc2: Layer, X, M: int, codes2, scales2, xl2, workspace, workspace_bytes: int,
+            stream=None, flags: int = 0):
+    """fc1 with its output handed to fc2 already quantized (svdq_mlp_fc1)."""
+    _check(load().svdq_mlp_fc1(fc1._h, fc2._h, _ptr(X), M, _ptr(codes2), _ptr(scales2), _ptr(xl2),
+                               _ptr(workspace), workspace_bytes, _stream(stream), flags), "svdq_mlp_fc1")
+
+
+def mlp_forward(fc1: Layer, fc2: Layer, X, M: int, Y, workspace, workspace_bytes: int, stream=None,
+                flags: int = 0):
+    """fc1 -> [GELU] -> fc2 (svdq_mlp_forward)."""
+    _check(load().svdq_mlp_forward(fc1._h, fc2._h, _ptr(X), M, _ptr(Y), _ptr(workspace), workspace_bytes,
+                                   _stream(stream), flags), "svdq_mlp_forward")

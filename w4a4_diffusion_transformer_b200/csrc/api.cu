@@ -39,6 +39,11 @@ struct svdq_layer {
   CUtensorMap tm_l2s_pair;               // 128-row boxes for the CTA-pair GEMMs
   CUtensorMap tm_wq_pair;                // INT4 weight codes, 128-row boxes (CTA-pair INT4 GEMM)
   int k2_kernel = 0;                     // NVFP4 GEMM: 0 = by size, 1 = single-CTA, 2 = CTA pairs
+  // LoRA adapter (svdq_set_lora): A^T rows for the down pass, (s B)^T rows for the up pass
+  __nv_bfloat16* d_lora_l1t = nullptr;   // [32][K]   A^T, zero rows past r
+  __nv_bfloat16* d_lora_l2s = nullptr;   // [N][32]   (bf16(s B) / alpha)^T (NVFP4 GEMM)
+  __nv_bfloat16* d_lora_l2t = nullptr;   // [N][64]   [L2b^T | bf16(s B)^T] (unfused up projection)
+  CUtensorMap tm_lora_l1t, tm_lora_l2s;
 };
 
 namespace {
@@ -60,6 +65,19 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   });
   return fn;
+}
+
+// 2D tensor [rows][cols] of `elem` bytes with rows `row_bytes` apart, box [box_rows][box_cols].
+bool make_map_strided(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,
+                      uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2D row-major tensor [rows][cols] of `elem` bytes, box [box_rows][box_cols].
@@ -149,12 +167,15 @@ struct WsLayout {
   size_t codes = 0, scales = 0, xl = 0, total = 0;
 };
 
+// Columns of the down projection XL: 32, plus 32 for X A when a LoRA adapter is attached.
+int xl_width(const HostPrep& h) { return h.lora_r > 0 ? 64 : 32; }
+
 WsLayout ws_layout(const HostPrep& h, int M) {
   WsLayout w;
   w.codes = 0;
   w.scales = align_up(act_code_bytes(h, M), 256);
   w.xl = w.scales + align_up(act_scale_bytes(h, M), 256);
-  w.total = w.xl + align_up((size_t)M * 32 * 2, 256);
+  w.total = w.xl + align_up((size_t)M * xl_width(h) * 2, 256);
   return w;
 }
 
@@ -179,7 +200,11 @@ void free_device(svdq_layer* L) {
   cudaFree(L->d_wpair);
   cudaFree(L->d_bias);
   cudaFree(L->d_err);
+  cudaFree(L->d_lora_l1t);
+  cudaFree(L->d_lora_l2s);
+  cudaFree(L->d_lora_l2t);
   L->d_inv_lam = nullptr;
+  L->d_lora_l1t = L->d_lora_l2s = L->d_lora_l2t = nullptr;
 }
 
 svdq_status upload_layer(svdq_layer* L, int device) {
@@ -307,6 +332,7 @@ K1Params k1_params(const svdq_layer* L, int M, void* codes, void* scales, void* 
   p.codes = static_cast<uint8_t*>(codes);
   p.scales = static_cast<uint8_t*>(scales);
   p.xl = static_cast<__nv_bfloat16*>(xl);
+  p.xl_stride = xl_width(h);
   p.err = L->d_err;
   p.budget_ns = L->budget_ns;
   return p;
@@ -332,19 +358,60 @@ svdq_status run_k1(const svdq_layer* L, const void* X, int M, void* codes, void*
                                                                                                     : SVDQ_ECUDA;
 }
 
-svdq_status run_k2_int4(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M,
-                        void* Y, cudaStream_t stream, bool branch, bool gelu) {
+// The LoRA adapter's down pass: XL columns 32..63 = bf16(X A), the first
+// kernel's down-projection-only mode over A^T.
+svdq_status run_k1_lora(const svdq_layer* L, const void* X, int M, void* xl, cudaStream_t stream) {
   const HostPrep& h = L->host;
-  CUtensorMap tm_a, tm_xl, tm_y;
+  CUtensorMap tm_x;
+  if (!make_map_kchunks(&tm_x, X, h.K, M, 32)) return SVDQ_ECUDA;
+  K1Params p = k1_params(L, M, nullptr, nullptr, static_cast<__nv_bfloat16*>(xl) + 32);
+  return launch_k1(tm_x, L->tm_lora_l1t, tm_x, p, kFmtNvfp4, 2, stream) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+}
+
+// The up-projection kernel adding xl ([M][width], row stride xlw) times l2t^T
+// ([N][width]) into Y [+ GELU].
+svdq_status run_upproj(const svdq_layer* L, const void* xl, int xlw, int width, const __nv_bfloat16* l2t, int M,
+                       void* Y, cudaStream_t stream, bool gelu) {
+  UpParams up;
+  up.M = M;
+  up.N = L->host.N;
+  up.width = width;
+  up.xl = static_cast<const __nv_bfloat16*>(xl);
+  up.xl_stride = xlw;
+  up.l2t = l2t;
+  up.gelu = gelu ? 1 : 0;
+  up.err = L->d_err;
+  up.budget_ns = L->budget_ns;
+  CUtensorMap tm_up;
+  if (!make_map(&tm_up, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L->host.N, M, 64, (uint32_t)upproj_box_rows(),
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ECUDA;
+  return launch_upproj(tm_up, up, stream) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+}
+
+svdq_status run_k2_int4(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M,
+                        void* Y, cudaStream_t stream, bool branch, bool gelu, bool lora_on) {
+  const HostPrep& h = L->host;
+  const bool lora = h.lora_r > 0 && lora_on;
+  CUtensorMap tm_a, tm_xl, tm_y, tm_xla;
   if (!make_map(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SVDQ_ECUDA;
   if (!make_map(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ECUDA;
   if (branch) {
-    if (!make_map(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_map_strided(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, M, (uint64_t)xl_width(h) * 2, 32, 128,
+                          CU_TENSOR_MAP_SWIZZLE_64B))
       return SVDQ_ECUDA;
   } else {
     tm_xl = tm_a;   // unused by the kernel
+  }
+  if (lora) {
+    // XL columns 32..63 (X A): the same rows, 64 bytes in
+    if (!make_map_strided(&tm_xla, static_cast<const __nv_bfloat16*>(xl) + 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32,
+                          M, (uint64_t)xl_width(h) * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return SVDQ_ECUDA;
+  } else {
+    tm_xla = tm_a;  // unused by the kernel
   }
   K2Int4Params p;
   p.M = M;
@@ -362,24 +429,41 @@ svdq_status run_k2_int4(const svdq_layer* L, const void* codes, const void* scal
   p.budget_ns = L->budget_ns;
   p.branch = branch ? 1 : 0;
   p.gelu = gelu ? 1 : 0;
-  const cudaError_t e = L->k2_kernel == 2
-                            ? launch_k2_int4_pair(tm_a, L->tm_wq_pair, tm_xl, L->tm_l2s_pair, tm_y, p, L->num_sms, stream)
-                            : launch_k2_int4(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream);
+  p.lora = lora ? 1 : 0;
+  const cudaError_t e =
+      L->k2_kernel == 2 && !lora
+          ? launch_k2_int4_pair(tm_a, L->tm_wq_pair, tm_xl, L->tm_l2s_pair, tm_y, p, L->num_sms, stream)
+          : launch_k2_int4(tm_a, L->tm_wq, tm_xl, L->tm_l2s, tm_y, tm_xla, lora ? L->tm_lora_l2s : L->tm_l2s, p,
+                           L->num_sms, stream);
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
 
+// The second kernel.  With a LoRA adapter (and lora_on) the NVFP4 GEMM adds
+// XL_lora (s B) in its own ring stage, the INT4 GEMM by reloading its branch
+// buffer within the tile; either way into the same accumulator.
 svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
-                   cudaStream_t stream, bool branch, bool gelu) {
-  if (L->host.format == SVDQ_INT4) return run_k2_int4(L, codes, scales, xl, M, Y, stream, branch, gelu);
+                   cudaStream_t stream, bool branch, bool gelu, bool lora_on = true) {
+  if (L->host.format == SVDQ_INT4) return run_k2_int4(L, codes, scales, xl, M, Y, stream, branch, gelu, lora_on);
   const HostPrep& h = L->host;
-  CUtensorMap tm_xl, tm_y;
+  const bool lora = h.lora_r > 0 && lora_on;
+  CUtensorMap tm_xl, tm_y, tm_xla;
   if (!make_map(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ECUDA;
+  const uint64_t xl_row = (uint64_t)xl_width(h) * 2;
   if (branch) {
-    if (!make_map(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_map_strided(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, M, xl_row, 32, 128,
+                          CU_TENSOR_MAP_SWIZZLE_64B))
       return SVDQ_ECUDA;
   } else {
     tm_xl = tm_y;   // unused by the kernel
+  }
+  if (lora) {
+    // XL columns 32..63 (X A): the same rows, 64 bytes in
+    if (!make_map_strided(&tm_xla, static_cast<const __nv_bfloat16*>(xl) + 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32,
+                          M, xl_row, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return SVDQ_ECUDA;
+  } else {
+    tm_xla = tm_y;   // unused by the kernel
   }
   K2Params p;
   p.M = M;
@@ -397,12 +481,110 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
   p.budget_ns = L->budget_ns;
   p.branch = branch ? 1 : 0;
   p.gelu = gelu ? 1 : 0;
+  p.lora = lora ? 1 : 0;
   // The CTA-pair kernel (256 x 256 tiles) is exact but measured slower than the
-  // single-CTA kernel on this part; it runs only when SVDQ_K2_KERNEL=pair.
-  const bool pair = L->k2_kernel == 2;
+  // single-CTA kernel on this part; it runs only when SVDQ_K2_KERNEL=pair, and
+  // only for layers without a LoRA adapter.
+  const bool pair = L->k2_kernel == 2 && !lora;
   const cudaError_t e = pair ? launch_k2_pair(tm_xl, L->tm_l2s_pair, tm_y, p, L->num_sms, stream)
-                             : launch_k2(tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream);
+                             : launch_k2(tm_xl, L->tm_l2s, tm_y, tm_xla, L->tm_lora_l2s, p, L->num_sms, stream);
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+}
+
+// ------------------------------------------------------------------ fc1 -> fc2 chain
+
+bool chainable(const svdq_layer* L1, const svdq_layer* L2) {
+  return L1->host.format == SVDQ_NVFP4 && L2->host.format == SVDQ_NVFP4 && L1->host.N == L2->host.K &&
+         L1->device == L2->device && L1->host.lora_r == 0 && L2->host.lora_r == 0;
+}
+
+// Workspace of the fused chain: [fc1's forward workspace][fc2 codes][fc2 scales]
+// [XL2][partials]; of the unfused chain: [fc1's workspace][Y1 BF16][fc2's workspace].
+struct ChainLayout {
+  size_t codes2 = 0, scales2 = 0, xl2 = 0, partials = 0, y1 = 0, ws2 = 0, total = 0;
+  int S = 1;
+};
+
+ChainLayout chain_layout(const svdq_layer* L1, const svdq_layer* L2, int M, bool unfused) {
+  ChainLayout c;
+  const size_t w1 = align_up(ws_layout(L1->host, M).total, 256);
+  if (unfused) {
+    c.y1 = w1;
+    c.ws2 = c.y1 + align_up((size_t)M * L1->host.N * 2, 256);
+    c.total = c.ws2 + ws_layout(L2->host, M).total;
+    return c;
+  }
+  c.S = k2_chain_splits(M, L1->host.N, L1->num_sms);
+  c.codes2 = w1;
+  c.scales2 = c.codes2 + align_up(act_code_bytes(L2->host, M), 256);
+  c.xl2 = c.scales2 + align_up(act_scale_bytes(L2->host, M), 256);
+  c.partials = c.xl2 + align_up((size_t)M * 32 * 2, 256);
+  c.total = c.partials + (size_t)pad_rows(M) * 2 * c.S * 32 * 4;
+  return c;
+}
+
+// fc1's first kernel, then its GEMM in chain mode (fc2's codes, scales and
+// down-projection partials), then the fixed-order sum of the partials into XL2.
+svdq_status run_chain_fc1(const svdq_layer* L1, const svdq_layer* L2, const void* X, int M, void* codes2,
+                          void* scales2, void* xl2, void* partials, int S, uint8_t* ws1, cudaStream_t s, bool gelu) {
+  const HostPrep& h1 = L1->host;
+  const HostPrep& h2 = L2->host;
+  const WsLayout w = ws_layout(h1, M);
+  void* codes1 = ws1 + w.codes;
+  void* scales1 = ws1 + w.scales;
+  void* xl1 = ws1 + w.xl;
+  const bool branch1 = h1.rank > 0, branch2 = h2.rank > 0;
+  svdq_status st = run_k1(L1, X, M, codes1, scales1, xl1, s, branch1 ? 0 : 1);
+  if (st != SVDQ_OK) return st;
+  CUtensorMap tm_xl;
+  if (branch1) {
+    if (!make_map(&tm_xl, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, M, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return SVDQ_ECUDA;
+  } else {
+    tm_xl = L1->tm_l2s;   // unused by the kernel
+  }
+  K2Params p;
+  p.M = M;
+  p.N = h1.N;
+  p.K = h1.K;
+  p.mpad = pad_rows(M);
+  p.acodes = static_cast<const uint8_t*>(codes1);
+  p.alpha = (float)std::ldexp(1.0, h1.g_x_exp + h1.g_w_exp);
+  p.sfa = static_cast<const uint8_t*>(scales1);
+  p.wmerged = L1->d_wmerged;
+  p.wpair = L1->d_wpair;
+  p.bias = L1->d_bias;
+  p.y = nullptr;
+  p.err = L1->d_err;
+  p.budget_ns = L1->budget_ns;
+  p.branch = branch1 ? 1 : 0;
+  p.gelu = gelu ? 1 : 0;
+  K2Chain& c = p.chain;
+  c.codes = static_cast<uint8_t*>(codes2);
+  c.scales = static_cast<uint8_t*>(scales2);
+  c.inv_lam = L2->d_inv_lam;
+  c.l1t = branch2 ? L2->d_l1t : nullptr;
+  c.partials = static_cast<float*>(partials);
+  c.K2 = h2.K;
+  c.nst = nvfp4_stages(h2.K);
+  c.S = S;
+  c.g_x_exp = h2.g_x_exp;
+  c.c_x = (float)std::ldexp((double)(1.0f / 6.0f), -h2.g_x_exp);
+  for (int m = 0; m < 8; ++m) {
+    c.rcp[m] = (float)(1.0 / (1.0 + m / 8.0));
+    c.rcp[8 + m] = m ? (float)(1.0 / m) : 0.0f;
+  }
+  if (launch_k2_chain(tm_xl, L1->tm_l2s, p, L1->num_sms, s) != cudaSuccess) return SVDQ_ECUDA;
+  if (branch2 && launch_xl_reduce(static_cast<const float*>(partials), 2 * S, M,
+                                  static_cast<__nv_bfloat16*>(xl2), s) != cudaSuccess)
+    return SVDQ_ECUDA;
+  return SVDQ_OK;
+}
+
+// The second kernel (the adapter, if any, is added inside it).
+svdq_status run_gemm_stage(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M,
+                           void* Y, cudaStream_t s, bool branch, bool gelu, bool lora_on) {
+  return run_k2(L, codes, scales, xl, M, Y, s, branch, gelu, lora_on);
 }
 
 }  // namespace
@@ -499,6 +681,8 @@ size_t svdq_tensor_bytes(const svdq_layer* L, int id) {
     case SVDQ_T_W_SCALES: return h.format == SVDQ_NVFP4 ? h.w_scales_e4m3.size() : h.w_scales_bf16.size() * 2;
     case SVDQ_T_BIAS: return h.bias.size() * 4;
     case SVDQ_T_GPTQ_U: return h.gptq_U.size() * 8;
+    case SVDQ_T_LORA_A: return h.lora_A.size() * 2;
+    case SVDQ_T_LORA_B: return h.lora_B.size() * 2;
   }
   return 0;
 }
@@ -524,6 +708,8 @@ svdq_status svdq_export(const svdq_layer* L, int id, void* dst, size_t bytes) {
       break;
     case SVDQ_T_BIAS: src = h.bias.data(); break;
     case SVDQ_T_GPTQ_U: src = h.gptq_U.data(); break;
+    case SVDQ_T_LORA_A: src = h.lora_A.data(); break;
+    case SVDQ_T_LORA_B: src = h.lora_B.data(); break;
     default: return SVDQ_EINVAL;
   }
   std::memcpy(dst, src, bytes);
@@ -591,12 +777,17 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int M, void* c
   if (!w4a4(L)) return SVDQ_EUNSUPPORTED;
   if (mode < 0 || mode > 2) return SVDQ_EINVAL;
   if (!scales && mode != 2) return SVDQ_EINVAL;
-  if (L->host.rank == 0 && mode == 2) return SVDQ_EINVAL;
-  if (L->host.rank == 0 && mode == 0) mode = 1;
-  if (L->host.rank > 0 && mode != 1 && !xl) return SVDQ_EINVAL;
+  const bool rank = L->host.rank > 0, lora = L->host.lora_r > 0;
+  const bool has_xl = rank || lora;
+  if (!has_xl && mode == 2) return SVDQ_EINVAL;
+  if (!has_xl && mode == 0) mode = 1;
+  if (has_xl && mode != 1 && !xl) return SVDQ_EINVAL;
   DeviceGuard g(L->device);
   if (!g.ok) return SVDQ_ECUDA;
-  return run_k1(L, X, M, codes, scales, xl, static_cast<cudaStream_t>(stream), mode);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (rank || mode != 2) st = run_k1(L, X, M, codes, scales, xl, s, rank ? mode : 1);
+  if (st == SVDQ_OK && lora && mode != 1) st = run_k1_lora(L, X, M, xl, s);
+  return st;
 }
 
 svdq_status svdq_gemm(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
@@ -605,12 +796,14 @@ svdq_status svdq_gemm(const svdq_layer* L, const void* codes, const void* scales
   if (st != SVDQ_OK) return st;
   if (!w4a4(L)) return SVDQ_EUNSUPPORTED;
   if (!scales) return SVDQ_EINVAL;
-  const bool branch = L->host.rank > 0 && !(flags & SVDQ_FWD_NO_BRANCH);
-  if (branch && !xl) return SVDQ_EINVAL;
+  const bool bare = (flags & SVDQ_FWD_NO_BRANCH) != 0;
+  const bool branch = L->host.rank > 0 && !bare;
+  const bool lora = L->host.lora_r > 0 && !bare;
+  if ((branch || lora) && !xl) return SVDQ_EINVAL;
   DeviceGuard g(L->device);
   if (!g.ok) return SVDQ_ECUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = run_k2(L, codes, scales, xl, M, Y, s, branch, (flags & SVDQ_FWD_GELU) != 0);
+  st = run_gemm_stage(L, codes, scales, xl, M, Y, s, branch, (flags & SVDQ_FWD_GELU) != 0, lora);
   if (st == SVDQ_OK && (flags & SVDQ_FWD_CHECK)) st = svdq_check(L, stream);
   return st;
 }
@@ -650,34 +843,163 @@ svdq_status svdq_linear_forward(const svdq_layer* L, const void* X, int M, void*
   void* scales = ws + w.scales;
   void* xl = ws + w.xl;
   const bool gelu = (flags & SVDQ_FWD_GELU) != 0;
+  const bool bare = (flags & SVDQ_FWD_NO_BRANCH) != 0;
   const bool has_branch = L->host.rank > 0;
-  if ((flags & SVDQ_FWD_UNFUSED) && has_branch) {
-    // measurement variant: down projection, quantize, bare GEMM, up projection
+  const bool lora = L->host.lora_r > 0 && !bare;
+  const int xlw = xl_width(L->host);
+  if ((flags & SVDQ_FWD_UNFUSED) && (has_branch || lora) && !bare) {
+    // measurement variant: down projection(s), quantize, bare GEMM, up projection.
+    // A rank-0 layer's L1d^T is all zero: its pass writes zero XL columns for
+    // the 64-wide up projection to read.
     st = run_k1(L, X, M, codes, scales, xl, s, 2);
+    if (st == SVDQ_OK && lora) st = run_k1_lora(L, X, M, xl, s);
     if (st == SVDQ_OK) st = run_k1(L, X, M, codes, scales, xl, s, 1);
-    if (st == SVDQ_OK) st = run_k2(L, codes, scales, xl, M, Y, s, false, false);
-    if (st == SVDQ_OK) {
-      UpParams up;
-      up.M = M;
-      up.N = L->host.N;
-      up.xl = static_cast<const __nv_bfloat16*>(xl);
-      up.l2t = L->d_l2t;
-      up.gelu = gelu ? 1 : 0;
-      up.err = L->d_err;
-      up.budget_ns = L->budget_ns;
-      CUtensorMap tm_up;
-      if (!make_map(&tm_up, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L->host.N, M, 64, (uint32_t)upproj_box_rows(),
-                    CU_TENSOR_MAP_SWIZZLE_128B))
-        st = SVDQ_ECUDA;
-      else
-        st = launch_upproj(tm_up, up, s) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
-    }
+    if (st == SVDQ_OK) st = run_k2(L, codes, scales, xl, M, Y, s, false, false, false);
+    // one up projection over the whole branch: [L2b^T | bf16(s B)^T] with an adapter
+    if (st == SVDQ_OK) st = run_upproj(L, xl, xlw, lora ? 64 : 32, lora ? L->d_lora_l2t : L->d_l2t, M, Y, s, gelu);
   } else {
-    const bool branch = has_branch && !(flags & SVDQ_FWD_NO_BRANCH);
+    const bool branch = has_branch && !bare;
     st = run_k1(L, X, M, codes, scales, xl, s, branch ? 0 : 1);
-    if (st == SVDQ_OK) st = run_k2(L, codes, scales, xl, M, Y, s, branch, gelu);
+    if (st == SVDQ_OK && lora) st = run_k1_lora(L, X, M, xl, s);
+    if (st == SVDQ_OK) st = run_gemm_stage(L, codes, scales, xl, M, Y, s, branch, gelu, lora);
   }
   if (st == SVDQ_OK && (flags & SVDQ_FWD_CHECK)) st = svdq_check(L, stream);
+  return st;
+}
+
+svdq_status svdq_set_lora(svdq_layer* L, int r, const uint16_t* A_bf16, const uint16_t* B_bf16, float scale) {
+  if (!L) return SVDQ_EINVAL;
+  if (L->host.format == SVDQ_W4A16_INT4) return SVDQ_EUNSUPPORTED;
+  if (r < 0) return SVDQ_EINVAL;
+  if (r > 32) return SVDQ_EUNSUPPORTED;
+  if (r > 0 && (!A_bf16 || !B_bf16 || !std::isfinite(scale))) return SVDQ_EINVAL;
+  HostPrep& h = L->host;
+  const int K = h.K, N = h.N;
+  try {
+    std::vector<uint16_t> a, b;
+    if (r > 0) {
+      a.assign(A_bf16, A_bf16 + (size_t)K * r);
+      b.resize((size_t)r * N);
+      for (size_t i = 0; i < b.size(); ++i)
+        b[i] = bf16_from_double((double)bf16_to_float(B_bf16[i]) * (double)scale);   // one rounding of s B
+    }
+    if (L->device >= 0) {
+      DeviceGuard g(L->device);
+      if (!g.ok) return SVDQ_ECUDA;
+      // no forward of this layer may be pending: the old buffers are released
+      if (cudaDeviceSynchronize() != cudaSuccess) return SVDQ_ECUDA;
+      cudaFree(L->d_lora_l1t);
+      cudaFree(L->d_lora_l2s);
+      cudaFree(L->d_lora_l2t);
+      L->d_lora_l1t = L->d_lora_l2s = L->d_lora_l2t = nullptr;
+      if (r > 0) {
+        // the GEMM's accumulator unit: alpha = g_x g_w (NVFP4) or 2^(ex + ew) (INT4)
+        const int alpha_exp = h.format == SVDQ_NVFP4 ? h.g_x_exp + h.g_w_exp : L->i4_ex + L->i4_ew;
+        // l2t: the unfused up projection's [N][64] = [L2b^T | bf16(s B)^T]
+        std::vector<uint16_t> l1t((size_t)32 * K, 0), l2s((size_t)N * 32, 0), l2t((size_t)N * 64, 0);
+        for (int i = 0; i < h.rank; ++i)
+          for (int n = 0; n < N; ++n) l2t[(size_t)n * 64 + i] = h.L2b[(size_t)i * N + n];
+        for (int i = 0; i < r; ++i) {
+          for (int k = 0; k < K; ++k) l1t[(size_t)i * K + k] = a[(size_t)k * r + i];
+          for (int n = 0; n < N; ++n) {
+            const uint16_t v = b[(size_t)i * N + n];
+            l2t[(size_t)n * 64 + 32 + i] = v;
+            l2s[(size_t)n * 32 + i] = bf16_from_double(std::ldexp((double)bf16_to_float(v), -alpha_exp));
+          }
+        }
+        cudaError_t e = upload(&L->d_lora_l1t, l1t.data(), l1t.size() * 2);
+        if (e == cudaSuccess) e = upload(&L->d_lora_l2s, l2s.data(), l2s.size() * 2);
+        if (e == cudaSuccess) e = upload(&L->d_lora_l2t, l2t.data(), l2t.size() * 2);
+        if (e != cudaSuccess || !make_map_kchunks(&L->tm_lora_l1t, L->d_lora_l1t, K, 32, 32) ||
+            !make_map(&L->tm_lora_l2s, L->d_lora_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
+                      CU_TENSOR_MAP_SWIZZLE_64B)) {
+          cudaFree(L->d_lora_l1t);
+          cudaFree(L->d_lora_l2s);
+          cudaFree(L->d_lora_l2t);
+          L->d_lora_l1t = L->d_lora_l2s = L->d_lora_l2t = nullptr;
+          h.lora_r = 0;
+          h.lora_A.clear();
+          h.lora_B.clear();
+          return e == cudaErrorMemoryAllocation ? SVDQ_ENOMEM : SVDQ_ECUDA;
+        }
+      }
+    }
+    h.lora_r = r;
+    h.lora_A.swap(a);
+    h.lora_B.swap(b);
+  } catch (const std::bad_alloc&) {
+    return SVDQ_ENOMEM;
+  }
+  return SVDQ_OK;
+}
+
+size_t svdq_mlp_workspace_bytes(const svdq_layer* fc1, const svdq_layer* fc2, int M, unsigned flags) {
+  if (!fc1 || !fc2 || M < 1 || fc1->device < 0 || !chainable(fc1, fc2)) return 0;
+  return chain_layout(fc1, fc2, M, (flags & SVDQ_FWD_UNFUSED) != 0).total;
+}
+
+svdq_status svdq_mlp_fc1(const svdq_layer* fc1, const svdq_layer* fc2, const void* X, int M, void* codes2,
+                         void* scales2, void* xl2, void* workspace, size_t workspace_bytes, void* stream,
+                         unsigned flags) {
+  svdq_status st = check_forward_args(fc1, X, M, codes2);
+  if (st != SVDQ_OK) return st;
+  if (!fc2 || !scales2) return SVDQ_EINVAL;
+  if (fc2->device < 0) return SVDQ_ESTATE;
+  if (!chainable(fc1, fc2)) return SVDQ_EUNSUPPORTED;
+  if (flags & ~(SVDQ_FWD_GELU | SVDQ_FWD_CHECK)) return SVDQ_EUNSUPPORTED;
+  if (fc2->host.rank > 0 && !xl2) return SVDQ_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(codes2) & 15) || (reinterpret_cast<uintptr_t>(scales2) & 15) ||
+      (reinterpret_cast<uintptr_t>(xl2) & 15))
+    return SVDQ_EINVAL;
+  const ChainLayout c = chain_layout(fc1, fc2, M, false);
+  if (!workspace || workspace_bytes < c.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return SVDQ_EINVAL;
+  DeviceGuard g(fc1->device);
+  if (!g.ok) return SVDQ_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  st = run_chain_fc1(fc1, fc2, X, M, codes2, scales2, xl2, ws + c.partials, c.S, ws, s,
+                     (flags & SVDQ_FWD_GELU) != 0);
+  if (st == SVDQ_OK && (flags & SVDQ_FWD_CHECK)) st = svdq_check(fc1, stream);
+  return st;
+}
+
+svdq_status svdq_mlp_forward(const svdq_layer* fc1, const svdq_layer* fc2, const void* X, int M, void* Y,
+                             void* workspace, size_t workspace_bytes, void* stream, unsigned flags) {
+  svdq_status st = check_forward_args(fc1, X, M, Y);
+  if (st != SVDQ_OK) return st;
+  if (!fc2) return SVDQ_EINVAL;
+  if (fc2->device < 0) return SVDQ_ESTATE;
+  if (!chainable(fc1, fc2)) return SVDQ_EUNSUPPORTED;
+  if (flags & ~(SVDQ_FWD_GELU | SVDQ_FWD_CHECK | SVDQ_FWD_UNFUSED)) return SVDQ_EUNSUPPORTED;
+  const bool unfused = (flags & SVDQ_FWD_UNFUSED) != 0;
+  const ChainLayout c = chain_layout(fc1, fc2, M, unfused);
+  if (!workspace || workspace_bytes < c.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return SVDQ_EINVAL;
+  DeviceGuard g(fc1->device);
+  if (!g.ok) return SVDQ_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool gelu = (flags & SVDQ_FWD_GELU) != 0;
+  const bool branch2 = fc2->host.rank > 0;
+  if (unfused) {
+    // the two layers one after the other, fc1's output through HBM in BF16
+    const WsLayout w1 = ws_layout(fc1->host, M), w2 = ws_layout(fc2->host, M);
+    uint8_t* ws2 = ws + c.ws2;
+    void* y1 = ws + c.y1;
+    const bool branch1 = fc1->host.rank > 0;
+    st = run_k1(fc1, X, M, ws + w1.codes, ws + w1.scales, ws + w1.xl, s, branch1 ? 0 : 1);
+    if (st == SVDQ_OK) st = run_k2(fc1, ws + w1.codes, ws + w1.scales, ws + w1.xl, M, y1, s, branch1, gelu);
+    if (st == SVDQ_OK) st = run_k1(fc2, y1, M, ws2 + w2.codes, ws2 + w2.scales, ws2 + w2.xl, s, branch2 ? 0 : 1);
+    if (st == SVDQ_OK) st = run_k2(fc2, ws2 + w2.codes, ws2 + w2.scales, ws2 + w2.xl, M, Y, s, branch2, false);
+  } else {
+    st = run_chain_fc1(fc1, fc2, X, M, ws + c.codes2, ws + c.scales2, ws + c.xl2, ws + c.partials, c.S, ws, s,
+                       gelu);
+    if (st == SVDQ_OK) st = run_k2(fc2, ws + c.codes2, ws + c.scales2, ws + c.xl2, M, Y, s, branch2, false);
+  }
+  if (st == SVDQ_OK && (flags & SVDQ_FWD_CHECK)) {
+    st = svdq_check(fc1, stream);
+    const svdq_status st2 = svdq_check(fc2, stream);
+    if (st == SVDQ_OK) st = st2;
+  }
   return st;
 }
 

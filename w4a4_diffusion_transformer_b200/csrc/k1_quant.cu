@@ -34,17 +34,19 @@
 // its scales group-major, [K/64][M padded to 128] BF16, the order the INT4 GEMM
 // stages them in.
 //
-// NVFP4 quantizer arithmetic per group of 16 (bit-exact with the CPU oracle): a =
-// max|v|; t = fp32(a * c_x) with c_x = fp32(1/6) 2^-gx; s = E4M3_rn_satfinite(t);
-// s == 0 -> all codes +0; inv = fp32(1 / (s * g_x)); code =
-// E2M1_rn_satfinite(fp32(v * inv)).  The reciprocal is exact without a
-// division: for s = (1 + m/8) 2^(e-7) (or m 2^-9 when e = 0) it equals
-// fp32(1/(1 + m/8)) 2^(7-e-gx) (or fp32(1/m) 2^(9-gx)), a power-of-two scaling
-// of one of 15 correctly rounded constants computed on the host.
+// NVFP4 quantizer arithmetic per group of 16 (bit-exact with the CPU oracle; the
+// device code is nvfp4_quant32 in nvfp4_quant.cuh): a = max|v|; t = fp32(a *
+// c_x) with c_x = fp32(1/6) 2^-gx; s = E4M3_rn_satfinite(t); s == 0 -> all
+// codes +0; inv = fp32(1 / (s * g_x)); code = E2M1_rn_satfinite(fp32(v *
+// inv)).  The reciprocal is exact without a division: for s = (1 + m/8)
+// 2^(e-7) (or m 2^-9 when e = 0) it equals fp32(1/(1 + m/8)) 2^(7-e-gx) (or
+// fp32(1/m) 2^(9-gx)), a power-of-two scaling of one of 15 correctly rounded
+// constants computed on the host.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "kernels.h"
+#include "nvfp4_quant.cuh"
 #include "sm100.cuh"
 
 namespace svdq {
@@ -340,29 +342,7 @@ __global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
             v[i * 4 + e] = __fmul2_rn(make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)),
                                       iv[e]);
         }
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          a0 = dev::fmax3(a0, fabsf(v[i].x), fabsf(v[i].y));
-          a1 = dev::fmax3(a1, fabsf(v[8 + i].x), fabsf(v[8 + i].y));
-        }
-        sb2 = dev::cvt_e4m3x2(__fmul_rn(a0, p.c_x), __fmul_rn(a1, p.c_x));
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const uint32_t sb = (sb2 >> (8 * g)) & 0xFFu;
-          if (sb != 0u) {
-            const uint32_t e = sb >> 3, m = sb & 7u;
-            const int p2 = (e ? 7 - (int)e : 9) - p.g_x_exp;
-            const float invs = rcp[(e ? 0 : 8) + m] * __int_as_float((p2 + 127) << 23);
-            const float2 inv2 = make_float2(invs, invs);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int b = g * 8 + h * 4;
-              packed[2 * g + h] = dev::cvt_e2m1x8(__fmul2_rn(v[b], inv2), __fmul2_rn(v[b + 1], inv2),
-                                                  __fmul2_rn(v[b + 2], inv2), __fmul2_rn(v[b + 3], inv2));
-            }
-          }
-        }
+        sb2 = dev::nvfp4_quant32(v, p.c_x, p.g_x_exp, rcp, packed);
       }
       // the stage's inputs have been read
       __syncwarp();
@@ -453,9 +433,10 @@ __global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
     const int row = row0 + fm * 16 + (fl >> 2);
     const int col = fn * 8 + 2 * (fl & 3);
     if (row < p.M)
-      *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)row * 32 + col) = __floats2bfloat162_rn(sum.x, sum.y);
+      *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)row * p.xl_stride + col) = __floats2bfloat162_rn(sum.x, sum.y);
     if (row + 8 < p.M)
-      *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)(row + 8) * 32 + col) = __floats2bfloat162_rn(sum.z, sum.w);
+      *reinterpret_cast<__nv_bfloat162*>(p.xl + (size_t)(row + 8) * p.xl_stride + col) =
+          __floats2bfloat162_rn(sum.z, sum.w);
   }
 }
 

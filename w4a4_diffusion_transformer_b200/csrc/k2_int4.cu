@@ -105,11 +105,6 @@ __device__ __forceinline__ void record_error(int* err, volatile int* abort_flag,
   *abort_flag = 1;
 }
 
-__device__ __forceinline__ float gelu_tanh(float y) {
-  const float k0 = 0.7978845608028654f;   // sqrt(2/pi)
-  return 0.5f * y * (1.0f + tanhf(k0 * (y + 0.044715f * y * y * y)));
-}
-
 // Instruction descriptor: FP16 x FP16 -> FP32, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -130,10 +125,18 @@ __device__ __forceinline__ void dequant_word(uint32_t w, __half2 s2, uint32_t (&
   }
 }
 
+// A LoRA adapter (p.lora) reuses the branch buffer within each tile: the
+// producer reloads it with XL_lora and (s B / alpha)^T once the tile's branch
+// MMAs have read it (after issuing group kLoraLoadG), and the MMA warp adds the
+// adapter after group kLoraMmaG, so the reload overlaps the group stream.  The
+// buffer's barriers then complete twice per tile; both sides count the phases.
+constexpr int kLoraLoadG = 2, kLoraMmaG = 5;
+
 __global__ void __launch_bounds__(kThreads, 1)
     k2_int4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2,
-                   const __grid_constant__ CUtensorMap tm_y, K2Int4Params p) {
+                   const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_xla,
+                   const __grid_constant__ CUtensorMap tm_l2a, K2Int4Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* oring = smem;                                          // operand ring (1 KiB aligned)
@@ -202,13 +205,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::tma_prefetch_desc(&tm_xl);
         dev::tma_prefetch_desc(&tm_l2);
       }
-      int it = 0, tcount = 0;
+      if (p.lora) {
+        dev::tma_prefetch_desc(&tm_xla);
+        dev::tma_prefetch_desc(&tm_l2a);
+      }
+      const int lora_g = min(kLoraLoadG, G - 1);
+      int it = 0, bc = 0;                           // bc: branch-buffer loads so far
       bool ok = true, deps_ready = false;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m0 = (tile % tiles_m) * kBM;
         const int n0 = (tile / tiles_m) * kBN;
         if (p.branch) {
-          if (!dev::mbar_wait(bempty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+          if (!dev::mbar_wait(bempty, ((uint32_t)bc & 1u) ^ 1u, abort_flag, p.budget_ns)) {
             record_error(p.err, abort_flag, 0x301);
             break;
           }
@@ -219,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             deps_ready = true;
           }
           dev::tma_load_2d(brbuf, &tm_xl, bfull, 0, m0);
+          ++bc;
         }
         for (int g = 0; g < G; ++g, ++it) {
           const int s = it % kPStages;
@@ -238,6 +247,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           dev::tma_load_2d(st + kPA, &tm_a, &pfull[s], g * 32, m0);
           dev::bulk_load(st + kPSA, p.sa + (size_t)g * p.mpad + m0, kBM * 2, &pfull[s]);
+          if (p.lora && g == lora_g) {
+            // the adapter's tiles, once the tile's branch MMAs have read the buffer
+            if (!dev::mbar_wait(bempty, ((uint32_t)bc & 1u) ^ 1u, abort_flag, p.budget_ns)) {
+              record_error(p.err, abort_flag, 0x306);
+              ok = false;
+              break;
+            }
+            dev::mbar_arrive_expect_tx(bfull, kBrBytes);
+            dev::tma_load_2d(brbuf + kBrABytes, &tm_l2a, bfull, 0, n0);
+            dev::tma_load_2d(brbuf, &tm_xla, bfull, 0, m0);
+            ++bc;
+          }
         }
       }
       // every exit path waits for the preceding grid, so that this grid never
@@ -245,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!deps_ready) dev::griddep_wait();
       for (int j = max(0, it - kPStages); j < it; ++j)
         if (!dev::mbar_wait(&pfull[j % kPStages], (uint32_t)(j / kPStages) & 1u, abort_flag, p.budget_ns)) break;
-      if (p.branch && tcount > 0) dev::mbar_wait(bfull, (uint32_t)(tcount - 1) & 1u, abort_flag, p.budget_ns);
+      if (bc > 0) dev::mbar_wait(bfull, (uint32_t)(bc - 1) & 1u, abort_flag, p.budget_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -253,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id16 = idesc_f16(kBM, kBN);
       const uint32_t idbf = dev::idesc_bf16(kBM, kBN);
-      int it = 0, tcount = 0;
+      const int lora_g = min(kLoraMmaG, G - 1);
+      int it = 0, tcount = 0, bc = 0;               // bc: branch-buffer phases consumed
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
         const int ab = tcount & 1;
@@ -265,10 +287,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::tc_fence_after();
         uint32_t accumulate = 0;
         if (p.branch) {
-          if (!dev::mbar_wait(bfull, (uint32_t)tcount & 1u, abort_flag, p.budget_ns)) {
+          if (!dev::mbar_wait(bfull, (uint32_t)bc & 1u, abort_flag, p.budget_ns)) {
             record_error(p.err, abort_flag, 0x304);
             break;
           }
+          ++bc;
           dev::tc_fence_after();
           const uint32_t a0 = dev::smem_u32(brbuf);
           const uint32_t b0 = a0 + kBrABytes;
@@ -297,6 +320,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             accumulate = 1;
           }
           dev::tc_commit(&oempty[s]);
+          if (p.lora && g == lora_g) {
+            if (!dev::mbar_wait(bfull, (uint32_t)bc & 1u, abort_flag, p.budget_ns)) {
+              record_error(p.err, abort_flag, 0x307);
+              ok = false;
+              break;
+            }
+            ++bc;
+            dev::tc_fence_after();
+            const uint32_t la = dev::smem_u32(brbuf);
+            const uint32_t lb = la + kBrABytes;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              dev::mma_bf16(dacc, dev::smem_desc(la + 32 * j, 16, 512, 4), dev::smem_desc(lb + 32 * j, 16, 512, 4),
+                            idbf, 1u);
+            dev::tc_commit(bempty);
+          }
         }
         if (!ok) break;
         dev::tc_commit(&acc_full[ab]);
@@ -422,8 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float y0 = p.alpha * __uint_as_float(cur[i0]) + bias[i0];
             float y1 = p.alpha * __uint_as_float(cur[i0 + 1]) + bias[i0 + 1];
             if (p.gelu) {
-              y0 = gelu_tanh(y0);
-              y1 = gelu_tanh(y1);
+              y0 = dev::gelu_tanh(y0);
+              y1 = dev::gelu_tanh(y1);
             }
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
             packed[e] = *reinterpret_cast<const uint32_t*>(&h2);
@@ -464,8 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_k2_int4(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
-                           const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Int4Params& p, int num_sms,
-                           cudaStream_t stream) {
+                           const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const CUtensorMap& tm_xla,
+                           const CUtensorMap& tm_l2a, const K2Int4Params& p, int num_sms, cudaStream_t stream) {
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -491,7 +530,7 @@ cudaError_t launch_k2_int4(const CUtensorMap& tm_a, const CUtensorMap& tm_b, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k2_int4_kernel, tm_a, tm_b, tm_xl, tm_l2, tm_y, p);
+  return cudaLaunchKernelEx(&cfg, k2_int4_kernel, tm_a, tm_b, tm_xl, tm_l2, tm_y, tm_xla, tm_l2a, p);
 }
 
 }  // namespace svdq

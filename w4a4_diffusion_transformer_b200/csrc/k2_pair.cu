@@ -103,11 +103,6 @@ __device__ __forceinline__ void record_error(int* err, volatile int* abort_flag,
   *abort_flag = 1;
 }
 
-__device__ __forceinline__ float gelu_tanh(float y) {
-  const float k0 = 0.7978845608028654f;   // sqrt(2/pi)
-  return 0.5f * y * (1.0f + tanhf(k0 * (y + 0.044715f * y * y * y)));
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     k2_pair_kernel(const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2,
                    const __grid_constant__ CUtensorMap tm_y, K2Params p) {
@@ -426,8 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float y0 = p.alpha * __uint_as_float(cur[i0]) + bias[i0];
             float y1 = p.alpha * __uint_as_float(cur[i0 + 1]) + bias[i0 + 1];
             if (p.gelu) {
-              y0 = gelu_tanh(y0);
-              y1 = gelu_tanh(y1);
+              y0 = dev::gelu_tanh(y0);
+              y1 = dev::gelu_tanh(y1);
             }
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
             packed[e] = *reinterpret_cast<const uint32_t*>(&h2);

@@ -24,9 +24,31 @@ struct K1Params {
   const float* inv_lam;         // [K]
   uint8_t* codes;               // NVFP4: tiled layout (act_tile_offset); INT4: [M][K/2]
   uint8_t* scales;              // NVFP4: tensor-core scale layout, mpad rows; INT4: BF16 [K/64][mpad]
-  __nv_bfloat16* xl;            // [M][32]
+  __nv_bfloat16* xl;            // [M][32] with row stride xl_stride elements
+  int xl_stride;                // 32, or 64 when a LoRA adapter's XL_lora shares the rows
   int* err;                     // device error word
   unsigned long long budget_ns; // bound on each wait
+};
+
+// fc1 -> fc2 chain: the NVFP4 GEMM of fc1 hands fc2 its input already
+// quantized (fc1's N is fc2's K).  Per output tile the epilogue rounds
+// y = [gelu](alpha acc + b) to BF16 -- the value fc2 would read -- quantizes
+// x_hat = fp32(y * inv_lam2) into fc2's activation codes and scales (the first
+// kernel's layouts and arithmetic), and accumulates y L1d2 (fc2's down
+// projection) over the tiles of one 128-row block that the CTA owns; the
+// per-CTA partial sums are added in a fixed order by launch_xl_reduce.
+struct K2Chain {
+  uint8_t* codes;               // fc2 activation codes, tiled layout (act_tile_offset over K2), mpad rows
+  uint8_t* scales;              // fc2 activation scales, tensor-core layout over K2, mpad rows
+  const float* inv_lam;         // fc2's 1/lam, [K2]
+  const __nv_bfloat16* l1t;     // fc2's L1d^T, [32][K2]; null when fc2 has no branch
+  float* partials;              // [mpad][2 S][32] partial sums of y L1d2 (with l1t)
+  int K2;                       // = N of this GEMM
+  int nst;                      // ceil(K2 / 256)
+  int S;                        // CTAs that share one 128-row block (N-tile ranges)
+  int g_x_exp;                  // fc2's activation tensor scale 2^g_x_exp
+  float c_x;                    // fp32(1/6) * 2^-g_x_exp
+  float rcp[16];                // the quantizer's reciprocal constants (K1Params::rcp)
 };
 
 struct K2Params {
@@ -43,6 +65,8 @@ struct K2Params {
   unsigned long long budget_ns;
   int branch;                   // 1: add XL (L2b / alpha) into the accumulator
   int gelu;                     // 1: tanh-GELU epilogue
+  int lora;                     // 1: one more ring stage per tile adds XL_lora (s B / alpha) (tm_xla, tm_l2a)
+  K2Chain chain;                // launch_k2_chain only
 };
 
 struct K2Int4Params {
@@ -58,12 +82,15 @@ struct K2Int4Params {
   unsigned long long budget_ns;
   int branch;                   // 1: add XL (L2b / alpha) into the accumulator
   int gelu;                     // 1: tanh-GELU epilogue
+  int lora;                     // 1: add XL_lora (s B / alpha) too (tm_xla, tm_l2a), same accumulator
 };
 
 struct UpParams {
   int M, N;
-  const __nv_bfloat16* xl;      // [M][32]
-  const __nv_bfloat16* l2t;     // [N][32] = L2b^T
+  int width;                    // branch width: 32, or 64 with a LoRA adapter
+  const __nv_bfloat16* xl;      // [M][width], row stride xl_stride elements
+  int xl_stride;
+  const __nv_bfloat16* l2t;     // [N][width] = L2b^T (with bf16(s B)^T beside it)
   int gelu;
   int* err;                     // device error word (a wait that ran out)
   unsigned long long budget_ns;
@@ -93,10 +120,22 @@ cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CU
 int k1_rows_per_cta();
 
 // NVFP4 GEMM: operands from p.acodes / p.sfa (the first kernel's layouts) and
-// p.wmerged; tm_xl / tm_l2 the branch tiles, tm_y the output.
+// p.wmerged; tm_xl / tm_l2 the branch tiles, tm_y the output; with p.lora,
+// tm_xla / tm_l2a the LoRA tiles (XL_lora [M][32], (s B / alpha)^T [N][32]; the
+// same boxes and swizzle as tm_xl / tm_l2).
 cudaError_t launch_k2(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
-                      const K2Params& p, int num_sms, cudaStream_t stream);
+                      const CUtensorMap& tm_xla, const CUtensorMap& tm_l2a, const K2Params& p, int num_sms,
+                      cudaStream_t stream);
 int k2_block_n();
+// The same GEMM in chain mode (p.chain; Y is not written): CTA c owns 128-row
+// block c / S and the c % S-th of S contiguous ranges of N tiles.
+// k2_chain_splits gives S for an M x N GEMM on num_sms SMs.
+cudaError_t launch_k2_chain(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const K2Params& p, int num_sms,
+                            cudaStream_t stream);
+int k2_chain_splits(int M, int N, int num_sms);
+// xl[m][j] = bf16(sum_{i < nparts} partials[m][i][j]) in order i = 0, 1, ...
+// (m < M, j < 32); launched as a programmatic dependent of the chain GEMM.
+cudaError_t launch_xl_reduce(const float* partials, int nparts, int M, __nv_bfloat16* xl, cudaStream_t stream);
 // The single-CTA GEMM's weight layout: per (256-row block, 256-K stage) the 32 KB
 // of tiled codes (wgt_tile_offset) followed by the 4 KB of scale factors of the
 // block's 256 rows (tensor-core layout, zero past K): one contiguous copy per stage.
@@ -118,8 +157,8 @@ void k2_pair_pack_weights(const uint8_t* tiled_codes, const uint8_t* sf, int N, 
 // INT4 GEMM: A = activation codes [M][K/2] (box 32 B x 128 rows), B = weight
 // codes [N][K/2] (box 32 B x 256 rows), both unswizzled.
 cudaError_t launch_k2_int4(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
-                           const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Int4Params& p, int num_sms,
-                           cudaStream_t stream);
+                           const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const CUtensorMap& tm_xla,
+                           const CUtensorMap& tm_l2a, const K2Int4Params& p, int num_sms, cudaStream_t stream);
 // The INT4 GEMM on CTA pairs (256 x 256 tiles, clusters of two): tm_b and tm_l2
 // with boxes of k2_int4_pair_rows_b() rows.
 int k2_int4_pair_rows_b();

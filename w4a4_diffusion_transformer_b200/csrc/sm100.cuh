@@ -162,6 +162,29 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Named barrier that also ANDs a predicate over the `threads` participants:
+// every participant gets the same answer, so they can leave a loop together.
+__device__ __forceinline__ bool named_barrier_and(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
+// 16-byte asynchronous copy global -> shared; src_bytes < 16 zero-fills the
+// rest (0: nothing is read and the 16 bytes become zero).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // ------------------------------------------------------------------ tcgen05
 
 // Allocate `ncols` TMEM columns (power of two >= 32); the address is written
@@ -491,6 +514,16 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// tanh-form GELU, 0.5 y (1 + tanh(u)) with u = sqrt(2/pi) (y + 0.044715 y^3),
+// evaluated as y / (1 + e^(-2u)): the same function, since 0.5 (1 + tanh u) is
+// the logistic function of 2u.  One exponential and one fast division keep the
+// relative error near 1e-6, far below the BF16 rounding of the result; for
+// very negative y the quotient underflows to zero, the function's limit.
+__device__ __forceinline__ float gelu_tanh(float y) {
+  const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
+  return __fdividef(y, 1.0f + __expf(-2.0f * u));
 }
 
 // ------------------------------------------------------------------ conversions

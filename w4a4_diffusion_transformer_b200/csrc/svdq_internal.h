@@ -31,6 +31,9 @@ struct HostPrep {
   float x_amax = 0.0f;                      // max |fp32(Xc / lam)| over the calibration batch
   float w_amax = 0.0f;                      // largest group maximum the residual quantizer saw
   std::vector<double> gptq_U;               // [K][K] GPTQ factor (kept only on request)
+  int lora_r = 0;                           // LoRA adapter rank (0: none)
+  std::vector<uint16_t> lora_A;             // [K][lora_r] BF16 bits, as given
+  std::vector<uint16_t> lora_B;             // [lora_r][N] BF16 bits of bf16(scale * B)
   std::vector<uint8_t> w_codes;             // [N][K/2]
   std::vector<uint8_t> w_scales_e4m3;       // [N][K/16]   (NVFP4)
   std::vector<uint16_t> w_scales_bf16;      // [N][K/64]   (INT4 / W4A16)

@@ -1,4 +1,5 @@
-// Unfused low-rank up projection (measurement variant only).
+// Unfused low-rank up projection (measurement variant only).  With a LoRA
+// adapter the branch is 64 wide ([XL | X A] times [L2b ; bf16(s B)]), one pass.
 //
 // The SOTA-314 practice page ("Do this") reports that running the rank-32
 // branch as separate 16-bit kernels adds 57% latency, from "the extra 16-bit
@@ -31,13 +32,11 @@ constexpr int kTileM = 64;     // 4 warps x 16 rows
 constexpr int kTileN = 128;    // two 64-column TMA boxes
 constexpr int kBoxBytes = 64 * 128;
 
-__device__ __forceinline__ float gelu_tanh(float y) {
-  const float k0 = 0.7978845608028654f;
-  return 0.5f * y * (1.0f + tanhf(k0 * (y + 0.044715f * y * y * y)));
-}
-
 __device__ __forceinline__ uint32_t ld32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
+// kKS k-steps of 16: the branch width is 32 (2) or, with a LoRA adapter
+// concatenated into it, 64 (4); l2t rows are then kKS * 16 wide.
+template <int kKS>
 __global__ void __launch_bounds__(128) upproj_kernel(const __grid_constant__ CUtensorMap tm_y, UpParams p) {
   __shared__ __align__(1024) uint8_t tile[2 * kBoxBytes];
   __shared__ uint64_t full;
@@ -57,16 +56,17 @@ __global__ void __launch_bounds__(128) upproj_kernel(const __grid_constant__ CUt
     dev::mbar_arrive_expect_tx(&full, (uint32_t)(nbox * kBoxBytes));
     for (int b = 0; b < nbox; ++b) dev::tma_load_2d(tile + b * kBoxBytes, &tm_y, &full, n0 + 64 * b, m0);
   }
-  // A fragments of this warp's 16 XL rows (two k-steps of 16)
+  // A fragments of this warp's 16 XL rows (kKS k-steps of 16)
   const int ra = m0 + warp * 16 + g, rb = ra + 8;
-  uint32_t a[2][4];
+  constexpr int kW = kKS * 16;                                // branch width
+  uint32_t a[kKS][4];
 #pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
+  for (int ks = 0; ks < kKS; ++ks) {
     const int k = ks * 16 + 2 * t4;
-    a[ks][0] = ra < p.M ? ld32(p.xl + (size_t)ra * 32 + k) : 0u;
-    a[ks][1] = rb < p.M ? ld32(p.xl + (size_t)rb * 32 + k) : 0u;
-    a[ks][2] = ra < p.M ? ld32(p.xl + (size_t)ra * 32 + k + 8) : 0u;
-    a[ks][3] = rb < p.M ? ld32(p.xl + (size_t)rb * 32 + k + 8) : 0u;
+    a[ks][0] = ra < p.M ? ld32(p.xl + (size_t)ra * p.xl_stride + k) : 0u;
+    a[ks][1] = rb < p.M ? ld32(p.xl + (size_t)rb * p.xl_stride + k) : 0u;
+    a[ks][2] = ra < p.M ? ld32(p.xl + (size_t)ra * p.xl_stride + k + 8) : 0u;
+    a[ks][3] = rb < p.M ? ld32(p.xl + (size_t)rb * p.xl_stride + k + 8) : 0u;
   }
   const bool got = dev::mbar_wait(&full, 0, &abort_flag, p.budget_ns);
   if (!__syncthreads_and(got)) {
@@ -80,9 +80,9 @@ __global__ void __launch_bounds__(128) upproj_kernel(const __grid_constant__ CUt
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     const bool bv = nb + g < p.N;
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      const uint32_t b0 = bv ? ld32(p.l2t + (size_t)(nb + g) * 32 + ks * 16 + 2 * t4) : 0u;
-      const uint32_t b1 = bv ? ld32(p.l2t + (size_t)(nb + g) * 32 + ks * 16 + 2 * t4 + 8) : 0u;
+    for (int ks = 0; ks < kKS; ++ks) {
+      const uint32_t b0 = bv ? ld32(p.l2t + (size_t)(nb + g) * kW + ks * 16 + 2 * t4) : 0u;
+      const uint32_t b1 = bv ? ld32(p.l2t + (size_t)(nb + g) * kW + ks * 16 + 2 * t4 + 8) : 0u;
       asm volatile(
           "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
           "{%0, %1, %2, %3};"
@@ -98,8 +98,8 @@ __global__ void __launch_bounds__(128) upproj_kernel(const __grid_constant__ CUt
       const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(e));
       float y0 = y.x + c[2 * h], y1 = y.y + c[2 * h + 1];
       if (p.gelu) {
-        y0 = gelu_tanh(y0);
-        y1 = gelu_tanh(y1);
+        y0 = dev::gelu_tanh(y0);
+        y1 = dev::gelu_tanh(y1);
       }
       *reinterpret_cast<__nv_bfloat162*>(e) = __floats2bfloat162_rn(y0, y1);
     }
@@ -117,7 +117,12 @@ __global__ void __launch_bounds__(128) upproj_kernel(const __grid_constant__ CUt
 
 cudaError_t launch_upproj(const CUtensorMap& tm_y, const UpParams& p, cudaStream_t stream) {
   dim3 grid((p.N + kTileN - 1) / kTileN, (p.M + kTileM - 1) / kTileM);
-  upproj_kernel<<<grid, 128, 0, stream>>>(tm_y, p);
+  if (p.width == 64)
+    upproj_kernel<4><<<grid, 128, 0, stream>>>(tm_y, p);
+  else if (p.width == 32)
+    upproj_kernel<2><<<grid, 128, 0, stream>>>(tm_y, p);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
