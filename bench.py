@@ -45,6 +45,8 @@ RANK = 32
 NOMINAL_FP4_DENSE_TFLOPS = 9000.0
 N_SETS = 6                   # rotating input sets, 6 x ~70 MB > L2
 FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 PF / 2.25 PF)
+INT8_OVER_BF16 = 2.0         # nominal dense ratio (4.5 POPS / 2.25 PF)
+W8A8_RANK = 16
 
 
 def layer_flops(M, K, N, r=RANK):
@@ -420,10 +422,11 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
 
     def w4a4_layer(d, fmt, X, flags, key, n_sets=2):
         M, K, N = X.shape[0], d["W"].shape[0], d["W"].shape[1]
+        r = W8A8_RANK if fmt == "w8a8" else RANK
         sets = []
         for _ in range(n_sets):
             L = pkg.Layer.prepare(syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]), syn.bf16_bits(d["Xc"]),
-                                  fmt=fmt, rank=RANK, device=dev)
+                                  fmt=fmt, rank=r, device=dev)
             x = X.clone() if isinstance(X, torch.Tensor) else torch.from_numpy(X).to(torch.bfloat16).cuda()
             sets.append((L, x, torch.empty((M, N), dtype=torch.bfloat16, device="cuda"),
                          torch.empty(L.act_code_bytes(M), dtype=torch.uint8, device="cuda"),
@@ -451,14 +454,15 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
         iso = time_events(stream, max(10, n // 4), flush_l2, lambda: k2(0))
         for st in sets:
             st[0].check(stream)
-        k2t = k2_flops(M, K, N) / (k2_ms * 1e-3) / 1e12
-        peak = bf16_peak * (FP4_OVER_BF16 if fmt == "nvfp4" else 1.0)
-        out[key] = {"shape": f"{M}x{K}->{N}", "format": fmt, "us_per_layer": lay * 1e3, "k2_us": k2_ms * 1e3,
-                    "layer_tflops": layer_flops(M, K, N) / (lay * 1e-3) / 1e12, "k2_tflops": k2t,
-                    "k2_frac": k2t / peak, "isolated_k2_us": iso * 1e3, "rotating_sets": n_sets,
-                    "k2_peak": f"{peak:g} TFLOP/s = measured bf16 burst" +
-                               (f" x {FP4_OVER_BF16:g}" if fmt == "nvfp4" else " (FP16 tensor rate, the INT4 "
-                                                                             "GEMM's dequantized operands)")}
+        k2t = k2_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12
+        ratio = {"nvfp4": FP4_OVER_BF16, "w8a8": INT8_OVER_BF16}.get(fmt, 1.0)
+        peak = bf16_peak * ratio
+        note = {"nvfp4": f" x {FP4_OVER_BF16:g}", "w8a8": f" x {INT8_OVER_BF16:g} (INT8 dense rate)"}.get(
+            fmt, " (FP16 tensor rate, the INT4 GEMM's dequantized operands)")
+        out[key] = {"shape": f"{M}x{K}->{N}", "format": fmt, "rank": r, "us_per_layer": lay * 1e3,
+                    "k2_us": k2_ms * 1e3, "layer_tflops": layer_flops(M, K, N, r) / (lay * 1e-3) / 1e12,
+                    "k2_tflops": k2t, "k2_frac": k2t / peak, "isolated_k2_us": iso * 1e3, "rotating_sets": n_sets,
+                    "k2_peak": f"{peak:g} TFLOP/s = measured bf16 burst" + note}
         y0 = sets[0][2]
         for st in sets:
             st[0].close()
@@ -467,6 +471,9 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
     # INT4 variant
     d = syn.layer("qkv_int4")
     w4a4_layer(d, "int4", d["X"], 0, "int4_qkv")
+    # W8A8 variant (rank 16 at 8 bits) on the attention-output shape
+    d = syn.layer("attn_out")
+    w4a4_layer(d, "w8a8", d["X"], 0, "w8a8_attn_out")
     # MLP pair: fc1 (GELU), then fc2 on fc1's output; fc2 calibrates on fc1's output for its calibration batch
     d1 = syn.layer("mlp", "fc1")
     h = w4a4_layer(d1, "nvfp4", d1["X"], pkg.FWD_GELU, "fc1_gelu")

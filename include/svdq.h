@@ -59,10 +59,14 @@ typedef enum {
 typedef enum {
   SVDQ_NVFP4 = 0,           /* W4A4, E2M1 g16, E4M3 scales, FP32 tensor scales     */
   SVDQ_INT4 = 1,            /* W4A4, symmetric INT4 g64, BF16 scales               */
-  SVDQ_W4A16_INT4 = 2       /* weight-only INT4 g64 (adaptive-norm linears)        */
+  SVDQ_W4A16_INT4 = 2,      /* weight-only INT4 g64 (adaptive-norm linears)        */
+  SVDQ_W8A8_INT8 = 3        /* W8A8: INT8, one FP32 scale per token / output channel,
+                               low-rank branch of rank 16                           */
 } svdq_format;
 
-/* Offline configuration.  rank: 32 (or 0 = no low-rank branch); alpha:
+/* Offline configuration.  rank: 32 for the 4-bit formats, 16 for SVDQ_W8A8_INT8
+ * (SOTA-314 practice page, "Do this": rank 32 at 4 bits, 16 at 8 bits), or 0
+ * = no low-rank branch; alpha:
  * smoothing migration strength (0.5).  flags: SVDQ_PREP_* bits (0 = the
  * round-to-nearest residual). */
 typedef struct {
@@ -130,7 +134,8 @@ typedef enum {
   SVDQ_T_RESIDUAL = 6,      /* float [K][N]    R = fp32(W_hat - diag(lam) L1d L2b)  */
   SVDQ_T_SIGMA = 7,         /* double [r]      leading singular values of W_hat     */
   SVDQ_T_W_CODES = 8,       /* uint8 [N][K/2]  residual codes, K-major, even k low  */
-  SVDQ_T_W_SCALES = 9,      /* NVFP4: uint8 [N][K/16] E4M3; INT4: uint16 [N][K/64] BF16 */
+  SVDQ_T_W_SCALES = 9,      /* NVFP4: uint8 [N][K/16] E4M3; INT4: uint16 [N][K/64] BF16;
+                               W8A8: float [N] (W_CODES is then int8 [N][K])         */
   SVDQ_T_BIAS = 10,         /* float [N]                                            */
   SVDQ_T_GPTQ_U = 11,       /* double [K][K]   GPTQ factor U (upper, H^-1 = U^T U); only
                                with SVDQ_PREP_GPTQ | SVDQ_PREP_KEEP_GPTQ_FACTOR      */
@@ -223,6 +228,10 @@ size_t svdq_workspace_bytes(const svdq_layer* layer, int M);
  *   Y          device, [M][N] BF16 row-major, 16-byte aligned; fully overwritten.
  *   workspace  device, >= svdq_workspace_bytes(layer, M), 256-byte aligned.
  *   flags      SVDQ_FWD_* bits.
+ * SVDQ_W8A8_INT8 enqueues three: a per-token scale pass over X (the largest
+ * smoothed magnitude of each row), the first kernel (INT8 codes, rank-16 down
+ * projection) and an INT8 tensor-core GEMM (exact int32 products, both scales
+ * and the branch applied in the epilogue).
  * W4A4 formats enqueue two kernels: the fused down-projection + quantize pass
  * over X ("Down Projection with Quantize, because they read the same input")
  * and the block-scaled tensor-core GEMM whose epilogue adds the up-projection
@@ -245,13 +254,14 @@ svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, v
                                 void* workspace, size_t workspace_bytes,
                                 void* stream, unsigned flags);
 
-/* The first kernel alone (NVFP4/INT4): writes the activation codes (device,
+/* The first kernel alone (NVFP4/INT4/W8A8): writes the activation codes (device,
  * svdq_act_code_bytes(layer, M) bytes, two codes per byte with the even k in
  * the low nibble; INT4 codes are 4-bit two's complement, row-major [M][K/2];
  * NVFP4 codes are in the GEMM's tiled layout, see svdq_act_codes_to_logical),
  * the activation scales (device, svdq_act_scale_bytes(layer, M)
  * bytes: NVFP4 E4M3 in the tensor-core layout, INT4 BF16 [K/64][M rounded up
- * to 128], group-major, padding rows zero) and, when
+ * to 128], group-major, W8A8 FP32 [s_x | 1/s_x], each M rounded up to 128
+ * entries; padding rows zero) and, when
  * the layer has a branch, XL = bf16(X L1d) (device [M][rank] BF16; [M][64]
  * with a LoRA adapter, see svdq_set_lora).  xl may be NULL for rank 0 without
  * an adapter.  `mode` 0 = fused, 1 = quantize only, 2 = down projection only. */
@@ -265,7 +275,8 @@ svdq_status svdq_gemm(const svdq_layer* layer, const void* codes, const void* sc
                       const void* xl, int M, void* Y, void* stream, unsigned flags);
 
 /* Bytes of the activation codes for M tokens in the layout the GEMM reads:
- * INT4 M * K/2; NVFP4 ceil(M/128)*128 * ceil(K/256) * 128 (tiled). */
+ * INT4 M * K/2; NVFP4 ceil(M/128)*128 * ceil(K/256) * 128 (tiled); W8A8
+ * ceil(M/128)*128 * ceil(K/128) * 128 (tiled, one byte per code). */
 size_t svdq_act_code_bytes(const svdq_layer* layer, int M);
 
 /* Host-side: convert a host copy of activation codes in the GEMM's layout
@@ -274,7 +285,8 @@ size_t svdq_act_code_bytes(const svdq_layer* layer, int M);
  * (128 bytes of a row), one contiguous 16 KiB block in which byte j of row r
  * sits at (r % 128) * 128 + (((j / 16) ^ (r % 8)) * 16) + j % 16: the order in
  * which the tensor core reads a 128-byte-swizzled operand tile, so the GEMM
- * fetches each stage with one contiguous copy. */
+ * fetches each stage with one contiguous copy.  W8A8 uses the same blocks for
+ * stages of 128 one-byte codes and converts to int8 [M][K]. */
 svdq_status svdq_act_codes_to_logical(const svdq_layer* layer, const void* device_layout,
                                       int M, void* logical);
 
@@ -283,7 +295,7 @@ size_t svdq_act_scale_bytes(const svdq_layer* layer, int M);
 
 /* Host-side: convert a host copy of activation scales in the GEMM's layout
  * (svdq_act_scale_bytes bytes) into the logical layout: NVFP4 uint8 [M][K/16],
- * INT4 uint16 [M][K/64] (BF16 bits). */
+ * INT4 uint16 [M][K/64] (BF16 bits), W8A8 float [M] (s_x). */
 svdq_status svdq_act_scales_to_logical(const svdq_layer* layer, const void* device_layout,
                                        int M, void* logical);
 

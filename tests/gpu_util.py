@@ -34,7 +34,7 @@ def oracle_prep_from(L, gptq_U=None) -> dict:
     (residual quantized by GPTQ with factor ``gptq_U`` when one is given)."""
     info = L.info
     r = info["rank"]
-    fmt = "int4" if info["format"] == lib.INT4 else "nvfp4"
+    fmt = {lib.INT4: "int4", lib.W8A8_INT8: "w8a8"}.get(info["format"], "nvfp4")
     p = {"fmt": fmt, "rank": r, "K": info["K"], "N": info["N"],
          "lam": L.export("lambda"), "inv_lam": L.export("inv_lambda"),
          "L1d": syn.from_bf16_bits(L.export("L1d")).astype(np.float64) if r else np.zeros((info["K"], 0)),

@@ -23,8 +23,8 @@ LIB_PATH = os.path.join(_HERE, "libsvdq.so")
 # status codes (svdq_status)
 OK, EINVAL, EUNSUPPORTED, ENOMEM, ECUDA, ENOCONVERGE, ETIMEOUT, ESTATE = range(8)
 # formats (svdq_format)
-NVFP4, INT4, W4A16_INT4 = 0, 1, 2
-FORMATS = {"nvfp4": NVFP4, "int4": INT4, "w4a16": W4A16_INT4}
+NVFP4, INT4, W4A16_INT4, W8A8_INT8 = 0, 1, 2, 3
+FORMATS = {"nvfp4": NVFP4, "int4": INT4, "w4a16": W4A16_INT4, "w8a8": W8A8_INT8}
 # forward flags
 FWD_GELU, FWD_UNFUSED, FWD_NO_BRANCH, FWD_CHECK = 0x1, 0x2, 0x4, 0x8
 # exportable tensors (svdq_tensor)
@@ -185,13 +185,14 @@ class Layer:
         info = self.info
         K, N, r = info["K"], info["N"], info["rank"]
         if dt is None:
-            dt = np.uint8 if info["format"] == NVFP4 else np.uint16
+            dt = {NVFP4: np.uint8, W8A8_INT8: np.float32}.get(info["format"], np.uint16)
         nbytes = load().svdq_tensor_bytes(self._h, tid)
         buf = np.empty(nbytes // np.dtype(dt).itemsize, dtype=dt)
         _check(load().svdq_export(self._h, tid, _ptr(buf), nbytes), f"svdq_export({name})")
+        w8 = info["format"] == W8A8_INT8
         shapes = {"lambda": (K,), "inv_lambda": (K,), "L1": (K, r), "L2": (r, N), "L1d": (K, r),
-                  "L2b": (r, N), "R": (K, N), "sigma": (r,), "w_codes": (N, K // 2), "bias": (N,),
-                  "w_scales": (N, -1), "gptq_U": (K, K), "lora_A": (K, -1), "lora_B": (-1, N)}
+                  "L2b": (r, N), "R": (K, N), "sigma": (r,), "w_codes": (N, K if w8 else K // 2), "bias": (N,),
+                  "w_scales": (N,) if w8 else (N, -1), "gptq_U": (K, K), "lora_A": (K, -1), "lora_B": (-1, N)}
         return buf.reshape(shapes[name])
 
     def set_lora(self, A_bits: Optional[np.ndarray], B_bits: Optional[np.ndarray], scale: float = 1.0):
@@ -217,8 +218,13 @@ class Layer:
         return int(load().svdq_act_code_bytes(self._h, M))
 
     def act_codes_to_logical(self, device_layout: np.ndarray, M: int) -> np.ndarray:
-        """Activation codes in the GEMM's layout -> uint8 [M][K/2] (two codes per byte)."""
-        out = np.empty((M, self.info["K"] // 2), dtype=np.uint8)
+        """Activation codes in the GEMM's layout -> uint8 [M][K/2] (two codes per
+        byte); W8A8: int8 [M][K]."""
+        info = self.info
+        if info["format"] == W8A8_INT8:
+            out = np.empty((M, info["K"]), dtype=np.int8)
+        else:
+            out = np.empty((M, info["K"] // 2), dtype=np.uint8)
         src = np.ascontiguousarray(device_layout, dtype=np.uint8)
         _check(load().svdq_act_codes_to_logical(self._h, _ptr(src), M, _ptr(out)), "svdq_act_codes_to_logical")
         return out
@@ -242,10 +248,13 @@ class Layer:
                                 flags), "svdq_gemm")
 
     def act_scales_to_logical(self, device_layout: np.ndarray, M: int) -> np.ndarray:
-        """NVFP4: uint8 [M][K/16] E4M3 bytes; INT4: uint16 [M][K/64] BF16 bits."""
+        """NVFP4: uint8 [M][K/16] E4M3 bytes; INT4: uint16 [M][K/64] BF16 bits;
+        W8A8: float32 [M] (one scale per token)."""
         info = self.info
         if info["format"] == INT4:
             out = np.empty((M, info["K"] // 64), dtype=np.uint16)
+        elif info["format"] == W8A8_INT8:
+            out = np.empty((M,), dtype=np.float32)
         else:
             out = np.empty((M, info["K"] // 16), dtype=np.uint8)
         src = np.ascontiguousarray(device_layout, dtype=np.uint8)

@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsvdq.so")
 
-CUDA_SOURCES = ["api.cu", "k1_quant.cu", "k2_gemm.cu", "k2_pair.cu", "k2_int4.cu", "k2_int4_pair.cu", "upproj.cu", "static_ws.cu", "w4a16.cu", "selftest.cu", "chain.cu"]
+CUDA_SOURCES = ["api.cu", "k1_quant.cu", "k2_gemm.cu", "k2_pair.cu", "k2_int4.cu", "k2_int4_pair.cu", "upproj.cu", "static_ws.cu", "w4a16.cu", "selftest.cu", "chain.cu", "k2_int8.cu"]
 CXX_SOURCES = ["prepare.cpp"]
 HEADERS = [os.path.join(CSRC, h) for h in ("sm100.cuh", "kernels.h", "svdq_internal.h", "nvfp4_quant.cuh")] + [
     os.path.join(INCLUDE, "svdq.h")]

@@ -128,7 +128,12 @@ struct DeviceGuard {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 
-bool w4a4(const svdq_layer* L) { return L->host.format == SVDQ_NVFP4 || L->host.format == SVDQ_INT4; }
+// Formats with quantized activations (the two-kernel forward): NVFP4, INT4, W8A8.
+bool w4a4(const svdq_layer* L) {
+  return L->host.format == SVDQ_NVFP4 || L->host.format == SVDQ_INT4 || L->host.format == SVDQ_W8A8_INT8;
+}
+bool w8a8(const HostPrep& h) { return h.format == SVDQ_W8A8_INT8; }
+int int8_stages(int K) { return (K + 127) / 128; }   // K stages of 128 int8 codes (128-byte rows)
 
 int pad_rows(int M) { return (M + 127) / 128 * 128; }
 int nvfp4_stages(int K) { return (K + 255) / 256; }   // K stages of 256 codes (128-byte rows)
@@ -137,6 +142,7 @@ int nvfp4_stages(int K) { return (K + 255) / 256; }   // K stages of 256 codes (
 // INT4 row-major [M][K/2].
 size_t act_code_bytes(const HostPrep& h, int M) {
   if (h.format == SVDQ_NVFP4) return (size_t)pad_rows(M) * (size_t)nvfp4_stages(h.K) * 128u;
+  if (h.format == SVDQ_W8A8_INT8) return (size_t)pad_rows(M) * (size_t)int8_stages(h.K) * 128u;
   return (size_t)M * (size_t)(h.K / 2);
 }
 
@@ -147,6 +153,7 @@ int pad_cols_int4(int N) { return (N + 255) / 256 * 256; }
 size_t act_scale_bytes(const HostPrep& h, int M) {
   if (h.format == SVDQ_NVFP4) return (size_t)((M + 127) / 128) * (size_t)(h.K / 64) * 512;
   if (h.format == SVDQ_INT4) return (size_t)(h.K / 64) * (size_t)pad_rows(M) * 2;   // BF16 [K/64][mpad]
+  if (h.format == SVDQ_W8A8_INT8) return (size_t)pad_rows(M) * 8;                   // s_x [mpad], 1/s_x [mpad]
   return 0;
 }
 
@@ -226,10 +233,20 @@ svdq_status upload_layer(svdq_layer* L, int device) {
   chk(cudaMalloc(reinterpret_cast<void**>(&L->d_err), sizeof(int)));
   if (e == cudaSuccess) chk(cudaMemset(L->d_err, 0, sizeof(int)));
   chk(upload(&L->d_bias, h.bias.data(), sizeof(float) * N));
-  if (h.format == SVDQ_NVFP4 || h.format == SVDQ_INT4) {
+  if (h.format == SVDQ_NVFP4 || h.format == SVDQ_INT4 || h.format == SVDQ_W8A8_INT8) {
     chk(upload(&L->d_inv_lam, h.inv_lam.data(), sizeof(float) * K));
     std::vector<uint8_t> tiled;
-    if (h.format == SVDQ_NVFP4) {
+    if (h.format == SVDQ_W8A8_INT8) {
+      // int8 weight codes in (256-row, 128-column) blocks of the GEMM's tiled
+      // layout (wgt_tile_offset over 128-byte rows), rows padded with zeros
+      const int nst8 = (K + 127) / 128;
+      tiled.assign(k2_int8_weight_bytes(N, K), 0);
+      for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k)
+          tiled[wgt_tile_offset(n, k >> 7, (k & 127) >> 4, nst8) + (k & 15)] = h.w_codes[(size_t)n * K + k];
+      chk(upload(&L->d_wq, tiled.data(), tiled.size()));
+      chk(upload(&L->d_ws, h.w_scales_f32.data(), sizeof(float) * N));
+    } else if (h.format == SVDQ_NVFP4) {
       // weight codes in the GEMM's tiled layout (wgt_tile_offset), rows padded to 256 with zeros
       const int nst = nvfp4_stages(K);
       tiled.assign((size_t)((N + 255) / 256) * (size_t)nst * 32768u, 0);
@@ -239,8 +256,12 @@ svdq_status upload_layer(svdq_layer* L, int device) {
     } else {
       chk(upload(&L->d_wq, h.w_codes.data(), h.w_codes.size()));
     }
-    int alpha_exp = h.g_x_exp + h.g_w_exp;
-    if (h.format == SVDQ_NVFP4) {
+    // the branch's up factor is divided by the GEMM's accumulator unit alpha
+    // (NVFP4: g_x g_w; INT4: 2^(ex + ew)); W8A8 keeps a branch accumulator of its own
+    int alpha_exp = h.format == SVDQ_W8A8_INT8 ? 0 : h.g_x_exp + h.g_w_exp;
+    if (h.format == SVDQ_W8A8_INT8) {
+      // nothing more: codes and scales are uploaded above
+    } else if (h.format == SVDQ_NVFP4) {
       // weight scales in the tensor-core layout, rows padded to a multiple of 256
       const int npad = (N + 255) / 256 * 256;
       std::vector<uint8_t> ws((size_t)(npad / 128) * (K / 64) * 512, 0);
@@ -329,6 +350,7 @@ K1Params k1_params(const svdq_layer* L, int M, void* codes, void* scales, void* 
     p.rcp[8 + m] = m ? (float)(1.0 / m) : 0.0f;
   }
   p.inv_lam = L->d_inv_lam;
+  p.inv_sx = nullptr;
   p.codes = static_cast<uint8_t*>(codes);
   p.scales = static_cast<uint8_t*>(scales);
   p.xl = static_cast<__nv_bfloat16*>(xl);
@@ -348,14 +370,53 @@ svdq_status run_k1(const svdq_layer* L, const void* X, int M, void* codes, void*
   // 16 bytes wide for NVFP4 (32 columns), 32 bytes for INT4 (64 columns)
   // NVFP4 codes are written tiled from registers; INT4 codes in 32-row x 32-byte
   // tiles by TMA (one per quantizer warp and stage)
-  const bool nv = h.format == SVDQ_NVFP4;
-  if (mode != 2 && !nv &&
+  const bool nv = h.format == SVDQ_NVFP4, i8 = w8a8(h);
+  if (mode != 2 && !nv && !i8 &&
       !make_map(&tm_c, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.K / 2, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SVDQ_ECUDA;
-  if (mode == 2 || nv) tm_c = tm_x;   // unused
+  if (mode == 2 || nv || i8) tm_c = tm_x;   // unused
   K1Params p = k1_params(L, M, codes, scales, xl);
-  return launch_k1(tm_x, L->tm_l1t, tm_c, p, nv ? kFmtNvfp4 : kFmtInt4, mode, stream) == cudaSuccess ? SVDQ_OK
-                                                                                                    : SVDQ_ECUDA;
+  if (i8 && mode != 2) {
+    // W8A8: the per-token scales first ([s_x | 1/s_x] in the scales buffer)
+    const int mpad = pad_rows(M);
+    float* sx = static_cast<float*>(scales);
+    if (launch_rowscale(static_cast<const __nv_bfloat16*>(X), L->d_inv_lam, M, h.K, mpad, sx, sx + mpad, stream) !=
+        cudaSuccess)
+      return SVDQ_ECUDA;
+    p.inv_sx = sx + mpad;
+  }
+  const int fmt = nv ? kFmtNvfp4 : i8 ? kFmtInt8 : kFmtInt4;
+  return launch_k1(tm_x, L->tm_l1t, tm_c, p, fmt, mode, stream) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+}
+
+svdq_status run_k2_int8(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
+                        cudaStream_t stream, bool branch, bool gelu) {
+  const HostPrep& h = L->host;
+  CUtensorMap tm_xl, tm_y;
+  if (!make_map(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.N, M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return SVDQ_ECUDA;
+  if (branch) {
+    if (!make_map_strided(&tm_xl, xl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, M, (uint64_t)xl_width(h) * 2, 32, 128,
+                          CU_TENSOR_MAP_SWIZZLE_64B))
+      return SVDQ_ECUDA;
+  } else {
+    tm_xl = tm_y;   // unused by the kernel
+  }
+  K2Int8Params p;
+  p.M = M;
+  p.N = h.N;
+  p.K = h.K;
+  p.acodes = static_cast<const uint8_t*>(codes);
+  p.wq = L->d_wq;
+  p.sx = static_cast<const float*>(scales);
+  p.sw = reinterpret_cast<const float*>(L->d_ws);
+  p.bias = L->d_bias;
+  p.y = static_cast<__nv_bfloat16*>(Y);
+  p.err = L->d_err;
+  p.budget_ns = L->budget_ns;
+  p.branch = branch ? 1 : 0;
+  p.gelu = gelu ? 1 : 0;
+  return launch_k2_int8(tm_xl, L->tm_l2s, tm_y, p, L->num_sms, stream) == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
 
 // The LoRA adapter's down pass: XL columns 32..63 = bf16(X A), the first
@@ -444,6 +505,7 @@ svdq_status run_k2_int4(const svdq_layer* L, const void* codes, const void* scal
 svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
                    cudaStream_t stream, bool branch, bool gelu, bool lora_on = true) {
   if (L->host.format == SVDQ_INT4) return run_k2_int4(L, codes, scales, xl, M, Y, stream, branch, gelu, lora_on);
+  if (w8a8(L->host)) return run_k2_int8(L, codes, scales, xl, M, Y, stream, branch, gelu);
   const HostPrep& h = L->host;
   const bool lora = h.lora_r > 0 && lora_on;
   CUtensorMap tm_xl, tm_y, tm_xla;
@@ -612,7 +674,7 @@ svdq_status svdq_prepare(const svdq_config* cfg, int K, int N, const uint16_t* W
   if (!out) return SVDQ_EINVAL;
   *out = nullptr;
   if (!cfg || !W_bf16 || K <= 0 || N <= 0) return SVDQ_EINVAL;
-  if (cfg->format < SVDQ_NVFP4 || cfg->format > SVDQ_W4A16_INT4) return SVDQ_EINVAL;
+  if (cfg->format < SVDQ_NVFP4 || cfg->format > SVDQ_W8A8_INT8) return SVDQ_EINVAL;
   const bool wo = cfg->format == SVDQ_W4A16_INT4;
   if (cfg->flags & ~(SVDQ_PREP_GPTQ | SVDQ_PREP_KEEP_GPTQ_FACTOR)) return SVDQ_EINVAL;
   if ((cfg->flags & SVDQ_PREP_KEEP_GPTQ_FACTOR) && !(cfg->flags & SVDQ_PREP_GPTQ)) return SVDQ_EINVAL;
@@ -620,7 +682,10 @@ svdq_status svdq_prepare(const svdq_config* cfg, int K, int N, const uint16_t* W
   if (!wo) {
     if (!calib_bf16 || M_calib < 1) return SVDQ_EINVAL;
     if (!(cfg->alpha > 0.0f && cfg->alpha < 1.0f)) return SVDQ_EINVAL;
-    if (cfg->rank != 0 && cfg->rank != 32) return SVDQ_EUNSUPPORTED;
+    // rank 32 at 4 bits, 16 at 8 bits (or no branch)
+    const int want = cfg->format == SVDQ_W8A8_INT8 ? 16 : 32;
+    if (cfg->rank != 0 && cfg->rank != want) return SVDQ_EUNSUPPORTED;
+    if (cfg->format == SVDQ_W8A8_INT8 && (cfg->flags & SVDQ_PREP_GPTQ)) return SVDQ_EUNSUPPORTED;
   }
   // W4A4 needs N % 16 for its TMA tiles; the weight-only GEMV takes any N
   if (K % 64 != 0 || (!wo && N % 16 != 0)) return SVDQ_EUNSUPPORTED;
@@ -678,7 +743,10 @@ size_t svdq_tensor_bytes(const svdq_layer* L, int id) {
     case SVDQ_T_RESIDUAL: return h.R.size() * 4;
     case SVDQ_T_SIGMA: return h.sigma.size() * 8;
     case SVDQ_T_W_CODES: return h.w_codes.size();
-    case SVDQ_T_W_SCALES: return h.format == SVDQ_NVFP4 ? h.w_scales_e4m3.size() : h.w_scales_bf16.size() * 2;
+    case SVDQ_T_W_SCALES:
+      return h.format == SVDQ_NVFP4 ? h.w_scales_e4m3.size()
+             : w8a8(h)              ? h.w_scales_f32.size() * 4
+                                    : h.w_scales_bf16.size() * 2;
     case SVDQ_T_BIAS: return h.bias.size() * 4;
     case SVDQ_T_GPTQ_U: return h.gptq_U.size() * 8;
     case SVDQ_T_LORA_A: return h.lora_A.size() * 2;
@@ -704,7 +772,9 @@ svdq_status svdq_export(const svdq_layer* L, int id, void* dst, size_t bytes) {
     case SVDQ_T_SIGMA: src = h.sigma.data(); break;
     case SVDQ_T_W_CODES: src = h.w_codes.data(); break;
     case SVDQ_T_W_SCALES:
-      src = h.format == SVDQ_NVFP4 ? (const void*)h.w_scales_e4m3.data() : (const void*)h.w_scales_bf16.data();
+      src = h.format == SVDQ_NVFP4 ? (const void*)h.w_scales_e4m3.data()
+            : w8a8(h)              ? (const void*)h.w_scales_f32.data()
+                                   : (const void*)h.w_scales_bf16.data();
       break;
     case SVDQ_T_BIAS: src = h.bias.data(); break;
     case SVDQ_T_GPTQ_U: src = h.gptq_U.data(); break;
@@ -738,6 +808,13 @@ svdq_status svdq_act_codes_to_logical(const svdq_layer* L, const void* device_la
   if (!w4a4(L)) return SVDQ_EUNSUPPORTED;
   const uint8_t* src = static_cast<const uint8_t*>(device_layout);
   uint8_t* dst = static_cast<uint8_t*>(logical);
+  if (w8a8(h)) {
+    const int nst8 = int8_stages(h.K);
+    for (int r = 0; r < M; ++r)
+      for (int k = 0; k < h.K; ++k)
+        dst[(size_t)r * h.K + k] = src[act_tile_offset(r, k >> 7, (k & 127) >> 4, nst8) + (k & 15)];
+    return SVDQ_OK;
+  }
   const size_t row = (size_t)(h.K / 2);
   if (h.format == SVDQ_INT4) {
     std::memcpy(dst, src, (size_t)M * row);
@@ -759,6 +836,10 @@ svdq_status svdq_act_scales_to_logical(const svdq_layer* L, const void* device_l
     const int G = h.K / 64, mpad = pad_rows(M);
     for (int r = 0; r < M; ++r)
       for (int gi = 0; gi < G; ++gi) dst[(size_t)r * G + gi] = src[(size_t)gi * mpad + r];
+    return SVDQ_OK;
+  }
+  if (w8a8(h)) {
+    std::memcpy(logical, device_layout, (size_t)M * sizeof(float));   // s_x, one per token
     return SVDQ_OK;
   }
   if (h.format != SVDQ_NVFP4) return SVDQ_EUNSUPPORTED;
@@ -869,7 +950,7 @@ svdq_status svdq_linear_forward(const svdq_layer* L, const void* X, int M, void*
 
 svdq_status svdq_set_lora(svdq_layer* L, int r, const uint16_t* A_bf16, const uint16_t* B_bf16, float scale) {
   if (!L) return SVDQ_EINVAL;
-  if (L->host.format == SVDQ_W4A16_INT4) return SVDQ_EUNSUPPORTED;
+  if (L->host.format == SVDQ_W4A16_INT4 || L->host.format == SVDQ_W8A8_INT8) return SVDQ_EUNSUPPORTED;
   if (r < 0) return SVDQ_EINVAL;
   if (r > 32) return SVDQ_EUNSUPPORTED;
   if (r > 0 && (!A_bf16 || !B_bf16 || !std::isfinite(scale))) return SVDQ_EINVAL;

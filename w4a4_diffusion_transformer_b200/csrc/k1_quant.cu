@@ -75,7 +75,7 @@ constexpr int kCodeBytes = 8 * 1024;                       // code staging tiles
 // groups of 16), INT4 warps own 64 columns (one group of 64).
 template <int F>
 struct K1Shape {
-  static constexpr int quant_warps = F == kFmtNvfp4 ? 8 : 4;
+  static constexpr int quant_warps = F == kFmtInt4 ? 4 : 8;
   static constexpr int cols = kBK / quant_warps;                     // columns per quantizer warp
   static constexpr int code_tile = kRows * cols / 2;                 // its codes: 32 rows x cols/2 B
   static constexpr int consumer_warps = quant_warps + kMmaWarps;
@@ -307,6 +307,70 @@ __global__ void __launch_bounds__(K1Shape<kFmt>::threads, 1)
     if (lane == 0) dev::bulk_wait_group_all();
     return;
   }
+  if (quant_warp && kFmt == kFmtInt8) {
+    // ---------------------------------------------------------- INT8 quantizer
+    // Warp w owns columns 32w..32w+31 of each 256-column stage, lane l row l;
+    // code = clamp(rint_even(fp32(v * inv_sx)), -127, 127) with v = fp32(x *
+    // inv_lam) and the row's 1/s_x from the per-token scale pass.  The 32
+    // codes go to the GEMM's tiled layout in 128-column stages: stage 2 it +
+    // w / 4, 16-byte chunks 2 (w % 4) and 2 (w % 4) + 1.
+    const int grow = row0 + lane;                     // < mpad
+    const int nst8 = (K + 127) / 128;
+    float invs = 0.f;
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % kXStages;
+      if (!dev::mbar_wait(&xfull[s], (uint32_t)(it / kXStages) & 1u, abort_flag, p.budget_ns)) {
+        record_error(p.err, abort_flag, 0x105);
+        break;
+      }
+      // the per-token scales come from the preceding kernel: read them only
+      // after the first X stage, which the X producer loads after waiting for it
+      if (it == 0) invs = p.inv_sx[grow];             // zero for padding rows: zero codes
+      const uint8_t* st = smem + s * kXStageBytes;
+      const int k0 = it * kBK;
+      const int kvalid = min(kBK, K - k0);
+      const int col0 = warp * 32;
+      const bool active = col0 < kvalid;              // kvalid is a multiple of 64
+      uint32_t w8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      if (active) {
+        const uint8_t* xt = st + (col0 >> 6) * 4096;
+        const int c0 = (col0 & 63) >> 3;
+        const float4* inv4 = reinterpret_cast<const float4*>(st + kXBytes) + (col0 >> 2);
+        const float2 is2 = make_float2(invs, invs);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(xt + sw128(lane, c0 + i));
+          const float4 ia = inv4[2 * i], ib = inv4[2 * i + 1];
+          const float2 iv[4] = {make_float2(ia.x, ia.y), make_float2(ia.z, ia.w), make_float2(ib.x, ib.y),
+                                make_float2(ib.z, ib.w)};
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            // four codes (columns 8i + 2e .. +3) into one 32-bit word
+            const float2 v0 = __fmul2_rn(
+                make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)), iv[e]);
+            const float2 v1 = __fmul2_rn(
+                make_float2(__uint_as_float(w[e + 1] << 16), __uint_as_float(w[e + 1] & 0xFFFF0000u)), iv[e + 1]);
+            const float2 q0 = __fmul2_rn(v0, is2), q1 = __fmul2_rn(v1, is2);
+            const int c[4] = {max(-127, min(127, __float2int_rn(q0.x))), max(-127, min(127, __float2int_rn(q0.y))),
+                              max(-127, min(127, __float2int_rn(q1.x))), max(-127, min(127, __float2int_rn(q1.y)))};
+            w8[2 * i + (e >> 1)] = (uint32_t)(c[0] & 0xFF) | ((uint32_t)(c[1] & 0xFF) << 8) |
+                                   ((uint32_t)(c[2] & 0xFF) << 16) | ((uint32_t)(c[3] & 0xFF) << 24);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&xempty[s]);
+      if (active) {
+        const int t8 = 2 * it + (warp >> 2);
+        const int ch = (warp & 3) * 2;
+        *reinterpret_cast<uint4*>(p.codes + act_tile_offset(grow, t8, ch, nst8)) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        *reinterpret_cast<uint4*>(p.codes + act_tile_offset(grow, t8, ch + 1, nst8)) =
+            make_uint4(w8[4], w8[5], w8[6], w8[7]);
+      }
+    }
+    return;
+  }
   if (quant_warp) {
     // ---------------------------------------------------------- NVFP4 quantizer
     const int grow = row0 + lane;                     // this lane's row (may be >= M: zero padding)
@@ -481,8 +545,69 @@ cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CU
   } else if (fmt == kFmtInt4) {
     if (mode == 0) return launch_k1_t<kFmtInt4, true, true>(tm_x, tm_l, tm_c, p, stream);
     if (mode == 1) return launch_k1_t<kFmtInt4, true, false>(tm_x, tm_l, tm_c, p, stream);
+  } else if (fmt == kFmtInt8) {
+    if (mode == 0) return launch_k1_t<kFmtInt8, true, true>(tm_x, tm_l, tm_c, p, stream);
+    if (mode == 1) return launch_k1_t<kFmtInt8, true, false>(tm_x, tm_l, tm_c, p, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+namespace {
+
+// One warp per row: the row's largest |fp32(x * inv_lam)| (the same IEEE
+// products the quantizer forms), then s = fp32(a fp32(1/127)) and the
+// correctly rounded reciprocal.
+__global__ void __launch_bounds__(256) rowscale_kernel(const __nv_bfloat16* __restrict__ x,
+                                                       const float* __restrict__ inv_lam, int M, int K, int mpad,
+                                                       float* __restrict__ sx, float* __restrict__ inv_sx) {
+  // X may be the preceding kernel's output
+  dev::griddep_wait();
+  dev::griddep_launch_dependents();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= mpad) return;
+  float a = 0.f;
+  if (row < M) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * K);
+    const float4* il = reinterpret_cast<const float4*>(inv_lam);
+    for (int c = lane; c < K / 8; c += 32) {        // 8 columns per 16-byte chunk
+      const uint4 raw = xr[c];
+      const float4 i0 = il[2 * c], i1 = il[2 * c + 1];
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      const float2 iv[4] = {make_float2(i0.x, i0.y), make_float2(i0.z, i0.w), make_float2(i1.x, i1.y),
+                            make_float2(i1.z, i1.w)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 v = __fmul2_rn(make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)),
+                                    iv[e]);
+        a = dev::fmax3(a, fabsf(v.x), fabsf(v.y));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  }
+  if (lane == 0) {
+    const float s = __fmul_rn(a, 1.0f / 127.0f);
+    sx[row] = s;
+    inv_sx[row] = s == 0.f ? 0.f : __frcp_rn(s);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rowscale(const __nv_bfloat16* x, const float* inv_lam, int M, int K, int mpad, float* sx,
+                            float* inv_sx, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((mpad + 7) / 8);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, rowscale_kernel, x, inv_lam, M, K, mpad, sx, inv_sx);
 }
 
 }  // namespace svdq

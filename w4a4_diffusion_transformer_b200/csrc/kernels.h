@@ -13,6 +13,7 @@ namespace svdq {
 // Activation/weight formats of the W4A4 kernels.
 constexpr int kFmtNvfp4 = 0;
 constexpr int kFmtInt4 = 1;
+constexpr int kFmtInt8 = 2;    // W8A8: one scale per token
 
 struct K1Params {
   int M, K;
@@ -22,7 +23,9 @@ struct K1Params {
   int g_x_exp;                  // activation tensor scale g_x = 2^g_x_exp
   float rcp[16];                // fp32(1/(1 + m/8)) for m = 0..7, then fp32(1/m) (index 8 + m)
   const float* inv_lam;         // [K]
-  uint8_t* codes;               // NVFP4: tiled layout (act_tile_offset); INT4: [M][K/2]
+  const float* inv_sx;          // INT8: per-token 1/s_x [mpad] (zero for padding rows)
+  uint8_t* codes;               // NVFP4: tiled layout (act_tile_offset); INT4: [M][K/2];
+                                // INT8: tiled in 128-column stages (act_tile_offset, nst = ceil(K/128))
   uint8_t* scales;              // NVFP4: tensor-core scale layout, mpad rows; INT4: BF16 [K/64][mpad]
   __nv_bfloat16* xl;            // [M][32] with row stride xl_stride elements
   int xl_stride;                // 32, or 64 when a LoRA adapter's XL_lora shares the rows
@@ -85,6 +88,20 @@ struct K2Int4Params {
   int lora;                     // 1: add XL_lora (s B / alpha) too (tm_xla, tm_l2a), same accumulator
 };
 
+struct K2Int8Params {
+  int M, N, K;
+  const uint8_t* acodes;        // int8 activation codes, tiled in 128-column stages (act_tile_offset), mpad rows
+  const uint8_t* wq;            // int8 weight codes, tiled in (256-row, 128-column) blocks (wgt_tile_offset)
+  const float* sx;              // per-token scales [mpad]
+  const float* sw;              // per-output-channel scales [N]
+  const float* bias;            // [N]
+  __nv_bfloat16* y;             // [M][N]
+  int* err;
+  unsigned long long budget_ns;
+  int branch;                   // 1: add XL L2b (rank 16) from its own accumulator
+  int gelu;
+};
+
 struct UpParams {
   int M, N;
   int width;                    // branch width: 32, or 64 with a LoRA adapter
@@ -118,6 +135,11 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t stream);
 cudaError_t launch_k1(const CUtensorMap& tm_x, const CUtensorMap& tm_l, const CUtensorMap& tm_c,
                       const K1Params& p, int fmt, int mode, cudaStream_t stream);
 int k1_rows_per_cta();
+// Per-token INT8 scales of x_hat = fp32(x * inv_lam): a = max_k |x_hat|,
+// s = fp32(a fp32(1/127)), inv = fp32(1/s) (0 when s == 0); sx and inv_sx get
+// mpad entries (padding rows zero).
+cudaError_t launch_rowscale(const __nv_bfloat16* x, const float* inv_lam, int M, int K, int mpad, float* sx,
+                            float* inv_sx, cudaStream_t stream);
 
 // NVFP4 GEMM: operands from p.acodes / p.sfa (the first kernel's layouts) and
 // p.wmerged; tm_xl / tm_l2 the branch tiles, tm_y the output; with p.lora,
@@ -165,6 +187,12 @@ int k2_int4_pair_rows_b();
 cudaError_t launch_k2_int4_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_xl,
                                 const CUtensorMap& tm_l2, const CUtensorMap& tm_y, const K2Int4Params& p,
                                 int num_sms, cudaStream_t stream);
+
+// W8A8 GEMM (tcgen05 kind::i8): tm_xl / tm_l2 the branch tiles (as for the
+// NVFP4 GEMM, L2b unscaled), tm_y the output.
+cudaError_t launch_k2_int8(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
+                           const K2Int8Params& p, int num_sms, cudaStream_t stream);
+size_t k2_int8_weight_bytes(int N, int K);
 
 // Y is read and rewritten through tm_y: a BF16 [M][N] map with boxes of 64
 // columns x upproj_box_rows() rows and the 128-byte swizzle.

@@ -686,10 +686,35 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
         }
 
     // ---- residual quantization, groups along K for each output column n
-    P.w_codes.assign((size_t)N * K / 2, 0);
     float amax = 0.0f;
     for (float v : P.R) amax = std::max(amax, std::fabs(v));
     P.w_amax = amax;
+    if (cfg.format == SVDQ_W8A8_INT8) {
+      // INT8, one group per output channel: s = fp32(a fp32(1/127)),
+      // code = clamp(rint(fp32(v fp32(1/s))), -127, 127)
+      P.w_codes.assign((size_t)N * K, 0);
+      P.w_scales_f32.assign(N, 0.0f);
+#pragma omp parallel for schedule(static)
+      for (int n = 0; n < N; ++n) {
+        float a = 0.0f;
+        for (int k = 0; k < K; ++k) a = std::max(a, std::fabs(P.R[(size_t)k * N + n]));
+        const float c127 = 1.0f / 127.0f;
+        volatile float t = a * c127;
+        const float sc = t;
+        P.w_scales_f32[n] = sc;
+        if (sc == 0.0f) continue;
+        volatile float iv = 1.0f / sc;
+        const float inv = iv;
+        for (int k = 0; k < K; ++k) {
+          volatile float q = P.R[(size_t)k * N + n] * inv;
+          float rq = std::nearbyint((float)q);
+          rq = std::min(127.0f, std::max(-127.0f, rq));
+          P.w_codes[(size_t)n * K + k] = (uint8_t)(int8_t)rq;
+        }
+      }
+      return SVDQ_OK;
+    }
+    P.w_codes.assign((size_t)N * K / 2, 0);
     if (cfg.flags & SVDQ_PREP_GPTQ) {
       const bool nvfp4 = cfg.format == SVDQ_NVFP4;
       if (nvfp4) {

@@ -34,9 +34,10 @@ struct HostPrep {
   int lora_r = 0;                           // LoRA adapter rank (0: none)
   std::vector<uint16_t> lora_A;             // [K][lora_r] BF16 bits, as given
   std::vector<uint16_t> lora_B;             // [lora_r][N] BF16 bits of bf16(scale * B)
-  std::vector<uint8_t> w_codes;             // [N][K/2]
+  std::vector<uint8_t> w_codes;             // [N][K/2] (4-bit formats), [N][K] int8 (W8A8)
   std::vector<uint8_t> w_scales_e4m3;       // [N][K/16]   (NVFP4)
   std::vector<uint16_t> w_scales_bf16;      // [N][K/64]   (INT4 / W4A16)
+  std::vector<float> w_scales_f32;          // [N]         (W8A8: one scale per output channel)
   std::vector<float> bias;                  // [N]
   int svd_iterations = 0;
   double svd_tail_energy = 0.0;
