@@ -217,7 +217,23 @@ const char* svdq_status_string(svdq_status s);
 svdq_status svdq_set_lora(svdq_layer* layer, int r, const uint16_t* A_bf16, const uint16_t* B_bf16,
                           float scale);
 
-/* ------------------------------------------------------------------ forward */
+/* Checkpoints.  svdq_serialize writes a prepared layer (scalars, lam, 1/lam,
+ * sigma, L1d, L2b, residual codes and scales, bias, and a LoRA adapter if one
+ * is attached) into `bytes` == svdq_serialized_bytes(layer) bytes of host
+ * memory `dst`; svdq_deserialize rebuilds the layer from such bytes, on
+ * `device` (or host-only with -1), without repeating the SVD or the
+ * quantization.  Preparation-only intermediates (the residual R, the float64
+ * L1 and L2, the GPTQ factor) are not stored: their svdq_tensor_bytes are 0 on
+ * a deserialized layer.  The byte layout is "SVDQ", a version, the scalar
+ * fields, then each array as a 64-bit byte count and its bytes (host byte
+ * order).  svdq_deserialize checks every size against the shape and format
+ * and returns SVDQ_EINVAL on any mismatch or truncation; SVDQ_ENOMEM,
+ * SVDQ_ECUDA as for svdq_prepare. */
+size_t svdq_serialized_bytes(const svdq_layer* layer);
+svdq_status svdq_serialize(const svdq_layer* layer, void* dst, size_t bytes);
+svdq_status svdq_deserialize(const void* src, size_t bytes, int device, svdq_layer** out);
+
+/* ------------------------------------------------------------------ forward *//* ------------------------------------------------------------------ forward */
 
 /* Workspace bytes a forward over M tokens needs (activation codes, scales in the
  * tensor-core layout and the BF16 down projection X L1d).  0 on bad input. */

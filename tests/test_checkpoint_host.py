@@ -1,0 +1,61 @@
+"""Checkpoints of prepared layers (svdq_serialize / svdq_deserialize), on the
+host: every stored tensor and the layer info survive the round trip for each
+format, with and without a LoRA adapter; damaged bytes are refused."""
+import numpy as np
+import pytest
+
+import synthetic as syn
+
+import w4a4_diffusion_transformer_b200 as lib
+
+KEPT = ["lambda", "inv_lambda", "sigma", "L1d", "L2b", "w_codes", "w_scales", "bias"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from w4a4_diffusion_transformer_b200 import build
+    build.build()
+    lib.load()
+
+
+def _layer(fmt, rank, lora=False):
+    d = syn.custom_layer(800 + rank, M=8, K=256, N=128)
+    L = lib.Layer.prepare(syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]),
+                          None if fmt == "w4a16" else syn.bf16_bits(d["Xc"]), fmt=fmt, rank=rank, device=-1)
+    if lora:
+        rng = np.random.default_rng(3)
+        L.set_lora(syn.bf16_bits(syn.to_bf16(rng.standard_normal((256, 8)))),
+                   syn.bf16_bits(syn.to_bf16(rng.standard_normal((8, 128)))), 0.5)
+    return L
+
+
+@pytest.mark.parametrize("fmt,rank,lora", [("nvfp4", 32, False), ("nvfp4", 32, True), ("int4", 32, True),
+                                           ("nvfp4", 0, False), ("w4a16", 0, False), ("w8a8", 16, False)])
+def test_round_trip(fmt, rank, lora):
+    L = _layer(fmt, rank, lora)
+    blob = L.serialize()
+    assert blob[:4] == b"SVDQ"
+    R = lib.Layer.deserialize(blob, device=-1)
+    assert R.info == L.info
+    for name in KEPT + (["lora_A", "lora_B"] if lora else []):
+        n = lib.load().svdq_tensor_bytes(L._h, lib.TENSORS[name][0])
+        assert lib.load().svdq_tensor_bytes(R._h, lib.TENSORS[name][0]) == n, name
+        if n:                                        # rank 0 has no branch tensors
+            np.testing.assert_array_equal(R.export(name), L.export(name), err_msg=name)
+    # preparation-only intermediates are not part of a checkpoint
+    for name in ("R", "L1", "L2"):
+        assert lib.load().svdq_tensor_bytes(R._h, lib.TENSORS[name][0]) == 0
+    assert R.serialize() == blob
+
+
+def test_damaged_bytes_are_refused():
+    blob = bytearray(_layer("nvfp4", 32).serialize())
+    for bad in (bytes(blob[:-1]), bytes(blob[:40]), b"XXXX" + bytes(blob[4:]), bytes(blob) + b"\0"):
+        with pytest.raises(lib.SvdqError) as e:
+            lib.Layer.deserialize(bad, device=-1)
+        assert e.value.status == lib.EINVAL
+    # a size field that disagrees with the shape
+    wrong = bytearray(blob)
+    wrong[8:12] = (int.from_bytes(blob[8:12], "little") + 64).to_bytes(4, "little")   # K
+    with pytest.raises(lib.SvdqError):
+        lib.Layer.deserialize(bytes(wrong), device=-1)

@@ -43,7 +43,7 @@ EXPORTED = [
     "svdq_gemm", "svdq_act_scale_bytes", "svdq_act_scales_to_logical", "svdq_check",
     "svdq_linear_forward_static", "svdq_act_code_bytes", "svdq_act_codes_to_logical",
     "svdq_selftest_wait_timeout", "svdq_mlp_workspace_bytes", "svdq_mlp_fc1", "svdq_mlp_forward",
-    "svdq_set_lora",
+    "svdq_set_lora", "svdq_serialized_bytes", "svdq_serialize", "svdq_deserialize",
 ]
 STATIC_WORKSPACE_BYTES = 16 << 20   # SVDQ_STATIC_WORKSPACE_BYTES
 
@@ -100,6 +100,9 @@ def load() -> ctypes.CDLL:
         "svdq_mlp_fc1": (I, [P, P, P, I, P, P, P, P, SZ, P, U]),
         "svdq_mlp_forward": (I, [P, P, P, I, P, P, SZ, P, U]),
         "svdq_set_lora": (I, [P, I, P, P, ctypes.c_float]),
+        "svdq_serialized_bytes": (SZ, [P]),
+        "svdq_serialize": (I, [P, P, SZ]),
+        "svdq_deserialize": (I, [P, SZ, I, ctypes.POINTER(P)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -161,6 +164,21 @@ class Layer:
         st = L.svdq_prepare(ctypes.byref(cfg), K, N, _ptr(W), _ptr(b), _ptr(c),
                             0 if c is None else c.shape[0], device, ctypes.byref(out))
         _check(st, "svdq_prepare")
+        return cls(out.value)
+
+    def serialize(self) -> bytes:
+        """The prepared layer as bytes (svdq_serialize)."""
+        n = int(load().svdq_serialized_bytes(self._h))
+        buf = np.empty(n, dtype=np.uint8)
+        _check(load().svdq_serialize(self._h, _ptr(buf), n), "svdq_serialize")
+        return buf.tobytes()
+
+    @classmethod
+    def deserialize(cls, data: bytes, device: int = 0) -> "Layer":
+        """Rebuild a layer from serialize()'s bytes (svdq_deserialize)."""
+        buf = np.frombuffer(data, dtype=np.uint8)
+        out = ctypes.c_void_p()
+        _check(load().svdq_deserialize(_ptr(buf), buf.size, device, ctypes.byref(out)), "svdq_deserialize")
         return cls(out.value)
 
     def close(self):

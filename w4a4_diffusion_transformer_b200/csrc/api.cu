@@ -553,6 +553,86 @@ svdq_status run_k2(const svdq_layer* L, const void* codes, const void* scales, c
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
 
+// (Re)build a layer's LoRA device buffers from the host copies (none when
+// lora_r == 0).  The device must be current and idle for this layer.
+svdq_status upload_lora(svdq_layer* L) {
+  const HostPrep& h = L->host;
+  const int K = h.K, N = h.N, r = h.lora_r;
+  cudaFree(L->d_lora_l1t);
+  cudaFree(L->d_lora_l2s);
+  cudaFree(L->d_lora_l2t);
+  L->d_lora_l1t = L->d_lora_l2s = L->d_lora_l2t = nullptr;
+  if (r == 0) return SVDQ_OK;
+  // the GEMM's accumulator unit: alpha = g_x g_w (NVFP4) or 2^(ex + ew) (INT4)
+  const int alpha_exp = h.format == SVDQ_NVFP4 ? h.g_x_exp + h.g_w_exp : L->i4_ex + L->i4_ew;
+  // l2t: the unfused up projection's [N][64] = [L2b^T | bf16(s B)^T]
+  std::vector<uint16_t> l1t((size_t)32 * K, 0), l2s((size_t)N * 32, 0), l2t((size_t)N * 64, 0);
+  for (int i = 0; i < h.rank; ++i)
+    for (int n = 0; n < N; ++n) l2t[(size_t)n * 64 + i] = h.L2b[(size_t)i * N + n];
+  for (int i = 0; i < r; ++i) {
+    for (int k = 0; k < K; ++k) l1t[(size_t)i * K + k] = h.lora_A[(size_t)k * r + i];
+    for (int n = 0; n < N; ++n) {
+      const uint16_t v = h.lora_B[(size_t)i * N + n];
+      l2t[(size_t)n * 64 + 32 + i] = v;
+      l2s[(size_t)n * 32 + i] = bf16_from_double(std::ldexp((double)bf16_to_float(v), -alpha_exp));
+    }
+  }
+  cudaError_t e = upload(&L->d_lora_l1t, l1t.data(), l1t.size() * 2);
+  if (e == cudaSuccess) e = upload(&L->d_lora_l2s, l2s.data(), l2s.size() * 2);
+  if (e == cudaSuccess) e = upload(&L->d_lora_l2t, l2t.data(), l2t.size() * 2);
+  if (e != cudaSuccess || !make_map_kchunks(&L->tm_lora_l1t, L->d_lora_l1t, K, 32, 32) ||
+      !make_map(&L->tm_lora_l2s, L->d_lora_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
+                CU_TENSOR_MAP_SWIZZLE_64B)) {
+    cudaFree(L->d_lora_l1t);
+    cudaFree(L->d_lora_l2s);
+    cudaFree(L->d_lora_l2t);
+    L->d_lora_l1t = L->d_lora_l2s = L->d_lora_l2t = nullptr;
+    return e == cudaErrorMemoryAllocation ? SVDQ_ENOMEM : SVDQ_ECUDA;
+  }
+  return SVDQ_OK;
+}
+
+// ------------------------------------------------------------------ serialization
+//
+// A prepared layer as bytes: "SVDQ", version, the scalar fields, then each
+// array as a 64-bit byte count followed by its bytes (lam, inv_lam, sigma,
+// L1d, L2b, w_codes, w_scales_e4m3, w_scales_bf16, w_scales_f32, bias,
+// lora_A, lora_B).  The preparation-only intermediates (R, L1, L2, the GPTQ
+// factor) are not part of it.
+
+constexpr uint32_t kSerialMagic = 0x51445653u;   // "SVDQ"
+constexpr uint32_t kSerialVersion = 1;
+
+struct SerialHeader {
+  uint32_t magic, version;
+  int32_t K, N, rank, format, g_x_exp, g_w_exp, lora_r, svd_iterations;
+  float alpha, x_amax, w_amax, pad;
+  double svd_tail_energy;
+};
+
+// f(array) for every serialized array of h, in order (h const or not).
+template <class F, class H>
+void serial_arrays(F&& f, H& h) {
+  f(h.lam);
+  f(h.inv_lam);
+  f(h.sigma);
+  f(h.L1d);
+  f(h.L2b);
+  f(h.w_codes);
+  f(h.w_scales_e4m3);
+  f(h.w_scales_bf16);
+  f(h.w_scales_f32);
+  f(h.bias);
+  f(h.lora_A);
+  f(h.lora_B);
+}
+
+size_t serialized_bytes(const HostPrep& h) {
+  size_t n = sizeof(SerialHeader);
+  serial_arrays([&](const auto& v) { n += 8 + v.size() * sizeof(v[0]); }, h);
+  return n;
+}
+
 // ------------------------------------------------------------------ fc1 -> fc2 chain
 
 bool chainable(const svdq_layer* L1, const svdq_layer* L2) {
@@ -948,6 +1028,122 @@ svdq_status svdq_linear_forward(const svdq_layer* L, const void* X, int M, void*
   return st;
 }
 
+size_t svdq_serialized_bytes(const svdq_layer* L) { return L ? serialized_bytes(L->host) : 0; }
+
+svdq_status svdq_serialize(const svdq_layer* L, void* dst, size_t bytes) {
+  if (!L || !dst) return SVDQ_EINVAL;
+  const HostPrep& h = L->host;
+  if (bytes != serialized_bytes(h)) return SVDQ_EINVAL;
+  SerialHeader hd = {};
+  hd.magic = kSerialMagic;
+  hd.version = kSerialVersion;
+  hd.K = h.K;
+  hd.N = h.N;
+  hd.rank = h.rank;
+  hd.format = h.format;
+  hd.g_x_exp = h.g_x_exp;
+  hd.g_w_exp = h.g_w_exp;
+  hd.lora_r = h.lora_r;
+  hd.svd_iterations = h.svd_iterations;
+  hd.alpha = h.alpha;
+  hd.x_amax = h.x_amax;
+  hd.w_amax = h.w_amax;
+  hd.svd_tail_energy = h.svd_tail_energy;
+  uint8_t* o = static_cast<uint8_t*>(dst);
+  std::memcpy(o, &hd, sizeof(hd));
+  o += sizeof(hd);
+  serial_arrays(
+      [&](const auto& v) {
+        const uint64_t n = v.size() * sizeof(v[0]);
+        std::memcpy(o, &n, 8);
+        if (n) std::memcpy(o + 8, v.data(), n);
+        o += 8 + n;
+      },
+      h);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_deserialize(const void* src, size_t bytes, int device, svdq_layer** out) {
+  if (!out) return SVDQ_EINVAL;
+  *out = nullptr;
+  if (!src || bytes < sizeof(SerialHeader)) return SVDQ_EINVAL;
+  SerialHeader hd;
+  std::memcpy(&hd, src, sizeof(hd));
+  if (hd.magic != kSerialMagic || hd.version != kSerialVersion) return SVDQ_EINVAL;
+  if (hd.format < SVDQ_NVFP4 || hd.format > SVDQ_W8A8_INT8 || hd.K <= 0 || hd.N <= 0 || hd.K % 64 ||
+      hd.rank < 0 || hd.rank > 32 || hd.lora_r < 0 || hd.lora_r > 32)
+    return SVDQ_EINVAL;
+  svdq_layer* L = new (std::nothrow) svdq_layer();
+  if (!L) return SVDQ_ENOMEM;
+  HostPrep& h = L->host;
+  h.K = hd.K;
+  h.N = hd.N;
+  h.rank = hd.rank;
+  h.format = hd.format;
+  h.g_x_exp = hd.g_x_exp;
+  h.g_w_exp = hd.g_w_exp;
+  h.lora_r = hd.lora_r;
+  h.svd_iterations = hd.svd_iterations;
+  h.alpha = hd.alpha;
+  h.x_amax = hd.x_amax;
+  h.w_amax = hd.w_amax;
+  h.svd_tail_energy = hd.svd_tail_energy;
+  const uint8_t* in = static_cast<const uint8_t*>(src) + sizeof(hd);
+  const uint8_t* end = static_cast<const uint8_t*>(src) + bytes;
+  bool ok = true;
+  try {
+    serial_arrays(
+        [&](auto& v) {
+          uint64_t n = 0;
+          if (!ok || end - in < 8) {
+            ok = false;
+            return;
+          }
+          std::memcpy(&n, in, 8);
+          in += 8;
+          if (n % sizeof(v[0]) || (uint64_t)(end - in) < n) {
+            ok = false;
+            return;
+          }
+          v.resize(n / sizeof(v[0]));
+          if (n) std::memcpy(v.data(), in, n);
+          in += n;
+        },
+        h);
+  } catch (const std::bad_alloc&) {
+    delete L;
+    return SVDQ_ENOMEM;
+  }
+  // every array must have the size the shape and format imply
+  const size_t K = h.K, N = h.N, r = h.rank, lr = h.lora_r;
+  const bool nv = h.format == SVDQ_NVFP4, i4 = h.format == SVDQ_INT4 || h.format == SVDQ_W4A16_INT4,
+             i8 = h.format == SVDQ_W8A8_INT8;
+  ok = ok && in == end && h.lam.size() == K && h.inv_lam.size() == K && h.sigma.size() == r &&
+       h.L1d.size() == K * r && h.L2b.size() == r * N && h.bias.size() == N &&
+       h.w_codes.size() == (i8 ? N * K : N * K / 2) && h.w_scales_e4m3.size() == (nv ? N * K / 16 : 0) &&
+       h.w_scales_bf16.size() == (i4 ? N * K / 64 : 0) && h.w_scales_f32.size() == (i8 ? N : 0) &&
+       h.lora_A.size() == K * lr && h.lora_B.size() == lr * N;
+  if (!ok) {
+    delete L;
+    return SVDQ_EINVAL;
+  }
+  svdq_status st = SVDQ_OK;
+  if (device >= 0) {
+    st = upload_layer(L, device);
+    if (st == SVDQ_OK && h.lora_r > 0) {
+      DeviceGuard g(device);
+      st = g.ok ? upload_lora(L) : SVDQ_ECUDA;
+    }
+    if (st != SVDQ_OK) free_device(L);
+  }
+  if (st != SVDQ_OK) {
+    delete L;
+    return st;
+  }
+  *out = L;
+  return SVDQ_OK;
+}
+
 svdq_status svdq_set_lora(svdq_layer* L, int r, const uint16_t* A_bf16, const uint16_t* B_bf16, float scale) {
   if (!L) return SVDQ_EINVAL;
   if (L->host.format == SVDQ_W4A16_INT4 || L->host.format == SVDQ_W8A8_INT8) return SVDQ_EUNSUPPORTED;
@@ -964,50 +1160,23 @@ svdq_status svdq_set_lora(svdq_layer* L, int r, const uint16_t* A_bf16, const ui
       for (size_t i = 0; i < b.size(); ++i)
         b[i] = bf16_from_double((double)bf16_to_float(B_bf16[i]) * (double)scale);   // one rounding of s B
     }
+    h.lora_r = r;
+    h.lora_A.swap(a);
+    h.lora_B.swap(b);
     if (L->device >= 0) {
       DeviceGuard g(L->device);
       if (!g.ok) return SVDQ_ECUDA;
       // no forward of this layer may be pending: the old buffers are released
       if (cudaDeviceSynchronize() != cudaSuccess) return SVDQ_ECUDA;
-      cudaFree(L->d_lora_l1t);
-      cudaFree(L->d_lora_l2s);
-      cudaFree(L->d_lora_l2t);
-      L->d_lora_l1t = L->d_lora_l2s = L->d_lora_l2t = nullptr;
-      if (r > 0) {
-        // the GEMM's accumulator unit: alpha = g_x g_w (NVFP4) or 2^(ex + ew) (INT4)
-        const int alpha_exp = h.format == SVDQ_NVFP4 ? h.g_x_exp + h.g_w_exp : L->i4_ex + L->i4_ew;
-        // l2t: the unfused up projection's [N][64] = [L2b^T | bf16(s B)^T]
-        std::vector<uint16_t> l1t((size_t)32 * K, 0), l2s((size_t)N * 32, 0), l2t((size_t)N * 64, 0);
-        for (int i = 0; i < h.rank; ++i)
-          for (int n = 0; n < N; ++n) l2t[(size_t)n * 64 + i] = h.L2b[(size_t)i * N + n];
-        for (int i = 0; i < r; ++i) {
-          for (int k = 0; k < K; ++k) l1t[(size_t)i * K + k] = a[(size_t)k * r + i];
-          for (int n = 0; n < N; ++n) {
-            const uint16_t v = b[(size_t)i * N + n];
-            l2t[(size_t)n * 64 + 32 + i] = v;
-            l2s[(size_t)n * 32 + i] = bf16_from_double(std::ldexp((double)bf16_to_float(v), -alpha_exp));
-          }
-        }
-        cudaError_t e = upload(&L->d_lora_l1t, l1t.data(), l1t.size() * 2);
-        if (e == cudaSuccess) e = upload(&L->d_lora_l2s, l2s.data(), l2s.size() * 2);
-        if (e == cudaSuccess) e = upload(&L->d_lora_l2t, l2t.data(), l2t.size() * 2);
-        if (e != cudaSuccess || !make_map_kchunks(&L->tm_lora_l1t, L->d_lora_l1t, K, 32, 32) ||
-            !make_map(&L->tm_lora_l2s, L->d_lora_l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, N, 32, 256,
-                      CU_TENSOR_MAP_SWIZZLE_64B)) {
-          cudaFree(L->d_lora_l1t);
-          cudaFree(L->d_lora_l2s);
-          cudaFree(L->d_lora_l2t);
-          L->d_lora_l1t = L->d_lora_l2s = L->d_lora_l2t = nullptr;
-          h.lora_r = 0;
-          h.lora_A.clear();
-          h.lora_B.clear();
-          return e == cudaErrorMemoryAllocation ? SVDQ_ENOMEM : SVDQ_ECUDA;
-        }
+      const svdq_status st = upload_lora(L);
+      if (st != SVDQ_OK) {
+        h.lora_r = 0;
+        h.lora_A.clear();
+        h.lora_B.clear();
+        return st;
       }
     }
-    h.lora_r = r;
-    h.lora_A.swap(a);
-    h.lora_B.swap(b);
+    return SVDQ_OK;
   } catch (const std::bad_alloc&) {
     return SVDQ_ENOMEM;
   }

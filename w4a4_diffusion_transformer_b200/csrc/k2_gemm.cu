@@ -56,7 +56,13 @@ constexpr int kBN = 256;
 // in the 128-byte swizzle: the tiled layout the operands are stored in.
 constexpr int kKB = 4;
 constexpr int kBKBytes = kKB * 32;           // E2M1 bytes per operand row per stage
-constexpr int kStages = 3;
+// Ring depth: the default mode runs 4 stages (its low-rank branch is a ring
+// stage and its epilogue stores from registers, which frees the shared memory
+// of the branch buffer and the output staging); chain mode keeps 3 stages, the
+// branch buffer and the staging its epilogue works in.
+#ifndef SVDQ_K2_DEEP
+#define SVDQ_K2_DEEP 1
+#endif
 constexpr uint32_t kSwz = 2u;                          // descriptor layout: 128-byte swizzle
 constexpr uint32_t kSwzAtom = 8u * kBKBytes;           // bytes between 8-row groups
 constexpr int kEpiWarps = 8;
@@ -86,15 +92,24 @@ static_assert(kStageBytes % 1024 == 0, "stage alignment");
 constexpr int kBrXL = kBM * 64;
 constexpr int kBrBytes = kBrXL + kBN * 64;
 static_assert(kBrBytes % 1024 == 0, "branch buffer alignment");
-constexpr int kSmemBytes = kStages * kStageBytes + kBrBytes + kEpiWarps * kEpiWarpBytes + 1024 + 256;
-static_assert(kSmemBytes <= 232448, "shared memory per block");
+
 constexpr int kTmemCols = 512;
 // Scale factors in TMEM, one region per pipeline stage (so a region is only
 // rewritten after the MMAs that read it have completed): 4 columns per 128-row
 // x 64-K block, 16 for A and 32 for B per stage.
 constexpr int kSFCol0 = 256;
 constexpr int kSFStageCols = 12 * kKB;       // 4 columns of A + 8 of B per K block
-static_assert(kSFCol0 + kStages * kSFStageCols <= kTmemCols, "TMEM budget");
+
+template <bool kChain>
+struct K2Layout {
+  static constexpr bool deep = !kChain && SVDQ_K2_DEEP;
+  static constexpr int stages = deep ? 4 : 3;
+  static constexpr int br_bytes = deep ? 0 : kBrBytes;
+  static constexpr int epi_warp_bytes = deep ? 512 : kEpiWarpBytes;   // deep: 128 bias floats only
+  static constexpr int smem = stages * kStageBytes + br_bytes + kEpiWarps * epi_warp_bytes + 1024 + 256;
+  static_assert(smem <= 232448, "shared memory per block");
+  static_assert(kSFCol0 + stages * kSFStageCols <= kTmemCols, "TMEM budget");
+};
 
 __device__ __forceinline__ void record_error(int* err, volatile int* abort_flag, int code) {
   atomicCAS(err, 0, code);
@@ -135,11 +150,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     k2_kernel(const __grid_constant__ CUtensorMap tm_xl, const __grid_constant__ CUtensorMap tm_l2,
               const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_xla,
               const __grid_constant__ CUtensorMap tm_l2a, K2Params p) {
+  using Lay = K2Layout<kChain>;
+  constexpr int kStages = Lay::stages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* brbuf = smem + kStages * kStageBytes;
-  uint8_t* epi_buf = brbuf + kBrBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(epi_buf + kEpiWarps * kEpiWarpBytes);
+  uint8_t* epi_buf = brbuf + Lay::br_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_buf + kEpiWarps * Lay::epi_warp_bytes);
   uint64_t* empty = full + kStages;
   uint64_t* sf_full = empty + kStages;             // a stage's scale factors are in shared memory
   uint64_t* sf_ready = sf_full + kStages;          // ... and in TMEM
@@ -160,10 +177,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const TileSeq<kChain> ts{tiles_m, tiles_n, kChain ? p.chain.S : 1};
   const int kblocks = K >> 6;                     // 64-element K blocks
   const int ktiles = (kblocks + kKB - 1) / kKB;
-  // A LoRA adapter is one more ring stage in front of each tile's K stages:
-  // XL_lora rows in the A slot, (s B / alpha)^T rows in the B slot (64-byte
-  // rows), two BF16 MMAs; its scale-factor slots are not read.
+  // Extra ring stages in front of each tile's K stages, each with XL rows in
+  // the A slot and (L2 / alpha)^T rows in the B slot (64-byte rows) for two
+  // BF16 MMAs; their scale-factor slots are moved but not read.  Stage 0: the
+  // low-rank branch (deep mode; otherwise it has a buffer of its own); then a
+  // LoRA adapter's XL_lora and (s B / alpha)^T.
   const int lora = kChain ? 0 : p.lora;
+  const int br_stage = (Lay::deep && p.branch) ? 1 : 0;
+  const int nextra = br_stage + lora;
+  const bool br_buf = p.branch && !Lay::deep;
 
   if (threadIdx.x == 0) {
     // the next kernel on the stream may launch now; it waits for this grid's
@@ -204,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool pa = warp == kProdA;
       if (p.branch) dev::tma_prefetch_desc(pa ? &tm_xl : &tm_l2);
       if (lora) dev::tma_prefetch_desc(pa ? &tm_xla : &tm_l2a);
+      const CUtensorMap* xmap[2] = {pa ? &tm_xl : &tm_l2, pa ? &tm_xla : &tm_l2a};
       // the activations come from the preceding kernel (launched as a
       // dependency); the weights do not, so their stream starts at once
       if (pa) dev::griddep_wait();
@@ -213,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = ts.first(u); t < ts.last(u) && ok; ++t, ++tcount) {
           const int m0 = ts.m0(u);
           const int n0 = ts.n0(u, t);
-          if (p.branch) {
+          if (br_buf) {
             // the previous tile's branch MMAs have read the buffer
             if (!dev::mbar_wait(br_empty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag, p.budget_ns)) {
               record_error(p.err, abort_flag, 0x201);
@@ -228,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               dev::tma_load_2d(brbuf + kBrXL, &tm_l2, br_full, 0, n0);
             }
           }
-          if (lora) {
+          for (int e = 0; e < nextra && ok; ++e, ++it) {
             const int s = it % kStages;
             if (!dev::mbar_wait(&empty[s], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
               record_error(p.err, abort_flag, 0x209);
@@ -236,16 +259,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             uint8_t* st = smem + s * kStageBytes;
+            const CUtensorMap* map = xmap[e < br_stage ? 0 : 1];
             dev::mbar_arrive_expect_tx(&sf_full[s], 0u);   // no scale factors in this stage
             if (pa) {
               dev::mbar_arrive_expect_tx(&full[s], (uint32_t)(kBM * 64));
-              dev::tma_load_2d(st, &tm_xla, &full[s], 0, m0);
+              dev::tma_load_2d(st, map, &full[s], 0, m0);
             } else {
               dev::mbar_arrive_expect_tx(&full[s], (uint32_t)(kBN * 64));
-              dev::tma_load_2d(st + kOffB, &tm_l2a, &full[s], 0, n0);
+              dev::tma_load_2d(st + kOffB, map, &full[s], 0, n0);
             }
-            ++it;
           }
+          if (!ok) break;
           for (int kt = 0; kt < ktiles; ++kt, ++it) {
             const int s = it % kStages;
             if (!dev::mbar_wait(&empty[s], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort_flag, p.budget_ns)) {
@@ -280,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!dev::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns) ||
             !dev::mbar_wait(&sf_full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag, p.budget_ns))
           break;
-      if (p.branch && tcount > 0) dev::mbar_wait(br_full, (uint32_t)(tcount - 1) & 1u, abort_flag, p.budget_ns);
+      if (br_buf && tcount > 0) dev::mbar_wait(br_full, (uint32_t)(tcount - 1) & 1u, abort_flag, p.budget_ns);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -299,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           dev::tc_fence_after();
           uint32_t accumulate = 0;
-          if (p.branch) {
+          if (br_buf) {
             if (!dev::mbar_wait(br_full, (uint32_t)tcount & 1u, abort_flag, p.budget_ns)) {
               record_error(p.err, abort_flag, 0x204);
               ok = false;
@@ -317,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             dev::tc_commit(br_empty);
           }
-          if (lora) {
+          for (int e = 0; e < nextra && ok; ++e, ++it) {
             const int s = it % kStages;
             if (!dev::mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns) ||
                 !dev::mbar_wait(&sf_ready[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns)) {
@@ -336,8 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               accumulate = 1;
             }
             dev::tc_commit(&empty[s]);
-            ++it;
           }
+          if (!ok) break;
           for (int kt = 0; kt < ktiles; ++kt, ++it) {
             const int s = it % kStages;
             if (!dev::mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns) ||
@@ -381,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < ts.units() && ok; u += gridDim.x) {
       for (int t = ts.first(u); t < ts.last(u) && ok; ++t) {
-        for (int kt = 0; kt < ktiles + lora; ++kt, ++it) {   // the LoRA stage's slots are moved too, unread
+        for (int kt = 0; kt < ktiles + nextra; ++kt, ++it) {   // the extra stages' slots are moved too, unread
           const int st = it % kStages;
           const bool got = dev::mbar_wait(&sf_full[st], (uint32_t)(it / kStages) & 1u, abort_flag, p.budget_ns);
           if (!__all_sync(0xffffffffu, got)) {
@@ -420,9 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                          // TMEM lane quarter of this warp
     const int half = (warp - kEpiWarp0) >> 2;       // which 128 of the 256 columns
     if (!kChain) {
-      uint8_t* wbuf = epi_buf + (warp - kEpiWarp0) * kEpiWarpBytes;
-      float* bias_s = reinterpret_cast<float*>(wbuf + 2 * kEpiBufBytes);
-      if (lane == 0) dev::tma_prefetch_desc(&tm_y);
+      uint8_t* wbuf = epi_buf + (warp - kEpiWarp0) * Lay::epi_warp_bytes;
+      float* bias_s = reinterpret_cast<float*>(Lay::deep ? wbuf : wbuf + 2 * kEpiBufBytes);
+      if (!Lay::deep && lane == 0) dev::tma_prefetch_desc(&tm_y);
       int tcount = 0, chunk = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < ts.units() && ok; u += gridDim.x) {
@@ -459,6 +483,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           dev::tc_fence_before();
           __syncwarp();
           if (lane == 0) dev::mbar_arrive(acc_empty);
+          if (Lay::deep) {
+            // each lane stores its row's 128 columns, 16 bytes at a time
+            const int row = m0 + q * 32 + lane;
+            __nv_bfloat16* yrow = p.y + (size_t)row * N;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t (&cur)[32] = c == 0 ? va : c == 1 ? vb : c == 2 ? vc : vd;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                uint32_t packed[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 b2 = reinterpret_cast<const float2*>(bias_s)[c * 16 + j * 4 + e];
+                  float y0 = p.alpha * __uint_as_float(cur[j * 8 + 2 * e]) + b2.x;
+                  float y1 = p.alpha * __uint_as_float(cur[j * 8 + 2 * e + 1]) + b2.y;
+                  if (p.gelu) {
+                    y0 = dev::gelu_tanh(y0);
+                    y1 = dev::gelu_tanh(y1);
+                  }
+                  const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+                  packed[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                const int col = n0 + c * 32 + j * 8;     // N is a multiple of 16: chunks are whole
+                if (row < M && col < N)
+                  *reinterpret_cast<uint4*>(yrow + col) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              }
+            }
+            __syncwarp();                                 // bias_s is restaged for the next tile
+          } else {
 #pragma unroll
           for (int c = 0; c < 4; ++c, ++chunk) {
             uint32_t (&cur)[32] = c == 0 ? va : c == 1 ? vb : c == 2 ? vc : vd;
@@ -493,9 +546,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           __syncwarp();
+          }
         }
       }
-      if (lane == 0) dev::bulk_wait_group_all();
+      if (!Lay::deep && lane == 0) dev::bulk_wait_group_all();
     } else {
       // ---------------------------------------------- chain: fc2's input
       // Shared memory of the epilogue in this mode: one 32 x 32 BF16 chunk
@@ -726,7 +780,8 @@ cudaError_t configure_k2() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device == dev) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k2_kernel<kChain>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e =
+      cudaFuncSetAttribute(k2_kernel<kChain>, cudaFuncAttributeMaxDynamicSharedMemorySize, K2Layout<kChain>::smem);
   if (e != cudaSuccess) return e;
   // the warpgroups' register budgets add up to exactly 128 per thread
   cudaFuncAttributes fa;
@@ -749,7 +804,7 @@ cudaError_t launch_k2_impl(const CUtensorMap& tm_xl, const CUtensorMap& tm_l2, c
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = K2Layout<kChain>::smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
