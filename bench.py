@@ -408,7 +408,7 @@ def block_b4(pkg, syn, stream, n, peaks, fp4_peak):
     return out
 
 
-def other_layers(pkg, syn, stream, flush_l2, n, peaks):
+def other_layers(pkg, syn, stream, flush_l2, n, peaks, only=None):
     """The other hot-path rows on their FLUX.1-shaped layers (not the headline):
     the INT4 variant (fused QKV 4608x3072->9216), the MLP pair (fc1 with the GELU
     epilogue, fc2 on fc1's output) and the W4A16 adaptive-norm GEMV (4x3072->18432).
@@ -468,13 +468,29 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
             st[0].close()
         return y0
 
+    def want(name):
+        return only is None or name in only
+
     # INT4 variant
-    d = syn.layer("qkv_int4")
-    w4a4_layer(d, "int4", d["X"], 0, "int4_qkv")
+    if want("int4"):
+        d = syn.layer("qkv_int4")
+        w4a4_layer(d, "int4", d["X"], 0, "int4_qkv")
     # W8A8 variant (rank 16 at 8 bits) on the attention-output shape
-    d = syn.layer("attn_out")
-    w4a4_layer(d, "w8a8", d["X"], 0, "w8a8_attn_out")
-    # MLP pair: fc1 (GELU), then fc2 on fc1's output; fc2 calibrates on fc1's output for its calibration batch
+    if want("w8a8"):
+        d = syn.layer("attn_out")
+        w4a4_layer(d, "w8a8", d["X"], 0, "w8a8_attn_out")
+    if want("mlp"):
+        mlp_pair(pkg, syn, stream, n, w4a4_layer, dev, out)
+    if want("w4a16"):
+        w4a16_adaln(pkg, syn, stream, flush_l2, n, peaks, dev, out)
+    return out
+
+
+def mlp_pair(pkg, syn, stream, n, w4a4_layer, dev, out):
+    """The MLP pair: fc1 (GELU), then fc2 on fc1's output (fc2 calibrates on
+    fc1's output for fc1's calibration batch), then the same pair through the
+    chain and as two separate layers."""
+    import torch
     d1 = syn.layer("mlp", "fc1")
     h = w4a4_layer(d1, "nvfp4", d1["X"], pkg.FWD_GELU, "fc1_gelu")
     L1 = pkg.Layer.prepare(syn.bf16_bits(d1["W"]), syn.bf16_bits(d1["bias"]), syn.bf16_bits(d1["Xc"]),
@@ -533,7 +549,11 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
         st[0].close()
         st[1].close()
     del csets
-    # W4A16 adaptive-norm GEMV (30 MB of weights per set)
+
+
+def w4a16_adaln(pkg, syn, stream, flush_l2, n, peaks, dev, out):
+    """The W4A16 adaptive-norm GEMV (30 MB of weights per set)."""
+    import torch
     da = syn.layer("block_b4", "adaln", with_run=False)
     Ma, Ka, Na = 4, da["W"].shape[0], da["W"].shape[1]
     n_sets = N_SETS
@@ -554,7 +574,6 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks):
                           "isolated_us": t_iso * 1e3, "rotating_sets": n_sets}
     for L in La:
         L.close()
-    return out
 
 
 def main():
@@ -565,6 +584,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-layers", action="store_true")
+    ap.add_argument("--only", default=None,
+                    help="comma-separated other-layer sections to run (int4, w8a8, mlp, w4a16, block); "
+                         "the library probes run only with all sections (the default)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -724,9 +746,13 @@ def main():
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
+    only = None if args.only is None else set(args.only.split(","))
     if rank == 0 and world == 1 and not args.no_other_layers:
-        out["other_layers"] = other_layers(pkg, syn, stream, flush_l2, max(30, min(200, args.steps)), peaks)
-        out["other_layers"]["block_b4"] = block_b4(pkg, syn, stream, max(20, min(100, args.steps)), peaks, fp4_peak)
+        out["other_layers"] = other_layers(pkg, syn, stream, flush_l2, max(30, min(200, args.steps)), peaks, only)
+        if only is None or "block" in only:
+            out["other_layers"]["block_b4"] = block_b4(pkg, syn, stream, max(20, min(100, args.steps)), peaks,
+                                                       fp4_peak)
+    if rank == 0 and world == 1 and not args.no_other_layers and only is None:
         lib_us = library_nvfp4_gemm_us(M, K, N, n_k)
         out["library_context"] = {
             "cublaslt_nvfp4_gemm_us": lib_us, "k2_us": k2_ms * 1e3, "bare_k2_us": bare_k2_ms * 1e3,

@@ -56,12 +56,14 @@ constexpr int kBN = 256;
 // in the 128-byte swizzle: the tiled layout the operands are stored in.
 constexpr int kKB = 4;
 constexpr int kBKBytes = kKB * 32;           // E2M1 bytes per operand row per stage
-// Ring depth: the default mode runs 4 stages (its low-rank branch is a ring
-// stage and its epilogue stores from registers, which frees the shared memory
-// of the branch buffer and the output staging); chain mode keeps 3 stages, the
-// branch buffer and the staging its epilogue works in.
+// Ring depth: 3 stages beside the branch buffer and the epilogue's staging.
+// SVDQ_K2_DEEP=1 builds a 4-stage default mode instead (the low-rank branch
+// becomes a ring stage and the epilogue stores Y straight from registers,
+// which frees that shared memory); measured slower at the attention-output
+// shape (31.0 vs 25.9 us): a lane holds one row, so each 16-byte store of the
+// epilogue touches 32 rows, and that costs more than the deeper ring gains.
 #ifndef SVDQ_K2_DEEP
-#define SVDQ_K2_DEEP 1
+#define SVDQ_K2_DEEP 0
 #endif
 constexpr uint32_t kSwz = 2u;                          // descriptor layout: 128-byte swizzle
 constexpr uint32_t kSwzAtom = 8u * kBKBytes;           // bytes between 8-row groups
