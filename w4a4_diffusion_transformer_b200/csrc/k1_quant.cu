@@ -570,7 +570,8 @@ __global__ void __launch_bounds__(256) rowscale_kernel(const __nv_bfloat16* __re
   if (row < M) {
     const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * K);
     const float4* il = reinterpret_cast<const float4*>(inv_lam);
-    for (int c = lane; c < K / 8; c += 32) {        // 8 columns per 16-byte chunk
+#pragma unroll 4
+    for (int c = lane; c < K / 8; c += 32) {        // 8 columns per 16-byte chunk (4 chunks in flight per lane)
       const uint4 raw = xr[c];
       const float4 i0 = il[2 * c], i1 = il[2 * c + 1];
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
