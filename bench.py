@@ -481,6 +481,8 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks, only=None):
         w4a4_layer(d, "w8a8", d["X"], 0, "w8a8_attn_out")
     if want("mlp"):
         mlp_pair(pkg, syn, stream, n, w4a4_layer, dev, out)
+    if want("lora"):
+        lora_layer(pkg, syn, stream, n, dev, out)
     if want("w4a16"):
         w4a16_adaln(pkg, syn, stream, flush_l2, n, peaks, dev, out)
     return out
@@ -551,6 +553,53 @@ def mlp_pair(pkg, syn, stream, n, w4a4_layer, dev, out):
     del csets
 
 
+def lora_layer(pkg, syn, stream, n, dev, out):
+    """The attention-output layer with a rank-32 LoRA adapter in its branch
+    (svdq_set_lora) against the same layer without one, back to back over
+    rotating sets; fused and unfused."""
+    import numpy as np
+    import torch
+    d = syn.layer("attn_out")
+    M, K = d["X"].shape
+    N = d["W"].shape[1]
+    g = np.random.default_rng([5, K, N])
+    A = syn.to_bf16(g.standard_normal((K, 32)) / np.sqrt(K))
+    B = syn.to_bf16(g.standard_normal((32, N)) * 0.1)
+    sets = []
+    for _ in range(3):
+        L = pkg.Layer.prepare(syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]), syn.bf16_bits(d["Xc"]),
+                              fmt="nvfp4", rank=RANK, device=dev)
+        sets.append([L, torch.from_numpy(d["X"]).to(torch.bfloat16).cuda(),
+                     torch.empty((M, N), dtype=torch.bfloat16, device="cuda"), None])
+
+    def alloc():
+        for st in sets:
+            st[3] = torch.empty(st[0].workspace_bytes(M), dtype=torch.uint8, device="cuda")
+
+    def fwd(flags):
+        def f(i):
+            L, x, y, ws = sets[i % len(sets)]
+            L.forward(x, M, y, ws, ws.numel(), stream, flags)
+        return f
+
+    alloc()
+    t0 = time_rotating(stream, n, fwd(0))
+    for st in sets:
+        st[0].set_lora(syn.bf16_bits(A), syn.bf16_bits(B), 0.5)
+    alloc()
+    for i in range(len(sets)):
+        fwd(pkg.FWD_CHECK)(i)
+    t1 = time_rotating(stream, n, fwd(0))
+    t2 = time_rotating(stream, n, fwd(pkg.FWD_UNFUSED))
+    for st in sets:
+        st[0].check(stream)
+        st[0].close()
+    out["lora_attn_out"] = {"shape": f"{M}x{K}->{N}", "format": "nvfp4", "rank": RANK, "lora_rank": 32,
+                            "us_without": t0 * 1e3, "us_with": t1 * 1e3, "us_with_unfused": t2 * 1e3,
+                            "note": "adapter appended to the 16-bit branch: one more down-projection pass "
+                                    "of the first kernel and one more ring stage per output tile"}
+
+
 def w4a16_adaln(pkg, syn, stream, flush_l2, n, peaks, dev, out):
     """The W4A16 adaptive-norm GEMV (30 MB of weights per set)."""
     import torch
@@ -585,7 +634,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-layers", action="store_true")
     ap.add_argument("--only", default=None,
-                    help="comma-separated other-layer sections to run (int4, w8a8, mlp, w4a16, block); "
+                    help="comma-separated other-layer sections to run (int4, w8a8, mlp, lora, w4a16, block); "
                          "the library probes run only with all sections (the default)")
     args = ap.parse_args()
     if args.warmup < 3:
