@@ -447,47 +447,111 @@ void gptq_hessian(const uint16_t* calib, int M, int K, const std::vector<float>&
   for (int k = 0; k < K; ++k) H[(size_t)k * K + k] += add;
 }
 
-// In place: the upper triangle of A (symmetric positive definite, [K][K]) becomes
-// the upper-triangular T with positive diagonal and A = T T^T -- Cholesky run
-// from the last column backwards.  false if a pivot is not positive.
-bool reverse_cholesky(std::vector<double>& A, int K) {
-  for (int j = K - 1; j >= 0; --j) {
-    double* rj = A.data() + (size_t)j * K;
-    double d = rj[j];
-    for (int k = j + 1; k < K; ++k) d -= rj[k] * rj[k];
-    if (!(d > 0.0) || !std::isfinite(d)) return false;
-    const double tjj = std::sqrt(d);
-    rj[j] = tjj;
-#pragma omp parallel for schedule(static) if (j >= 64)
-    for (int i = 0; i < j; ++i) {
-      double* ri = A.data() + (size_t)i * K;
-      double s = ri[j];                     // still H_ij: column j is being formed
-      for (int k = j + 1; k < K; ++k) s -= ri[k] * rj[k];
-      ri[j] = s / tjj;
+// The GPTQ factor U (upper triangular, positive diagonal, H^-1 = U^T U) of the
+// damped Hessian H ([K][K], symmetric positive definite), blocked for the cache
+// and the cores.  With J the order reversal, P = J H J = L L^T (lower
+// Cholesky), so H = T T^T with T = J L J upper and U = T^-1 = J L^-1 J.
+//   * L: right-looking blocked Cholesky of P in place (the diagonal block by
+//     the textbook loop, the panel by a triangular solve, the trailing matrix
+//     by block products in parallel);
+//   * L^-1: column blocks in parallel, each solved block row by block row.
+// false if a pivot is not positive (non-finite calibration).
+constexpr int kFactorBlock = 64;
+
+bool gptq_factor(const std::vector<double>& H, int K, std::vector<double>& U) {
+  const int B = kFactorBlock;
+  const int nb = (K + B - 1) / B;
+  std::vector<double> P((size_t)K * K);
+  // P = J H J (the lower triangle is what the factorization uses)
+#pragma omp parallel for schedule(static)
+  for (int i = 0; i < K; ++i)
+    for (int j = 0; j < K; ++j) P[(size_t)i * K + j] = H[(size_t)(K - 1 - i) * K + (K - 1 - j)];
+  auto at = [&](int i, int j) -> double& { return P[(size_t)i * K + j]; };
+  std::vector<double> Lt((size_t)B * K);            // the current panel, transposed
+  bool ok = true;
+  for (int kb = 0; kb < nb && ok; ++kb) {
+    const int k0 = kb * B, k1 = std::min(K, k0 + B);
+    // diagonal block
+    for (int j = k0; j < k1 && ok; ++j) {
+      double d = at(j, j);
+      for (int k = k0; k < j; ++k) d -= at(j, k) * at(j, k);
+      if (!(d > 0.0) || !std::isfinite(d)) {
+        ok = false;
+        break;
+      }
+      const double ljj = std::sqrt(d);
+      at(j, j) = ljj;
+      for (int i = j + 1; i < k1; ++i) {
+        double v = at(i, j);
+        for (int k = k0; k < j; ++k) v -= at(i, k) * at(j, k);
+        at(i, j) = v / ljj;
+      }
+    }
+    if (!ok) break;
+    // panel: rows below the block, L[i, k0:k1] = P[i, k0:k1] L[k0:k1, k0:k1]^-T
+#pragma omp parallel for schedule(static)
+    for (int i = k1; i < K; ++i)
+      for (int j = k0; j < k1; ++j) {
+        double v = at(i, j);
+        for (int k = k0; k < j; ++k) v -= at(i, k) * at(j, k);
+        at(i, j) = v / at(j, j);
+      }
+    // trailing update of the lower triangle: P[i, j] -= sum_k L[i, k] L[j, k],
+    // as row updates P[i, j0:j1] -= L[i, k] Lt[k, j0:j1] over a transposed copy
+    // of the panel, so the inner loop runs along contiguous columns
+    const int rem = nb - kb - 1;
+    if (rem > 0) {
+      const int w = k1 - k0;
+#pragma omp parallel for schedule(static)
+      for (int j = k1; j < K; ++j)
+        for (int k = 0; k < w; ++k) Lt[(size_t)k * K + j] = at(j, k0 + k);
+#pragma omp parallel for schedule(dynamic, 1)
+      for (int t = 0; t < rem * (rem + 1) / 2; ++t) {
+        int ib = 0;
+        while ((ib + 1) * (ib + 2) / 2 <= t) ++ib;     // block row ib, block column jb <= ib
+        const int jb = t - ib * (ib + 1) / 2;
+        const int i0 = k1 + ib * B, i1 = std::min(K, i0 + B);
+        const int j0 = k1 + jb * B, j1 = std::min(K, j0 + B);
+        for (int i = i0; i < i1; ++i) {
+          double* pi = &P[(size_t)i * K];
+          const int je = std::min(j1, i + 1);
+          for (int k = 0; k < w; ++k) {
+            const double lik = pi[k0 + k];
+            const double* lt = &Lt[(size_t)k * K];
+            for (int j = j0; j < je; ++j) pi[j] -= lik * lt[j];
+          }
+        }
+      }
     }
   }
-  return true;
-}
-
-// U = T^-1 for the upper-triangular T in the upper triangle of A; then
-// H^-1 = T^-T T^-1 = U^T U, so U is the upper Cholesky factor of H^-1.
-void upper_inverse(const std::vector<double>& A, int K, std::vector<double>& U) {
+  if (!ok) return false;
+  // X = L^-1 (lower), one block of B columns per task: rows i >= j0 of the
+  // block by forward substitution, X[i][c] = (delta_ic - sum_{k<i} L[i][k]
+  // X[k][c]) / L[i][i], in a private row-major [K][B] buffer so that the
+  // update runs along contiguous rows; then U = J X J.
   U.assign((size_t)K * K, 0.0);
 #pragma omp parallel
   {
-    std::vector<double> u(K);
-#pragma omp for schedule(dynamic, 8)
-    for (int j = K - 1; j >= 0; --j) {
-      u[j] = 1.0 / A[(size_t)j * K + j];
-      for (int i = j - 1; i >= 0; --i) {
-        const double* ti = A.data() + (size_t)i * K;
-        double s = 0.0;
-        for (int k = i + 1; k <= j; ++k) s += ti[k] * u[k];
-        u[i] = -s / ti[i];
+    std::vector<double> W((size_t)K * B);
+#pragma omp for schedule(dynamic, 1)
+    for (int jb = 0; jb < nb; ++jb) {
+      const int j0 = jb * B, w = std::min(K, j0 + B) - j0;
+      for (int i = j0; i < K; ++i) {
+        double* wi = &W[(size_t)(i - j0) * B];
+        for (int c = 0; c < w; ++c) wi[c] = (i == j0 + c) ? 1.0 : 0.0;
+        const double* li = &P[(size_t)i * K];
+        for (int k = j0; k < i; ++k) {
+          const double lik = li[k];
+          const double* wk = &W[(size_t)(k - j0) * B];
+          for (int c = 0; c < w; ++c) wi[c] -= lik * wk[c];
+        }
+        for (int c = 0; c < w; ++c) wi[c] = wi[c] / li[i];
+        double* urow = &U[(size_t)(K - 1 - i) * K];
+        for (int c = 0; c < w; ++c) urow[K - 1 - (j0 + c)] = wi[c];
       }
-      for (int i = 0; i <= j; ++i) U[(size_t)i * K + j] = u[i];
     }
   }
+  return true;
 }
 
 // Magnitude of a 3-bit E2M1 code.
@@ -725,8 +789,7 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
       }
       std::vector<double> H, U;
       gptq_hessian(calib, M_calib, K, P.inv_lam, H);
-      if (!reverse_cholesky(H, K)) return SVDQ_ENOCONVERGE;
-      upper_inverse(H, K, U);
+      if (!gptq_factor(H, K, U)) return SVDQ_ENOCONVERGE;
       std::vector<double>().swap(H);
       gptq_columns(P.R, K, N, U, nvfp4, P);
       if (nvfp4) P.g_x_exp = pow2_ceil_exponent(4.0 * (double)P.x_amax / 2688.0);
