@@ -59,3 +59,20 @@ def test_damaged_bytes_are_refused():
     wrong[8:12] = (int.from_bytes(blob[8:12], "little") + 64).to_bytes(4, "little")   # K
     with pytest.raises(lib.SvdqError):
         lib.Layer.deserialize(bytes(wrong), device=-1)
+
+
+def test_chain_and_adapter_rules_on_host_only_layers():
+    # the MLP chain needs device layers: host-only layers get no workspace and a state error
+    d1 = syn.custom_layer(830, M=8, K=256, N=512)
+    d2 = syn.custom_layer(831, M=8, K=512, N=256)
+    L1 = lib.Layer.prepare(syn.bf16_bits(d1["W"]), None, syn.bf16_bits(d1["Xc"]), device=-1)
+    L2 = lib.Layer.prepare(syn.bf16_bits(d2["W"]), None, syn.bf16_bits(d2["Xc"]), device=-1)
+    assert lib.mlp_workspace_bytes(L1, L2, 8) == 0
+    st = lib.load().svdq_mlp_forward(L1._h, L2._h, 16, 8, 16, 16, 1 << 20, None, 0)
+    assert st == lib.ESTATE
+    # an adapter on a host-only layer is stored and survives a checkpoint
+    rng = np.random.default_rng(9)
+    L1.set_lora(syn.bf16_bits(syn.to_bf16(rng.standard_normal((256, 4)))),
+                syn.bf16_bits(syn.to_bf16(rng.standard_normal((4, 512)))), 2.0)
+    R = lib.Layer.deserialize(L1.serialize(), device=-1)
+    np.testing.assert_array_equal(R.export("lora_B"), L1.export("lora_B"))
