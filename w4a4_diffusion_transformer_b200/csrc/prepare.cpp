@@ -31,6 +31,9 @@
 #ifdef _OPENMP
 #include <omp.h>
 #endif
+#if defined(__AVX2__) && defined(__FMA__)
+#include <immintrin.h>
+#endif
 
 #include "svdq_internal.h"
 
@@ -122,89 +125,222 @@ struct Rng {
   }
 };
 
-// Y[K][b] = A[K][N] * Z[N][b]   (all row-major)
-void gemm_AZ(const double* A, int K, int N, const double* Z, int b, double* Y) {
-#pragma omp parallel for schedule(static)
-  for (int k0 = 0; k0 < K; k0 += 8) {
-    const int k1 = std::min(K, k0 + 8);
-    double acc[8][128];
-    for (int i = 0; i < k1 - k0; ++i)
-      for (int j = 0; j < b; ++j) acc[i][j] = 0.0;
-    for (int n = 0; n < N; ++n) {
-      const double* z = Z + (size_t)n * b;
-      for (int i = 0; i < k1 - k0; ++i) {
-        const double a = A[(size_t)(k0 + i) * N + n];
-        double* ac = acc[i];
-        for (int j = 0; j < b; ++j) ac[j] += a * z[j];
-      }
-    }
-    for (int i = 0; i < k1 - k0; ++i)
-      std::memcpy(Y + (size_t)(k0 + i) * b, acc[i], sizeof(double) * b);
+// Row blocks of a fixed size for reductions over rows: the partial sums of each
+// block are added in block order, so the result does not depend on the thread
+// count.
+constexpr int kRowChunk = 256;
+
+inline int row_chunks(int rows) { return (rows + kRowChunk - 1) / kRowChunk; }
+
+// sum_r x[r] y[r] over [0, n) with four interleaved partial sums.
+inline double dot4(const double* x, const double* y, int n) {
+  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+  int r = 0;
+  for (; r + 4 <= n; r += 4) {
+    s0 += x[r] * y[r];
+    s1 += x[r + 1] * y[r + 1];
+    s2 += x[r + 2] * y[r + 2];
+    s3 += x[r + 3] * y[r + 3];
   }
+  for (; r < n; ++r) s0 += x[r] * y[r];
+  return (s0 + s1) + (s2 + s3);
 }
 
-// Z[N][b] = A^T * Q   with A[K][N], Q[K][b]
-void gemm_AtQ(const double* A, int K, int N, const double* Q, int b, double* Z) {
-#pragma omp parallel for schedule(static)
-  for (int n0 = 0; n0 < N; n0 += 32) {
-    const int n1 = std::min(N, n0 + 32);
-    double* zb = Z + (size_t)n0 * b;
-    std::fill(zb, zb + (size_t)(n1 - n0) * b, 0.0);
-    for (int k = 0; k < K; ++k) {
-      const double* q = Q + (size_t)k * b;
-      const double* a = A + (size_t)k * N;
-      for (int n = n0; n < n1; ++n) {
-        const double av = a[n];
-        double* z = Z + (size_t)n * b;
-        for (int j = 0; j < b; ++j) z[j] += av * q[j];
-      }
-    }
+// ---- packed float64 GEMM
+//
+// C[m][n] = op(A) op(B) with op(A)(i, p) = A[i * ars + p * acs] and
+// op(B)(p, j) = B[p * brs + j * bcs]; C is row-major with leading dimension
+// ldc.  Panels of op(A) (kMR rows) and op(B) (kNR columns) are packed per
+// kKC-deep slice; a 4 x 8 register tile accumulates each slice with fused
+// multiply-adds in ascending p and is then added to C, slice after slice.  Each
+// element of C belongs to one thread, so the result is the same for every
+// thread count.
+constexpr int kMR = 4, kNR = 8, kMC = 64, kKC = 256, kNC = 1024;
+
+inline void micro_tile(const double* ap, const double* bp, int kc, double* c) {
+#if defined(__AVX2__) && defined(__FMA__)
+  __m256d c00 = _mm256_setzero_pd(), c01 = _mm256_setzero_pd(), c10 = _mm256_setzero_pd(),
+          c11 = _mm256_setzero_pd(), c20 = _mm256_setzero_pd(), c21 = _mm256_setzero_pd(),
+          c30 = _mm256_setzero_pd(), c31 = _mm256_setzero_pd();
+  for (int p = 0; p < kc; ++p) {
+    const __m256d b0 = _mm256_loadu_pd(bp + kNR * p), b1 = _mm256_loadu_pd(bp + kNR * p + 4);
+    __m256d a = _mm256_broadcast_sd(ap + kMR * p);
+    c00 = _mm256_fmadd_pd(a, b0, c00);
+    c01 = _mm256_fmadd_pd(a, b1, c01);
+    a = _mm256_broadcast_sd(ap + kMR * p + 1);
+    c10 = _mm256_fmadd_pd(a, b0, c10);
+    c11 = _mm256_fmadd_pd(a, b1, c11);
+    a = _mm256_broadcast_sd(ap + kMR * p + 2);
+    c20 = _mm256_fmadd_pd(a, b0, c20);
+    c21 = _mm256_fmadd_pd(a, b1, c21);
+    a = _mm256_broadcast_sd(ap + kMR * p + 3);
+    c30 = _mm256_fmadd_pd(a, b0, c30);
+    c31 = _mm256_fmadd_pd(a, b1, c31);
   }
+  _mm256_storeu_pd(c, c00);
+  _mm256_storeu_pd(c + 4, c01);
+  _mm256_storeu_pd(c + 8, c10);
+  _mm256_storeu_pd(c + 12, c11);
+  _mm256_storeu_pd(c + 16, c20);
+  _mm256_storeu_pd(c + 20, c21);
+  _mm256_storeu_pd(c + 24, c30);
+  _mm256_storeu_pd(c + 28, c31);
+#else
+  for (int i = 0; i < kMR * kNR; ++i) c[i] = 0.0;
+  for (int p = 0; p < kc; ++p)
+    for (int i = 0; i < kMR; ++i)
+      for (int j = 0; j < kNR; ++j) c[i * kNR + j] = std::fma(ap[kMR * p + i], bp[kNR * p + j], c[i * kNR + j]);
+#endif
 }
 
-// Orthonormalise the b columns of row-major X[rows][b] in place (modified
-// Gram-Schmidt, two passes).  A column that vanishes is replaced by a random
-// direction orthogonal to the previous ones.
-void orthonormalize(double* X, int rows, int b, Rng& rng) {
-  std::vector<double> C((size_t)rows * b);
-  for (int r = 0; r < rows; ++r)
-    for (int j = 0; j < b; ++j) C[(size_t)j * rows + r] = X[(size_t)r * b + j];
-  for (int j = 0; j < b; ++j) {
-    double* cj = C.data() + (size_t)j * rows;
-    double n0 = 0.0;
-    for (int r = 0; r < rows; ++r) n0 += cj[r] * cj[r];
-    n0 = std::sqrt(n0);
-    for (int attempt = 0; attempt < 4; ++attempt) {
-      for (int pass = 0; pass < 2; ++pass) {
-        for (int i = 0; i < j; ++i) {
-          const double* ci = C.data() + (size_t)i * rows;
-          double d = 0.0;
-          for (int r = 0; r < rows; ++r) d += ci[r] * cj[r];
-          for (int r = 0; r < rows; ++r) cj[r] -= d * ci[r];
+void gemm(int m, int n, int k, const double* A, size_t ars, size_t acs, const double* B, size_t brs,
+          size_t bcs, double* C, size_t ldc) {
+#pragma omp parallel for schedule(static)
+  for (int i = 0; i < m; ++i) std::fill(C + (size_t)i * ldc, C + (size_t)i * ldc + n, 0.0);
+  if (k <= 0 || m <= 0 || n <= 0) return;
+  const int npan_max = (std::min(n, kNC) + kNR - 1) / kNR;
+  std::vector<double> Bp((size_t)npan_max * kKC * kNR);
+  for (int jc = 0; jc < n; jc += kNC) {
+    const int nc = std::min(kNC, n - jc);
+    const int np = (nc + kNR - 1) / kNR;
+    for (int pc = 0; pc < k; pc += kKC) {
+      const int kc = std::min(kKC, k - pc);
+#pragma omp parallel
+      {
+#pragma omp for schedule(static)
+        for (int jp = 0; jp < np; ++jp) {
+          double* dst = Bp.data() + (size_t)jp * kc * kNR;
+          for (int p = 0; p < kc; ++p)
+            for (int jj = 0; jj < kNR; ++jj) {
+              const int j = jp * kNR + jj;
+              dst[(size_t)p * kNR + jj] = j < nc ? B[(size_t)(pc + p) * brs + (size_t)(jc + j) * bcs] : 0.0;
+            }
+        }
+        std::vector<double> Ap((size_t)kMC * kc);
+        double tile[kMR * kNR];
+#pragma omp for schedule(static)
+        for (int ib = 0; ib < (m + kMC - 1) / kMC; ++ib) {
+          const int ic = ib * kMC, mc = std::min(kMC, m - ic);
+          const int mp = (mc + kMR - 1) / kMR;
+          for (int ip = 0; ip < mp; ++ip)
+            for (int p = 0; p < kc; ++p)
+              for (int ii = 0; ii < kMR; ++ii) {
+                const int i = ip * kMR + ii;
+                Ap[((size_t)ip * kc + p) * kMR + ii] =
+                    i < mc ? A[(size_t)(ic + i) * ars + (size_t)(pc + p) * acs] : 0.0;
+              }
+          for (int jp = 0; jp < np; ++jp)
+            for (int ip = 0; ip < mp; ++ip) {
+              micro_tile(Ap.data() + (size_t)ip * kc * kMR, Bp.data() + (size_t)jp * kc * kNR, kc, tile);
+              const int ie = std::min(kMR, mc - ip * kMR), je = std::min(kNR, nc - jp * kNR);
+              for (int ii = 0; ii < ie; ++ii) {
+                double* c = C + (size_t)(ic + ip * kMR + ii) * ldc + jc + jp * kNR;
+                for (int jj = 0; jj < je; ++jj) c[jj] += tile[ii * kNR + jj];
+              }
+            }
         }
       }
-      double nn = 0.0;
-      for (int r = 0; r < rows; ++r) nn += cj[r] * cj[r];
-      nn = std::sqrt(nn);
-      if (nn > 1e-10 * std::max(n0, 1e-300) && nn > 1e-200) {
-        for (int r = 0; r < rows; ++r) cj[r] /= nn;
-        break;
-      }
-      for (int r = 0; r < rows; ++r) cj[r] = rng.normal();
-      n0 = 0.0;
-      for (int r = 0; r < rows; ++r) n0 += cj[r] * cj[r];
-      n0 = std::sqrt(n0);
     }
   }
-  for (int r = 0; r < rows; ++r)
-    for (int j = 0; j < b; ++j) X[(size_t)r * b + j] = C[(size_t)j * rows + r];
+}
+
+// Orthonormalise the b columns of row-major X[rows][b] in place: classical
+// Gram-Schmidt with one re-orthogonalisation (twice is enough), the inner
+// products summed in fixed row blocks.  A column that vanishes is replaced by
+// a random direction orthogonal to the previous ones.
+void orthonormalize(double* X, int rows, int b, Rng& rng) {
+  std::vector<double> C((size_t)rows * b);
+  const int nch = row_chunks(rows);
+  std::vector<double> part((size_t)nch * (b + 1)), d(b + 1);
+  double n0 = 0.0, nn = 0.0;
+  bool done = false;
+#pragma omp parallel
+  {
+#pragma omp for schedule(static)
+    for (int j = 0; j < b; ++j)
+      for (int r = 0; r < rows; ++r) C[(size_t)j * rows + r] = X[(size_t)r * b + j];
+    for (int j = 0; j < b; ++j) {
+      double* cj = C.data() + (size_t)j * rows;
+#pragma omp for schedule(static)
+      for (int ch = 0; ch < nch; ++ch) {
+        const int r0 = ch * kRowChunk, r1 = std::min(rows, r0 + kRowChunk);
+        part[ch] = dot4(cj + r0, cj + r0, r1 - r0);
+      }
+#pragma omp single
+      {
+        double s = 0.0;
+        for (int ch = 0; ch < nch; ++ch) s += part[ch];
+        n0 = std::sqrt(s);
+        done = false;
+      }
+      for (int attempt = 0; attempt < 4 && !done; ++attempt) {
+        for (int pass = 0; pass < 2; ++pass) {              // c_j -= C_{<j} (C_{<j}^T c_j)
+#pragma omp for schedule(static)
+          for (int ch = 0; ch < nch; ++ch) {
+            const int r0 = ch * kRowChunk, r1 = std::min(rows, r0 + kRowChunk);
+            for (int i = 0; i < j; ++i)
+              part[(size_t)ch * (b + 1) + i] = dot4(C.data() + (size_t)i * rows + r0, cj + r0, r1 - r0);
+          }
+#pragma omp single
+          for (int i = 0; i < j; ++i) {
+            double s = 0.0;
+            for (int ch = 0; ch < nch; ++ch) s += part[(size_t)ch * (b + 1) + i];
+            d[i] = s;
+          }
+#pragma omp for schedule(static)
+          for (int ch = 0; ch < nch; ++ch) {
+            const int r0 = ch * kRowChunk, r1 = std::min(rows, r0 + kRowChunk);
+            for (int i = 0; i < j; ++i) {
+              const double* ci = C.data() + (size_t)i * rows;
+              const double di = d[i];
+              for (int r = r0; r < r1; ++r) cj[r] -= di * ci[r];
+            }
+          }
+        }
+#pragma omp for schedule(static)
+        for (int ch = 0; ch < nch; ++ch) {
+          const int r0 = ch * kRowChunk, r1 = std::min(rows, r0 + kRowChunk);
+          part[ch] = dot4(cj + r0, cj + r0, r1 - r0);
+        }
+#pragma omp single
+        {
+          double s = 0.0;
+          for (int ch = 0; ch < nch; ++ch) s += part[ch];
+          nn = std::sqrt(s);
+          if (nn > 1e-10 * std::max(n0, 1e-300) && nn > 1e-200) {
+            for (int r = 0; r < rows; ++r) cj[r] /= nn;
+            done = true;
+          } else {
+            for (int r = 0; r < rows; ++r) cj[r] = rng.normal();
+            s = 0.0;
+            for (int ch = 0; ch < nch; ++ch) {
+              const int r0 = ch * kRowChunk, r1 = std::min(rows, r0 + kRowChunk);
+              s += dot4(cj + r0, cj + r0, r1 - r0);
+            }
+            n0 = std::sqrt(s);
+          }
+        }
+      }
+    }
+#pragma omp for schedule(static)
+    for (int r = 0; r < rows; ++r)
+      for (int j = 0; j < b; ++j) X[(size_t)r * b + j] = C[(size_t)j * rows + r];
+  }
 }
 
 // Symmetric eigen-decomposition of T[b][b] (cyclic Jacobi).  On return the
-// eigenvalues are in w (descending) and the eigenvectors are the columns of E.
-void sym_eig(std::vector<double> T, int b, std::vector<double>& w, std::vector<double>& E) {
-  E.assign((size_t)b * b, 0.0);
-  for (int i = 0; i < b; ++i) E[(size_t)i * b + i] = 1.0;
+// eigenvalues are in w (descending) and, when `vectors` is set, the
+// eigenvectors are the columns of E.  A rotation in the (p, q) plane rotates
+// rows p and q, mirrors them into columns p and q, and sets the 2 x 2 block
+// from the rotation's tangent t: T'pp = Tpp - t Tpq, T'qq = Tqq + t Tpq,
+// T'pq = 0.  The eigenvectors are kept as rows so that each rotation touches
+// two contiguous rows.
+void sym_eig(std::vector<double> T, int b, std::vector<double>& w, std::vector<double>& E, bool vectors) {
+  std::vector<double> V;
+  if (vectors) {
+    V.assign((size_t)b * b, 0.0);
+    for (int i = 0; i < b; ++i) V[(size_t)i * b + i] = 1.0;
+  }
   auto at = [&](int i, int j) -> double& { return T[(size_t)i * b + j]; };
   for (int sweep = 0; sweep < 100; ++sweep) {
     double off = 0.0, tot = 0.0;
@@ -221,20 +357,30 @@ void sym_eig(std::vector<double> T, int b, std::vector<double>& w, std::vector<d
         const double theta = (at(q, q) - at(p, p)) / (2.0 * apq);
         const double t = (theta >= 0 ? 1.0 : -1.0) / (std::fabs(theta) + std::sqrt(theta * theta + 1.0));
         const double c = 1.0 / std::sqrt(t * t + 1.0), s = t * c;
+        const double app = at(p, p) - t * apq, aqq = at(q, q) + t * apq;
+        double* rp = &at(p, 0);
+        double* rq = &at(q, 0);
         for (int k = 0; k < b; ++k) {
-          const double akp = at(k, p), akq = at(k, q);
-          at(k, p) = c * akp - s * akq;
-          at(k, q) = s * akp + c * akq;
+          const double x = rp[k], y = rq[k];
+          rp[k] = c * x - s * y;
+          rq[k] = s * x + c * y;
         }
+        rp[p] = app;
+        rq[q] = aqq;
+        rp[q] = rq[p] = 0.0;
         for (int k = 0; k < b; ++k) {
-          const double apk = at(p, k), aqk = at(q, k);
-          at(p, k) = c * apk - s * aqk;
-          at(q, k) = s * apk + c * aqk;
+          if (k == p || k == q) continue;
+          at(k, p) = rp[k];
+          at(k, q) = rq[k];
         }
-        for (int k = 0; k < b; ++k) {
-          const double ekp = E[(size_t)k * b + p], ekq = E[(size_t)k * b + q];
-          E[(size_t)k * b + p] = c * ekp - s * ekq;
-          E[(size_t)k * b + q] = s * ekp + c * ekq;
+        if (vectors) {
+          double* vp = V.data() + (size_t)p * b;
+          double* vq = V.data() + (size_t)q * b;
+          for (int k = 0; k < b; ++k) {
+            const double x = vp[k], y = vq[k];
+            vp[k] = c * x - s * y;
+            vq[k] = s * x + c * y;
+          }
         }
       }
   }
@@ -242,77 +388,143 @@ void sym_eig(std::vector<double> T, int b, std::vector<double>& w, std::vector<d
   for (int i = 0; i < b; ++i) idx[i] = i;
   std::sort(idx.begin(), idx.end(), [&](int x, int y) { return at(x, x) > at(y, y); });
   w.resize(b);
-  std::vector<double> E2((size_t)b * b);
-  for (int c = 0; c < b; ++c) {
-    w[c] = at(idx[c], idx[c]);
-    for (int k = 0; k < b; ++k) E2[(size_t)k * b + c] = E[(size_t)k * b + idx[c]];
+  for (int c = 0; c < b; ++c) w[c] = at(idx[c], idx[c]);
+  if (vectors) {
+    E.assign((size_t)b * b, 0.0);
+    for (int c = 0; c < b; ++c)
+      for (int k = 0; k < b; ++k) E[(size_t)k * b + c] = V[(size_t)idx[c] * b + k];
   }
-  E.swap(E2);
 }
 
-// G[b][b] = X^T X for row-major X[rows][b]
-void gram(const double* X, int rows, int b, std::vector<double>& G) {
-  G.assign((size_t)b * b, 0.0);
-  const int nt = 1
-#ifdef _OPENMP
-      * omp_get_max_threads()
-#endif
-      ;
-  std::vector<double> part((size_t)nt * b * b, 0.0);
-#pragma omp parallel
-  {
-    int t = 0;
-#ifdef _OPENMP
-    t = omp_get_thread_num();
-#endif
-    double* g = part.data() + (size_t)t * b * b;
-#pragma omp for schedule(static)
-    for (int r = 0; r < rows; ++r) {
+// G[b][b] = X^T Y for row-major X[rows][b] and Y[rows][b], summed in fixed row
+// blocks.
+void gram_xy(const double* X, const double* Y, int rows, int b, std::vector<double>& G) {
+  const int nch = row_chunks(rows);
+  std::vector<double> part((size_t)nch * b * b, 0.0);
+#pragma omp parallel for schedule(static)
+  for (int ch = 0; ch < nch; ++ch) {
+    double* g = part.data() + (size_t)ch * b * b;
+    const int r0 = ch * kRowChunk, r1 = std::min(rows, r0 + kRowChunk);
+    for (int r = r0; r < r1; ++r) {
       const double* x = X + (size_t)r * b;
+      const double* y = Y + (size_t)r * b;
       for (int i = 0; i < b; ++i) {
         const double xi = x[i];
-        for (int j = 0; j < b; ++j) g[(size_t)i * b + j] += xi * x[j];
+        for (int j = 0; j < b; ++j) g[(size_t)i * b + j] += xi * y[j];
       }
     }
   }
-  for (int t = 0; t < nt; ++t)
-    for (size_t i = 0; i < (size_t)b * b; ++i) G[i] += part[(size_t)t * b * b + i];
+  G.assign((size_t)b * b, 0.0);
+  for (int ch = 0; ch < nch; ++ch)
+    for (size_t i = 0; i < (size_t)b * b; ++i) G[i] += part[(size_t)ch * b * b + i];
 }
 
 // Top-r SVD of A[K][N]: L1 = U Sigma[:, :r] ([K][r]), L2 = V^T[:r, :] ([r][N]).
+//
+// Block subspace iteration (block b = r + 32): Q = orth(A Z), Z = orth(A^T Q),
+// with the Ritz values of B B^T (B = Q^T A) after every step; it stops when
+// the captured energy sum_{i<r} sigma_i^2 stops changing.  The energy settles
+// like (sigma_{b+1} / sigma_r)^(2t), which is slow when the spectrum is flat
+// around sigma_r.  When the observed rate says the remaining steps on A cost
+// more than forming the Gram matrix of the smaller side (G = A^T A or A A^T,
+// min(K, N)^2 entries) and stepping on it (2 min(K,N)^2 b flops a step against
+// 4 K N b), the iteration moves to G.  The last step and the extraction run on
+// A itself, so the factors keep the accuracy of the plain iteration.
 svdq_status truncated_svd(const std::vector<double>& A, int K, int N, int r,
                           std::vector<double>& L1, std::vector<double>& L2,
                           std::vector<double>& sigma, int& iters, double& tail) {
+  constexpr double kTol = 1e-13;                        // relative change of the energy
+  constexpr int kMaxSteps = 300, kMaxGramSteps = 1000;
   const int b = std::min(std::min(r + 32, K), N);
   const int re = std::min(r, b);                        // directions beyond rank(A) stay zero
   Rng rng(0x5EED5EEDull);
   std::vector<double> Z((size_t)N * b), Zraw((size_t)N * b), Q((size_t)K * b), T, w, E;
   for (auto& z : Z) z = rng.normal();
   orthonormalize(Z.data(), N, b, rng);
-  double prev = -1.0, energy = 0.0;
-  bool converged = false;
   const bool exact_block = (b == std::min(K, N));      // the block spans the whole range
-  const int max_iter = 300;
-  int it = 0;
-  for (; it < max_iter; ++it) {
-    gemm_AZ(A.data(), K, N, Z.data(), b, Q.data());     // Q <- A Z
-    orthonormalize(Q.data(), K, b, rng);
-    gemm_AtQ(A.data(), K, N, Q.data(), b, Zraw.data()); // Zraw <- A^T Q  (= B^T, B = Q^T A)
-    gram(Zraw.data(), N, b, T);                         // B B^T
-    sym_eig(T, b, w, E);
-    energy = 0.0;
-    for (int i = 0; i < re; ++i) energy += std::max(w[i], 0.0);
-    if (exact_block || (it >= 3 && std::fabs(energy - prev) <= 1e-13 * energy)) {
+  auto top_energy = [&]() {
+    double e = 0.0;
+    for (int i = 0; i < re; ++i) e += std::max(w[i], 0.0);
+    return e;
+  };
+  auto step_on_A = [&](bool from_Z) {
+    if (from_Z) {
+      gemm(K, b, N, A.data(), N, 1, Z.data(), b, 1, Q.data(), b);    // Q <- A Z
+      orthonormalize(Q.data(), K, b, rng);
+    }
+    gemm(N, b, K, A.data(), 1, N, Q.data(), b, 1, Zraw.data(), b);   // Zraw <- A^T Q (= B^T)
+    gram_xy(Zraw.data(), Zraw.data(), N, b, T);                       // B B^T
+    sym_eig(T, b, w, E, false);
+  };
+  const int ns = std::min(K, N);
+  const double cost_a = 4.0 * K * N * b, cost_g = 2.0 * ns * ns * b, cost_form = 2.0 * ns * ns * std::max(K, N);
+  double prev = -1.0, delta_prev = -1.0, energy = 0.0;
+  bool converged = false, to_gram = false;
+  int steps = 0;
+  for (int it = 0; it < kMaxSteps; ++it) {
+    step_on_A(true);
+    ++steps;
+    energy = top_energy();
+    if (exact_block || (it >= 3 && std::fabs(energy - prev) <= kTol * energy)) {
       converged = true;
       break;
     }
+    const double delta = std::fabs(energy - prev);
+    if (it >= 4 && delta_prev > 0.0) {
+      const double rho = delta / delta_prev;
+      const double left = (rho > 0.0 && rho < 1.0) ? std::log(kTol * energy / delta) / std::log(rho) : 1e30;
+      to_gram = left * (cost_a - cost_g) > cost_form;
+    }
+    delta_prev = it >= 1 ? delta : -1.0;
     prev = energy;
+    if (to_gram) break;
     Z = Zraw;
     orthonormalize(Z.data(), N, b, rng);
   }
-  iters = std::min(it + 1, max_iter);
+  if (to_gram) {
+    // Gram of the smaller side, started from the basis on that side
+    const bool right = N <= K;
+    std::vector<double> G((size_t)ns * ns), S, Y((size_t)ns * b);
+    if (right) {
+      gemm(N, N, K, A.data(), 1, N, A.data(), N, 1, G.data(), N);   // A^T A
+      S = Zraw;
+    } else {
+      gemm(K, K, N, A.data(), N, 1, A.data(), 1, N, G.data(), K);   // A A^T
+      S = Q;
+    }
+    orthonormalize(S.data(), ns, b, rng);
+    double gprev = -1.0;
+    for (int it = 0; it < kMaxGramSteps; ++it) {
+      gemm(ns, b, ns, G.data(), ns, 1, S.data(), b, 1, Y.data(), b);   // Y <- G S
+      ++steps;
+      gram_xy(S.data(), Y.data(), ns, b, T);                          // S^T G S
+      sym_eig(T, b, w, E, false);
+      energy = top_energy();
+      if (it >= 1 && std::fabs(energy - gprev) <= kTol * energy) {
+        converged = true;
+        break;
+      }
+      prev = gprev = energy;
+      S = Y;
+      orthonormalize(S.data(), ns, b, rng);
+    }
+    // last step and Rayleigh-Ritz on A
+    if (right) {
+      Z = Y;
+      orthonormalize(Z.data(), N, b, rng);
+      step_on_A(true);
+    } else {
+      Q = Y;
+      orthonormalize(Q.data(), K, b, rng);
+      step_on_A(false);
+    }
+    ++steps;
+    energy = top_energy();
+  }
+  iters = steps;
   if (!converged && std::fabs(energy - prev) > 1e-8 * std::max(energy, 1e-300))
     return SVDQ_ENOCONVERGE;
+  sym_eig(T, b, w, E, true);
   const std::vector<double>& Zf = Zraw;
   // Rayleigh-Ritz: B = Q^T A = Z^T, B B^T = E diag(w) E^T.
   // U = Q E, sigma = sqrt(w), V^T rows = E^T B / sigma = (Z E)^T / sigma.
@@ -334,9 +546,16 @@ svdq_status truncated_svd(const std::vector<double>& A, int K, int N, int r,
       for (int j = 0; j < b; ++j) v += Zf[(size_t)n * b + j] * E[(size_t)j * b + i];
       L2[(size_t)i * N + n] = sigma[i] > 0 ? v / sigma[i] : 0.0;
     }
+  const int nch = row_chunks(K);
+  std::vector<double> part(nch);
+#pragma omp parallel for schedule(static)
+  for (int ch = 0; ch < nch; ++ch) {
+    const int r0 = ch * kRowChunk, r1 = std::min(K, r0 + kRowChunk);
+    const double* a = A.data() + (size_t)r0 * N;
+    part[ch] = dot4(a, a, (r1 - r0) * N);
+  }
   double total = 0.0;
-#pragma omp parallel for reduction(+ : total) schedule(static)
-  for (size_t i = 0; i < A.size(); ++i) total += A[i] * A[i];
+  for (int ch = 0; ch < nch; ++ch) total += part[ch];
   double kept = 0.0;
   for (int i = 0; i < r; ++i) kept += sigma[i] * sigma[i];
   tail = total - kept;
