@@ -278,9 +278,9 @@ svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, v
  * bytes: NVFP4 E4M3 in the tensor-core layout, INT4 BF16 [K/64][M rounded up
  * to 128], group-major, W8A8 FP32 [s_x | 1/s_x], each M rounded up to 128
  * entries; padding rows zero) and, when
- * the layer has a branch, XL = bf16(X L1d) (device [M][rank] BF16; [M][64]
- * with a LoRA adapter, see svdq_set_lora).  xl may be NULL for rank 0 without
- * an adapter.  `mode` 0 = fused, 1 = quantize only, 2 = down projection only. */
+ * the layer has a branch, XL = bf16(X L1d) (device [M][32] BF16 whatever the
+ * rank: X L1d in the first `rank` columns, zeros after; [M][64] with a LoRA
+ * adapter, see svdq_set_lora).  xl may be NULL for rank 0 without an adapter.  `mode` 0 = fused, 1 = quantize only, 2 = down projection only. */
 svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int M,
                               void* codes, void* scales, void* xl,
                               void* stream, int mode);

@@ -7,7 +7,11 @@ the offline preparation, CUDA kernels for the forward).  There is no fallback:
 if the library is missing, importing ``lib`` raises.
 
 Device memory and streams come from the caller (for example PyTorch tensors:
-anything with ``data_ptr()``, or raw integer addresses).
+anything with ``data_ptr()``, or raw integer addresses).  PyTorch tensors and
+NumPy arrays are checked before the call: a device operand must be a
+contiguous CUDA tensor, a host operand host memory, and each must hold at
+least the bytes the call reads or writes (``ValueError`` otherwise).  Raw
+addresses and other objects are passed through unchecked.
 """
 from __future__ import annotations
 
@@ -129,6 +133,32 @@ def _ptr(x) -> Optional[int]:
     raise TypeError(f"cannot take the address of {type(x)}")
 
 
+def _held_bytes(x, what: str, device: bool) -> Optional[int]:
+    """Bytes held by a tensor or array argument after checking where it lives
+    and that it is contiguous; None for raw addresses and unknown objects."""
+    if x is None or isinstance(x, int):
+        return None
+    if isinstance(x, np.ndarray):
+        if device:
+            raise ValueError(f"{what}: a NumPy array is host memory; this operand is a device buffer")
+        if not x.flags.c_contiguous:
+            raise ValueError(f"{what}: not contiguous")
+        return int(x.nbytes)
+    if hasattr(x, "is_cuda") and hasattr(x, "numel"):
+        if bool(x.is_cuda) != device:
+            raise ValueError(f"{what}: must be a {'CUDA' if device else 'host'} tensor")
+        if not x.is_contiguous():
+            raise ValueError(f"{what}: not contiguous")
+        return int(x.numel()) * int(x.element_size())
+    return None
+
+
+def _need(x, nbytes: int, what: str, device: bool = True):
+    have = _held_bytes(x, what, device)
+    if have is not None and have < nbytes:
+        raise ValueError(f"{what}: holds {have} bytes, the call accesses {nbytes}")
+
+
 def _stream(s) -> Optional[int]:
     if s is None:
         return None
@@ -147,6 +177,13 @@ class Layer:
 
     def __init__(self, handle: int):
         self._h = ctypes.c_void_p(handle)
+        info = self.info
+        self._K, self._N = info["K"], info["N"]
+        self._xl_cols = self._xl_width()
+
+    def _xl_width(self) -> int:
+        # XL is [M][32] BF16 (zeros past the rank); [M][64] with a LoRA adapter
+        return 64 if load().svdq_tensor_bytes(self._h, TENSORS["lora_A"][0]) else 32
 
     @classmethod
     def prepare(cls, W_bits: np.ndarray, bias_bits: Optional[np.ndarray], calib_bits: Optional[np.ndarray],
@@ -156,9 +193,15 @@ class Layer:
         calib_bits: uint16 [M_calib][K] or None (W4A16); flags: PREP_* bits."""
         L = load()
         W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+        if W.ndim != 2:
+            raise ValueError(f"W_bits must be [K][N], got shape {W.shape}")
         K, N = W.shape
         b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
         c = None if calib_bits is None else np.ascontiguousarray(calib_bits, dtype=np.uint16)
+        if b is not None and b.size != N:
+            raise ValueError(f"bias_bits must hold N = {N} values, got shape {b.shape}")
+        if c is not None and (c.ndim != 2 or c.shape[1] != K):
+            raise ValueError(f"calib_bits must be [M_calib][K = {K}], got shape {c.shape}")
         cfg = Config(FORMATS[fmt], rank, alpha, flags)
         out = ctypes.c_void_p()
         st = L.svdq_prepare(ctypes.byref(cfg), K, N, _ptr(W), _ptr(b), _ptr(c),
@@ -217,14 +260,20 @@ class Layer:
         """Attach a LoRA adapter W -> W + scale A B (A_bits uint16 [K][r], B_bits
         uint16 [r][N], BF16 patterns) to the low-rank branch; None removes it."""
         if A_bits is None:
-            _check(load().svdq_set_lora(self._h, 0, None, None, 0.0), "svdq_set_lora")
+            try:
+                _check(load().svdq_set_lora(self._h, 0, None, None, 0.0), "svdq_set_lora")
+            finally:
+                self._xl_cols = self._xl_width()
             return
         A = np.ascontiguousarray(A_bits, dtype=np.uint16)
         B = np.ascontiguousarray(B_bits, dtype=np.uint16)
+        if A.ndim != 2 or B.ndim != 2 or A.shape[0] != self._K or B.shape != (A.shape[1], self._N):
+            raise ValueError(f"A is [K = {self._K}][r] and B is [r][N = {self._N}]; got {A.shape} and {B.shape}")
         r = A.shape[1]
-        if B.shape[0] != r:
-            raise ValueError("A is [K][r] and B is [r][N]")
-        _check(load().svdq_set_lora(self._h, r, _ptr(A), _ptr(B), float(scale)), "svdq_set_lora")
+        try:
+            _check(load().svdq_set_lora(self._h, r, _ptr(A), _ptr(B), float(scale)), "svdq_set_lora")
+        finally:
+            self._xl_cols = self._xl_width()
 
     def workspace_bytes(self, M: int) -> int:
         return int(load().svdq_workspace_bytes(self._h, M))
@@ -244,24 +293,44 @@ class Layer:
         else:
             out = np.empty((M, info["K"] // 2), dtype=np.uint8)
         src = np.ascontiguousarray(device_layout, dtype=np.uint8)
+        _need(src, self.act_code_bytes(M), "device_layout", device=False)
         _check(load().svdq_act_codes_to_logical(self._h, _ptr(src), M, _ptr(out)), "svdq_act_codes_to_logical")
         return out
 
+    def _need_act(self, M: int, X=None, Y=None, codes=None, scales=None, xl=None):
+        if M <= 0:
+            return                     # the library answers M <= 0 itself
+        if X is not None:
+            _need(X, M * self._K * 2, "X")
+        if Y is not None:
+            _need(Y, M * self._N * 2, "Y")
+        if codes is not None:
+            _need(codes, self.act_code_bytes(M), "codes")
+        if scales is not None:
+            _need(scales, self.act_scale_bytes(M), "scales")
+        if xl is not None:
+            _need(xl, M * self._xl_cols * 2, "xl")
+
     def forward(self, X, M: int, Y, workspace, workspace_bytes: int, stream=None, flags: int = 0):
+        self._need_act(M, X=X, Y=Y)
+        _need(workspace, workspace_bytes, "workspace")
         _check(load().svdq_linear_forward(self._h, _ptr(X), M, _ptr(Y), _ptr(workspace), workspace_bytes,
                                           _stream(stream), flags), "svdq_linear_forward")
 
     def forward_static(self, X, M: int, Y, stream=None, flags: int = 0):
         """Forward with the library's built-in device workspace (no caller workspace,
         no allocation); see svdq_linear_forward_static in include/svdq.h."""
+        self._need_act(M, X=X, Y=Y)
         _check(load().svdq_linear_forward_static(self._h, _ptr(X), M, _ptr(Y), _stream(stream), flags),
                "svdq_linear_forward_static")
 
     def quantize_act(self, X, M: int, codes, scales, xl, stream=None, mode: int = 0):
+        self._need_act(M, X=X, codes=codes, scales=scales, xl=xl)
         _check(load().svdq_quantize_act(self._h, _ptr(X), M, _ptr(codes), _ptr(scales), _ptr(xl),
                                         _stream(stream), mode), "svdq_quantize_act")
 
     def gemm(self, codes, scales, xl, M: int, Y, stream=None, flags: int = 0):
+        self._need_act(M, Y=Y, codes=codes, scales=scales, xl=xl)
         _check(load().svdq_gemm(self._h, _ptr(codes), _ptr(scales), _ptr(xl), M, _ptr(Y), _stream(stream),
                                 flags), "svdq_gemm")
 
@@ -276,6 +345,7 @@ class Layer:
         else:
             out = np.empty((M, info["K"] // 16), dtype=np.uint8)
         src = np.ascontiguousarray(device_layout, dtype=np.uint8)
+        _need(src, self.act_scale_bytes(M), "device_layout", device=False)
         _check(load().svdq_act_scales_to_logical(self._h, _ptr(src), M, _ptr(out)), "svdq_act_scales_to_logical")
         return out
 
@@ -298,6 +368,11 @@ def mlp_workspace_bytes(fc1: Layer, fc2: Layer, M: int, flags: int = 0) -> int:
 def mlp_fc1(fc1: Layer, fc2: Layer, X, M: int, codes2, scales2, xl2, workspace, workspace_bytes: int,
             stream=None, flags: int = 0):
     """fc1 with its output handed to fc2 already quantized (svdq_mlp_fc1)."""
+    fc1._need_act(M, X=X)
+    if M > 0 and xl2 is not None:
+        _need(xl2, M * 32 * 2, "xl2")
+    fc2._need_act(M, codes=codes2, scales=scales2)
+    _need(workspace, workspace_bytes, "workspace")
     _check(load().svdq_mlp_fc1(fc1._h, fc2._h, _ptr(X), M, _ptr(codes2), _ptr(scales2), _ptr(xl2),
                                _ptr(workspace), workspace_bytes, _stream(stream), flags), "svdq_mlp_fc1")
 
@@ -305,5 +380,8 @@ def mlp_fc1(fc1: Layer, fc2: Layer, X, M: int, codes2, scales2, xl2, workspace, 
 def mlp_forward(fc1: Layer, fc2: Layer, X, M: int, Y, workspace, workspace_bytes: int, stream=None,
                 flags: int = 0):
     """fc1 -> [GELU] -> fc2 (svdq_mlp_forward)."""
+    fc1._need_act(M, X=X)
+    fc2._need_act(M, Y=Y)
+    _need(workspace, workspace_bytes, "workspace")
     _check(load().svdq_mlp_forward(fc1._h, fc2._h, _ptr(X), M, _ptr(Y), _ptr(workspace), workspace_bytes,
                                    _stream(stream), flags), "svdq_mlp_forward")
