@@ -164,12 +164,13 @@ typedef enum {
  *   out        receives the new layer; owned by the caller, free with svdq_destroy.
  *
  * Runs on the host (multi-threaded), then copies the prepared buffers to
- * `device` with blocking copies.  Errors: SVDQ_EINVAL, SVDQ_EUNSUPPORTED (shape
+ * `device` with blocking copies.  Errors: SVDQ_EINVAL (also for a NaN or an
+ * infinity in W, the bias or the calibration batch), SVDQ_EUNSUPPORTED (shape
  * rules; for SVDQ_NVFP4 also a calibration batch whose largest smoothed
  * magnitude puts the activation tensor-scale exponent outside [-40, 30], i.e.
  * below about 3e-10 or above about 7e11), SVDQ_ENOMEM, SVDQ_ECUDA,
  * SVDQ_ENOCONVERGE (the SVD's energy check failed, or the GPTQ Hessian was
- * not positive definite after damping -- only with non-finite calibration).
+ * not positive definite after damping).
  * On error *out is set to NULL and nothing leaks. */
 svdq_status svdq_prepare(const svdq_config* cfg, int K, int N,
                          const uint16_t* W_bf16, const uint16_t* bias_bf16,

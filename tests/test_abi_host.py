@@ -206,3 +206,20 @@ def test_rank_above_matrix_rank():
     assert np.all(L1[:, 16:] == 0) and np.all(L2[16:] == 0)
     lam = L.export("lambda").astype(np.float64)
     np.testing.assert_allclose(L1 @ L2, lam[:, None] * d["W"], rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("where", ["W", "bias", "calib"])
+@pytest.mark.parametrize("bits", [0x7FC0, 0x7F80, 0xFF80])          # NaN, +inf, -inf
+def test_prepare_refuses_non_finite_inputs(where, bits):
+    import time
+    d = syn.custom_layer(17, M=8, K=256, N=128)
+    W, b, Xc = syn.bf16_bits(d["W"]).copy(), syn.bf16_bits(d["bias"]).copy(), syn.bf16_bits(d["Xc"]).copy()
+    {"W": W, "bias": b, "calib": Xc}[where].reshape(-1)[37] = bits
+    t = time.perf_counter()
+    with pytest.raises(lib.SvdqError) as e:
+        lib.Layer.prepare(W, b, Xc, device=-1)
+    assert e.value.status == lib.EINVAL
+    assert time.perf_counter() - t < 5.0                             # refused before any iteration
+    if where == "calib":                                            # weight-only layers ignore the batch
+        L = lib.Layer.prepare(W, b, Xc, fmt="w4a16", rank=0, device=-1)
+        assert L.info["rank"] == 0

@@ -880,6 +880,16 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
                          HostPrep& P) {
   try {
     const bool w4a16 = cfg.format == SVDQ_W4A16_INT4;
+    // NaN or infinity anywhere in the inputs (all exponent bits set) would only
+    // stall the iterations below: refuse it up front.
+    auto finite = [](const uint16_t* p, size_t n) {
+      for (size_t i = 0; i < n; ++i)
+        if ((p[i] & 0x7F80u) == 0x7F80u) return false;
+      return true;
+    };
+    if (!finite(W, (size_t)K * N) || (bias && !finite(bias, (size_t)N)) ||
+        (!w4a16 && calib && !finite(calib, (size_t)M_calib * K)))
+      return SVDQ_EINVAL;
     P.K = K; P.N = N; P.format = cfg.format;
     P.rank = w4a16 ? 0 : cfg.rank;
     P.alpha = cfg.alpha;
