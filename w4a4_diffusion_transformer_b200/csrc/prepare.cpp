@@ -193,6 +193,76 @@ inline void micro_tile(const double* ap, const double* bp, int kc, double* c) {
 #endif
 }
 
+// Pack op(A)[i0, i0+mc) x [p0, p0+kc) into kMR-row micro-panels Ap[ip][p][kMR]
+// (zero rows past mc).
+void pack_a(const double* A, size_t ars, size_t acs, int i0, int mc, int p0, int kc, double* Ap) {
+  const int mp = (mc + kMR - 1) / kMR;
+  for (int ip = 0; ip < mp; ++ip)
+    for (int p = 0; p < kc; ++p)
+      for (int ii = 0; ii < kMR; ++ii) {
+        const int i = ip * kMR + ii;
+        Ap[((size_t)ip * kc + p) * kMR + ii] = i < mc ? A[(size_t)(i0 + i) * ars + (size_t)(p0 + p) * acs] : 0.0;
+      }
+}
+
+// Pack micro-panels [jp0, jp1) of op(B)[p0, p0+kc) x [j0, j0+nc) into
+// Bp[jp][p][kNR] (zero columns past nc).
+void pack_b(const double* B, size_t brs, size_t bcs, int p0, int kc, int j0, int nc, int jp0, int jp1,
+            double* Bp) {
+  for (int jp = jp0; jp < jp1; ++jp) {
+    double* dst = Bp + (size_t)jp * kc * kNR;
+    for (int p = 0; p < kc; ++p)
+      for (int jj = 0; jj < kNR; ++jj) {
+        const int j = jp * kNR + jj;
+        dst[(size_t)p * kNR + jj] = j < nc ? B[(size_t)(p0 + p) * brs + (size_t)(j0 + j) * bcs] : 0.0;
+      }
+  }
+}
+
+// C[0, mc) x [0, nc) += (or -=) Ap Bp over one packed slice of depth kc.
+void slice_tiles(const double* Ap, int mc, const double* Bp, int nc, int kc, bool subtract, double* C,
+                 size_t ldc) {
+  double tile[kMR * kNR];
+  const int mp = (mc + kMR - 1) / kMR, np = (nc + kNR - 1) / kNR;
+  for (int jp = 0; jp < np; ++jp)
+    for (int ip = 0; ip < mp; ++ip) {
+      micro_tile(Ap + (size_t)ip * kc * kMR, Bp + (size_t)jp * kc * kNR, kc, tile);
+      const int ie = std::min(kMR, mc - ip * kMR), je = std::min(kNR, nc - jp * kNR);
+      for (int ii = 0; ii < ie; ++ii) {
+        double* c = C + (size_t)(ip * kMR + ii) * ldc + jp * kNR;
+        if (subtract)
+          for (int jj = 0; jj < je; ++jj) c[jj] -= tile[ii * kNR + jj];
+        else
+          for (int jj = 0; jj < je; ++jj) c[jj] += tile[ii * kNR + jj];
+      }
+    }
+}
+
+// C = op(A) op(B) on the calling thread alone (for use inside parallel tasks);
+// with `update` set, C -= op(A) op(B) instead.  Ap and Bp are scratch.
+void gemm_serial(int m, int n, int k, const double* A, size_t ars, size_t acs, const double* B, size_t brs,
+                 size_t bcs, double* C, size_t ldc, bool update, std::vector<double>& Ap,
+                 std::vector<double>& Bp) {
+  if (!update)
+    for (int i = 0; i < m; ++i) std::fill(C + (size_t)i * ldc, C + (size_t)i * ldc + n, 0.0);
+  if (k <= 0 || m <= 0 || n <= 0) return;
+  for (int ic = 0; ic < m; ic += kMC) {
+    const int mc = std::min(kMC, m - ic);
+    for (int jc = 0; jc < n; jc += kNC) {
+      const int nc = std::min(kNC, n - jc);
+      for (int pc = 0; pc < k; pc += kKC) {
+        const int kc = std::min(kKC, k - pc);
+        Ap.resize((size_t)kMC * kc);
+        Bp.resize((size_t)((nc + kNR - 1) / kNR) * kc * kNR);
+        pack_a(A, ars, acs, ic, mc, pc, kc, Ap.data());
+        pack_b(B, brs, bcs, pc, kc, jc, nc, 0, (nc + kNR - 1) / kNR, Bp.data());
+        slice_tiles(Ap.data(), mc, Bp.data(), nc, kc, update, C + (size_t)ic * ldc + jc, ldc);
+      }
+    }
+  }
+}
+
+// C[m][n] = op(A) op(B), the row blocks of C spread over the threads.
 void gemm(int m, int n, int k, const double* A, size_t ars, size_t acs, const double* B, size_t brs,
           size_t bcs, double* C, size_t ldc) {
 #pragma omp parallel for schedule(static)
@@ -208,36 +278,13 @@ void gemm(int m, int n, int k, const double* A, size_t ars, size_t acs, const do
 #pragma omp parallel
       {
 #pragma omp for schedule(static)
-        for (int jp = 0; jp < np; ++jp) {
-          double* dst = Bp.data() + (size_t)jp * kc * kNR;
-          for (int p = 0; p < kc; ++p)
-            for (int jj = 0; jj < kNR; ++jj) {
-              const int j = jp * kNR + jj;
-              dst[(size_t)p * kNR + jj] = j < nc ? B[(size_t)(pc + p) * brs + (size_t)(jc + j) * bcs] : 0.0;
-            }
-        }
+        for (int jp = 0; jp < np; ++jp) pack_b(B, brs, bcs, pc, kc, jc, nc, jp, jp + 1, Bp.data());
         std::vector<double> Ap((size_t)kMC * kc);
-        double tile[kMR * kNR];
 #pragma omp for schedule(static)
         for (int ib = 0; ib < (m + kMC - 1) / kMC; ++ib) {
           const int ic = ib * kMC, mc = std::min(kMC, m - ic);
-          const int mp = (mc + kMR - 1) / kMR;
-          for (int ip = 0; ip < mp; ++ip)
-            for (int p = 0; p < kc; ++p)
-              for (int ii = 0; ii < kMR; ++ii) {
-                const int i = ip * kMR + ii;
-                Ap[((size_t)ip * kc + p) * kMR + ii] =
-                    i < mc ? A[(size_t)(ic + i) * ars + (size_t)(pc + p) * acs] : 0.0;
-              }
-          for (int jp = 0; jp < np; ++jp)
-            for (int ip = 0; ip < mp; ++ip) {
-              micro_tile(Ap.data() + (size_t)ip * kc * kMR, Bp.data() + (size_t)jp * kc * kNR, kc, tile);
-              const int ie = std::min(kMR, mc - ip * kMR), je = std::min(kNR, nc - jp * kNR);
-              for (int ii = 0; ii < ie; ++ii) {
-                double* c = C + (size_t)(ic + ip * kMR + ii) * ldc + jc + jp * kNR;
-                for (int jj = 0; jj < je; ++jj) c[jj] += tile[ii * kNR + jj];
-              }
-            }
+          pack_a(A, ars, acs, ic, mc, pc, kc, Ap.data());
+          slice_tiles(Ap.data(), mc, Bp.data(), nc, kc, false, C + (size_t)ic * ldc + jc, ldc);
         }
       }
     }
@@ -671,11 +718,13 @@ void gptq_hessian(const uint16_t* calib, int M, int K, const std::vector<float>&
 // and the cores.  With J the order reversal, P = J H J = L L^T (lower
 // Cholesky), so H = T T^T with T = J L J upper and U = T^-1 = J L^-1 J.
 //   * L: right-looking blocked Cholesky of P in place (the diagonal block by
-//     the textbook loop, the panel by a triangular solve, the trailing matrix
-//     by block products in parallel);
-//   * L^-1: column blocks in parallel, each solved block row by block row.
-// false if a pivot is not positive (non-finite calibration).
-constexpr int kFactorBlock = 64;
+//     the textbook loop, the panel by a triangular solve, the trailing lower
+//     triangle by packed block products, one block pair per task);
+//   * X = L^-1: one block column per task; each block row takes the product
+//     of L's row block with the rows of X above it (a packed product), then a
+//     forward substitution through L's diagonal block.
+// false if a pivot is not positive.
+constexpr int kFactorBlock = 128;
 
 bool gptq_factor(const std::vector<double>& H, int K, std::vector<double>& U) {
   const int B = kFactorBlock;
@@ -686,10 +735,9 @@ bool gptq_factor(const std::vector<double>& H, int K, std::vector<double>& U) {
   for (int i = 0; i < K; ++i)
     for (int j = 0; j < K; ++j) P[(size_t)i * K + j] = H[(size_t)(K - 1 - i) * K + (K - 1 - j)];
   auto at = [&](int i, int j) -> double& { return P[(size_t)i * K + j]; };
-  std::vector<double> Lt((size_t)B * K);            // the current panel, transposed
   bool ok = true;
   for (int kb = 0; kb < nb && ok; ++kb) {
-    const int k0 = kb * B, k1 = std::min(K, k0 + B);
+    const int k0 = kb * B, k1 = std::min(K, k0 + B), w = k1 - k0;
     // diagonal block
     for (int j = k0; j < k1 && ok; ++j) {
       double d = at(j, j);
@@ -715,58 +763,55 @@ bool gptq_factor(const std::vector<double>& H, int K, std::vector<double>& U) {
         for (int k = k0; k < j; ++k) v -= at(i, k) * at(j, k);
         at(i, j) = v / at(j, j);
       }
-    // trailing update of the lower triangle: P[i, j] -= sum_k L[i, k] L[j, k],
-    // as row updates P[i, j0:j1] -= L[i, k] Lt[k, j0:j1] over a transposed copy
-    // of the panel, so the inner loop runs along contiguous columns
+    // trailing lower triangle: P[I, J] -= L[I, k0:k1] L[J, k0:k1]^T for block
+    // rows I and block columns J <= I (a diagonal block is updated whole; its
+    // upper part is never read)
     const int rem = nb - kb - 1;
     if (rem > 0) {
-      const int w = k1 - k0;
-#pragma omp parallel for schedule(static)
-      for (int j = k1; j < K; ++j)
-        for (int k = 0; k < w; ++k) Lt[(size_t)k * K + j] = at(j, k0 + k);
-#pragma omp parallel for schedule(dynamic, 1)
-      for (int t = 0; t < rem * (rem + 1) / 2; ++t) {
-        int ib = 0;
-        while ((ib + 1) * (ib + 2) / 2 <= t) ++ib;     // block row ib, block column jb <= ib
-        const int jb = t - ib * (ib + 1) / 2;
-        const int i0 = k1 + ib * B, i1 = std::min(K, i0 + B);
-        const int j0 = k1 + jb * B, j1 = std::min(K, j0 + B);
-        for (int i = i0; i < i1; ++i) {
-          double* pi = &P[(size_t)i * K];
-          const int je = std::min(j1, i + 1);
-          for (int k = 0; k < w; ++k) {
-            const double lik = pi[k0 + k];
-            const double* lt = &Lt[(size_t)k * K];
-            for (int j = j0; j < je; ++j) pi[j] -= lik * lt[j];
-          }
+#pragma omp parallel
+      {
+        std::vector<double> Ap, Bp;
+#pragma omp for schedule(dynamic, 1)
+        for (int t = 0; t < rem * (rem + 1) / 2; ++t) {
+          int ib = 0;
+          while ((ib + 1) * (ib + 2) / 2 <= t) ++ib;     // block row ib, block column jb <= ib
+          const int jb = t - ib * (ib + 1) / 2;
+          const int i0 = k1 + ib * B, i1 = std::min(K, i0 + B);
+          const int j0 = k1 + jb * B, j1 = std::min(K, j0 + B);
+          gemm_serial(i1 - i0, j1 - j0, w, &P[(size_t)i0 * K + k0], K, 1, &P[(size_t)j0 * K + k0], 1, K,
+                      &P[(size_t)i0 * K + j0], K, true, Ap, Bp);
         }
       }
     }
   }
   if (!ok) return false;
-  // X = L^-1 (lower), one block of B columns per task: rows i >= j0 of the
-  // block by forward substitution, X[i][c] = (delta_ic - sum_{k<i} L[i][k]
-  // X[k][c]) / L[i][i], in a private row-major [K][B] buffer so that the
-  // update runs along contiguous rows; then U = J X J.
   U.assign((size_t)K * K, 0.0);
 #pragma omp parallel
   {
-    std::vector<double> W((size_t)K * B);
+    std::vector<double> X, Ap, Bp;
 #pragma omp for schedule(dynamic, 1)
     for (int jb = 0; jb < nb; ++jb) {
       const int j0 = jb * B, w = std::min(K, j0 + B) - j0;
-      for (int i = j0; i < K; ++i) {
-        double* wi = &W[(size_t)(i - j0) * B];
-        for (int c = 0; c < w; ++c) wi[c] = (i == j0 + c) ? 1.0 : 0.0;
-        const double* li = &P[(size_t)i * K];
-        for (int k = j0; k < i; ++k) {
-          const double lik = li[k];
-          const double* wk = &W[(size_t)(k - j0) * B];
-          for (int c = 0; c < w; ++c) wi[c] -= lik * wk[c];
+      X.assign((size_t)(K - j0) * w, 0.0);               // rows j0.., row-major [K - j0][w]
+      for (int ib = jb; ib < nb; ++ib) {
+        const int i0 = ib * B, i1 = std::min(K, i0 + B);
+        double* xi0 = &X[(size_t)(i0 - j0) * w];
+        // S = L[i0:i1, j0:i0] X[j0:i0, :], kept negated in the rows' slots
+        if (i0 > j0)
+          gemm_serial(i1 - i0, w, i0 - j0, &P[(size_t)i0 * K + j0], K, 1, X.data(), w, 1, xi0, w, true, Ap, Bp);
+        for (int i = i0; i < i1; ++i) {
+          double* xr = &X[(size_t)(i - j0) * w];
+          if (i - j0 < w) xr[i - j0] += 1.0;             // the identity's column
+          const double* li = &P[(size_t)i * K];
+          for (int k = i0; k < i; ++k) {
+            const double lik = li[k];
+            const double* xk = &X[(size_t)(k - j0) * w];
+            for (int c = 0; c < w; ++c) xr[c] -= lik * xk[c];
+          }
+          for (int c = 0; c < w; ++c) xr[c] = xr[c] / li[i];
+          double* urow = &U[(size_t)(K - 1 - i) * K];
+          for (int c = 0; c < w; ++c) urow[K - 1 - (j0 + c)] = xr[c];
         }
-        for (int c = 0; c < w; ++c) wi[c] = wi[c] / li[i];
-        double* urow = &U[(size_t)(K - 1 - i) * K];
-        for (int c = 0; c < w; ++c) urow[K - 1 - (j0 + c)] = wi[c];
       }
     }
   }
