@@ -20,7 +20,10 @@
 // The truncated SVD is a block subspace iteration in float64 (block r + 32,
 // Gaussian start, re-orthonormalised every half step) with a Rayleigh-Ritz
 // extraction; it stops when the captured energy sum_{i<r} sigma_i^2 stops
-// changing.
+// changing.  On a slowly converging (flat) spectrum it steps on the Gram
+// matrix of the smaller side instead and returns to W_hat for the extraction.
+// Every reduction adds its partial sums in a fixed order, so the prepared
+// bytes are the same for any number of host threads.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
