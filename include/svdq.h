@@ -49,7 +49,8 @@ typedef enum {
   SVDQ_OK = 0,
   SVDQ_EINVAL = 1,          /* null pointer, bad enum, inconsistent sizes          */
   SVDQ_EUNSUPPORTED = 2,    /* shape or option this build does not implement       */
-  SVDQ_ENOMEM = 3,          /* host or device allocation failed (prepare only)     */
+  SVDQ_ENOMEM = 3,          /* host or device allocation failed (prepare, set_lora,
+                               deserialize; never a forward)                        */
   SVDQ_ECUDA = 4,           /* a CUDA runtime/driver call failed                   */
   SVDQ_ENOCONVERGE = 5,     /* the truncated SVD did not converge                  */
   SVDQ_ETIMEOUT = 6,        /* a bounded device wait expired (read with CHECK)     */
@@ -110,7 +111,8 @@ typedef struct {
   int K, N, rank, format;
   int device;               /* CUDA ordinal, or -1 for a host-only layer           */
   int g_x_exp, g_w_exp;     /* NVFP4 tensor scales g = 2^exp (0 for INT4)          */
-  int svd_iterations;       /* subspace iterations the SVD took                    */
+  int svd_iterations;       /* subspace steps the SVD took (on W_hat and, for a
+                               flat spectrum, on its smaller Gram matrix)        */
   double svd_tail_energy;   /* ||W_hat||_F^2 - sum_{i<r} sigma_i^2                 */
 } svdq_layer_info;
 
@@ -212,8 +214,8 @@ const char* svdq_status_string(svdq_status s);
  * and svdq_workspace_bytes grows accordingly.  Blocking: synchronizes the
  * device before replacing the adapter's device buffers, so no forward of this
  * layer may be pending on another thread.  Errors: SVDQ_EINVAL (r < 0, null
- * factors, non-finite scale), SVDQ_EUNSUPPORTED (r > 32, SVDQ_W4A16_INT4),
- * SVDQ_ENOMEM, SVDQ_ECUDA.  The fc1 -> fc2 chain (svdq_mlp_*) does not take
+ * factors, non-finite scale), SVDQ_EUNSUPPORTED (r > 32, a SVDQ_W4A16_INT4 or
+ * SVDQ_W8A8_INT8 layer), SVDQ_ENOMEM, SVDQ_ECUDA.  The fc1 -> fc2 chain (svdq_mlp_*) does not take
  * layers with an adapter (SVDQ_EUNSUPPORTED). */
 svdq_status svdq_set_lora(svdq_layer* layer, int r, const uint16_t* A_bf16, const uint16_t* B_bf16,
                           float scale);
@@ -234,7 +236,7 @@ size_t svdq_serialized_bytes(const svdq_layer* layer);
 svdq_status svdq_serialize(const svdq_layer* layer, void* dst, size_t bytes);
 svdq_status svdq_deserialize(const void* src, size_t bytes, int device, svdq_layer** out);
 
-/* ------------------------------------------------------------------ forward *//* ------------------------------------------------------------------ forward */
+/* ------------------------------------------------------------------ forward */
 
 /* Workspace bytes a forward over M tokens needs (activation codes, scales in the
  * tensor-core layout and the BF16 down projection X L1d).  0 on bad input. */
@@ -260,8 +262,9 @@ size_t svdq_workspace_bytes(const svdq_layer* layer, int M);
  * the calibration batch's largest smoothed activation and about 220 times it;
  * a group whose smoothed activations exceed that upper limit is clamped to it
  * (its contribution shrinks by the ratio), and smaller scales are rounded to
- * FP16 subnormals (an absolute error below 2^-32 of the calibration maximum).  SVDQ_W4A16_INT4 (the adaptive-norm
- * linears, "stay W4A16") enqueues one weight-only GEMV kernel meant for a few
+ * FP16 subnormals (an absolute error below 2^-32 of the calibration maximum).
+ * SVDQ_W4A16_INT4 (the adaptive-norm linears, "stay W4A16") enqueues one
+ * weight-only GEMV kernel meant for a few
  * rows (M <= 16), needs no workspace (pass NULL, 0) and accepts only
  * SVDQ_FWD_CHECK among the flags.  The W4A4 kernels are programmatic dependent
  * launches: their prologues may overlap the preceding kernel on the stream,
@@ -271,17 +274,22 @@ svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, v
                                 void* workspace, size_t workspace_bytes,
                                 void* stream, unsigned flags);
 
-/* The first kernel alone (NVFP4/INT4/W8A8): writes the activation codes (device,
- * svdq_act_code_bytes(layer, M) bytes, two codes per byte with the even k in
- * the low nibble; INT4 codes are 4-bit two's complement, row-major [M][K/2];
- * NVFP4 codes are in the GEMM's tiled layout, see svdq_act_codes_to_logical),
- * the activation scales (device, svdq_act_scale_bytes(layer, M)
- * bytes: NVFP4 E4M3 in the tensor-core layout, INT4 BF16 [K/64][M rounded up
- * to 128], group-major, W8A8 FP32 [s_x | 1/s_x], each M rounded up to 128
- * entries; padding rows zero) and, when
- * the layer has a branch, XL = bf16(X L1d) (device [M][32] BF16 whatever the
- * rank: X L1d in the first `rank` columns, zeros after; [M][64] with a LoRA
- * adapter, see svdq_set_lora).  xl may be NULL for rank 0 without an adapter.  `mode` 0 = fused, 1 = quantize only, 2 = down projection only. */
+/* The first kernel alone (NVFP4/INT4/W8A8).  Writes
+ *   codes   device, svdq_act_code_bytes(layer, M) bytes: the 4-bit formats hold
+ *           two codes per byte, the even k in the low nibble (INT4: 4-bit two's
+ *           complement, row-major [M][K/2]; NVFP4: the GEMM's tiled layout, see
+ *           svdq_act_codes_to_logical); W8A8 one int8 per byte in the tiled
+ *           layout;
+ *   scales  device, svdq_act_scale_bytes(layer, M) bytes: NVFP4 E4M3 in the
+ *           tensor-core layout, INT4 BF16 [K/64][M rounded up to 128]
+ *           (group-major), W8A8 FP32 [s_x | 1/s_x], each M rounded up to 128
+ *           entries; padding rows zero;
+ *   xl      when the layer has a branch, XL = bf16(X L1d): device [M][32] BF16
+ *           whatever the rank (X L1d in the first `rank` columns, zeros after),
+ *           [M][64] with a LoRA adapter (see svdq_set_lora); may be NULL for
+ *           rank 0 without an adapter.
+ * W8A8 runs its per-token scale pass first (not in mode 2).  `mode` 0 = fused,
+ * 1 = quantize only, 2 = down projection only. */
 svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int M,
                               void* codes, void* scales, void* xl,
                               void* stream, int mode);
