@@ -343,8 +343,8 @@ svdq_status svdq_check(const svdq_layer* layer, void* stream);
  * order differs from the first kernel's, so XL2 may differ from it by a BF16
  * rounding).  fc1's BF16 output and fc2's first kernel disappear from the path.
  *
- * Both layers: SVDQ_NVFP4, prepared on the same device, fc1's N equal to
- * fc2's K (else SVDQ_EUNSUPPORTED).  fc2's calibration batch (its lam and
+ * Both layers: SVDQ_NVFP4, prepared on the same device, without a LoRA
+ * adapter, fc1's N equal to fc2's K (else SVDQ_EUNSUPPORTED).  fc2's calibration batch (its lam and
  * activation tensor scale) is used as is.
  *
  * svdq_mlp_workspace_bytes: workspace of svdq_mlp_forward (and of
