@@ -179,17 +179,23 @@ svdq_status svdq_prepare(const svdq_config* cfg, int K, int N,
                          const uint16_t* calib_bf16, int M_calib,
                          int device, svdq_layer** out);
 
+/* Frees the layer and its device buffers; NULL is a no-op. */
 void svdq_destroy(svdq_layer* layer);
 
+/* Fills *info; SVDQ_EINVAL for a NULL argument. */
 svdq_status svdq_get_info(const svdq_layer* layer, svdq_layer_info* info);
 
-/* Bytes of tensor `id` (0 if the layer's format has no such tensor). */
+/* Bytes of tensor `id` (0 if the layer's format has no such tensor, for an
+ * unknown id or a NULL layer). */
 size_t svdq_tensor_bytes(const svdq_layer* layer, int id);
 
 /* Copy tensor `id` into host memory `dst` of `bytes` (must equal
- * svdq_tensor_bytes).  Host-side; no GPU work. */
+ * svdq_tensor_bytes, which must not be 0; else SVDQ_EINVAL).  Host-side; no
+ * GPU work. */
 svdq_status svdq_export(const svdq_layer* layer, int id, void* dst, size_t bytes);
 
+/* A short English description of `s`; never NULL ("unknown status" for a
+ * value outside svdq_status). */
 const char* svdq_status_string(svdq_status s);
 
 /* svdq_set_lora -- attach a LoRA adapter (W -> W + scale A B) to the layer's
