@@ -233,11 +233,12 @@ svdq_status svdq_set_lora(svdq_layer* layer, int r, const uint16_t* A_bf16, cons
  * `device` (or host-only with -1), without repeating the SVD or the
  * quantization.  Preparation-only intermediates (the residual R, the float64
  * L1 and L2, the GPTQ factor) are not stored: their svdq_tensor_bytes are 0 on
- * a deserialized layer.  The byte layout is "SVDQ", a version, the scalar
- * fields, then each array as a 64-bit byte count and its bytes (host byte
- * order).  svdq_deserialize checks every size against the shape and format
- * and returns SVDQ_EINVAL on any mismatch or truncation; SVDQ_ENOMEM,
- * SVDQ_ECUDA as for svdq_prepare. */
+ * a deserialized layer.  The byte layout is "SVDQ", a version (2), the scalar
+ * fields, then each array as a 64-bit byte count and its bytes, then a 64-bit
+ * FNV-1a checksum of all the bytes before it (host byte order throughout).
+ * svdq_deserialize checks the checksum and every size against the shape and
+ * format, and returns SVDQ_EINVAL on any mismatch, corruption or truncation;
+ * SVDQ_ENOMEM, SVDQ_ECUDA as for svdq_prepare. */
 size_t svdq_serialized_bytes(const svdq_layer* layer);
 svdq_status svdq_serialize(const svdq_layer* layer, void* dst, size_t bytes);
 svdq_status svdq_deserialize(const void* src, size_t bytes, int device, svdq_layer** out);

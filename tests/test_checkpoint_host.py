@@ -1,6 +1,8 @@
 """Checkpoints of prepared layers (svdq_serialize / svdq_deserialize), on the
 host: every stored tensor and the layer info survive the round trip for each
-format, with and without a LoRA adapter; damaged bytes are refused."""
+format, with and without a LoRA adapter; damaged bytes are refused, both by
+the checksum and, for bytes re-signed after the change, by the checks of
+each field against the shape and format."""
 import numpy as np
 import pytest
 
@@ -48,17 +50,63 @@ def test_round_trip(fmt, rank, lora):
     assert R.serialize() == blob
 
 
+def _fnv1a64(data: bytes) -> int:
+    """FNV-1a, 64-bit (Fowler, Noll and Vo), from its published definition."""
+    h = 0xCBF29CE484222325
+    for b in data:
+        h = ((h ^ b) * 0x100000001B3) & 0xFFFFFFFFFFFFFFFF
+    return h
+
+
+def _resign(blob: bytearray) -> bytes:
+    """The bytes with their trailing checksum recomputed."""
+    body = bytes(blob[:-8])
+    return body + _fnv1a64(body).to_bytes(8, "little")
+
+
+def test_checksum_is_fnv1a_of_the_rest():
+    blob = _layer("int4", 32, lora=True).serialize()
+    assert int.from_bytes(blob[-8:], "little") == _fnv1a64(blob[:-8])
+    assert int.from_bytes(blob[4:8], "little") == 2                     # format version
+
+
+def test_every_single_byte_change_is_refused():
+    blob = _layer("nvfp4", 32).serialize()
+    rng = np.random.default_rng(11)
+    positions = sorted(set(range(0, 96)) | set(rng.integers(0, len(blob), 300).tolist()) |
+                       set(range(len(blob) - 8, len(blob))))
+    for pos in positions:
+        bad = bytearray(blob)
+        bad[pos] ^= 1 << int(rng.integers(0, 8))
+        with pytest.raises(lib.SvdqError) as e:
+            lib.Layer.deserialize(bytes(bad), device=-1)
+        assert e.value.status == lib.EINVAL, pos
+
+
 def test_damaged_bytes_are_refused():
     blob = bytearray(_layer("nvfp4", 32).serialize())
     for bad in (bytes(blob[:-1]), bytes(blob[:40]), b"XXXX" + bytes(blob[4:]), bytes(blob) + b"\0"):
         with pytest.raises(lib.SvdqError) as e:
             lib.Layer.deserialize(bad, device=-1)
         assert e.value.status == lib.EINVAL
-    # a size field that disagrees with the shape
+    # fields that disagree with the shape or format, re-signed so that only the
+    # field checks can refuse them
+    assert lib.Layer.deserialize(_resign(bytearray(blob)), device=-1).info["K"] == 256
+    for off, delta in ((8, 64), (12, 16), (16, 1), (20, 7), (32, 40)):   # K, N, rank, format, lora_r
+        wrong = bytearray(blob)
+        wrong[off:off + 4] = ((int.from_bytes(blob[off:off + 4], "little") + delta) % 2 ** 32).to_bytes(4, "little")
+        with pytest.raises(lib.SvdqError) as e:
+            lib.Layer.deserialize(_resign(wrong), device=-1)
+        assert e.value.status == lib.EINVAL, off
+    # an array's byte count that no longer matches its bytes
+    hdr = 64
     wrong = bytearray(blob)
-    wrong[8:12] = (int.from_bytes(blob[8:12], "little") + 64).to_bytes(4, "little")   # K
-    with pytest.raises(lib.SvdqError):
-        lib.Layer.deserialize(bytes(wrong), device=-1)
+    n0 = int.from_bytes(blob[hdr:hdr + 8], "little")                    # lam: K floats
+    assert n0 == 256 * 4
+    wrong[hdr:hdr + 8] = (n0 - 4).to_bytes(8, "little")
+    with pytest.raises(lib.SvdqError) as e:
+        lib.Layer.deserialize(_resign(wrong), device=-1)
+    assert e.value.status == lib.EINVAL
 
 
 def test_chain_and_adapter_rules_on_host_only_layers():

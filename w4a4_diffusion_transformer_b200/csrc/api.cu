@@ -597,11 +597,23 @@ svdq_status upload_lora(svdq_layer* L) {
 // A prepared layer as bytes: "SVDQ", version, the scalar fields, then each
 // array as a 64-bit byte count followed by its bytes (lam, inv_lam, sigma,
 // L1d, L2b, w_codes, w_scales_e4m3, w_scales_bf16, w_scales_f32, bias,
-// lora_A, lora_B).  The preparation-only intermediates (R, L1, L2, the GPTQ
-// factor) are not part of it.
+// lora_A, lora_B), then a 64-bit FNV-1a checksum of everything before it.
+// The preparation-only intermediates (R, L1, L2, the GPTQ factor) are not
+// part of it.
 
 constexpr uint32_t kSerialMagic = 0x51445653u;   // "SVDQ"
-constexpr uint32_t kSerialVersion = 1;
+constexpr uint32_t kSerialVersion = 2;
+
+// FNV-1a, 64-bit (Fowler, Noll and Vo): xor in each byte, then multiply by
+// the FNV prime, starting from the offset basis.
+uint64_t fnv1a64(const uint8_t* p, size_t n) {
+  uint64_t h = 0xCBF29CE484222325ull;
+  for (size_t i = 0; i < n; ++i) {
+    h ^= p[i];
+    h *= 0x100000001B3ull;
+  }
+  return h;
+}
 
 struct SerialHeader {
   uint32_t magic, version;
@@ -628,7 +640,7 @@ void serial_arrays(F&& f, H& h) {
 }
 
 size_t serialized_bytes(const HostPrep& h) {
-  size_t n = sizeof(SerialHeader);
+  size_t n = sizeof(SerialHeader) + 8;   // header and checksum
   serial_arrays([&](const auto& v) { n += 8 + v.size() * sizeof(v[0]); }, h);
   return n;
 }
@@ -1060,16 +1072,21 @@ svdq_status svdq_serialize(const svdq_layer* L, void* dst, size_t bytes) {
         o += 8 + n;
       },
       h);
+  const uint64_t sum = fnv1a64(static_cast<const uint8_t*>(dst), (size_t)(o - static_cast<uint8_t*>(dst)));
+  std::memcpy(o, &sum, 8);
   return SVDQ_OK;
 }
 
 svdq_status svdq_deserialize(const void* src, size_t bytes, int device, svdq_layer** out) {
   if (!out) return SVDQ_EINVAL;
   *out = nullptr;
-  if (!src || bytes < sizeof(SerialHeader)) return SVDQ_EINVAL;
+  if (!src || bytes < sizeof(SerialHeader) + 8) return SVDQ_EINVAL;
   SerialHeader hd;
   std::memcpy(&hd, src, sizeof(hd));
   if (hd.magic != kSerialMagic || hd.version != kSerialVersion) return SVDQ_EINVAL;
+  uint64_t sum = 0;
+  std::memcpy(&sum, static_cast<const uint8_t*>(src) + bytes - 8, 8);
+  if (sum != fnv1a64(static_cast<const uint8_t*>(src), bytes - 8)) return SVDQ_EINVAL;   // corrupted
   if (hd.format < SVDQ_NVFP4 || hd.format > SVDQ_W8A8_INT8 || hd.K <= 0 || hd.N <= 0 || hd.K % 64 ||
       hd.rank < 0 || hd.rank > 32 || hd.lora_r < 0 || hd.lora_r > 32)
     return SVDQ_EINVAL;
@@ -1089,7 +1106,7 @@ svdq_status svdq_deserialize(const void* src, size_t bytes, int device, svdq_lay
   h.w_amax = hd.w_amax;
   h.svd_tail_energy = hd.svd_tail_energy;
   const uint8_t* in = static_cast<const uint8_t*>(src) + sizeof(hd);
-  const uint8_t* end = static_cast<const uint8_t*>(src) + bytes;
+  const uint8_t* end = static_cast<const uint8_t*>(src) + bytes - 8;
   bool ok = true;
   try {
     serial_arrays(
