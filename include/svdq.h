@@ -162,7 +162,9 @@ typedef enum {
  *              maxima and the activation tensor scale); required for the W4A4
  *              formats, ignored (may be NULL) for SVDQ_W4A16_INT4.
  *   device     CUDA ordinal that receives the prepared buffers, or -1 to keep
- *              the layer on the host (export only; forwards return SVDQ_ESTATE).
+ *              the layer on the host (export only; forwards return SVDQ_ESTATE);
+ *              below -1: SVDQ_EINVAL; a device the process cannot use:
+ *              SVDQ_ECUDA.
  *   out        receives the new layer; owned by the caller, free with svdq_destroy.
  *
  * Runs on the host (multi-threaded), then copies the prepared buffers to

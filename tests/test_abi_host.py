@@ -223,3 +223,26 @@ def test_prepare_refuses_non_finite_inputs(where, bits):
     if where == "calib":                                            # weight-only layers ignore the batch
         L = lib.Layer.prepare(W, b, Xc, fmt="w4a16", rank=0, device=-1)
         assert L.info["rank"] == 0
+
+
+def test_device_argument():
+    d = syn.custom_layer(19, M=8, K=128, N=64)
+    args = (syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]), syn.bf16_bits(d["Xc"]))
+    blob = lib.Layer.prepare(*args, device=-1).serialize()
+    for call in (lambda: lib.Layer.prepare(*args, device=-2), lambda: lib.Layer.deserialize(blob, device=-2)):
+        with pytest.raises(lib.SvdqError) as e:
+            call()
+        assert e.value.status == lib.EINVAL
+
+
+def test_device_placement_without_a_gpu_fails_cleanly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("this machine has a GPU: placement succeeds")
+    d = syn.custom_layer(20, M=8, K=128, N=64)
+    args = (syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]), syn.bf16_bits(d["Xc"]))
+    blob = lib.Layer.prepare(*args, device=-1).serialize()
+    for call in (lambda: lib.Layer.prepare(*args, device=0), lambda: lib.Layer.deserialize(blob, device=0)):
+        with pytest.raises(lib.SvdqError) as e:
+            call()
+        assert e.value.status == lib.ECUDA

@@ -765,7 +765,7 @@ svdq_status svdq_prepare(const svdq_config* cfg, int K, int N, const uint16_t* W
                          const uint16_t* calib_bf16, int M_calib, int device, svdq_layer** out) {
   if (!out) return SVDQ_EINVAL;
   *out = nullptr;
-  if (!cfg || !W_bf16 || K <= 0 || N <= 0) return SVDQ_EINVAL;
+  if (!cfg || !W_bf16 || K <= 0 || N <= 0 || device < -1) return SVDQ_EINVAL;
   if (cfg->format < SVDQ_NVFP4 || cfg->format > SVDQ_W8A8_INT8) return SVDQ_EINVAL;
   const bool wo = cfg->format == SVDQ_W4A16_INT4;
   if (cfg->flags & ~(SVDQ_PREP_GPTQ | SVDQ_PREP_KEEP_GPTQ_FACTOR)) return SVDQ_EINVAL;
@@ -1080,7 +1080,7 @@ svdq_status svdq_serialize(const svdq_layer* L, void* dst, size_t bytes) {
 svdq_status svdq_deserialize(const void* src, size_t bytes, int device, svdq_layer** out) {
   if (!out) return SVDQ_EINVAL;
   *out = nullptr;
-  if (!src || bytes < sizeof(SerialHeader) + 8) return SVDQ_EINVAL;
+  if (!src || bytes < sizeof(SerialHeader) + 8 || device < -1) return SVDQ_EINVAL;
   SerialHeader hd;
   std::memcpy(&hd, src, sizeof(hd));
   if (hd.magic != kSerialMagic || hd.version != kSerialVersion) return SVDQ_EINVAL;
