@@ -297,14 +297,16 @@ svdq_status svdq_linear_forward(const svdq_layer* layer, const void* X, int M, v
  *           whatever the rank (X L1d in the first `rank` columns, zeros after),
  *           [M][64] with a LoRA adapter (see svdq_set_lora); may be NULL for
  *           rank 0 without an adapter.
- * W8A8 runs its per-token scale pass first (not in mode 2).  `mode` 0 = fused,
- * 1 = quantize only, 2 = down projection only. */
+ * X and every output buffer 16-byte aligned (else SVDQ_EINVAL).  W8A8 runs its
+ * per-token scale pass first (not in mode 2).  `mode` 0 = fused, 1 = quantize
+ * only, 2 = down projection only. */
 svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int M,
                               void* codes, void* scales, void* xl,
                               void* stream, int mode);
 
-/* The second kernel alone: Y from the first kernel's outputs.  flags:
- * SVDQ_FWD_GELU, SVDQ_FWD_NO_BRANCH, SVDQ_FWD_CHECK. */
+/* The second kernel alone: Y from the first kernel's outputs (codes, scales,
+ * xl and Y 16-byte aligned, else SVDQ_EINVAL).  flags: SVDQ_FWD_GELU,
+ * SVDQ_FWD_NO_BRANCH, SVDQ_FWD_CHECK. */
 svdq_status svdq_gemm(const svdq_layer* layer, const void* codes, const void* scales,
                       const void* xl, int M, void* Y, void* stream, unsigned flags);
 

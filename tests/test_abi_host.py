@@ -246,3 +246,23 @@ def test_device_placement_without_a_gpu_fails_cleanly():
         with pytest.raises(lib.SvdqError) as e:
             call()
         assert e.value.status == lib.ECUDA
+
+
+def test_operand_alignment_is_checked_before_the_layer_state():
+    # raw addresses (never dereferenced: the host-only layer stops every call)
+    d = syn.custom_layer(21, M=8, K=128, N=64)
+    L = lib.Layer.prepare(syn.bf16_bits(d["W"]), None, syn.bf16_bits(d["Xc"]), device=-1)
+    A, B = 0x10000, 0x10008                                     # 16-byte aligned / not
+    for fn in (lambda x, y: L.forward(x, 8, y, 0x20000, 1 << 20), lambda x, y: L.forward_static(x, 8, y)):
+        for x, y, want in ((A, A, lib.ESTATE), (B, A, lib.EINVAL), (A, B, lib.EINVAL)):
+            with pytest.raises(lib.SvdqError) as e:
+                fn(x, y)
+            assert e.value.status == want, (hex(x), hex(y))
+    for codes, scales, xl, want in ((A, A, A, lib.ESTATE), (B, A, A, lib.EINVAL), (A, B, A, lib.EINVAL),
+                                    (A, A, B, lib.EINVAL)):
+        with pytest.raises(lib.SvdqError) as e:
+            L.quantize_act(A, 8, codes, scales, xl)
+        assert e.value.status == want
+        with pytest.raises(lib.SvdqError) as e:
+            L.gemm(codes, scales, xl, 8, A)
+        assert e.value.status == want

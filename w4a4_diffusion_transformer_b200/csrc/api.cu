@@ -329,10 +329,11 @@ svdq_status upload_layer(svdq_layer* L, int device) {
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
 }
 
+// Arguments first (SVDQ_EINVAL), then the layer's state (SVDQ_ESTATE).
 svdq_status check_forward_args(const svdq_layer* L, const void* X, int M, const void* Y) {
   if (!L || !X || !Y || M < 1) return SVDQ_EINVAL;
-  if (L->device < 0) return SVDQ_ESTATE;
   if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(Y) & 15)) return SVDQ_EINVAL;
+  if (L->device < 0) return SVDQ_ESTATE;
   return SVDQ_OK;
 }
 
@@ -945,6 +946,7 @@ svdq_status svdq_act_scales_to_logical(const svdq_layer* L, const void* device_l
 
 svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int M, void* codes, void* scales, void* xl,
                               void* stream, int mode) {
+  if ((reinterpret_cast<uintptr_t>(scales) & 15) || (reinterpret_cast<uintptr_t>(xl) & 15)) return SVDQ_EINVAL;
   svdq_status st = check_forward_args(L, X, M, codes);
   if (st != SVDQ_OK) return st;
   if (!w4a4(L)) return SVDQ_EUNSUPPORTED;
@@ -965,6 +967,7 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int M, void* c
 
 svdq_status svdq_gemm(const svdq_layer* L, const void* codes, const void* scales, const void* xl, int M, void* Y,
                       void* stream, unsigned flags) {
+  if ((reinterpret_cast<uintptr_t>(scales) & 15) || (reinterpret_cast<uintptr_t>(xl) & 15)) return SVDQ_EINVAL;
   svdq_status st = check_forward_args(L, codes, M, Y);
   if (st != SVDQ_OK) return st;
   if (!w4a4(L)) return SVDQ_EUNSUPPORTED;

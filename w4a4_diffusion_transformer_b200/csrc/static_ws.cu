@@ -47,6 +47,7 @@ cudaError_t static_workspace_address(int device, void** out) {
 extern "C" svdq_status svdq_linear_forward_static(const svdq_layer* layer, const void* X, int M, void* Y,
                                                   void* stream, unsigned flags) {
   if (!layer || !X || !Y || M < 1) return SVDQ_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(Y) & 15)) return SVDQ_EINVAL;
   svdq_layer_info info;
   svdq_status st = svdq_get_info(layer, &info);
   if (st != SVDQ_OK) return st;
