@@ -152,3 +152,14 @@ def test_mlp_operand_sizes():
         lib.mlp_fc1(L1, L2, X, M, codes2, scales2, FakeCuda(M * 64 - 2), ws, 1 << 20)
     with pytest.raises(ValueError):
         lib.mlp_fc1(L1, L2, X, M, FakeCuda(L2.act_code_bytes(M) - 2), scales2, FakeCuda(M * 64), ws, 1 << 20)
+
+
+def test_layer_as_a_context_manager():
+    d = syn.custom_layer(66, M=8, K=128, N=64)
+    with lib.Layer.prepare(syn.bf16_bits(d["W"]), None, syn.bf16_bits(d["Xc"]), device=-1) as L:
+        assert L.info["K"] == 128
+        blob = L.serialize()
+    assert L._h is None                                          # freed on leaving the block
+    with lib.Layer.deserialize(blob, device=-1) as R:
+        assert R.info["N"] == 64
+    assert R._h is None

@@ -235,6 +235,13 @@ class Layer:
         except Exception:
             pass
 
+    def __enter__(self) -> "Layer":
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+        return False
+
     @property
     def info(self) -> dict:
         i = LayerInfo()
