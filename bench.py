@@ -186,6 +186,17 @@ def allreduce_max(x, world):
     return float(t.item())
 
 
+def guarded(errors, name, fn):
+    """Run one secondary section.  Its failure is recorded under `name` in
+    `errors` (so it shows in the JSON line) instead of ending the run: the
+    headline numbers are measured before any secondary section starts."""
+    try:
+        return fn()
+    except Exception as e:          # noqa: BLE001 - recorded, not hidden
+        errors[name] = f"{type(e).__name__}: {e}"[:400]
+        return None
+
+
 def whole_job_tflops(flops_per_step, world, step_ms_max):
     """Whole-job throughput: every rank runs its own replica of the step, and
     the job takes as long as its slowest rank."""
@@ -471,20 +482,27 @@ def other_layers(pkg, syn, stream, flush_l2, n, peaks, only=None):
     def want(name):
         return only is None or name in only
 
+    errors = {}
     # INT4 variant
     if want("int4"):
-        d = syn.layer("qkv_int4")
-        w4a4_layer(d, "int4", d["X"], 0, "int4_qkv")
+        def int4():
+            d = syn.layer("qkv_int4")
+            w4a4_layer(d, "int4", d["X"], 0, "int4_qkv")
+        guarded(errors, "int4", int4)
     # W8A8 variant (rank 16 at 8 bits) on the attention-output shape
     if want("w8a8"):
-        d = syn.layer("attn_out")
-        w4a4_layer(d, "w8a8", d["X"], 0, "w8a8_attn_out")
+        def w8a8():
+            d = syn.layer("attn_out")
+            w4a4_layer(d, "w8a8", d["X"], 0, "w8a8_attn_out")
+        guarded(errors, "w8a8", w8a8)
     if want("mlp"):
-        mlp_pair(pkg, syn, stream, n, w4a4_layer, dev, out)
+        guarded(errors, "mlp", lambda: mlp_pair(pkg, syn, stream, n, w4a4_layer, dev, out))
     if want("lora"):
-        lora_layer(pkg, syn, stream, n, dev, out)
+        guarded(errors, "lora", lambda: lora_layer(pkg, syn, stream, n, dev, out))
     if want("w4a16"):
-        w4a16_adaln(pkg, syn, stream, flush_l2, n, peaks, dev, out)
+        guarded(errors, "w4a16", lambda: w4a16_adaln(pkg, syn, stream, flush_l2, n, peaks, dev, out))
+    if errors:
+        out["section_errors"] = errors
     return out
 
 
@@ -796,24 +814,35 @@ def main():
         "clocks": clk.summary(),
     }
     only = None if args.only is None else set(args.only.split(","))
+    errors = {}
     if rank == 0 and world == 1 and not args.no_other_layers:
-        out["other_layers"] = other_layers(pkg, syn, stream, flush_l2, max(30, min(200, args.steps)), peaks, only)
+        others = guarded(errors, "other_layers", lambda: other_layers(pkg, syn, stream, flush_l2,
+                                                                       max(30, min(200, args.steps)), peaks, only))
+        out["other_layers"] = others if others is not None else {}
         if only is None or "block" in only:
-            out["other_layers"]["block_b4"] = block_b4(pkg, syn, stream, max(20, min(100, args.steps)), peaks,
-                                                       fp4_peak)
+            blk = guarded(errors, "block_b4", lambda: block_b4(pkg, syn, stream, max(20, min(100, args.steps)),
+                                                                peaks, fp4_peak))
+            if blk is not None:
+                out["other_layers"]["block_b4"] = blk
     if rank == 0 and world == 1 and not args.no_other_layers and only is None:
-        lib_us = library_nvfp4_gemm_us(M, K, N, n_k)
-        out["library_context"] = {
-            "cublaslt_nvfp4_gemm_us": lib_us, "k2_us": k2_ms * 1e3, "bare_k2_us": bare_k2_ms * 1e3,
-            "note": "bare NVFP4 GEMM of the same shape through torch._scaled_mm (no low-rank branch, no bias), "
-                    "back to back over rotating operand sets; context, not a baseline"}
-        probe = nvfp4_peak_probe(dev)
-        if probe is not None:
-            out["nvfp4_peak_measured"] = probe
-            out["pct_nvfp4_peak"]["of_cublaslt_8192"] = value / world / probe["tflops"]
-            out["roofline"]["frac_of_cublaslt_8192"] = k2_achieved / probe["tflops"]
+        def library_probes():
+            lib_us = library_nvfp4_gemm_us(M, K, N, n_k)
+            out["library_context"] = {
+                "cublaslt_nvfp4_gemm_us": lib_us, "k2_us": k2_ms * 1e3, "bare_k2_us": bare_k2_ms * 1e3,
+                "note": "bare NVFP4 GEMM of the same shape through torch._scaled_mm (no low-rank branch, no bias), "
+                        "back to back over rotating operand sets; context, not a baseline"}
+            probe = nvfp4_peak_probe(dev)
+            if probe is not None:
+                out["nvfp4_peak_measured"] = probe
+                out["pct_nvfp4_peak"]["of_cublaslt_8192"] = value / world / probe["tflops"]
+                out["roofline"]["frac_of_cublaslt_8192"] = k2_achieved / probe["tflops"]
+        guarded(errors, "library_probes", library_probes)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(d, M, K, N)
+        cpu = guarded(errors, "cpu_baseline", lambda: cpu_baseline(d, M, K, N))
+        if cpu is not None:
+            out["cpu_baseline"] = cpu
+    if errors:
+        out["section_errors"] = errors
     for st in sets:
         st.L.close()
     if world > 1:

@@ -67,3 +67,16 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     args = types.SimpleNamespace(gpus=2, steps=1, warmup=0)
     assert bench.run_reference(args) is None
     assert capsys.readouterr().out == ""
+
+
+def test_a_failing_secondary_section_is_recorded_not_fatal():
+    errors = {}
+    assert bench.guarded(errors, "ok", lambda: 7) == 7
+    assert errors == {}
+
+    def broken():
+        raise RuntimeError("device lost " + "x" * 1000)
+
+    assert bench.guarded(errors, "lora", broken) is None
+    assert list(errors) == ["lora"] and errors["lora"].startswith("RuntimeError: device lost")
+    assert len(errors["lora"]) <= 400
