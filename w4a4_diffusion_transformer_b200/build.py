@@ -54,26 +54,42 @@ def _run(cmd, log):
     return r.stdout
 
 
+def _compile(cmd, obj, log):
+    """One compile into a temporary object, renamed into place on success, so
+    an interrupted build never leaves a truncated object that looks fresh."""
+    tmp = obj + ".tmp"
+    _run(cmd + ["-o", tmp], log)
+    os.replace(tmp, obj)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every source for sm_100a and link libsvdq.so; returns its path."""
+    """Compile every source for sm_100a and link libsvdq.so; returns its path.
+    Stale sources compile in parallel (one process each)."""
+    from concurrent.futures import ThreadPoolExecutor
+
     os.makedirs(BUILD, exist_ok=True)
     log: list = []
-    objs = []
+    objs, jobs = [], []
     changed = force or not os.path.exists(LIB)
-    for src in CUDA_SOURCES:
+    for src in CUDA_SOURCES + CXX_SOURCES:
         s = os.path.join(CSRC, src)
         o = os.path.join(BUILD, src + ".o")
         objs.append(o)
         if force or _stale(o, s):
-            _run([_nvcc()] + ARCH + NVCC_FLAGS + ["-c", s, "-o", o], log)
-            changed = True
-    for src in CXX_SOURCES:
-        s = os.path.join(CSRC, src)
-        o = os.path.join(BUILD, src + ".o")
-        objs.append(o)
-        if force or _stale(o, s):
-            _run(["g++"] + CXX_FLAGS + ["-c", s, "-o", o], log)
-            changed = True
+            cxx = src in CXX_SOURCES
+            cmd = (["g++"] + CXX_FLAGS if cxx else [_nvcc()] + ARCH + NVCC_FLAGS) + ["-c", s]
+            jobs.append((cmd, o))
+    if jobs:
+        logs = [[] for _ in jobs]
+        with ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as pool:
+            futures = [pool.submit(_compile, cmd, o, lg) for (cmd, o), lg in zip(jobs, logs)]
+            errors = [f.exception() for f in futures]
+        for lg in logs:
+            log.extend(lg)
+        failed = [e for e in errors if e is not None]
+        if failed:
+            raise failed[0]
+        changed = True
     if changed or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
         tmp = LIB + ".tmp"
         _run([_nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-Xcompiler", "-fopenmp", "-lgomp"], log)
