@@ -9,6 +9,7 @@ Hessian of the same calibration batch.
 """
 import numpy as np
 import pytest
+from hypothesis import HealthCheck, given, settings, strategies as st
 
 import synthetic as syn
 from oracle import svdq_oracle as o
@@ -105,3 +106,21 @@ def test_flags_validation():
     L0 = _prep(d, "nvfp4", flags=0)
     q = o.quantize_weights(L0.export("R"), "nvfp4")
     np.testing.assert_array_equal(L0.export("w_codes"), o.pack_nibbles(q["w_codes"]))
+
+
+
+@settings(max_examples=20, deadline=None, derandomize=True, suppress_health_check=list(HealthCheck))
+@given(fmt=st.sampled_from(["nvfp4", "int4"]), kb=st.integers(1, 6), nb=st.integers(1, 8),
+       seed=st.integers(0, 10 ** 6), mcal=st.integers(8, 160), latent=st.sampled_from([0, 4, 16]),
+       rank=st.sampled_from([0, 32]))
+def test_codes_bit_exact_over_random_shapes(fmt, kb, nb, seed, mcal, latent, rank):
+    # K and N span several factor blocks of 128 and ragged tails; calibration
+    # batches both smaller and larger than K
+    K, N = 64 * kb, 16 * nb
+    d = syn.custom_layer(seed, 4, K, N, latent_rank=latent, calib_tokens=mcal)
+    L = _prep(d, fmt, rank=rank)
+    q, codes, scales = _oracle_codes(L, fmt)
+    np.testing.assert_array_equal(L.export("w_codes"), codes)
+    np.testing.assert_array_equal(L.export("w_scales"), scales)
+    Uo = o.gptq_factor(o.gptq_hessian(d["Xc"], L.export("inv_lambda")))
+    assert np.max(np.abs(L.export("gptq_U") - Uo)) <= 1e-10 * np.max(np.abs(Uo))
