@@ -5,6 +5,7 @@ the checksum and, for bytes re-signed after the change, by the checks of
 each field against the shape and format."""
 import numpy as np
 import pytest
+from hypothesis import HealthCheck, given, settings, strategies as st
 
 import synthetic as syn
 
@@ -124,3 +125,26 @@ def test_chain_and_adapter_rules_on_host_only_layers():
                 syn.bf16_bits(syn.to_bf16(rng.standard_normal((4, 512)))), 2.0)
     R = lib.Layer.deserialize(L1.serialize(), device=-1)
     np.testing.assert_array_equal(R.export("lora_B"), L1.export("lora_B"))
+
+
+@settings(max_examples=25, deadline=None, derandomize=True, suppress_health_check=list(HealthCheck))
+@given(fmt=st.sampled_from(["nvfp4", "int4", "w8a8", "w4a16"]), kb=st.integers(1, 4), nb=st.integers(1, 12),
+       seed=st.integers(0, 10 ** 6), lora_r=st.integers(0, 32), with_rank=st.booleans())
+def test_round_trip_over_random_layers(fmt, kb, nb, seed, lora_r, with_rank):
+    K, N = 64 * kb, 16 * nb
+    rank = 0 if fmt == "w4a16" or not with_rank else (16 if fmt == "w8a8" else 32)
+    d = syn.custom_layer(seed, M=4, K=K, N=N)
+    L = lib.Layer.prepare(syn.bf16_bits(d["W"]), syn.bf16_bits(d["bias"]),
+                          None if fmt == "w4a16" else syn.bf16_bits(d["Xc"]), fmt=fmt, rank=rank, device=-1)
+    adapter = lora_r > 0 and fmt in ("nvfp4", "int4")
+    if adapter:
+        rng = np.random.default_rng(seed)
+        L.set_lora(syn.bf16_bits(syn.to_bf16(rng.standard_normal((K, lora_r)))),
+                   syn.bf16_bits(syn.to_bf16(rng.standard_normal((lora_r, N)))), 0.25)
+    blob = L.serialize()
+    R = lib.Layer.deserialize(blob, device=-1)
+    assert R.info == L.info
+    assert R.serialize() == blob
+    for name in KEPT + (["lora_A", "lora_B"] if adapter else []):
+        if lib.load().svdq_tensor_bytes(L._h, lib.TENSORS[name][0]):
+            np.testing.assert_array_equal(R.export(name), L.export(name), err_msg=name)
