@@ -1009,10 +1009,20 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
         }
       }
     } else {
-      for (size_t i = 0; i < Wh.size(); ++i) P.R[i] = (float)Wh[i];
+#pragma omp parallel for schedule(static)
+      for (int k = 0; k < K; ++k)
+        for (int n = 0; n < N; ++n) P.R[(size_t)k * N + n] = (float)Wh[(size_t)k * N + n];
       if (!w4a16) {
+        const int nch = row_chunks(K);
+        std::vector<double> part(nch);
+#pragma omp parallel for schedule(static)
+        for (int ch = 0; ch < nch; ++ch) {
+          const int r0 = ch * kRowChunk, r1 = std::min(K, r0 + kRowChunk);
+          const double* a = Wh.data() + (size_t)r0 * N;
+          part[ch] = dot4(a, a, (r1 - r0) * N);
+        }
         double tot = 0.0;
-        for (double v : Wh) tot += v * v;
+        for (int ch = 0; ch < nch; ++ch) tot += part[ch];
         P.svd_tail_energy = tot;
       }
     }
@@ -1027,8 +1037,9 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
         }
 
     // ---- residual quantization, groups along K for each output column n
-    float amax = 0.0f;
-    for (float v : P.R) amax = std::max(amax, std::fabs(v));
+    float amax = 0.0f;                      // a maximum: exact in any order
+#pragma omp parallel for schedule(static) reduction(max : amax)
+    for (size_t i = 0; i < P.R.size(); ++i) amax = std::max(amax, std::fabs(P.R[i]));
     P.w_amax = amax;
     if (cfg.format == SVDQ_W8A8_INT8) {
       // INT8, one group per output channel: s = fp32(a fp32(1/127)),
@@ -1078,31 +1089,44 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
       const float g = (float)std::ldexp(1.0, P.g_w_exp);
       const float c = (float)std::ldexp((double)(1.0f / 6.0f), -P.g_w_exp);
       P.w_scales_e4m3.assign((size_t)N * K / 16, 0);
+      // 16 output columns per task, so that each group's 16 rows are read as
+      // contiguous 64-byte row segments
 #pragma omp parallel for schedule(static)
-      for (int n = 0; n < N; ++n) {
-        float col[16];
+      for (int nb = 0; nb < (N + 15) / 16; ++nb) {
+        const int n0 = nb * 16, nc = std::min(16, N - n0);
+        float blk[16][16];
         uint8_t codes[16];
         for (int g16 = 0; g16 < K / 16; ++g16) {
-          for (int i = 0; i < 16; ++i) col[i] = P.R[(size_t)(g16 * 16 + i) * N + n];
-          P.w_scales_e4m3[(size_t)n * (K / 16) + g16] = nvfp4_group(col, c, g, codes);
-          for (int i = 0; i < 8; ++i)
-            P.w_codes[(size_t)n * (K / 2) + g16 * 8 + i] = (uint8_t)(codes[2 * i] | (codes[2 * i + 1] << 4));
+          for (int i = 0; i < 16; ++i)
+            for (int j = 0; j < nc; ++j) blk[j][i] = P.R[(size_t)(g16 * 16 + i) * N + n0 + j];
+          for (int j = 0; j < nc; ++j) {
+            const int n = n0 + j;
+            P.w_scales_e4m3[(size_t)n * (K / 16) + g16] = nvfp4_group(blk[j], c, g, codes);
+            for (int i = 0; i < 8; ++i)
+              P.w_codes[(size_t)n * (K / 2) + g16 * 8 + i] = (uint8_t)(codes[2 * i] | (codes[2 * i + 1] << 4));
+          }
         }
       }
       // activation tensor scale from the calibration batch, 4x headroom
       P.g_x_exp = pow2_ceil_exponent(4.0 * (double)P.x_amax / 2688.0);
     } else {
       P.w_scales_bf16.assign((size_t)N * K / 64, 0);
+      // 16 output columns per task (contiguous 64-byte row segments)
 #pragma omp parallel for schedule(static)
-      for (int n = 0; n < N; ++n) {
-        float col[64];
+      for (int nb = 0; nb < (N + 15) / 16; ++nb) {
+        const int n0 = nb * 16, nc = std::min(16, N - n0);
+        float blk[16][64];
         int8_t codes[64];
         for (int g64 = 0; g64 < K / 64; ++g64) {
-          for (int i = 0; i < 64; ++i) col[i] = P.R[(size_t)(g64 * 64 + i) * N + n];
-          P.w_scales_bf16[(size_t)n * (K / 64) + g64] = int4_group(col, codes);
-          for (int i = 0; i < 32; ++i)
-            P.w_codes[(size_t)n * (K / 2) + g64 * 32 + i] =
-                (uint8_t)((codes[2 * i] & 0xF) | ((codes[2 * i + 1] & 0xF) << 4));
+          for (int i = 0; i < 64; ++i)
+            for (int j = 0; j < nc; ++j) blk[j][i] = P.R[(size_t)(g64 * 64 + i) * N + n0 + j];
+          for (int j = 0; j < nc; ++j) {
+            const int n = n0 + j;
+            P.w_scales_bf16[(size_t)n * (K / 64) + g64] = int4_group(blk[j], codes);
+            for (int i = 0; i < 32; ++i)
+              P.w_codes[(size_t)n * (K / 2) + g64 * 32 + i] =
+                  (uint8_t)((codes[2 * i] & 0xF) | ((codes[2 * i + 1] & 0xF) << 4));
+          }
         }
       }
     }
