@@ -998,14 +998,20 @@ svdq_status host_prepare(const svdq_config& cfg, int K, int N, const uint16_t* W
       for (size_t i = 0; i < P.L2b.size(); ++i) P.L2b[i] = bf16_from_double(P.L2[i]);
       std::vector<double> L2v((size_t)r * N);
       for (size_t i = 0; i < L2v.size(); ++i) L2v[i] = bf16_to_float(P.L2b[i]);
-#pragma omp parallel for schedule(static)
-      for (int k = 0; k < K; ++k) {
-        double lk[128];
-        for (int i = 0; i < r; ++i) lk[i] = (double)P.lam[k] * (double)bf16_to_float(P.L1d[(size_t)k * r + i]);
-        for (int n = 0; n < N; ++n) {
-          double br = 0.0;
-          for (int i = 0; i < r; ++i) br += lk[i] * L2v[(size_t)i * N + n];
-          P.R[(size_t)k * N + n] = (float)(Wh[(size_t)k * N + n] - br);
+      // each element sums its r products in ascending i; a whole row at a
+      // time, so that the inner loop runs along contiguous columns
+#pragma omp parallel
+      {
+        std::vector<double> br(N);
+#pragma omp for schedule(static)
+        for (int k = 0; k < K; ++k) {
+          std::fill(br.begin(), br.end(), 0.0);
+          for (int i = 0; i < r; ++i) {
+            const double lki = (double)P.lam[k] * (double)bf16_to_float(P.L1d[(size_t)k * r + i]);
+            const double* l2 = &L2v[(size_t)i * N];
+            for (int n = 0; n < N; ++n) br[n] += lki * l2[n];
+          }
+          for (int n = 0; n < N; ++n) P.R[(size_t)k * N + n] = (float)(Wh[(size_t)k * N + n] - br[n]);
         }
       }
     } else {
